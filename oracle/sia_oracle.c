@@ -1,0 +1,299 @@
+/*
+ * sia_oracle.c -- plain, slow CPU oracle for indexed sparse attention over paged caches.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may call, link or load this file:
+ * only tests/, __graft_entry__.smoke() and the cpu_baseline / reference legs of bench.py use
+ * it.  It shares no code, header, table or constant with the CUDA library.
+ *
+ * What it computes follows the naive five-step decode chain printed in "Day 0 Inference
+ * Adaptation and Performance Optimization for Hybrid Sparse Attention LLMs" (section
+ * "Operator Fusion and Multi-Stream Scheduling"): score every historical position, weight and
+ * sum the heads, pick the Top-K positions, gather those rows of the primary paged KV cache and
+ * run softmax attention over them.  The index score is fixed as
+ *      I[t,s] = sum_h w[t,h] * ReLU(q[t,h] . k[s])
+ * (one index key per position shared by all heads), ties in Top-K go to the lower position,
+ * and every floating-point value is carried in fp64.
+ *
+ * Readings of points the pages leave open (each one is listed in the design doc):
+ *   - causal: query j of sequence b at position p sees positions 0..p (itself included);
+ *   - quantised index cache: value = e4m3 code decoded exactly, times its per-token scale
+ *     ("high-precision computation + low-precision cache": dequantise, then compute);
+ *   - Top-K output: the selected positions in ascending order, padded with -1 when fewer
+ *     than K positions are visible;
+ *   - the Top-K decision is taken on scores rounded to fp32, the precision the GPU ranks in
+ *     (for the integer-valued inputs used in tests that rounding is exact);
+ *   - attention (MLA absorbed form): logits use all DL+DR dims of the latent row, the output
+ *     is the softmax-weighted sum of the first DL dims; lse is the natural-log sum-exp.
+ *
+ * Parity pins: tests/test_oracle.py checks every function here against closed forms,
+ * brute force and special cases that do not reuse this code.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_OK 0
+#define ORACLE_BAD_INPUT 1
+
+/* ---- element decoding (from the format definitions) -------------------------------------- */
+
+/* bfloat16: the upper 16 bits of an IEEE-754 binary32. */
+double oracle_bf16_value(uint16_t bits) {
+    uint32_t u = ((uint32_t)bits) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* OCP FP8 E4M3 ("fn" variant): 1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits,
+ * no infinities, S.1111.111 is NaN.  Exponent field 0 encodes subnormals 2^-6 * m/8. */
+double oracle_e4m3_value(uint8_t bits) {
+    int sign = (bits >> 7) & 1;
+    int e = (bits >> 3) & 15;
+    int m = bits & 7;
+    double mag;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) mag = ldexp((double)m / 8.0, 1 - 7);
+    else mag = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return sign ? -mag : mag;
+}
+
+static double elem_value(const void* base, long idx, int fp8) {
+    if (fp8) return oracle_e4m3_value(((const uint8_t*)base)[idx]);
+    return oracle_bf16_value(((const uint16_t*)base)[idx]);
+}
+
+/* ---- step a1: page-table translation ---------------------------------------------------- */
+
+/* Physical row (page * P + offset) holding logical position s of sequence b, or -1 when the
+ * page id is outside the pool. */
+static long physical_row(const int32_t* page_table, int max_pages, int P, int num_pages,
+                         int b, int s) {
+    int page = page_table[(long)b * max_pages + s / P];
+    if (page < 0 || page >= num_pages) return -1;
+    return (long)page * P + (s % P);
+}
+
+static int query_position(const int32_t* seq_lens, const int32_t* q_pos, int J, int b, int j) {
+    if (q_pos) return q_pos[(long)b * J + j];
+    return seq_lens[b] - J + j;
+}
+
+/* ---- steps a2-a4: relevance scoring, head-weighted aggregation, causal mask --------------- */
+
+/*
+ * scores[(b*J + j) * Lpad + s] for s <= p (p = the query's position), NaN elsewhere, with
+ * Lpad = max_pages * P.  n_visible[b*J + j] = p + 1 (0 when p < 0).
+ * rows: optional list of flattened (b*J + j) rows to compute (NULL = all of them).
+ */
+int oracle_index_scores(int B, int J, int H, int D, int P, int max_pages, int num_pages,
+                        int fp8, const void* q, const float* q_scale, const float* w,
+                        const void* k_cache, const float* k_scale,
+                        const int32_t* page_table, const int32_t* seq_lens,
+                        const int32_t* q_pos, const int32_t* rows, int n_rows,
+                        double* scores, int32_t* n_visible) {
+    long Lpad = (long)max_pages * P;
+    int total = rows ? n_rows : B * J;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (int r = 0; r < total; ++r) {
+        int bj = rows ? rows[r] : r;
+        int b = bj / J, j = bj % J;
+        int p = query_position(seq_lens, q_pos, J, b, j);
+        double* out = scores + (long)bj * Lpad;
+        for (long s = 0; s < Lpad; ++s) out[s] = NAN;
+        if (p >= seq_lens[b] || p >= Lpad) { bad = 1; n_visible[bj] = 0; continue; }
+        n_visible[bj] = p + 1 > 0 ? p + 1 : 0;
+        double qs = q_scale ? (double)q_scale[bj] : 1.0;
+        for (int s = 0; s <= p; ++s) {
+            long row = physical_row(page_table, max_pages, P, num_pages, b, s);
+            if (row < 0) { bad = 1; continue; }
+            double ks = k_scale ? (double)k_scale[row] : 1.0;
+            double total_score = 0.0;
+            for (int h = 0; h < H; ++h) {
+                double dot = 0.0;
+                for (int d = 0; d < D; ++d) {
+                    double qv = elem_value(q, ((long)bj * H + h) * D + d, fp8) * qs;
+                    double kv = elem_value(k_cache, row * D + d, fp8) * ks;
+                    dot += qv * kv;
+                }
+                double relu = dot > 0.0 ? dot : 0.0;
+                total_score += (double)w[(long)bj * H + h] * relu;
+            }
+            out[s] = total_score;
+        }
+    }
+    return bad ? ORACLE_BAD_INPUT : ORACLE_OK;
+}
+
+/* ---- step a5: Top-K selection ------------------------------------------------------------ */
+
+typedef struct { double score; int32_t pos; } scored_pos;
+
+/* Rank order: larger score first; equal scores -> lower position first.  -0.0 and +0.0
+ * compare equal, so the position decides between them. */
+static int by_score_desc_pos_asc(const void* a, const void* b) {
+    const scored_pos* x = (const scored_pos*)a;
+    const scored_pos* y = (const scored_pos*)b;
+    if (x->score > y->score) return -1;
+    if (x->score < y->score) return 1;
+    return (x->pos > y->pos) - (x->pos < y->pos);
+}
+
+static int by_int_asc(const void* a, const void* b) {
+    int32_t x = *(const int32_t*)a, y = *(const int32_t*)b;
+    return (x > y) - (x < y);
+}
+
+/* One query row: the K best of scores[0..n_visible) -> out[0..K), ascending, -1 padded. */
+int oracle_topk_row(const double* scores, int n_visible, int K, int32_t* out) {
+    int take = n_visible < K ? n_visible : K;
+    scored_pos* all = (scored_pos*)malloc(sizeof(scored_pos) * (size_t)(n_visible > 0 ? n_visible : 1));
+    if (!all) return ORACLE_BAD_INPUT;
+    for (int s = 0; s < n_visible; ++s) {
+        all[s].score = (double)(float)scores[s]; /* rank in the GPU's precision */
+        all[s].pos = s;
+    }
+    qsort(all, (size_t)n_visible, sizeof(scored_pos), by_score_desc_pos_asc);
+    for (int i = 0; i < take; ++i) out[i] = all[i].pos;
+    qsort(out, (size_t)take, sizeof(int32_t), by_int_asc);
+    for (int i = take; i < K; ++i) out[i] = -1;
+    free(all);
+    return ORACLE_OK;
+}
+
+/* Rows of a score matrix [n_rows_total, Lpad] -> topk [n_rows_total, K]. */
+int oracle_topk(const double* scores, const int32_t* n_visible, long Lpad, int K,
+                const int32_t* rows, int n_rows, int total_rows, int32_t* topk) {
+    int total = rows ? n_rows : total_rows;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (int r = 0; r < total; ++r) {
+        int bj = rows ? rows[r] : r;
+        bad |= oracle_topk_row(scores + (long)bj * Lpad, n_visible[bj], K, topk + (long)bj * K);
+    }
+    return bad ? ORACLE_BAD_INPUT : ORACLE_OK;
+}
+
+/* ---- steps a6-a7: gather the selected latent rows, softmax attention --------------------- */
+
+/*
+ * q   bf16 [B, J, H, DL+DR];  kv bf16 [num_pages, P, DL+DR];  topk int32 [B, J, K] (-1 = none)
+ * out [B, J, H, DL] = sum_s softmax_s(z) * c[s][0:DL],  z_s = scale * q[h] . c[s]
+ * lse [B, J, H]     = log sum_s exp(z_s)  (-inf and out = 0 when the list is empty)
+ */
+int oracle_sparse_attend(int B, int J, int H, int DL, int DR, int P, int max_pages,
+                         int num_pages, double scale, const uint16_t* q, const uint16_t* kv,
+                         const int32_t* page_table, const int32_t* seq_lens,
+                         const int32_t* topk, int K, const int32_t* rows, int n_rows,
+                         double* out, double* lse) {
+    int DC = DL + DR;
+    int total = rows ? n_rows : B * J;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (int r = 0; r < total; ++r) {
+        int bj = rows ? rows[r] : r;
+        int b = bj / J;
+        const int32_t* sel = topk + (long)bj * K;
+        long* phys = (long*)malloc(sizeof(long) * (size_t)K);
+        double* z = (double*)malloc(sizeof(double) * (size_t)K);
+        int n = 0;
+        for (int i = 0; i < K; ++i) {
+            int s = sel[i];
+            if (s < 0) continue;
+            if (s >= seq_lens[b]) { bad = 1; continue; }
+            long row = physical_row(page_table, max_pages, P, num_pages, b, s);
+            if (row < 0) { bad = 1; continue; }
+            phys[n++] = row;
+        }
+        for (int h = 0; h < H; ++h) {
+            const uint16_t* qh = q + ((long)bj * H + h) * DC;
+            double* oh = out + ((long)bj * H + h) * DL;
+            double m = -INFINITY;
+            for (int i = 0; i < n; ++i) {
+                const uint16_t* c = kv + phys[i] * DC;
+                double dot = 0.0;
+                for (int d = 0; d < DC; ++d) dot += oracle_bf16_value(qh[d]) * oracle_bf16_value(c[d]);
+                z[i] = scale * dot;
+                if (z[i] > m) m = z[i];
+            }
+            double denom = 0.0;
+            for (int i = 0; i < n; ++i) denom += exp(z[i] - m);
+            for (int d = 0; d < DL; ++d) {
+                double acc = 0.0;
+                for (int i = 0; i < n; ++i) acc += exp(z[i] - m) * oracle_bf16_value(kv[phys[i] * DC + d]);
+                oh[d] = n > 0 ? acc / denom : 0.0;
+            }
+            lse[(long)bj * H + h] = n > 0 ? m + log(denom) : -INFINITY;
+        }
+        free(phys);
+        free(z);
+    }
+    return bad ? ORACLE_BAD_INPUT : ORACLE_OK;
+}
+
+/*
+ * Second, independent formulation used to pin the first: dense attention of the query over
+ * every causal position 0..p, with the logit of each position outside the allowed set forced
+ * to -inf before the softmax.  allowed: uint8 [B*J, Lpad] (1 = take part).
+ */
+int oracle_dense_masked_attend(int B, int J, int H, int DL, int DR, int P, int max_pages,
+                               int num_pages, double scale, const uint16_t* q,
+                               const uint16_t* kv, const int32_t* page_table,
+                               const int32_t* seq_lens, const int32_t* q_pos,
+                               const uint8_t* allowed, double* out, double* lse) {
+    int DC = DL + DR;
+    long Lpad = (long)max_pages * P;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (int bj = 0; bj < B * J; ++bj) {
+        int b = bj / J, j = bj % J;
+        int p = query_position(seq_lens, q_pos, J, b, j);
+        double* logits = (double*)malloc(sizeof(double) * (size_t)(p + 1 > 0 ? p + 1 : 1));
+        for (int h = 0; h < H; ++h) {
+            const uint16_t* qh = q + ((long)bj * H + h) * DC;
+            for (int s = 0; s <= p; ++s) {
+                long row = physical_row(page_table, max_pages, P, num_pages, b, s);
+                if (row < 0) { bad = 1; logits[s] = -INFINITY; continue; }
+                if (!allowed[(long)bj * Lpad + s]) { logits[s] = -INFINITY; continue; }
+                double dot = 0.0;
+                for (int d = 0; d < DC; ++d)
+                    dot += oracle_bf16_value(qh[d]) * oracle_bf16_value(kv[row * DC + d]);
+                logits[s] = scale * dot;
+            }
+            double m = -INFINITY;
+            for (int s = 0; s <= p; ++s) if (logits[s] > m) m = logits[s];
+            double* oh = out + ((long)bj * H + h) * DL;
+            if (m == -INFINITY) {
+                for (int d = 0; d < DL; ++d) oh[d] = 0.0;
+                lse[(long)bj * H + h] = -INFINITY;
+                continue;
+            }
+            double denom = 0.0;
+            for (int s = 0; s <= p; ++s) denom += exp(logits[s] - m);
+            for (int d = 0; d < DL; ++d) {
+                double acc = 0.0;
+                for (int s = 0; s <= p; ++s) {
+                    if (logits[s] == -INFINITY) continue;
+                    long row = physical_row(page_table, max_pages, P, num_pages, b, s);
+                    acc += exp(logits[s] - m) * oracle_bf16_value(kv[row * DC + d]);
+                }
+                oh[d] = acc / denom;
+            }
+            lse[(long)bj * H + h] = m + log(denom);
+        }
+        free(logits);
+    }
+    return bad ? ORACLE_BAD_INPUT : ORACLE_OK;
+}
+
+/* Number of threads the OpenMP runtime uses for the loops above (1 without OpenMP). */
+#ifdef _OPENMP
+#include <omp.h>
+int oracle_num_threads(void) { return omp_get_max_threads(); }
+void oracle_set_num_threads(int n) { omp_set_num_threads(n); }
+#else
+int oracle_num_threads(void) { return 1; }
+void oracle_set_num_threads(int n) { (void)n; }
+#endif

@@ -1,0 +1,345 @@
+"""Pins for the CPU oracle: each check is fixed by something other than the oracle itself
+(hand-worked examples, closed forms, invariants, brute force, library routines)."""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+from scipy.special import logsumexp, softmax
+
+import oracle
+from indexed_sparse_attention_paged_b200 import workloads
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def bf16(a):
+    return torch.tensor(np.asarray(a, dtype=np.float32)).to(torch.bfloat16)
+
+
+def rng(seed):
+    return np.random.default_rng(seed)
+
+
+# ---------------------------------------------------------------- element decoding
+
+def test_bf16_decode_matches_torch_for_every_pattern():
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    ref = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    got = np.array([oracle.bf16_value(int(b)) for b in bits[::7]])
+    np.testing.assert_array_equal(np.isnan(got), np.isnan(ref[::7]))
+    ok = ~np.isnan(ref[::7])
+    np.testing.assert_array_equal(got[ok], ref[::7][ok])
+
+
+def test_e4m3_decode_matches_torch_for_every_code():
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = np.array([oracle.e4m3_value(int(c)) for c in codes])
+    np.testing.assert_array_equal(np.isnan(got), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    np.testing.assert_array_equal(got[ok], ref[ok])
+    assert oracle.e4m3_value(0x7E) == 448.0          # largest finite value of the format
+    assert oracle.e4m3_value(0x01) == 2.0 ** -9      # smallest subnormal
+
+
+# ---------------------------------------------------------------- scores (steps 1-2)
+
+def _golden_index():
+    with open(os.path.join(GOLDEN, "worked_index_example.json")) as f:
+        return json.load(f)
+
+
+def test_scores_hand_worked_example():
+    g = _golden_index()
+    q = bf16(g["q"])
+    k = bf16(g["k_cache"])
+    w = np.array(g["w"], dtype=np.float32)
+    pt = np.array(g["page_table"], dtype=np.int32)
+    sl = np.array([g["seq_len"]], dtype=np.int32)
+    scores, nvis, st = oracle.index_scores(q, w, k, pt, sl, page_size=g["page_size"])
+    assert st == 0 and nvis[0, 0] == 3
+    np.testing.assert_array_equal(scores[0, 0, :3], g["scores"])
+    assert np.isnan(scores[0, 0, 3])          # past the query: not scored
+    tk, _, _ = oracle.index_topk(q, w, k, pt, sl, page_size=g["page_size"], top_k=2)
+    assert tk[0, 0].tolist() == g["top2"]
+    tk, _, _ = oracle.index_topk(q, w, k, pt, sl, page_size=g["page_size"], top_k=4)
+    assert tk[0, 0].tolist() == g["top4"]
+
+
+def _small_index_case(seed, B=2, J=1, H=3, D=8, P=4, L=11, fp8=False):
+    r = rng(seed)
+    pages = (L + P - 1) // P
+    num_pages = B * pages
+    perm = r.permutation(num_pages).astype(np.int32)
+    pt = perm.reshape(B, pages)
+    q = r.integers(-3, 4, (B, J, H, D)).astype(np.float32)
+    k = r.integers(-3, 4, (num_pages, P, D)).astype(np.float32)
+    w = r.integers(-2, 3, (B, J, H)).astype(np.float32)
+    sl = np.full(B, L, dtype=np.int32)
+    return q, k, w, pt, sl
+
+
+def _logical_k(k, pt, P, b, L):
+    """Logical-order key rows of sequence b, read through the page table by hand."""
+    return np.stack([k[pt[b, s // P], s % P] for s in range(L)])
+
+
+def test_scores_closed_form_without_relu():
+    # with w = 1 and non-negative q, k every dot is >= 0, ReLU is the identity and the head
+    # sum factors: I[s] = (sum_h q_h) . k[s]
+    q, k, w, pt, sl = _small_index_case(1)
+    q, k, w = np.abs(q), np.abs(k), np.ones_like(w)
+    scores, _, st = oracle.index_scores(bf16(q), w, bf16(k), pt, sl, page_size=4)
+    assert st == 0
+    for b in range(2):
+        expect = _logical_k(k, pt, 4, b, 11) @ q[b, 0].sum(axis=0)
+        np.testing.assert_array_equal(scores[b, 0, :11], expect)
+
+
+def test_scores_single_head_weight_selects_relu_of_that_head():
+    q, k, w, pt, sl = _small_index_case(2)
+    for h in range(3):
+        wh = np.zeros_like(w)
+        wh[..., h] = 1.0
+        scores, _, _ = oracle.index_scores(bf16(q), wh, bf16(k), pt, sl, page_size=4)
+        for b in range(2):
+            dots = _logical_k(k, pt, 4, b, 11) @ q[b, 0, h]
+            np.testing.assert_array_equal(scores[b, 0, :11], np.maximum(dots, 0.0))
+
+
+def test_scores_linear_in_head_weights_and_scales():
+    q, k, w, pt, sl = _small_index_case(3)
+    w2 = rng(33).integers(-2, 3, w.shape).astype(np.float32)
+    s1, _, _ = oracle.index_scores(bf16(q), w, bf16(k), pt, sl, page_size=4)
+    s2, _, _ = oracle.index_scores(bf16(q), w2, bf16(k), pt, sl, page_size=4)
+    s12, _, _ = oracle.index_scores(bf16(q), w + w2, bf16(k), pt, sl, page_size=4)
+    np.testing.assert_array_equal(s12[..., :11], s1[..., :11] + s2[..., :11])
+    # per-token power-of-two key scales and a per-query scale multiply the score exactly
+    ks = np.power(2.0, rng(34).integers(-4, 5, k.shape[:2])).astype(np.float32)
+    qs = np.array([[0.5], [4.0]], dtype=np.float32)
+    k8 = torch.tensor(k).to(torch.float8_e4m3fn)
+    q8 = torch.tensor(q).to(torch.float8_e4m3fn)
+    sc, _, _ = oracle.index_scores(q8, w, k8, pt, sl, page_size=4, fp8=True, k_scale=ks, q_scale=qs)
+    for b in range(2):
+        for s in range(11):
+            row = pt[b, s // 4] * 4 + s % 4
+            assert sc[b, 0, s] == s1[b, 0, s] * ks.reshape(-1)[row] * qs[b, 0]
+
+
+def test_scores_independent_of_physical_page_placement():
+    q, k, w, pt, sl = _small_index_case(4)
+    base, _, _ = oracle.index_scores(bf16(q), w, bf16(k), pt, sl, page_size=4)
+    # move every page to a new physical slot and rewrite the table to match
+    perm = rng(44).permutation(k.shape[0])
+    k_moved = np.empty_like(k)
+    k_moved[perm] = k
+    moved, _, _ = oracle.index_scores(bf16(q), w, bf16(k_moved), perm[pt].astype(np.int32), sl,
+                                      page_size=4)
+    np.testing.assert_array_equal(base, moved)
+
+
+def test_fp8_and_bf16_storage_give_identical_scores():
+    # integers in [-3,3] are exact in both formats, so the quantised index path must agree
+    # with the bf16 baseline exactly (Top-K hit rate 100%)
+    q, k, w, pt, sl = _small_index_case(5)
+    sb, _, _ = oracle.index_scores(bf16(q), w, bf16(k), pt, sl, page_size=4)
+    s8, _, _ = oracle.index_scores(torch.tensor(q).to(torch.float8_e4m3fn), w,
+                                   torch.tensor(k).to(torch.float8_e4m3fn), pt, sl, page_size=4,
+                                   fp8=True)
+    np.testing.assert_array_equal(sb, s8)
+
+
+def test_causal_visibility_and_query_positions():
+    q, k, w, pt, sl = _small_index_case(6, J=2)
+    scores, nvis, st = oracle.index_scores(bf16(q), w, bf16(k), pt, sl, page_size=4)
+    assert st == 0
+    # default positions: seq_len - J + j -> draft at L-2 sees L-1 positions, verify sees L
+    assert nvis.tolist() == [[10, 11], [10, 11]]
+    assert np.isnan(scores[0, 0, 10]) and not np.isnan(scores[0, 1, 10])
+    qp = np.array([[0, 5], [3, 3]], dtype=np.int32)
+    scores, nvis, _ = oracle.index_scores(bf16(q), w, bf16(k), pt, sl, page_size=4, q_pos=qp)
+    assert nvis.tolist() == [[1, 6], [4, 4]]
+    assert np.isnan(scores[0, 0, 1]) and not np.isnan(scores[0, 0, 0])
+
+
+def test_bad_page_id_is_reported_not_read():
+    q, k, w, pt, sl = _small_index_case(7)
+    pt = pt.copy()
+    pt[1, 1] = k.shape[0] + 5
+    _, _, st = oracle.index_scores(bf16(q), w, bf16(k), pt, sl, page_size=4)
+    assert st != 0
+
+
+# ---------------------------------------------------------------- Top-K (step 3)
+
+def _brute_force_topk(scores, k):
+    """The unique K-subset that beats every outsider under (score desc, position asc),
+    found by enumerating every subset."""
+    n = len(scores)
+    if n <= k:
+        return list(range(n)) + [-1] * (k - n)
+    found = []
+    for sub in itertools.combinations(range(n), k):
+        inside = set(sub)
+        if all((scores[i] > scores[j]) or (scores[i] == scores[j] and i < j)
+               for i in inside for j in range(n) if j not in inside):
+            found.append(list(sub))
+    assert len(found) == 1
+    return found[0]
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_topk_matches_brute_force_with_heavy_ties(seed):
+    r = rng(100 + seed)
+    n = int(r.integers(1, 11))
+    k = int(r.integers(1, 6))
+    scores = r.integers(-2, 3, n).astype(np.float64)     # few distinct values -> many ties
+    got = oracle.topk_row(scores, n, k).tolist()
+    assert got == _brute_force_topk(list(scores), k)
+
+
+def test_topk_invariants_on_large_rows():
+    r = rng(200)
+    for n, k in [(5000, 2048), (3000, 64), (2048, 2048), (100, 2048)]:
+        scores = r.integers(-50, 50, n).astype(np.float64)
+        got = oracle.topk_row(scores, n, k)
+        sel = got[got >= 0]
+        assert len(sel) == min(n, k)
+        assert np.all(np.diff(sel) > 0)                    # ascending, no repeats
+        if n > k:
+            mask = np.zeros(n, bool)
+            mask[sel] = True
+            thr = scores[mask].min()
+            assert scores[~mask].max() <= thr
+            # among positions scoring exactly the threshold, the lowest ones are taken
+            eq = np.flatnonzero(scores == thr)
+            taken = np.flatnonzero(mask & (scores == thr))
+            assert taken.tolist() == eq[:len(taken)].tolist()
+
+
+def test_topk_special_cases():
+    assert oracle.topk_row(np.zeros(10), 10, 4).tolist() == [0, 1, 2, 3]
+    assert oracle.topk_row(np.array([-0.0, 0.0, -0.0]), 3, 1).tolist() == [0]
+    assert oracle.topk_row(np.array([0.0, -0.0, 1.0]), 3, 2).tolist() == [0, 2]
+    assert oracle.topk_row(np.array([3.0, 1.0]), 2, 4).tolist() == [0, 1, -1, -1]
+    assert oracle.topk_row(np.array([]), 0, 3).tolist() == [-1, -1, -1]
+
+
+# ---------------------------------------------------------------- attention (steps 4-5)
+
+def _attn_case(seed, B=2, J=2, H=3, DL=8, DR=4, P=4, L=13, K=5):
+    r = rng(seed)
+    pages = (L + P - 1) // P
+    num_pages = B * pages
+    pt = r.permutation(num_pages).astype(np.int32).reshape(B, pages)
+    q = r.standard_normal((B, J, H, DL + DR)).astype(np.float32)
+    kv = r.standard_normal((num_pages, P, DL + DR)).astype(np.float32)
+    sl = np.full(B, L, dtype=np.int32)
+    topk = np.full((B, J, K), -1, dtype=np.int32)
+    for b in range(B):
+        for j in range(J):
+            p = L - J + j
+            sel = np.sort(r.choice(p + 1, size=min(K, p + 1), replace=False))
+            topk[b, j, :len(sel)] = sel
+    return bf16(q), bf16(kv), pt, sl, topk
+
+
+def test_attention_hand_worked_example():
+    with open(os.path.join(GOLDEN, "worked_attention_example.json")) as f:
+        g = json.load(f)
+    q = bf16(np.array(g["q"]).reshape(1, 1, 1, 3))
+    kv = bf16(np.array(g["rows"] + [[0, 0, 0]]).reshape(1, 4, 3))
+    pt = np.array([[0]], dtype=np.int32)
+    sl = np.array([3], dtype=np.int32)
+    out, lse, st = oracle.sparse_attend(q, kv, pt, sl, np.array([[[0, 2]]], dtype=np.int32),
+                                        page_size=4, d_latent=2, scale=1.0)
+    assert st == 0
+    np.testing.assert_allclose(out[0, 0, 0], [3.0, 2.0], rtol=0, atol=1e-15)
+    np.testing.assert_allclose(lse[0, 0, 0], 2.0 + math.log(2.0), rtol=0, atol=1e-15)
+    out, lse, _ = oracle.sparse_attend(q, kv, pt, sl, np.array([[[0, 1]]], dtype=np.int32),
+                                       page_size=4, d_latent=2, scale=1.0)
+    e = math.e
+    np.testing.assert_allclose(out[0, 0, 0], [2 * e / (e + 1), (4 * e + 2) / (e + 1)], atol=1e-15)
+    np.testing.assert_allclose(lse[0, 0, 0], 2.0 + math.log(1 + 1 / e), atol=1e-15)
+
+
+def test_sparse_gather_equals_dense_masked_attention():
+    q, kv, pt, sl, topk = _attn_case(300)
+    Lpad = pt.shape[1] * 4
+    allowed = np.zeros((2, 2, Lpad), np.uint8)
+    for b in range(2):
+        for j in range(2):
+            allowed[b, j, topk[b, j][topk[b, j] >= 0]] = 1
+    o1, l1, s1 = oracle.sparse_attend(q, kv, pt, sl, topk, page_size=4, d_latent=8, scale=0.3)
+    o2, l2, s2 = oracle.dense_masked_attend(q, kv, pt, sl, allowed, page_size=4, d_latent=8,
+                                            scale=0.3)
+    assert s1 == 0 and s2 == 0
+    np.testing.assert_allclose(o1, o2, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(l1, l2, rtol=0, atol=1e-12)
+
+
+def test_topk_covering_the_history_reduces_to_dense_causal_attention():
+    q, kv, pt, sl, _ = _attn_case(301, K=16)
+    L = 13
+    topk = np.full((2, 2, 16), -1, dtype=np.int32)
+    for j in range(2):
+        n = L - 2 + j + 1
+        topk[:, j, :n] = np.arange(n)
+    o1, l1, _ = oracle.sparse_attend(q, kv, pt, sl, topk, page_size=4, d_latent=8, scale=0.3)
+    # library softmax over the full causal history, rows read through the page table by hand
+    qn = q.to(torch.float64).numpy()
+    kvn = kv.to(torch.float64).numpy()
+    for b in range(2):
+        for j in range(2):
+            n = L - 2 + j + 1
+            rows = np.stack([kvn[pt[b, s // 4], s % 4] for s in range(n)])
+            z = 0.3 * rows @ qn[b, j].T                      # [n, H]
+            np.testing.assert_allclose(o1[b, j], (softmax(z, axis=0).T @ rows[:, :8]), atol=1e-12)
+            np.testing.assert_allclose(l1[b, j], logsumexp(z, axis=0), atol=1e-12)
+
+
+def test_attention_special_cases():
+    q, kv, pt, sl, _ = _attn_case(302, K=4)
+    kvn = kv.to(torch.float64).numpy()
+    # one selected row: the output is that row's latent part and lse is its logit
+    topk = np.full((2, 2, 4), -1, dtype=np.int32)
+    topk[:, :, 0] = 7
+    o, l, _ = oracle.sparse_attend(q, kv, pt, sl, topk, page_size=4, d_latent=8, scale=0.3)
+    for b in range(2):
+        row = kvn[pt[b, 1], 3]
+        for j in range(2):
+            np.testing.assert_array_equal(o[b, j], np.broadcast_to(row[:8], (3, 8)))
+            zq = 0.3 * q[b, j].to(torch.float64).numpy() @ row
+            np.testing.assert_allclose(l[b, j], zq, atol=1e-12)
+    # zero query: uniform weights -> mean of the selected rows, lse = log(count)
+    qz = torch.zeros_like(q)
+    topk[:, :, :3] = [2, 5, 9]
+    o, l, _ = oracle.sparse_attend(qz, kv, pt, sl, topk, page_size=4, d_latent=8, scale=0.3)
+    for b in range(2):
+        rows = np.stack([kvn[pt[b, s // 4], s % 4] for s in (2, 5, 9)])
+        np.testing.assert_allclose(o[b, 0, 0], rows[:, :8].mean(axis=0), atol=1e-12)
+    np.testing.assert_allclose(l, math.log(3.0), atol=1e-12)
+    # an empty list gives zeros and lse = -inf
+    topk[:] = -1
+    o, l, _ = oracle.sparse_attend(q, kv, pt, sl, topk, page_size=4, d_latent=8, scale=0.3)
+    assert np.all(o == 0) and np.all(np.isneginf(l))
+
+
+# ---------------------------------------------------------------- generators
+
+def test_workload_generator_is_deterministic_and_shaped():
+    wl = workloads.WORKLOADS[1]
+    a = workloads.make_inputs(wl)
+    b = workloads.make_inputs(wl)
+    for key in ("q_idx", "k_cache", "w", "q_attn", "kv_cache", "page_table"):
+        assert torch.equal(a[key].view(torch.uint8) if a[key].dtype != torch.float32 else a[key],
+                           b[key].view(torch.uint8) if b[key].dtype != torch.float32 else b[key])
+    assert a["page_table"].shape == (1, 16)
+    assert sorted(a["page_table"].flatten().tolist()) == list(range(16))
+    assert a["q_idx"].shape == (1, 1, 4, 32) and a["kv_cache"].shape == (16, 16, 80)
+    v = a["q_idx"].float()
+    assert v.min() >= -3 and v.max() <= 3 and torch.equal(v, v.round())
