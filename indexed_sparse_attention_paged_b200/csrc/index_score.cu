@@ -1,0 +1,424 @@
+// index_score.cu -- the indexer's scoring stage on the sm_100a tensor cores.
+//
+// Computes, for every query (b, j) and every causal position s <= p(b, j),
+//     I[s] = q_scale[b,j] * k_scale[s] * sum_h w[b,j,h] * ReLU(q[b,j,h] . k[s])
+// reading k[s] straight out of the paged index-K cache ("Rapid Adaptation and Inference
+// Optimization: Key Engineering Practices for Day0 LLM Support", section IV.4.1; the score form
+// is the spec's fixed reading of the "score, then weight and sum the heads" steps in "Day 0
+// Inference Adaptation and Performance Optimization for Hybrid Sparse Attention LLMs", section
+// "Operator Fusion and Multi-Stream Scheduling").  Prefill and decode share this one kernel, as
+// the pages ask of the fused indexer.
+//
+// Design (B200): one tcgen05 MMA per (128-position tile, query sub-block):
+//   A = K tile   [128 positions x D]   (TMA, K-major, swizzled; M = 128 = TMEM lanes)
+//   B = Q group  [nq_sub*HP rows x D]  (threads, K-major, swizzled; N = queries x heads)
+//   D = TMEM     [128 lanes x N fp32 columns]
+// so that in the epilogue each thread owns one position and reduces sum_h w*ReLU(d) over its
+// own registers, without shuffles.  The grid is persistent (one CTA per SM); the flat list of
+// (query group, tile) work is split evenly between CTAs, which balances ragged context lengths
+// and the causal "light at the start, heavy at the end" prefill load.
+//
+// Exactness: for integer-valued q, k, w (the tests' inputs) every product and every partial
+// sum is an integer below 2^24, so the fp32 result equals the exact score whatever order the
+// tensor core and the epilogue add in.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "sia_common.cuh"
+#include "sia_internal.h"
+#include "sia_ptx.cuh"
+
+namespace sia {
+namespace {
+
+struct IndexBarriers {
+  uint64_t k_full[8];
+  uint64_t k_empty[8];
+  uint64_t acc_full[2][2];
+  uint64_t acc_empty[2][2];
+  uint64_t q_full;
+  uint64_t q_empty;
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int abort;
+  int start_item, start_tile, count;
+};
+
+struct GroupInfo {
+  int b, g;         // sequence, query group
+  int max_pos;      // largest visible position among the group's queries (-1: none)
+  int n_tiles;
+};
+
+__device__ __forceinline__ GroupInfo group_info(const IndexKernelParams& p, int item) {
+  GroupInfo gi;
+  gi.b = item / p.groups_per_seq;
+  gi.g = item - gi.b * p.groups_per_seq;
+  int mp = -1;
+  const int j0 = gi.g * p.qg;
+  const int j1 = min(p.J, j0 + p.qg);
+  if (p.q_pos == nullptr) {
+    mp = query_position(p.seq_lens, nullptr, p.J, gi.b, j1 - 1, p.Lpad);
+  } else {
+    for (int j = j0; j < j1; ++j) mp = max(mp, query_position(p.seq_lens, p.q_pos, p.J, gi.b, j, p.Lpad));
+  }
+  gi.max_pos = mp;
+  gi.n_tiles = mp < 0 ? 0 : mp / kIndexTileRows + 1;
+  return gi;
+}
+
+// Warp 0 finds where this CTA's share of the flat tile list starts.
+__device__ void locate_start(const IndexKernelParams& p, IndexBarriers* sb) {
+  const int lane = threadIdx.x & 31;
+  const int items = p.B * p.groups_per_seq;
+  long long total = 0;
+  for (int base = 0; base < items; base += 32) {
+    const int it = base + lane;
+    long long t = it < items ? group_info(p, it).n_tiles : 0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    total += t;
+  }
+  const long long begin = total * blockIdx.x / gridDim.x;
+  const long long end = total * (blockIdx.x + 1) / gridDim.x;
+  int start_item = items, start_tile = 0;
+  long long before = 0;
+  for (int base = 0; base < items; base += 32) {
+    const int it = base + lane;
+    const long long t = it < items ? group_info(p, it).n_tiles : 0;
+    long long incl = t;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const long long excl = before + incl - t;
+    const bool here = t > 0 && begin >= excl && begin < excl + t;
+    const unsigned m = __ballot_sync(0xffffffffu, here);
+    if (m) {
+      const int src = __ffs(m) - 1;
+      start_item = __shfl_sync(0xffffffffu, it, src);
+      start_tile = (int)(begin - __shfl_sync(0xffffffffu, excl, src));
+      break;
+    }
+    before += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  if (lane == 0) {
+    sb->start_item = start_item;
+    sb->start_tile = start_tile;
+    sb->count = (int)(end - begin);
+  }
+}
+
+template <int NSUB>
+__global__ void __launch_bounds__(64 + 128 * NSUB, 1)
+    index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexKernelParams p) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  IndexBarriers* sb = reinterpret_cast<IndexBarriers*>(smem + p.off_bar);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  constexpr int kEpiThreads = 128 * NSUB;
+
+  if ((smem_u32(smem) & 1023u) != 0) {  // the swizzled layouts need a 1024-byte aligned base
+    if (threadIdx.x == 0) report(p.status, SIA_DEV_TIMEOUT);
+    return;
+  }
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.k_stages; ++s) {
+      mbar_init(&sb->k_full[s], 1);
+      mbar_init(&sb->k_empty[s], 1);
+    }
+    for (int a = 0; a < p.acc_stages; ++a)
+      for (int s = 0; s < NSUB; ++s) {
+        mbar_init(&sb->acc_full[a][s], 1);
+        mbar_init(&sb->acc_empty[a][s], 128);
+      }
+    mbar_init(&sb->q_full, kEpiThreads);
+    mbar_init(&sb->q_empty, 1);
+    mbar_init(&sb->mma_done, 1);
+    sb->abort = 0;
+    fence_mbarrier_init();
+    tma_prefetch_desc(&kmap);
+  }
+  if (warp == 0) locate_start(p, sb);
+  if (warp == 1) {
+    tmem_alloc(&sb->tmem_base, p.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = sb->tmem_base;
+  volatile int* abort = &sb->abort;
+  const int start_item = sb->start_item;
+  const int start_tile = sb->start_tile;
+  const int my_count = sb->count;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    int it = 0;
+    int item = start_item, t0 = start_tile, remaining = my_count;
+    bool ok = true;
+    while (remaining > 0 && ok) {
+      const GroupInfo gi = group_info(p, item);
+      const int t1 = min(gi.n_tiles, t0 + remaining);
+      const int32_t* pt_row = p.page_table + (long long)gi.b * p.max_pages;
+      int cached_base = -1, cached_page = -1;
+      for (int t = t0; t < t1 && ok; ++t, ++it) {
+        const int stage = it % p.k_stages;
+        const uint32_t phase = (uint32_t)(it / p.k_stages) & 1u;
+        int go = 1;
+        if (lane == 0) go = mbar_wait(&sb->k_empty[stage], phase ^ 1u, abort, p.status);
+        go = __shfl_sync(0xffffffffu, go, 0);
+        if (!go) { ok = false; break; }
+        uint8_t* kst = smem + p.off_k + stage * p.k_stage_bytes;
+        const int chunks = kIndexTileRows / p.box_rows;
+        // page ids of this tile's chunks, read 32 logical pages at a time by the whole warp
+        uint32_t valid_mask = 0;
+        int pages_of_chunk[16];
+#pragma unroll 1
+        for (int c = 0; c < chunks; ++c) {
+          const int pos = t * kIndexTileRows + c * p.box_rows;
+          const int lp = pos / p.P;
+          if (lp < cached_base || lp >= cached_base + 32) {
+            cached_base = lp;
+            cached_page = (lp + lane < p.max_pages) ? pt_row[lp + lane] : -1;
+          }
+          const int page = __shfl_sync(0xffffffffu, cached_page, lp - cached_base);
+          pages_of_chunk[c] = page;
+          if (pos <= gi.max_pos) {
+            if (page >= 0 && page < p.num_pages) valid_mask |= 1u << c;
+            else if (lane == 0) report(p.status, SIA_DEV_BAD_PAGE);
+          }
+        }
+        if (lane == 0) {
+          const uint32_t bytes = (uint32_t)__popc(valid_mask) * p.n_kblocks * p.box_rows * p.kbw;
+          mbar_arrive_expect_tx(&sb->k_full[stage], bytes);
+          for (int c = 0; c < chunks; ++c) {
+            if (!(valid_mask >> c & 1u)) continue;
+            const int pos = t * kIndexTileRows + c * p.box_rows;
+            const int y = pages_of_chunk[c] * p.P + (pos % p.P);
+            for (int kb = 0; kb < p.n_kblocks; ++kb)
+              tma_load_2d(kst + kb * p.k_kblock_bytes + c * p.box_rows * p.kbw, &kmap,
+                          &sb->k_full[stage], kb * p.kbw / (p.fp8 ? 1 : 2), y);
+          }
+        }
+        __syncwarp();
+      }
+      remaining -= (t1 - t0);
+      ++item;
+      t0 = 0;
+    }
+    // do not leave while loads into our shared memory may still be landing
+    if (lane == 0 && it > 0) {
+      const int first = it > p.k_stages ? it - p.k_stages : 0;
+      for (int i = first; i < it; ++i)
+        mbar_wait(&sb->k_full[i % p.k_stages], (uint32_t)(i / p.k_stages) & 1u, abort, p.status);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = p.fp8 ? umma_idesc(0, 0, false, false, p.n_cols, 128)
+                                   : umma_idesc(1, 1, false, false, p.n_cols, 128);
+      const uint32_t layout = umma_layout_type(p.kbw);
+      const uint32_t sbo = 8 * p.kbw;
+      int it = 0, acc_it = 0, seg = 0;
+      int item = start_item, t0 = start_tile, remaining = my_count;
+      bool ok = true;
+      while (remaining > 0 && ok) {
+        const GroupInfo gi = group_info(p, item);
+        const int t1 = min(gi.n_tiles, t0 + remaining);
+        if (t1 > t0) {
+          if (!mbar_wait(&sb->q_full, (uint32_t)seg & 1u, abort, p.status)) { ok = false; break; }
+          tc_fence_after();
+          for (int t = t0; t < t1; ++t, ++it, ++acc_it) {
+            const int stage = it % p.k_stages;
+            if (!mbar_wait(&sb->k_full[stage], (uint32_t)(it / p.k_stages) & 1u, abort, p.status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const int as = acc_it % p.acc_stages;
+            const uint32_t aph = (uint32_t)(acc_it / p.acc_stages) & 1u;
+            const uint32_t a_base = smem_u32(smem + p.off_k + stage * p.k_stage_bytes);
+            for (int sub = 0; sub < NSUB; ++sub) {
+              if (!mbar_wait(&sb->acc_empty[as][sub], aph ^ 1u, abort, p.status)) { ok = false; break; }
+              tc_fence_after();
+              const uint32_t d_tmem = tmem_base + (uint32_t)((as * NSUB + sub) * p.n_cols);
+              const uint32_t b_base = smem_u32(smem + p.off_q + sub * p.q_sub_bytes);
+              for (int kb = 0; kb < p.n_kblocks; ++kb)
+                for (int ks = 0; ks < p.ksteps_per_block; ++ks) {
+                  const uint64_t ad =
+                      umma_smem_desc(a_base + kb * p.k_kblock_bytes + ks * 32, 16, sbo, layout);
+                  const uint64_t bd =
+                      umma_smem_desc(b_base + kb * p.q_kblock_bytes + ks * 32, 16, sbo, layout);
+                  const bool acc = (kb | ks) != 0;
+                  if (p.fp8) umma_f8(d_tmem, ad, bd, idesc, acc);
+                  else umma_f16(d_tmem, ad, bd, idesc, acc);
+                }
+              umma_commit(&sb->acc_full[as][sub]);
+            }
+            if (!ok) break;
+            umma_commit(&sb->k_empty[stage]);
+          }
+          umma_commit(&sb->q_empty);
+          ++seg;
+        }
+        remaining -= (t1 - t0);
+        ++item;
+        t0 = 0;
+      }
+      umma_commit(&sb->mma_done);
+      mbar_wait(&sb->mma_done, 0, abort, p.status);
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- epilogue warps
+    const int et = threadIdx.x - 64;          // 0 .. kEpiThreads-1
+    const int sub = (warp - 2) >> 2;          // accumulator sub-block of this warp
+    const int quad = warp & 3;                // TMEM lane quarter this warp may access
+    const int row = quad * 32 + lane;         // position inside the tile
+    // w and per-query info are double-buffered by segment parity: a warp may start staging
+    // the next group while another still reads the current one (it cannot get two groups ahead,
+    // since every epilogue thread must stage a group before its MMAs can run)
+    const int w_words = p.qg * p.HP;
+    int acc_it = 0, seg = 0;
+    int item = start_item, t0 = start_tile, remaining = my_count;
+    bool ok = true;
+    while (remaining > 0 && ok) {
+      const GroupInfo gi = group_info(p, item);
+      const int t1 = min(gi.n_tiles, t0 + remaining);
+      if (t1 > t0) {
+        // -- stage this group's q (swizzled, zero-padded) and head weights
+        if (seg > 0 && !mbar_wait(&sb->q_empty, (uint32_t)(seg - 1) & 1u, abort, p.status)) { ok = false; break; }
+        float* w_s = reinterpret_cast<float*>(smem + p.off_w) + (seg & 1) * w_words;
+        int* info_pos = reinterpret_cast<int*>(smem + p.off_info) + (seg & 1) * 16;
+        float* info_qs = reinterpret_cast<float*>(smem + p.off_info + 128) + (seg & 1) * 16;
+        const int chunks16 = p.kbw / 16;
+        const int total16 = NSUB * p.n_kblocks * p.n_cols * chunks16;
+        for (int i = et; i < total16; i += kEpiThreads) {
+          const int c16 = i % chunks16;
+          int r = i / chunks16;
+          const int rr = r % p.n_cols;
+          r /= p.n_cols;
+          const int kb = r % p.n_kblocks;
+          const int sb_ = r / p.n_kblocks;
+          const int ql = rr / p.HP, h = rr - ql * p.HP;
+          const int j = gi.g * p.qg + sb_ * p.nq_sub + ql;
+          uint4 v = make_uint4(0u, 0u, 0u, 0u);
+          if (j < p.J && h < p.H)
+            v = *reinterpret_cast<const uint4*>(p.q + (((long long)gi.b * p.J + j) * p.H + h) * p.d_bytes +
+                                                kb * p.kbw + c16 * 16);
+          const uint32_t dst = smem_u32(smem + p.off_q + sb_ * p.q_sub_bytes + kb * p.q_kblock_bytes) +
+                               swizzled_offset(rr, c16 * 16, p.kbw);
+          st_shared_v4(dst, v.x, v.y, v.z, v.w);
+        }
+        for (int i = et; i < p.qg * p.HP; i += kEpiThreads) {
+          const int ql = i / p.HP, h = i - ql * p.HP;
+          const int j = gi.g * p.qg + ql;
+          w_s[i] = (j < p.J && h < p.H) ? p.w[((long long)gi.b * p.J + j) * p.H + h] : 0.0f;
+        }
+        if (et < p.qg) {
+          const int j = gi.g * p.qg + et;
+          info_pos[et] = j < p.J ? query_position(p.seq_lens, p.q_pos, p.J, gi.b, j, p.Lpad) : -1;
+          info_qs[et] = (j < p.J && p.q_scale) ? p.q_scale[(long long)gi.b * p.J + j] : 1.0f;
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&sb->q_full);
+        // every epilogue thread has staged its share (w_s / info are visible after this)
+        if (!mbar_wait(&sb->q_full, (uint32_t)seg & 1u, abort, p.status)) { ok = false; break; }
+        const int32_t* pt_row = p.page_table + (long long)gi.b * p.max_pages;
+        const long long out_row0 = (long long)gi.b * p.J;
+        for (int t = t0; t < t1; ++t, ++acc_it) {
+          const int as = acc_it % p.acc_stages;
+          const uint32_t aph = (uint32_t)(acc_it / p.acc_stages) & 1u;
+          const int s = t * kIndexTileRows + row;
+          // per-position scale and page check (independent of the accumulator: fetch first);
+          // a position whose page id is outside the pool is ranked last (-inf)
+          float ks = 1.0f;
+          if (s <= gi.max_pos) {
+            const int page = pt_row[s / p.P];
+            if (page < 0 || page >= p.num_pages) ks = __int_as_float(0xff800000);
+            else if (p.k_scale) ks = p.k_scale[(long long)page * p.P + (s % p.P)];
+          }
+          if (!mbar_wait(&sb->acc_full[as][sub], aph, abort, p.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t col0 = (uint32_t)((as * NSUB + sub) * p.n_cols);
+          for (int ql = 0; ql < p.nq_sub; ++ql) {
+            const int qloc = sub * p.nq_sub + ql;
+            const float* wq = w_s + qloc * p.HP;
+            float acc = 0.0f;
+            for (int hc = 0; hc * 16 < p.H; hc += 2) {
+              uint32_t v0[16], v1[16];
+              const uint32_t ta = tmem_addr(tmem_base, quad * 32, col0 + ql * p.HP + hc * 16);
+              tmem_ld16(ta, v0);
+              const bool two = (hc + 1) * 16 < p.H;
+              if (two) tmem_ld16(ta + 16, v1);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                acc = fmaf(wq[hc * 16 + i], fmaxf(__uint_as_float(v0[i]), 0.0f), acc);
+              if (two) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                  acc = fmaf(wq[hc * 16 + 16 + i], fmaxf(__uint_as_float(v1[i]), 0.0f), acc);
+              }
+            }
+            const int pos = info_pos[qloc];
+            if (s <= pos) {
+              const int j = gi.g * p.qg + qloc;
+              const float v = isinf(ks) ? ks : acc * ks * info_qs[qloc];
+              p.scores[(out_row0 + j) * p.Lpad + s] = v;
+            }
+          }
+          tc_fence_before();
+          mbar_arrive(&sb->acc_empty[as][sub]);
+        }
+        ++seg;
+      }
+      remaining -= (t1 - t0);
+      ++item;
+      t0 = 0;
+    }
+  }
+  pdl_launch_dependents();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, p.tmem_cols);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_index_score(const IndexKernelParams& p, const CUtensorMap& kmap, int grid,
+                               bool pdl, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(64 + 128 * p.n_sub, 1, 1);
+  cfg.dynamicSmemBytes = p.smem_bytes;
+  cfg.stream = stream;
+  int na = 0;
+  if (pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  cudaError_t e;
+  if (p.n_sub == 2) {
+    e = cudaFuncSetAttribute(index_score_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)p.smem_bytes);
+    if (e != cudaSuccess) return e;
+    return cudaLaunchKernelEx(&cfg, index_score_kernel<2>, kmap, p);
+  }
+  e = cudaFuncSetAttribute(index_score_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)p.smem_bytes);
+  if (e != cudaSuccess) return e;
+  return cudaLaunchKernelEx(&cfg, index_score_kernel<1>, kmap, p);
+}
+
+}  // namespace sia

@@ -1,0 +1,106 @@
+// sia_internal.h -- launch parameters shared between the C-ABI layer (sia_api.cu) and the
+// kernels of libsia.  Host and device code; no torch types.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "sia.h"
+
+namespace sia {
+
+// Rows (positions) per indexer tile: the M of every tcgen05 MMA of the indexer.
+constexpr int kIndexTileRows = 128;
+// Latent rows per attention tile.
+constexpr int kAttnTileRows = 64;
+// Largest Top-K slice one CTA keeps in shared memory (keys, 4 bytes each).
+constexpr int kTopkSliceMax = 16384;
+constexpr int kTopkThreads = 512;
+
+// -------------------------------------------------------------------------- indexer scoring
+struct IndexKernelParams {
+  int B, J, H, HP;            // batch, queries per sequence, heads, heads padded to 16
+  int P, max_pages, num_pages;
+  long long Lpad;             // score row length = max_pages * P
+  int d_bytes;                // bytes of one q / k row
+  int kbw;                    // bytes per K block row (128 or 64)
+  int n_kblocks;              // d_bytes / kbw
+  int ksteps_per_block;       // kbw / 32
+  int fp8;
+  int nq_sub;                 // queries per accumulator sub-block
+  int n_sub;                  // accumulator sub-blocks per A tile (1 or 2)
+  int qg;                     // queries per group = nq_sub * n_sub
+  int n_cols;                 // N of one MMA = nq_sub * HP
+  int groups_per_seq;         // ceil(J / qg)
+  int acc_stages;             // accumulator stages in TMEM
+  int k_stages;               // K-tile stages in shared memory
+  int box_rows;               // rows per TMA box = min(P, 128)
+  uint32_t tmem_cols;
+  // shared-memory layout, byte offsets from the 1024-aligned base
+  uint32_t off_k, k_stage_bytes, k_kblock_bytes;
+  uint32_t off_q, q_sub_bytes, q_kblock_bytes;
+  uint32_t off_w, off_info, off_bar, smem_bytes;
+  const uint8_t* q;
+  const float* q_scale;
+  const float* w;
+  const float* k_scale;
+  const int32_t* page_table;
+  const int32_t* seq_lens;
+  const int32_t* q_pos;
+  float* scores;
+  int32_t* status;
+};
+
+// -------------------------------------------------------------------------- Top-K
+struct TopkKernelParams {
+  int B, J, K;
+  long long Lpad;
+  int cluster;                // CTAs per query row
+  int slice;                  // keys per CTA (multiple of 32, <= kTopkSliceMax)
+  const float* scores;
+  const int32_t* seq_lens;
+  const int32_t* q_pos;
+  int32_t* topk;
+  int32_t* status;
+};
+
+// -------------------------------------------------------------------------- attention
+struct AttnKernelParams {
+  int B, J, H, DL, DR, P, max_pages, num_pages, K;
+  float scale_log2;           // softmax_scale * log2(e)
+  int splits;                 // Top-K splits per query (>1 -> partials + combine)
+  int rows_per_split;         // multiple of kAttnTileRows
+  int units;                  // B * J * splits
+  const int32_t* page_table;
+  const int32_t* seq_lens;
+  const int32_t* topk;
+  uint16_t* out;              // bf16 bits
+  float* lse;
+  float* part_o;              // [splits][B*J][H][DL] fp32 (splits > 1)
+  float* part_lse;            // [splits][B*J][H]
+  int32_t* status;
+};
+
+struct CombineKernelParams {
+  int BJ, H, DL, splits;
+  const float* part_o;
+  const float* part_lse;
+  uint16_t* out;
+  float* lse;
+};
+
+// Launchers (each returns cudaSuccess or the launch error).  `pdl` asks for programmatic
+// dependent launch on the previous kernel of the stream.
+cudaError_t launch_index_score(const IndexKernelParams& p, const CUtensorMap& kmap, int grid,
+                               bool pdl, cudaStream_t stream);
+cudaError_t launch_topk(const TopkKernelParams& p, bool pdl, cudaStream_t stream);
+cudaError_t launch_sparse_attend(const AttnKernelParams& p, const CUtensorMap* maps,
+                                 int n_clusters, bool pdl, cudaStream_t stream);
+cudaError_t launch_combine(const CombineKernelParams& p, bool pdl, cudaStream_t stream);
+
+// Shared memory the attention kernel needs for (d_latent, d_rope).
+size_t attend_smem_bytes(int dl, int dr);
+
+}  // namespace sia

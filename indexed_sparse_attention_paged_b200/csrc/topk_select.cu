@@ -1,0 +1,237 @@
+// topk_select.cu -- exact per-query Top-K of the index scores (radix select).
+//
+// For each query row, picks the K positions with the largest score, ties going to the lower
+// position, and writes them in ascending order, padded with -1 when fewer than K positions are
+// visible ("Day 0 Inference Adaptation and Performance Optimization for Hybrid Sparse Attention
+// LLMs", section "Operator Fusion and Multi-Stream Scheduling", step 3; the fused index
+// operator outputs only these indices, "Rapid Adaptation and Inference Optimization",
+// section IV.4.1).
+//
+// Design: one thread-block cluster of `cluster` CTAs per query row; each CTA keeps a slice of
+// the row's keys in shared memory.  Keys are the scores mapped to order-preserving uint32
+// (-0.0 folded onto +0.0).  Three MSB-first radix passes (11, 11, 10 bits) find the exact K-th
+// largest key T; the per-CTA digit histograms are summed across the cluster through
+// distributed shared memory.  The selection is then every key > T plus the lowest-positioned
+// keys == T, compacted in position order with block- and cluster-level prefix sums, which
+// makes the output ascending without a sort.
+#include <cuda_runtime.h>
+
+#include "sia_common.cuh"
+#include "sia_internal.h"
+#include "sia_ptx.cuh"
+
+namespace sia {
+namespace {
+
+constexpr int kBins = 2048;
+
+__device__ __forceinline__ uint32_t order_key(float f) {
+  uint32_t u = __float_as_uint(f);
+  if (u == 0x80000000u) u = 0u;  // -0.0 ranks as +0.0
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+struct TopkShared {
+  uint32_t hist[2][kBins];
+  int scan[kTopkThreads / 32];
+  int scan2[kTopkThreads / 32];
+  uint32_t sel_prefix;
+  int sel_krem;
+  int cta_gt, cta_eq;
+};
+
+// Block-wide exclusive prefix sum of (a, b) over threads in thread order; also returns totals.
+__device__ __forceinline__ void block_scan2(int a, int b, int& ea, int& eb, int& ta, int& tb,
+                                            TopkShared* sh) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int ia = a, ib = b;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int va = __shfl_up_sync(0xffffffffu, ia, o);
+    const int vb = __shfl_up_sync(0xffffffffu, ib, o);
+    if (lane >= o) { ia += va; ib += vb; }
+  }
+  if (lane == 31) { sh->scan[warp] = ia; sh->scan2[warp] = ib; }
+  __syncthreads();
+  int wa = 0, wb = 0;
+  ta = 0; tb = 0;
+  for (int w = 0; w < kTopkThreads / 32; ++w) {
+    if (w < warp) { wa += sh->scan[w]; wb += sh->scan2[w]; }
+    ta += sh->scan[w];
+    tb += sh->scan2[w];
+  }
+  ea = wa + ia - a;
+  eb = wb + ib - b;
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkKernelParams p) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  TopkShared* sh = reinterpret_cast<TopkShared*>(smem);
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem + sizeof(TopkShared));
+  const int tid = threadIdx.x, lane = tid & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int C = p.cluster;
+  const long long row = blockIdx.x / C;
+  const int b = (int)(row / p.J), j = (int)(row - (long long)b * p.J);
+  int32_t* out = p.topk + row * p.K;
+
+  pdl_wait_primary();  // scores come from the previous kernel on the stream
+
+  bool bad = false;
+  const int pos = query_position(p.seq_lens, p.q_pos, p.J, b, j, p.Lpad, &bad);
+  if (bad && rank == 0 && tid == 0) report(p.status, SIA_DEV_BAD_POSITION);
+  const int n = pos + 1;  // visible positions 0..pos
+  if (n <= p.K) {
+    // everything visible is selected: 0..n-1 then -1 padding (no scores needed)
+    for (int i = rank * kTopkThreads + tid; i < p.K; i += C * kTopkThreads) out[i] = i < n ? i : -1;
+    pdl_launch_dependents();
+    return;
+  }
+
+  // ---- load this CTA's slice of keys
+  const int s0 = rank * p.slice;
+  const int len = max(0, min(n - s0, p.slice));
+  const float* src = p.scores + row * p.Lpad + s0;
+  for (int i = tid; i < len; i += kTopkThreads) keys[i] = order_key(src[i]);
+
+  // ---- three radix passes to find the K-th largest key
+  uint32_t prefix = 0;
+  int krem = p.K;
+  const int shifts[3] = {21, 10, 0};
+  const int widths[3] = {11, 11, 10};
+  for (int pass = 0; pass < 3; ++pass) {
+    uint32_t* h = sh->hist[pass & 1];
+    for (int i = tid; i < kBins; i += kTopkThreads) h[i] = 0;
+    __syncthreads();
+    const int sh_ = shifts[pass];
+    const int hi_shift = sh_ + widths[pass];  // bits above this digit must equal the prefix
+    const uint32_t dmask = (1u << widths[pass]) - 1u;
+    const int rounds = (len + kTopkThreads - 1) / kTopkThreads;
+    for (int r = 0; r < rounds; ++r) {
+      const int i = r * kTopkThreads + tid;
+      uint32_t digit = 0xffffffffu;
+      if (i < len) {
+        const uint32_t k = keys[i];
+        const bool match = pass == 0 || (k >> hi_shift) == prefix;
+        if (match) digit = (k >> sh_) & dmask;
+      }
+      const unsigned same = __match_any_sync(0xffffffffu, digit);
+      if (digit != 0xffffffffu && lane == __ffs(same) - 1) atomicAdd(&h[digit], (uint32_t)__popc(same));
+    }
+    // make every CTA's histogram visible cluster-wide, then sum them
+    cluster_sync();
+    // each thread owns 4 consecutive bins; count of keys in bins above, found by a suffix scan
+    const int per = kBins / kTopkThreads;
+    uint32_t cnt[kBins / kTopkThreads];
+    int mine = 0;
+#pragma unroll
+    for (int q = 0; q < per; ++q) {
+      const int bin = tid * per + q;
+      uint32_t c = 0;
+      for (int r = 0; r < C; ++r) c += ld_cluster_u32(mapa_cluster(&h[bin], (uint32_t)r));
+      cnt[q] = c;
+      mine += (int)c;
+    }
+    // suffix sum over threads in descending bin order: scan with reversed thread index
+    int ex_a, ex_b, tot_a, tot_b;
+    // thread t's position in descending order is (kTopkThreads-1-t); compute the exclusive
+    // prefix over higher threads by scanning the reversed values
+    __syncthreads();
+    {
+      // place values in reversed order through shared scratch
+      __shared__ int rev[kTopkThreads];
+      rev[kTopkThreads - 1 - tid] = mine;
+      __syncthreads();
+      const int rv = rev[tid];
+      block_scan2(rv, 0, ex_a, ex_b, tot_a, tot_b, sh);
+      __syncthreads();
+      rev[kTopkThreads - 1 - tid] = ex_a;  // keys in bins of higher threads
+      __syncthreads();
+      ex_a = rev[tid];
+      __syncthreads();
+    }
+    int above = ex_a;  // keys in bins above this thread's bins
+#pragma unroll
+    for (int q = per - 1; q >= 0; --q) {
+      const int bin = tid * per + q;
+      const int c = (int)cnt[q];
+      if (above < krem && krem <= above + c) {
+        sh->sel_prefix = (prefix << widths[pass]) | (uint32_t)bin;
+        sh->sel_krem = krem - above;
+      }
+      above += c;
+    }
+    __syncthreads();
+    prefix = sh->sel_prefix;
+    krem = sh->sel_krem;
+    __syncthreads();
+  }
+  const uint32_t T = prefix;  // the K-th largest key; take every key > T and krem keys == T
+
+  // ---- compaction in position order
+  const int chunk = (len + kTopkThreads - 1) / kTopkThreads;
+  const int c0 = min(len, tid * chunk), c1 = min(len, c0 + chunk);
+  int gt = 0, eq = 0;
+  for (int i = c0; i < c1; ++i) {
+    gt += keys[i] > T;
+    eq += keys[i] == T;
+  }
+  int ex_gt, ex_eq, tot_gt, tot_eq;
+  block_scan2(gt, eq, ex_gt, ex_eq, tot_gt, tot_eq, sh);
+  if (tid == 0) { sh->cta_gt = tot_gt; sh->cta_eq = tot_eq; }
+  cluster_sync();
+  int off_gt = 0, off_eq = 0;
+  for (int r = 0; r < (int)rank; ++r) {
+    off_gt += (int)ld_cluster_u32(mapa_cluster(&sh->cta_gt, (uint32_t)r));
+    off_eq += (int)ld_cluster_u32(mapa_cluster(&sh->cta_eq, (uint32_t)r));
+  }
+  int gt_before = off_gt + ex_gt, eq_before = off_eq + ex_eq;
+  for (int i = c0; i < c1; ++i) {
+    const uint32_t k = keys[i];
+    if (k > T) {
+      out[gt_before + min(eq_before, krem)] = s0 + i;
+      ++gt_before;
+    } else if (k == T) {
+      if (eq_before < krem) out[gt_before + eq_before] = s0 + i;
+      ++eq_before;
+    }
+  }
+  pdl_launch_dependents();
+  cluster_sync();  // no CTA leaves while a peer may still read its shared memory
+}
+
+}  // namespace
+
+cudaError_t launch_topk(const TopkKernelParams& p, bool pdl, cudaStream_t stream) {
+  const size_t smem = sizeof(TopkShared) + (size_t)p.slice * sizeof(uint32_t);
+  cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  if (p.cluster > 8) {
+    e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  cfg.gridDim = dim3((unsigned)((long long)p.B * p.J * p.cluster), 1, 1);
+  cfg.blockDim = dim3(kTopkThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  int na = 0;
+  attr[na].id = cudaLaunchAttributeClusterDimension;
+  attr[na].val.clusterDim.x = p.cluster;
+  attr[na].val.clusterDim.y = 1;
+  attr[na].val.clusterDim.z = 1;
+  ++na;
+  if (pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, topk_kernel, p);
+}
+
+}  // namespace sia

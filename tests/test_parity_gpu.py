@@ -1,0 +1,303 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the same seeded
+inputs.  Index scores and Top-K lists must match exactly; attention outputs within max-abs 1e-2
+of the oracle's fp64 result (the spec's tolerance; the bf16 rounding of the output alone is at
+most 2^-9 relative)."""
+import functools
+
+import numpy as np
+import pytest
+import torch
+
+import indexed_sparse_attention_paged_b200 as sia
+import oracle
+from indexed_sparse_attention_paged_b200 import workloads
+
+pytestmark = pytest.mark.gpu
+
+ATOL = 1e-2
+DEV = "cuda:0"
+
+
+def _wl(number, **kw):
+    base = workloads.WORKLOADS[number]
+    return workloads.Workload(**{**base.__dict__, **kw})
+
+
+def run_index(h, d, top_k, with_scores=True):
+    B, J = h["batch"], h["n_q"]
+    Lpad = h["max_pages"] * h["workload"].page_size
+    scores = torch.full((B, J, Lpad), float("nan"), device=DEV) if with_scores else None
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    topk = sia.sparse_index_topk(d["q_idx"], d["w"], d["k_cache"], d["page_table"], d["seq_lens"],
+                                 top_k=top_k, k_scale=d["k_scale"], q_pos=d.get("q_pos"),
+                                 scores_out=scores, dev_status=status)
+    torch.cuda.synchronize()
+    return topk.cpu().numpy(), (scores.cpu().numpy() if with_scores else None), int(status.item())
+
+
+def oracle_index(h, top_k, rows=None, q_pos=None):
+    wl = h["workload"]
+    ks = None if h["k_scale"] is None else h["k_scale"].numpy()
+    return oracle.index_topk(h["q_idx"], h["w"].numpy(), h["k_cache"], h["page_table"].numpy(),
+                             h["seq_lens"].numpy(), page_size=wl.page_size, top_k=top_k,
+                             fp8=wl.idx_fp8, k_scale=ks,
+                             q_pos=None if q_pos is None else q_pos.numpy(), rows=rows)
+
+
+def run_attend(h, d, topk_np, with_lse=True):
+    wl = h["workload"]
+    topk = torch.from_numpy(np.ascontiguousarray(topk_np)).to(DEV)
+    B, J, H = h["batch"], h["n_q"], wl.attn_heads
+    lse = torch.full((B, J, H), float("nan"), device=DEV) if with_lse else None
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    out = sia.sparse_mla_attend(d["q_attn"], d["kv_cache"], d["page_table"], d["seq_lens"], topk,
+                                d_latent=wl.d_latent, softmax_scale=wl.softmax_scale, lse=lse,
+                                dev_status=status)
+    torch.cuda.synchronize()
+    return out.float().cpu().numpy(), (lse.cpu().numpy() if with_lse else None), int(status.item())
+
+
+def oracle_attend(h, topk_np, rows=None):
+    wl = h["workload"]
+    return oracle.sparse_attend(h["q_attn"], h["kv_cache"], h["page_table"].numpy(),
+                                h["seq_lens"].numpy(), topk_np, page_size=wl.page_size,
+                                d_latent=wl.d_latent, scale=wl.softmax_scale, rows=rows)
+
+
+def assert_scores_equal(got, ref, nvis_rows):
+    """Exact equality of every visible score (positions 0..p of each row)."""
+    for (b, j), n in nvis_rows:
+        g, r = got[b, j, :n], ref[b, j, :n].astype(np.float32)
+        bad = np.flatnonzero(g != r)
+        assert bad.size == 0, "row (%d,%d): %d scores differ, first at %d: %r vs %r" % (
+            b, j, bad.size, bad[0], g[bad[0]], r[bad[0]])
+
+
+def check_index_case(h, top_k, rows=None):
+    d = workloads.to_device(h, DEV)
+    got_topk, got_scores, st = run_index(h, d, top_k)
+    assert st == 0
+    ref_topk, ref_scores, ost = oracle_index(h, top_k, rows=rows)
+    assert ost == 0
+    B, J = h["batch"], h["n_q"]
+    flat = range(B * J) if rows is None else rows
+    nv = []
+    for r in flat:
+        b, j = divmod(int(r), J)
+        n = int(np.sum(~np.isnan(ref_scores[b, j])))
+        nv.append(((b, j), n))
+    assert_scores_equal(got_scores, ref_scores, nv)
+    for r in flat:
+        b, j = divmod(int(r), J)
+        assert np.array_equal(got_topk[b, j], ref_topk[b, j]), "top-k differs in row (%d,%d)" % (b, j)
+    return got_topk
+
+
+def check_attend_case(h, topk_np, rows=None):
+    d = workloads.to_device(h, DEV)
+    got, got_lse, st = run_attend(h, d, topk_np)
+    assert st == 0
+    ref, ref_lse, ost = oracle_attend(h, topk_np, rows=rows)
+    assert ost == 0
+    B, J = h["batch"], h["n_q"]
+    flat = range(B * J) if rows is None else rows
+    H = h["workload"].attn_heads
+    worst = 0.0
+    for r in flat:
+        b, j = divmod(int(r), J)
+        err = np.abs(got[b, j] - ref[b, j])
+        worst = max(worst, float(err.max()))
+        assert err.max() <= ATOL, "row (%d,%d): max-abs error %.3g" % (b, j, err.max())
+        e_lse = np.abs(got_lse[b, j] - ref_lse[b, j])
+        fin = np.isfinite(ref_lse[b, j])
+        assert np.all(np.isfinite(got_lse[b, j]) == fin)
+        assert np.all(e_lse[fin] <= 1e-3 * np.maximum(1.0, np.abs(ref_lse[b, j][fin]))), "lse row (%d,%d)" % (b, j)
+    return worst
+
+
+# ------------------------------------------------------------------ stage 1: index + Top-K
+
+INDEX_CASES = {
+    # name: (workload number, overrides, top_k)
+    "tiny_cfg1": (1, dict(), 16),
+    "bf16_ragged_p64": (2, dict(seq_lens=[300, 1000, 37, 129]), 64),
+    "bf16_l_lt_k": (2, dict(seq_lens=[100, 5, 1]), 128),
+    "bf16_j2_causal": (2, dict(seq_lens=[700, 256], n_q=2), 128),
+    "fp8_ragged": (3, dict(seq_lens=[513, 2000, 64]), 256),
+    "fp8_j2": (5, dict(seq_lens=[1500, 777], n_q=2), 300),
+    "prefill_chunk_300": (4, dict(seq_lens=[300], n_q=300), 64),
+}
+
+
+@pytest.mark.parametrize("name", sorted(INDEX_CASES))
+def test_index_topk_matches_oracle(name):
+    num, kw, top_k = INDEX_CASES[name]
+    h = workloads.make_inputs(workloads.WORKLOADS[num], **kw)
+    check_index_case(h, top_k)
+
+
+def test_index_all_equal_scores_take_lowest_positions():
+    h = workloads.make_inputs(workloads.WORKLOADS[2], seq_lens=[1000, 3000])
+    h["w"].zero_()                      # every score is 0: the tie rule decides everything
+    got = check_index_case(h, 256)
+    assert np.array_equal(got[0, 0], np.arange(256)) and np.array_equal(got[1, 0], np.arange(256))
+
+
+def test_index_negative_weights_give_no_negative_zero():
+    h = workloads.make_inputs(workloads.WORKLOADS[2], seq_lens=[900])
+    h["w"].copy_(-torch.abs(h["w"]) - 1.0)    # all w < 0 -> scores <= 0, many exact zeros
+    d = workloads.to_device(h, DEV)
+    _, scores, _ = run_index(h, d, 128)
+    z = scores[0, 0, :900]
+    assert np.all(z <= 0)
+    assert not np.any(np.signbit(z[z == 0])), "-0.0 written"
+    check_index_case(h, 128)
+
+
+def test_index_fp8_and_bf16_storage_select_the_same_positions():
+    hb = workloads.make_inputs(workloads.WORKLOADS[2], seq_lens=[3000, 1200])
+    h8 = dict(hb)
+    h8["workload"] = _wl(2, idx_fp8=True)
+    h8["q_idx"] = hb["q_idx"].float().to(torch.float8_e4m3fn)
+    h8["k_cache"] = hb["k_cache"].float().to(torch.float8_e4m3fn)
+    tb, _, _ = run_index(hb, workloads.to_device(hb, DEV), 512)
+    t8, _, _ = run_index(h8, workloads.to_device(h8, DEV), 512)
+    assert np.array_equal(tb, t8)
+
+
+def test_index_bad_page_id_sets_status_without_fault():
+    h = workloads.make_inputs(workloads.WORKLOADS[2], seq_lens=[500, 500])
+    h["page_table"][1, 2] = h["num_pages"] + 7
+    d = workloads.to_device(h, DEV)
+    topk, _, st = run_index(h, d, 64)
+    assert st & sia.SIA_DEV_BAD_PAGE
+    ref, _, _ = oracle_index(h, 64, rows=[0])
+    assert np.array_equal(topk[0, 0], ref[0, 0])      # the untouched sequence is still exact
+
+
+# ------------------------------------------------------------------ stage 2: sparse attention
+
+def _random_topk(h, top_k, seed, fill=1.0):
+    rng = np.random.default_rng(seed)
+    B, J = h["batch"], h["n_q"]
+    L = h["seq_lens"].numpy()
+    out = np.full((B, J, top_k), -1, dtype=np.int32)
+    for b in range(B):
+        for j in range(J):
+            p = L[b] - J + j
+            n = min(top_k, p + 1, max(1, int(fill * top_k)))
+            out[b, j, :n] = np.sort(rng.choice(p + 1, size=n, replace=False))
+    return out
+
+
+ATTN_CASES = {
+    "tiny_cfg1_heads8": (1, dict(), 16, 1.0),
+    "mla512_b1_splits": (2, dict(seq_lens=[5000]), 2048, 1.0),
+    "mla512_b3_ragged_lists": (2, dict(seq_lens=[3000, 130, 700]), 512, 0.7),
+    "mla512_j2": (2, dict(seq_lens=[900, 2500], n_q=2), 256, 1.0),
+    "mla512_short_list": (2, dict(seq_lens=[40]), 64, 1.0),
+}
+
+
+@pytest.mark.parametrize("name", sorted(ATTN_CASES))
+def test_attend_matches_oracle(name):
+    num, kw, top_k, fill = ATTN_CASES[name]
+    h = workloads.make_inputs(workloads.WORKLOADS[num], **kw)
+    topk = _random_topk(h, top_k, seed=7, fill=fill)
+    check_attend_case(h, topk)
+
+
+def test_attend_empty_list_gives_zero_and_minus_inf():
+    h = workloads.make_inputs(workloads.WORKLOADS[2], seq_lens=[300, 300])
+    topk = _random_topk(h, 128, seed=3)
+    topk[1] = -1
+    d = workloads.to_device(h, DEV)
+    out, lse, st = run_attend(h, d, topk)
+    assert st == 0
+    assert np.all(out[1] == 0) and np.all(np.isneginf(lse[1]))
+    check_attend_case(h, topk, rows=[0])
+
+
+def test_attend_bad_position_sets_status_and_is_skipped():
+    h = workloads.make_inputs(workloads.WORKLOADS[2], seq_lens=[300])
+    topk = _random_topk(h, 128, seed=5)
+    bad = topk.copy()
+    bad[0, 0, 10] = 100000                     # past the context: ignored, reported
+    d = workloads.to_device(h, DEV)
+    out, _, st = run_attend(h, d, bad)
+    assert st & sia.SIA_DEV_BAD_POSITION
+    keep = np.concatenate([topk[0, 0, :10], topk[0, 0, 11:], [-1]]).astype(np.int32)[None, None]
+    ref, _, _ = oracle_attend(h, keep)
+    assert np.abs(out - ref).max() <= ATOL
+
+
+# ------------------------------------------------------------------ the fused decode path
+
+@pytest.mark.parametrize("num,kw", [(1, {}), (2, dict(seq_lens=[2500, 4100])),
+                                    (3, dict(seq_lens=[1500, 3000, 2049])),
+                                    (5, dict(seq_lens=[4000, 2300]))])
+def test_fused_decode_matches_oracle(num, kw):
+    wl = workloads.WORKLOADS[num]
+    h = workloads.make_inputs(wl, **kw)
+    d = workloads.to_device(h, DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    out, topk = sia.fused_decode(d["q_idx"], d["w"], d["k_cache"], d["q_attn"], d["kv_cache"],
+                                 d["page_table"], d["seq_lens"], top_k=wl.top_k,
+                                 d_latent=wl.d_latent, softmax_scale=wl.softmax_scale,
+                                 k_scale=d["k_scale"], dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    ref_topk, _, _ = oracle_index(h, wl.top_k)
+    assert np.array_equal(topk.cpu().numpy(), ref_topk)
+    ref, _, _ = oracle_attend(h, ref_topk)
+    assert np.abs(out.float().cpu().numpy() - ref).max() <= ATOL
+
+
+# ------------------------------------------------------------------ full-size workloads, sampled
+
+@functools.lru_cache(maxsize=1)
+def _full(num):
+    return workloads.make_inputs(workloads.WORKLOADS[num])
+
+
+@pytest.mark.parametrize("num", [2, 3, 5, 4])
+def test_full_size_workload_sampled_rows(num):
+    wl = workloads.WORKLOADS[num]
+    h = _full(num)
+    d = workloads.to_device(h, DEV)
+    B, J = h["batch"], h["n_q"]
+    rng = np.random.default_rng(num)
+    n_rows = 3 if num != 4 else 6
+    rows = sorted(set(int(r) for r in rng.choice(B * J, size=n_rows, replace=False)) |
+                  ({B * J - 1} if num == 4 else set()))
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    if num == 4:
+        topk = sia.sparse_index_topk(d["q_idx"], d["w"], d["k_cache"], d["page_table"],
+                                     d["seq_lens"], top_k=wl.top_k, dev_status=status)
+        out = sia.sparse_mla_attend(d["q_attn"], d["kv_cache"], d["page_table"], d["seq_lens"], topk,
+                                    d_latent=wl.d_latent, softmax_scale=wl.softmax_scale,
+                                    dev_status=status)
+    else:
+        out, topk = sia.fused_decode(d["q_idx"], d["w"], d["k_cache"], d["q_attn"], d["kv_cache"],
+                                     d["page_table"], d["seq_lens"], top_k=wl.top_k,
+                                     d_latent=wl.d_latent, softmax_scale=wl.softmax_scale,
+                                     k_scale=d["k_scale"], dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    got_topk = topk.cpu().numpy()
+    ref_topk, _, _ = oracle_index(h, wl.top_k, rows=rows)
+    for r in rows:
+        b, j = divmod(r, J)
+        assert np.array_equal(got_topk[b, j], ref_topk[b, j]), "top-k row %d" % r
+    ref, _, _ = oracle_attend(h, got_topk, rows=rows)
+    got = out.float().cpu().numpy()
+    for r in rows:
+        b, j = divmod(r, J)
+        assert np.abs(got[b, j] - ref[b, j]).max() <= ATOL, "attention row %d" % r
+    # properties that hold for every row: ascending lists, -1 only as tail padding
+    t = got_topk.reshape(B * J, -1)
+    valid = t >= 0
+    assert np.all(valid[:, :-1] | ~valid[:, 1:])
+    d_ = np.diff(np.where(valid, t, np.iinfo(np.int32).max), axis=1)
+    assert np.all((d_ > 0) | ~valid[:, 1:])
+    assert np.all(np.isfinite(got))
