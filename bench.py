@@ -1,0 +1,376 @@
+"""Benchmark: fused sparse-attention decode throughput on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload 2]
+
+One step = one fused decode (indexer scoring + Top-K + sparse MLA attention + split merge) over
+one batch of the decode workload (batch 32, one query token per sequence, context 8192, page
+size 64, shuffled pages; indexer 64 heads x 128 dims bf16; Top-K 2048; 128 attention heads over
+512+64 latent dims).  Inputs are seeded synthetic tensors (indexed_sparse_attention_paged_b200.
+workloads), resident in HBM before timing.  L2 is flushed (a 512 MiB write) before every timed
+step and each step is timed alone with CUDA events on the launching stream; the reported time
+is the mean step time, maximum over ranks.  With N GPUs every rank runs its own independent
+batch (weak scaling, no collective on the data path).
+
+Prints one JSON line (rank 0).  `--impl reference` times the CPU oracle (the only reference
+implementation: the pages have no code) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", type=int, default=2, choices=[2, 3, 5])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def source_sha() -> str:
+    """Hash of the CUDA sources, to tell whether recorded ncu counters are still current."""
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "indexed_sparse_attention_paged_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def algorithmic_bytes(inputs) -> dict:
+    """Bytes the step must move at minimum: every visible index-K row once per sequence (plus its
+    scale), every selected latent row once per query, the queries, weights and page tables in,
+    the outputs (attention out, lse, Top-K) out.  Score and split workspaces are not counted."""
+    wl = inputs["workload"]
+    B, J = inputs["batch"], inputs["n_q"]
+    lens = [int(x) for x in inputs["seq_lens"]]
+    idx_elem = 1 if wl.idx_fp8 else 2
+    idx_k = sum(lens) * wl.idx_dim * idx_elem + (sum(lens) * 4 if wl.idx_fp8 else 0)
+    sel = sum(min(wl.top_k, L - J + j + 1) for L in lens for j in range(J))
+    kv = sel * (wl.d_latent + wl.d_rope) * 2
+    q_idx = B * J * wl.idx_heads * wl.idx_dim * idx_elem + B * J * wl.idx_heads * 4
+    q_attn = B * J * wl.attn_heads * (wl.d_latent + wl.d_rope) * 2
+    pt = sum((L + wl.page_size - 1) // wl.page_size for L in lens) * 4 * 2 + B * 4
+    out = B * J * wl.attn_heads * wl.d_latent * 2 + B * J * wl.attn_heads * 4 + B * J * wl.top_k * 4
+    stage1 = idx_k + q_idx + pt // 2 + B * J * wl.top_k * 4
+    stage2 = kv + q_attn + pt // 2 + B * J * wl.top_k * 4 + B * J * wl.attn_heads * (wl.d_latent * 2 + 4)
+    return dict(total=idx_k + kv + q_idx + q_attn + pt + out, stage1=stage1, stage2=stage2,
+                idx_k=idx_k, kv=kv)
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons every 200 ms while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.QUERY,
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def peaks() -> dict:
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "source": "fallback"}
+
+
+def recorded_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on this source."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            t = json.load(f)
+        rec = t.get(kernel)
+        if rec and rec.get("source_sha") == source_sha():
+            return rec.get("dram_bytes_per_launch")
+    except (OSError, ValueError):
+        pass
+    return None
+
+
+def cpu_baseline(inputs, rows):
+    """The oracle, as it stands, on a bounded sample of query rows: scoring, Top-K, attention."""
+    import oracle
+    wl = inputs["workload"]
+    ks = None if inputs["k_scale"] is None else inputs["k_scale"].numpy()
+    pt, sl = inputs["page_table"].numpy(), inputs["seq_lens"].numpy()
+    t0 = time.perf_counter()
+    topk, _, _ = oracle.index_topk(inputs["q_idx"], inputs["w"].numpy(), inputs["k_cache"], pt, sl,
+                                   page_size=wl.page_size, top_k=wl.top_k, fp8=wl.idx_fp8, k_scale=ks,
+                                   rows=rows)
+    oracle.sparse_attend(inputs["q_attn"], inputs["kv_cache"], pt, sl, topk, page_size=wl.page_size,
+                         d_latent=wl.d_latent, scale=wl.softmax_scale, rows=rows)
+    dt = time.perf_counter() - t0
+    return dict(value=len(rows) / dt, unit="queries/s", cores=oracle.num_threads(), kind="oracle",
+                sample="%d of the %d query rows (rows %d..%d), full scoring + Top-K + attention each; %.1f s"
+                       % (len(rows), inputs["batch"] * inputs["n_q"], rows[0], rows[-1], dt))
+
+
+def run_reference(args, rank, world):
+    from indexed_sparse_attention_paged_b200 import workloads
+    import oracle
+    if rank != 0:
+        return
+    wl = workloads.WORKLOADS[args.workload]
+    inputs = workloads.make_inputs(wl)
+    n = max(4, min(16, oracle.num_threads()))
+    rows = list(range(n))
+    for _ in range(args.warmup and 1):
+        cpu_baseline(inputs, rows[:1])
+    vals = []
+    for _ in range(args.steps):
+        vals.append(cpu_baseline(inputs, rows))
+    v = statistics.mean(x["value"] for x in vals)
+    cb = dict(vals[-1])
+    cb["value"] = v
+    line = dict(impl="reference", metric=metric_name(wl), value=v, unit="queries/s", n_gpus=args.gpus,
+                steps=args.steps, warmup=args.warmup, ms_per_step=1000.0 * len(rows) / v / 1.0,
+                higher_is_better=True, scaling="weak", vs_baseline=None, dtype="f64", data="synthetic",
+                config=config_of(wl, inputs, "cpu (no L2 flush)"), cpu_baseline=cb,
+                e2e={"value": v, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0})
+    print(json.dumps(line), flush=True)
+
+
+def metric_name(wl):
+    return "fused sparse-attn decode queries/s @B=%d ctx=%s; achieved HBM GB/s %% of peak" % (
+        wl.batch, "8K" if wl.context == 8192 else str(wl.context or "1k-32k"))
+
+
+def config_of(wl, inputs, l2):
+    return {"workload": wl.name, "batch": inputs["batch"], "n_q": inputs["n_q"],
+            "context": wl.context or "uniform[%d,%d]" % (wl.len_lo, wl.len_hi),
+            "page_size": wl.page_size, "idx_heads": wl.idx_heads, "idx_dim": wl.idx_dim,
+            "idx_dtype": "e4m3" if wl.idx_fp8 else "bf16", "top_k": wl.top_k,
+            "attn_heads": wl.attn_heads, "d_latent": wl.d_latent, "d_rope": wl.d_rope,
+            "l2": l2, "parallelism": "replicas"}
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import torch
+    import torch.distributed as dist
+    import indexed_sparse_attention_paged_b200 as sia
+    from indexed_sparse_attention_paged_b200 import build as cuda_build
+    from indexed_sparse_attention_paged_b200 import workloads
+
+    cuda_build.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev, timeout=__import__("datetime").timedelta(seconds=120))
+
+    wl = workloads.WORKLOADS[args.workload]
+    host = workloads.make_inputs(wl, seed=1000 + wl.number + 7919 * rank)
+    d = workloads.to_device(host, dev)
+    plan = sia.FusedDecodePlan(d, dev)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+
+    def timed(fn, steps):
+        ts = []
+        for _ in range(steps):
+            flush.fill_(1)
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record(stream)
+            fn()
+            e.record(stream)
+            ts.append((s, e))
+        torch.cuda.synchronize()
+        return [s.elapsed_time(e) for s, e in ts]
+
+    # warm-up
+    for _ in range(max(3, args.warmup)):
+        plan()
+    torch.cuda.synchronize()
+
+    # stage-only calls for the per-kernel roofline
+    ia, aa = plan.ia, plan.aa
+    import ctypes
+    lib = sia.load_library()
+    ws1 = torch.empty(max(256, lib.sia_index_workspace_size(ctypes.byref(ia))), dtype=torch.uint8, device=dev)
+    ws2 = torch.empty(max(256, lib.sia_attend_workspace_size(ctypes.byref(aa))), dtype=torch.uint8, device=dev)
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    st_ptr = ctypes.c_void_p(plan.status.data_ptr())
+
+    def stage1():
+        sia._check(lib.sia_sparse_index_topk(ctypes.byref(ia), ctypes.c_void_p(ws1.data_ptr()), ws1.numel(), st_ptr, sp))
+
+    def stage2():
+        sia._check(lib.sia_sparse_mla_attend(ctypes.byref(aa), ctypes.c_void_p(ws2.data_ptr()), ws2.numel(), st_ptr, sp))
+
+    for _ in range(3):
+        stage1()
+        stage2()
+    torch.cuda.synchronize()
+
+    # ---------------- timed region
+    sampler = ClockSampler(local)
+    sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_wall = time.perf_counter()
+    step_ms = timed(plan, args.steps)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    wall = time.perf_counter() - t_wall
+    s1_ms = timed(stage1, max(10, args.steps // 2))
+    s2_ms = timed(stage2, max(10, args.steps // 2))
+    clocks = sampler.stop()
+    if int(plan.status.item()) != 0:
+        raise RuntimeError("device status %#x during the benchmark" % int(plan.status.item()))
+
+    mean_ms = statistics.mean(step_ms)
+    if world > 1:
+        t = torch.tensor([mean_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        mean_ms = float(t.item())
+
+    # ---------------- end-to-end through the C ABI with host buffers
+    pin = {k: host[k].pin_memory() for k in ("q_idx", "w", "q_attn", "page_table", "seq_lens")}
+    out_h = torch.empty(plan.out.shape, dtype=plan.out.dtype).pin_memory()
+    lse_h = torch.empty(plan.lse.shape, dtype=plan.lse.dtype).pin_memory()
+    topk_h = torch.empty(plan.topk.shape, dtype=plan.topk.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in pin.values())
+    d2h = sum(t.numel() * t.element_size() for t in (out_h, lse_h, topk_h))
+
+    def e2e_step():
+        for k, t in pin.items():
+            d[k].copy_(t, non_blocking=True)
+        plan()
+        out_h.copy_(plan.out, non_blocking=True)
+        lse_h.copy_(plan.lse, non_blocking=True)
+        topk_h.copy_(plan.topk, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    e2e_ms = statistics.mean(timed(e2e_step, max(10, args.steps // 2)))
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    queries = host["batch"] * host["n_q"]
+    value = world * queries / (mean_ms / 1000.0)
+    ab = algorithmic_bytes(host)
+    pk = peaks()
+    s1, s2 = statistics.mean(s1_ms), statistics.mean(s2_ms)
+    dominant = "sparse_attend" if s2 >= s1 else "index_topk"
+    dom_bytes, dom_ms = (ab["stage2"], s2) if dominant == "sparse_attend" else (ab["stage1"], s1)
+    achieved = dom_bytes / (dom_ms / 1000.0) / 1e9
+    step_gbs = ab["total"] / (mean_ms / 1000.0) / 1e9
+    kernels_per_step = 3 + (1 if plan_splits(lib, aa) > 1 else 0)
+
+    line = {
+        "metric": metric_name(wl), "value": value, "unit": "queries/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": mean_ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": config_of(wl, host, "flushed before every timed step (512 MiB write); inputs 370 MB"),
+        "achieved_hbm_gbs": step_gbs,
+        "hbm_frac_of_measured": step_gbs / pk["hbm_gbs"],
+        "hbm_frac_of_8tbs": step_gbs / 8000.0,
+        "roofline": {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": pk["hbm_gbs"],
+                     "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "peak_source": pk["source"],
+                     "traffic": recorded_traffic(dominant),
+                     "algorithmic_bytes_per_launch": dom_bytes, "ms_per_launch": dom_ms},
+        "stages": {"index_topk_ms": s1, "sparse_attend_ms": s2,
+                   "index_topk_gbs": ab["stage1"] / (s1 / 1000.0) / 1e9,
+                   "sparse_attend_gbs": ab["stage2"] / (s2 / 1000.0) / 1e9,
+                   "step_algorithmic_bytes": ab["total"]},
+        "e2e": {"value": world * queries / (e2e_ms / 1000.0), "unit": "queries/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": kernels_per_step * args.steps,
+        "clocks": clocks,
+        "wall_s_timed_region": wall,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        n = max(4, min(16, oracle.num_threads()))
+        line["cpu_baseline"] = cpu_baseline(host, list(range(n)))
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def plan_splits(lib, aa) -> int:
+    """Top-K splits the library picks for this attention call (from its workspace size)."""
+    import ctypes
+    return 2 if lib.sia_attend_workspace_size(ctypes.byref(aa)) > 0 else 1
+
+
+if __name__ == "__main__":
+    main()

@@ -163,7 +163,7 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
       const GroupInfo gi = group_info(p, item);
       const int t1 = min(gi.n_tiles, t0 + remaining);
       const int32_t* pt_row = p.page_table + (long long)gi.b * p.max_pages;
-      int cached_base = -1, cached_page = -1;
+      int cached_base = -(1 << 30), cached_page = -1;  // nothing cached yet
       for (int t = t0; t < t1 && ok; ++t, ++it) {
         const int stage = it % p.k_stages;
         const uint32_t phase = (uint32_t)(it / p.k_stages) & 1u;
