@@ -31,6 +31,9 @@
 namespace sia {
 namespace {
 
+// Per K stage: 16 bytes of chunk mask, then one fp32 key scale per tile row.
+constexpr uint32_t kStageInfoBytes = 16 + 4 * kIndexTileRows;
+
 struct IndexBarriers {
   uint64_t k_full[8];
   uint64_t k_empty[8];
@@ -126,7 +129,7 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.k_stages; ++s) {
       mbar_init(&sb->k_full[s], 1);
-      mbar_init(&sb->k_empty[s], 1);
+      mbar_init(&sb->k_empty[s], 1 + 4 * NSUB);  // MMA commit + every epilogue warp
     }
     for (int a = 0; a < p.acc_stages; ++a)
       for (int s = 0; s < NSUB; ++s) {
@@ -192,7 +195,13 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
           }
         }
         if (lane == 0) {
-          const uint32_t bytes = (uint32_t)__popc(valid_mask) * p.n_kblocks * p.box_rows * p.kbw;
+          // per-stage info read by the epilogue: which chunks hold real pages, and (FP8) the
+          // per-token key scales of the tile, copied next to the K tile
+          uint8_t* info = smem + p.off_kinfo + stage * kStageInfoBytes;
+          *reinterpret_cast<uint32_t*>(info) = valid_mask;
+          const uint32_t scale_bytes = p.k_scale ? (uint32_t)p.box_rows * 4u : 0u;
+          const uint32_t bytes =
+              (uint32_t)__popc(valid_mask) * (p.n_kblocks * p.box_rows * p.kbw + scale_bytes);
           mbar_arrive_expect_tx(&sb->k_full[stage], bytes);
           for (int c = 0; c < chunks; ++c) {
             if (!(valid_mask >> c & 1u)) continue;
@@ -201,6 +210,9 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
             for (int kb = 0; kb < p.n_kblocks; ++kb)
               tma_load_2d(kst + kb * p.k_kblock_bytes + c * p.box_rows * p.kbw, &kmap,
                           &sb->k_full[stage], kb * p.kbw / (p.fp8 ? 1 : 2), y);
+            if (p.k_scale)
+              bulk_load(info + 16 + c * p.box_rows * 4, p.k_scale + (long long)y, scale_bytes,
+                        &sb->k_full[stage]);
           }
         }
         __syncwarp();
@@ -327,22 +339,24 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
         mbar_arrive(&sb->q_full);
         // every epilogue thread has staged its share (w_s / info are visible after this)
         if (!mbar_wait(&sb->q_full, (uint32_t)seg & 1u, abort, p.status)) { ok = false; break; }
-        const int32_t* pt_row = p.page_table + (long long)gi.b * p.max_pages;
         const long long out_row0 = (long long)gi.b * p.J;
         for (int t = t0; t < t1; ++t, ++acc_it) {
           const int as = acc_it % p.acc_stages;
           const uint32_t aph = (uint32_t)(acc_it / p.acc_stages) & 1u;
+          const int kstage = acc_it % p.k_stages;
           const int s = t * kIndexTileRows + row;
-          // per-position scale and page check (independent of the accumulator: fetch first);
+          if (!mbar_wait(&sb->acc_full[as][sub], aph, abort, p.status)) { ok = false; break; }
+          // the K stage of this tile is still held (k_empty also waits for us): its loads have
+          // landed, and waiting on k_full makes the scales and the chunk mask visible here
+          if (!mbar_wait(&sb->k_full[kstage], (uint32_t)(acc_it / p.k_stages) & 1u, abort, p.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint8_t* info = smem + p.off_kinfo + kstage * kStageInfoBytes;
           // a position whose page id is outside the pool is ranked last (-inf)
           float ks = 1.0f;
-          if (s <= gi.max_pos) {
-            const int page = pt_row[s / p.P];
-            if (page < 0 || page >= p.num_pages) ks = __int_as_float(0xff800000);
-            else if (p.k_scale) ks = p.k_scale[(long long)page * p.P + (s % p.P)];
-          }
-          if (!mbar_wait(&sb->acc_full[as][sub], aph, abort, p.status)) { ok = false; break; }
-          tc_fence_after();
+          if (!((*reinterpret_cast<const uint32_t*>(info) >> (row / p.box_rows)) & 1u))
+            ks = __int_as_float(0xff800000);
+          else if (p.k_scale)
+            ks = reinterpret_cast<const float*>(info + 16)[row];
           const uint32_t col0 = (uint32_t)((as * NSUB + sub) * p.n_cols);
           for (int ql = 0; ql < p.nq_sub; ++ql) {
             const int qloc = sub * p.nq_sub + ql;
@@ -373,6 +387,8 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
           }
           tc_fence_before();
           mbar_arrive(&sb->acc_empty[as][sub]);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sb->k_empty[kstage]);
         }
         ++seg;
       }

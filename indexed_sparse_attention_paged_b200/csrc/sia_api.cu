@@ -113,8 +113,8 @@ sia_status check_index(const sia_index_args* a) {
   if (!pow2(a->page_size) || a->page_size < 8 || a->page_size > 4096)
     return fail(SIA_ERR_UNSUPPORTED, "page_size must be a power of two in [8, 4096] (got %d)", a->page_size);
   if (!aligned(a->q, 16) || !aligned(a->k_cache, 16) || !aligned(a->w, 4) || !aligned(a->topk_out, 4) ||
-      (a->scores_out && !aligned(a->scores_out, 16)) || (a->k_scale && !aligned(a->k_scale, 4)))
-    return fail(SIA_ERR_INVALID_ARGUMENT, "q and k_cache must be 16-byte aligned, other arrays 4-byte aligned");
+      (a->scores_out && !aligned(a->scores_out, 16)) || (a->k_scale && !aligned(a->k_scale, 16)))
+    return fail(SIA_ERR_INVALID_ARGUMENT, "q, k_cache, k_scale and scores_out must be 16-byte aligned, other arrays 4-byte aligned");
   const long long lpad = (long long)a->max_pages_per_seq * a->page_size;
   if (lpad > (1ll << 30)) return fail(SIA_ERR_UNSUPPORTED, "max_pages_per_seq * page_size too large");
   if ((long long)a->num_pages * a->page_size > (1ll << 31) - 1)
@@ -163,9 +163,10 @@ sia_status plan_index(const sia_index_args* a, IndexPlan* pl, bool make_maps) {
   const uint32_t w_bytes = (uint32_t)round_up((size_t)2 * k.qg * k.HP * 4, 16);  // double-buffered
   const uint32_t info_bytes = 256;
   const uint32_t bar_bytes = 256;
+  const uint32_t kinfo_bytes = 16 + 4 * kIndexTileRows;  // per stage: chunk mask + key scales
   const uint32_t fixed = q_bytes + w_bytes + info_bytes + bar_bytes;
   const int limit = max_smem_optin();
-  int stages = (int)((limit - (int)fixed) / (int)k.k_stage_bytes);
+  int stages = (int)((limit - (int)fixed) / (int)(k.k_stage_bytes + kinfo_bytes));
   stages = std::min(stages, 8);
   if (stages < 2) return fail(SIA_ERR_UNSUPPORTED, "indexer tile does not fit in shared memory");
   k.k_stages = stages;
@@ -173,7 +174,8 @@ sia_status plan_index(const sia_index_args* a, IndexPlan* pl, bool make_maps) {
   k.off_q = k.k_stage_bytes * stages;
   k.off_w = k.off_q + q_bytes;
   k.off_info = k.off_w + w_bytes;
-  k.off_bar = k.off_info + info_bytes;
+  k.off_kinfo = k.off_info + info_bytes;
+  k.off_bar = k.off_kinfo + kinfo_bytes * stages;
   k.smem_bytes = k.off_bar + bar_bytes;
   k.q = static_cast<const uint8_t*>(a->q);
   k.q_scale = a->q_scale;
@@ -196,7 +198,10 @@ sia_status plan_index(const sia_index_args* a, IndexPlan* pl, bool make_maps) {
   while ((k.Lpad + cs - 1) / cs > kTopkSliceMax) cs <<= 1;
   if (cs > 16) return fail(SIA_ERR_UNSUPPORTED, "context too long for the Top-K kernel (max %d)", 16 * kTopkSliceMax);
   const long long rows = (long long)a->batch * a->n_q;
-  while (cs < 8 && rows * cs * 2 <= 2ll * pl->grid) cs <<= 1;
+  // rows of up to 16384 positions take one CTA each (no cluster); longer rows split across a
+  // cluster, widened while that still leaves SMs idle
+  if (cs > 1)
+    while (cs < 8 && rows * cs * 2 <= 2ll * pl->grid) cs <<= 1;
   t.cluster = cs;
   t.slice = (int)round_up((size_t)((k.Lpad + cs - 1) / cs), 32);
   if (rows * cs > 0x7fffffffll) return fail(SIA_ERR_UNSUPPORTED, "too many query rows");
@@ -248,6 +253,8 @@ sia_status check_attend(const sia_attend_args* a) {
   if (!((a->d_latent == 512 && a->d_rope == 64) || (a->d_latent == 64 && a->d_rope == 16)))
     return fail(SIA_ERR_UNSUPPORTED, "(d_latent, d_rope) must be (512, 64) or (64, 16) (got %d, %d)", a->d_latent, a->d_rope);
   if (a->n_heads < 1 || a->n_heads > 128) return fail(SIA_ERR_UNSUPPORTED, "n_heads must be 1..128 (got %d)", a->n_heads);
+  if (a->top_k > 8 * kAttnMaxSplitRows)
+    return fail(SIA_ERR_UNSUPPORTED, "top_k must be <= %d (got %d)", 8 * kAttnMaxSplitRows, a->top_k);
   if (!std::isfinite(a->softmax_scale)) return fail(SIA_ERR_INVALID_ARGUMENT, "softmax_scale must be finite");
   if (!aligned(a->q, 16) || !aligned(a->kv_cache, 16) || !aligned(a->out, 16) || !aligned(a->topk, 4) ||
       (a->lse && !aligned(a->lse, 4)))
@@ -278,9 +285,10 @@ sia_status plan_attend(const sia_attend_args* a, AttendPlan* pl, bool make_maps)
   const int pairs = std::max(1, sm_count() / 2);
   // pick the number of Top-K splits that minimises the rows one cluster has to stream
   const int max_splits = std::max(1, std::min(8, (a->top_k + kAttnTileRows - 1) / kAttnTileRows));
+  const int min_splits = (a->top_k + kAttnMaxSplitRows - 1) / kAttnMaxSplitRows;
   long long best = -1;
   int best_s = 1, best_rows = 0;
-  for (int s = 1; s <= max_splits; ++s) {
+  for (int s = min_splits; s <= max_splits; ++s) {
     const int rows = (int)round_up((size_t)((a->top_k + s - 1) / s), kAttnTileRows);
     const int s_eff = (a->top_k + rows - 1) / rows;
     const long long units = bj * s_eff;
@@ -291,6 +299,7 @@ sia_status plan_attend(const sia_attend_args* a, AttendPlan* pl, bool make_maps)
   k.rows_per_split = best_rows;
   if (bj * best_s > 0x7fffffffll) return fail(SIA_ERR_UNSUPPORTED, "too many attention work units");
   k.units = (int)(bj * best_s);
+  k.kv = a->kv_cache;
   k.page_table = a->page_table;
   k.seq_lens = a->seq_lens;
   k.topk = a->topk;

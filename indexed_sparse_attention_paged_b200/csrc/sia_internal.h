@@ -13,8 +13,10 @@ namespace sia {
 
 // Rows (positions) per indexer tile: the M of every tcgen05 MMA of the indexer.
 constexpr int kIndexTileRows = 128;
-// Latent rows per attention tile.
+// Latent rows per attention tile, and the most Top-K entries one attention unit (a split of a
+// query's list) may hold.
 constexpr int kAttnTileRows = 64;
+constexpr int kAttnMaxSplitRows = 2048;
 // Largest Top-K slice one CTA keeps in shared memory (keys, 4 bytes each).
 constexpr int kTopkSliceMax = 16384;
 constexpr int kTopkThreads = 512;
@@ -41,7 +43,7 @@ struct IndexKernelParams {
   // shared-memory layout, byte offsets from the 1024-aligned base
   uint32_t off_k, k_stage_bytes, k_kblock_bytes;
   uint32_t off_q, q_sub_bytes, q_kblock_bytes;
-  uint32_t off_w, off_info, off_bar, smem_bytes;
+  uint32_t off_w, off_info, off_kinfo, off_bar, smem_bytes;
   const uint8_t* q;
   const float* q_scale;
   const float* w;
@@ -73,6 +75,7 @@ struct AttnKernelParams {
   int splits;                 // Top-K splits per query (>1 -> partials + combine)
   int rows_per_split;         // multiple of kAttnTileRows
   int units;                  // B * J * splits
+  const void* kv;             // bf16 [num_pages * P, DL + DR]
   const int32_t* page_table;
   const int32_t* seq_lens;
   const int32_t* topk;

@@ -24,6 +24,7 @@
 // 2^8.  Splits of the Top-K list (to fill the GPU at small batch) write fp32 partials that
 // combine_kernel merges by log-sum-exp.
 #include <cuda.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include "sia_internal.h"
@@ -32,35 +33,55 @@
 namespace sia {
 namespace {
 
-constexpr int kAttnThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 softmax / epilogue
-constexpr int kStages = 2;         // latent-row tiles in flight per CTA
+constexpr int kProducerWarps = 4;   // cp.async gather (+ TMA for q)
+constexpr int kFirstProducerWarp = 4;
+constexpr int kMmaWarp = 8;
+constexpr int kAttnThreads = 288;   // warps 0-3 softmax/epilogue, 4-7 gather, 8 MMA
+// Registers per thread after the split (launch gives 168 x 288): the softmax warpgroup holds a
+// tile of fp32 logits plus the next tile's fp16 partials, the gather warpgroup needs little.
+constexpr int kSoftmaxRegs = 232;
+constexpr int kGatherRegs = 96;
+constexpr int kStages = 3;          // latent-row tiles in flight per CTA
 constexpr int kRows = kAttnTileRows;
 
 template <int DL, int DR>
 struct AttnLayout;
 
+// Per-CTA share of each latent row: CTA r gathers latent dims [DL/2 r, DL/2 (r+1)) (used by both
+// Q.C^T and P.C) and a share of the rope dims (used by Q.C^T only).
 template <>
 struct AttnLayout<512, 64> {
-  static constexpr int kLatBlocks = 4;    // 4 x 64 latent dims per CTA
+  static constexpr int kLatBlocks = 4;    // 4 x 64 latent dims per CTA, 128-byte swizzled rows
   static constexpr int kLatKbw = 128;
-  static constexpr int kRopeKbw = 64;     // 32 rope dims per CTA
+  static constexpr int kRopeKbw = 64;     // 32 rope dims per CTA, 64-byte swizzled rows
   static constexpr int kPvN = 256;
   static constexpr uint32_t kTmemCols = 512;
-  __device__ static int lat_x(int r, int i) { return 256 * r + 64 * i; }
   __device__ static bool has_rope(int) { return true; }
+  __device__ static int lat_x(int r, int i) { return 256 * r + 64 * i; }   // q columns (elements)
   __device__ static int rope_x(int r) { return 512 + 32 * r; }
+  __device__ static int chunks(int) { return 36; }                        // 16-byte pieces per row
+  __device__ static int chunk_src(int r, int k) { return k < 32 ? 512 * r + 16 * k : 1024 + 64 * r + 16 * (k - 32); }
+  __device__ static uint32_t chunk_dst(int row, int k) {
+    return k < 32 ? (uint32_t)(k >> 3) * (kAttnTileRows * 128) + swizzled_offset(row, (k & 7) * 16, 128)
+                  : 4u * (kAttnTileRows * 128) + swizzled_offset(row, (k - 32) * 16, 64);
+  }
 };
 
 template <>
 struct AttnLayout<64, 16> {
-  static constexpr int kLatBlocks = 1;    // 32 latent dims per CTA
+  static constexpr int kLatBlocks = 1;    // 32 latent dims per CTA, 64-byte swizzled rows
   static constexpr int kLatKbw = 64;
-  static constexpr int kRopeKbw = 32;     // all 16 rope dims on CTA 0
+  static constexpr int kRopeKbw = 32;     // all 16 rope dims on CTA 0, 32-byte swizzled rows
   static constexpr int kPvN = 32;
   static constexpr uint32_t kTmemCols = 256;
-  __device__ static int lat_x(int r, int) { return 32 * r; }
   __device__ static bool has_rope(int r) { return r == 0; }
+  __device__ static int lat_x(int r, int) { return 32 * r; }
   __device__ static int rope_x(int) { return 64; }
+  __device__ static int chunks(int r) { return r == 0 ? 6 : 4; }
+  __device__ static int chunk_src(int r, int k) { return k < 4 ? 64 * r + 16 * k : 128 + 16 * (k - 4); }
+  __device__ static uint32_t chunk_dst(int row, int k) {
+    return k < 4 ? swizzled_offset(row, k * 16, 64) : (uint32_t)(kAttnTileRows * 64) + swizzled_offset(row, (k - 4) * 16, 32);
+  }
 };
 
 struct AttnMaps {
@@ -76,19 +97,24 @@ struct AttnSmem {
   static constexpr uint32_t kCStageBytes = Lay::kLatBlocks * kCLatBytes + kCRopeBytes;
   static constexpr uint32_t kOffQ = 0;
   static constexpr uint32_t kOffC = kOffQ + Lay::kLatBlocks * kQLatBytes + kQRopeBytes;
-  static constexpr uint32_t kOffP = kOffC + kStages * kCStageBytes;
-  static constexpr uint32_t kOffSx = kOffP + 128 * 128;                 // P: 128 x 64 bf16
-  static constexpr uint32_t kOffBar = kOffSx + kRows * 128 * 4;         // Sx: 64 x 128 fp32
+  static constexpr uint32_t kOffSx = kOffC + kStages * kCStageBytes;   // peer logits, fp16
+  static constexpr uint32_t kOffRows = kOffSx + kRows * 128 * 2;
+  // per unit (double-buffered): physical cache row of each Top-K entry, validity bits, and
+  // each gather warp's lowest position of a -1 entry
+  static constexpr uint32_t kOffMask = kOffRows + 2 * kAttnMaxSplitRows * 4;
+  static constexpr uint32_t kOffFirstNeg = kOffMask + 2 * (kAttnMaxSplitRows / 8);
+  static constexpr uint32_t kOffBar = kOffFirstNeg + 2 * kProducerWarps * 4;
   static constexpr uint32_t kBytes = kOffBar + 256;
 };
 
 struct AttnBarriers {
   uint64_t c_full[kStages], c_empty[kStages];
   uint64_t s_full[2], s_empty[2];
-  uint64_t p_full, p_empty;
+  uint64_t p_full[2], p_empty[2];
   uint64_t q_full, q_empty;
   uint64_t o_full, o_empty;
   uint64_t sx_ready, sx_free;
+  uint64_t tab_full[2], tab_free[2];
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort;
@@ -100,29 +126,19 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-// Does tile t of unit (bj, split) exist?  A tile exists when its first Top-K entry is a
-// position (valid entries come first in a Top-K row, -1 padding after them).
-__device__ __forceinline__ bool tile_exists(const AttnKernelParams& p, long long row_base,
-                                            int row0, int row_end, int t) {
-  const int r = row0 + t * kRows;
-  return r < row_end && p.topk[row_base + r] >= 0;
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
 }
 
-// Physical cache row of Top-K entry idx of sequence b, or -1 when the entry is padding or
-// points outside the context / page pool.
-__device__ __forceinline__ int phys_row(const AttnKernelParams& p, int b, int idx, int L,
-                                        bool report_bad) {
-  if (idx < 0) return -1;
-  if (idx >= L) {
-    if (report_bad) report(p.status, SIA_DEV_BAD_POSITION);
-    return -1;
-  }
-  const int page = p.page_table[(long long)b * p.max_pages + idx / p.P];
-  if (page < 0 || page >= p.num_pages) {
-    if (report_bad) report(p.status, SIA_DEV_BAD_PAGE);
-    return -1;
-  }
-  return page * p.P + idx % p.P;
+__device__ __forceinline__ float2 unpack_f16x2(uint32_t v) {
+  __half2 h = *reinterpret_cast<__half2*>(&v);
+  return __half22float2(h);
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
 
 template <int DL, int DR>
@@ -132,12 +148,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   using Sm = AttnSmem<Lay>;
   extern __shared__ __align__(1024) uint8_t smem[];
   AttnBarriers* sb = reinterpret_cast<AttnBarriers*>(smem + Sm::kOffBar);
+  int32_t* rows_tab = reinterpret_cast<int32_t*>(smem + Sm::kOffRows);        // [2][max rows]
+  uint32_t* mask_tab = reinterpret_cast<uint32_t*>(smem + Sm::kOffMask);      // [2][max rows/32]
+  int32_t* fneg_tab = reinterpret_cast<int32_t*>(smem + Sm::kOffFirstNeg);    // [2][gather warps]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
   const uint32_t peer = rank ^ 1u;
   const int cluster_id = blockIdx.x >> 1;
   const int n_clusters = gridDim.x >> 1;
   const bool rope = Lay::has_rope((int)rank);
+  const int DC = p.DL + p.DR;
 
   if ((smem_u32(smem) & 1023u) != 0) {
     if (threadIdx.x == 0) report(p.status, SIA_DEV_TIMEOUT);
@@ -145,15 +165,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&sb->c_full[s], 1);
+      mbar_init(&sb->c_full[s], kProducerWarps * 32);  // one cp.async completion per gather thread
       mbar_init(&sb->c_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sb->s_full[s], 1);
       mbar_init(&sb->s_empty[s], 128);
+      mbar_init(&sb->p_full[s], 128);
+      mbar_init(&sb->p_empty[s], 1);
+      mbar_init(&sb->tab_full[s], kProducerWarps * 32);
+      mbar_init(&sb->tab_free[s], 128);
     }
-    mbar_init(&sb->p_full, 128);
-    mbar_init(&sb->p_empty, 1);
     mbar_init(&sb->q_full, 1);
     mbar_init(&sb->q_empty, 1);
     mbar_init(&sb->o_full, 1);
@@ -165,10 +187,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     fence_mbarrier_init();
     tma_prefetch_desc(&maps.q_lat);
     tma_prefetch_desc(&maps.q_rope);
-    tma_prefetch_desc(&maps.kv_lat);
-    tma_prefetch_desc(&maps.kv_rope);
   }
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tmem_alloc(&sb->tmem_base, Lay::kTmemCols);
     tmem_relinquish();
   }
@@ -177,12 +197,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = sb->tmem_base;
   volatile int* abort = &sb->abort;
-  const uint32_t o_col = 0, s_col = Lay::kPvN;
+  const uint32_t o_col = 0, s_col = Lay::kPvN, p_col = Lay::kPvN + 2 * kRows;
 
   pdl_wait_primary();  // the Top-K lists come from the previous kernel on the stream
 
-  if (warp == 0) {
-    // ---------------------------------------------------------------- TMA producer
+  if (warp >= kFirstProducerWarp && warp < kFirstProducerWarp + kProducerWarps) {
+    // ---------------------------------------------------------------- gather (4 warps)
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kGatherRegs));
+    const int ptid = threadIdx.x - kFirstProducerWarp * 32;   // 0..127
+    const int pwarp = warp - kFirstProducerWarp;
+    const uint8_t* kv = static_cast<const uint8_t*>(p.kv);
+    const int nch = Lay::chunks((int)rank);
     int it = 0, u_it = 0;
     bool ok = true;
     for (int u = cluster_id; u < p.units && ok; u += n_clusters, ++u_it) {
@@ -191,84 +216,104 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int L = p.seq_lens[b];
       const long long row_base = (long long)bj * p.K;
       const int row0 = split * p.rows_per_split;
-      const int row_end = min(p.K, row0 + p.rows_per_split);
-      // query rows of all heads
-      int go = 1;
-      if (lane == 0) go = mbar_wait(&sb->q_empty, ((uint32_t)u_it & 1u) ^ 1u, abort, p.status);
-      if (!__shfl_sync(0xffffffffu, go, 0)) { ok = false; break; }
-      if (lane == 0) {
-        const uint32_t qbytes = Lay::kLatBlocks * Sm::kQLatBytes + (rope ? Sm::kQRopeBytes : 0);
-        mbar_arrive_expect_tx(&sb->q_full, qbytes);
-        const int y = bj * p.H;
-        for (int i = 0; i < Lay::kLatBlocks; ++i)
-          tma_load_2d(smem + Sm::kOffQ + i * Sm::kQLatBytes, &maps.q_lat, &sb->q_full,
-                      Lay::lat_x((int)rank, i), y);
-        if (rope)
-          tma_load_2d(smem + Sm::kOffQ + Lay::kLatBlocks * Sm::kQLatBytes, &maps.q_rope,
-                      &sb->q_full, Lay::rope_x((int)rank), y);
-      }
-      for (int t = 0; tile_exists(p, row_base, row0, row_end, t); ++t, ++it) {
-        const int stage = it % kStages;
-        if (lane == 0) go = mbar_wait(&sb->c_empty[stage], ((uint32_t)(it / kStages) & 1u) ^ 1u, abort, p.status);
-        if (!__shfl_sync(0xffffffffu, go, 0)) { ok = false; break; }
-        // lanes 0..15 each gather one group of 4 rows
-        int y[4] = {0, 0, 0, 0};
-        if (lane < 16) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int r = row0 + t * kRows + lane * 4 + i;
-            const int idx = r < row_end ? p.topk[row_base + r] : -1;
-            const int pr = phys_row(p, b, idx, L, rank == 0);
-            y[i] = pr < 0 ? 0 : pr;   // absent rows read row 0 (finite data) and are masked
-          }
-        }
-        if (lane == 0)
-          mbar_arrive_expect_tx(&sb->c_full[stage], Lay::kLatBlocks * Sm::kCLatBytes + (rope ? Sm::kCRopeBytes : 0));
-        __syncwarp();
-        if (lane < 16) {
-          uint8_t* cst = smem + Sm::kOffC + stage * Sm::kCStageBytes;
-#pragma unroll
+      const int nrows = min(p.K, row0 + p.rows_per_split) - row0;
+      const int nrows_pad = (nrows + kRows - 1) / kRows * kRows;
+      const int buf = u_it & 1;
+      // query rows of all heads (TMA; independent of the Top-K list)
+      if (ptid == 0) {
+        if (mbar_wait(&sb->q_empty, ((uint32_t)u_it & 1u) ^ 1u, abort, p.status)) {
+          const uint32_t qbytes = Lay::kLatBlocks * Sm::kQLatBytes + (rope ? Sm::kQRopeBytes : 0);
+          mbar_arrive_expect_tx(&sb->q_full, qbytes);
+          const int y = bj * p.H;
           for (int i = 0; i < Lay::kLatBlocks; ++i)
-            tma_gather4(cst + i * Sm::kCLatBytes + lane * 4 * Lay::kLatKbw, &maps.kv_lat,
-                        &sb->c_full[stage], Lay::lat_x((int)rank, i), y[0], y[1], y[2], y[3]);
+            tma_load_2d(smem + Sm::kOffQ + i * Sm::kQLatBytes, &maps.q_lat, &sb->q_full, Lay::lat_x((int)rank, i), y);
           if (rope)
-            tma_gather4(cst + Lay::kLatBlocks * Sm::kCLatBytes + lane * 4 * Lay::kRopeKbw,
-                        &maps.kv_rope, &sb->c_full[stage], Lay::rope_x((int)rank), y[0], y[1],
-                        y[2], y[3]);
+            tma_load_2d(smem + Sm::kOffQ + Lay::kLatBlocks * Sm::kQLatBytes, &maps.q_rope, &sb->q_full,
+                        Lay::rope_x((int)rank), y);
         }
-        __syncwarp();
+      }
+      // resolve this unit's Top-K entries to physical cache rows: 16 entries per thread, all
+      // loads of a thread in flight at once
+      if (!mbar_wait(&sb->tab_free[buf], ((uint32_t)(u_it >> 1) & 1u) ^ 1u, abort, p.status)) { ok = false; break; }
+      int32_t* rt = rows_tab + buf * kAttnMaxSplitRows;
+      uint32_t* mt = mask_tab + buf * (kAttnMaxSplitRows / 32);
+      const int32_t* tk = p.topk + row_base + row0;
+      const int32_t* pt_row = p.page_table + (long long)b * p.max_pages;
+      constexpr int kPer = kAttnMaxSplitRows / (kProducerWarps * 32);
+      int idx[kPer], pg[kPer];
+#pragma unroll
+      for (int k = 0; k < kPer; ++k) {
+        const int r = ptid + k * kProducerWarps * 32;
+        idx[k] = r < nrows ? tk[r] : -1;
+      }
+#pragma unroll
+      for (int k = 0; k < kPer; ++k) pg[k] = (idx[k] >= 0 && idx[k] < L) ? pt_row[idx[k] / p.P] : -1;
+      int fneg = nrows;
+#pragma unroll
+      for (int k = 0; k < kPer; ++k) {
+        const int r = ptid + k * kProducerWarps * 32;
+        if (k * kProducerWarps * 32 < nrows_pad) {     // warp-uniform (nrows_pad is a multiple of 64)
+          if (r < nrows && idx[k] < 0) fneg = min(fneg, r);
+          const bool pos_ok = idx[k] >= 0 && idx[k] < L;
+          const bool page_ok = pg[k] >= 0 && pg[k] < p.num_pages;
+          if (rank == 0 && idx[k] >= 0) {
+            if (idx[k] >= L) report(p.status, SIA_DEV_BAD_POSITION);
+            else if (!page_ok) report(p.status, SIA_DEV_BAD_PAGE);
+          }
+          const bool v = pos_ok && page_ok;
+          rt[r] = v ? pg[k] * p.P + idx[k] % p.P : 0;   // absent rows read row 0 (finite data)
+          const unsigned bits = __ballot_sync(0xffffffffu, v);
+          if (lane == 0) mt[(r - lane) / 32] = bits;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) fneg = min(fneg, __shfl_xor_sync(0xffffffffu, fneg, o));
+      if (lane == 0) fneg_tab[buf * kProducerWarps + pwarp] = fneg;
+      mbar_arrive(&sb->tab_full[buf]);
+      if (!mbar_wait(&sb->tab_full[buf], (uint32_t)(u_it >> 1) & 1u, abort, p.status)) { ok = false; break; }
+      int first_neg = nrows;
+#pragma unroll
+      for (int w = 0; w < kProducerWarps; ++w) first_neg = min(first_neg, fneg_tab[buf * kProducerWarps + w]);
+      const int ntiles = (first_neg + kRows - 1) / kRows;
+      for (int t = 0; t < ntiles; ++t, ++it) {
+        const int stage = it % kStages;
+        if (!mbar_wait(&sb->c_empty[stage], ((uint32_t)(it / kStages) & 1u) ^ 1u, abort, p.status)) { ok = false; break; }
+        const uint32_t cst = smem_u32(smem + Sm::kOffC + stage * Sm::kCStageBytes);
+        const int32_t* rows = rt + t * kRows;
+        for (int i = ptid; i < kRows * nch; i += kProducerWarps * 32) {
+          const int row = i / nch, k = i - row * nch;
+          cp_async16(cst + Lay::chunk_dst(row, k), kv + (size_t)(uint32_t)rows[row] * (DC * 2) + Lay::chunk_src((int)rank, k));
+        }
+        asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(&sb->c_full[stage])) : "memory");
       }
     }
-    if (lane == 0) {  // let in-flight gathers land before the CTA may leave
-      const int first = it > kStages ? it - kStages : 0;
-      for (int i = first; i < it; ++i)
-        mbar_wait(&sb->c_full[i % kStages], (uint32_t)(i / kStages) & 1u, abort, p.status);
-    }
-  } else if (warp == 1) {
+    asm volatile("cp.async.wait_all;" ::: "memory");  // our copies have landed before we may leave
+    if (ptid == 0 && u_it > 0) mbar_wait(&sb->q_full, (uint32_t)(u_it - 1) & 1u, abort, p.status);
+  } else if (warp == kMmaWarp) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       const uint32_t idesc_qk = umma_idesc(1, 1, false, false, kRows, 128);
       const uint32_t idesc_pv = umma_idesc(1, 1, false, true, Lay::kPvN, 128);
       const uint32_t q_base = smem_u32(smem + Sm::kOffQ);
-      const uint32_t p_base = smem_u32(smem + Sm::kOffP);
       int it = 0, s_it = 0, pv_it = 0, u_it = 0;
       bool ok = true;
       for (int u = cluster_id; u < p.units && ok; u += n_clusters, ++u_it) {
-        const int bj = u / p.splits, split = u - bj * p.splits;
-        const long long row_base = (long long)bj * p.K;
-        const int row0 = split * p.rows_per_split;
-        const int row_end = min(p.K, row0 + p.rows_per_split);
+        const int buf = u_it & 1;
+        if (!mbar_wait(&sb->tab_full[buf], (uint32_t)(u_it >> 1) & 1u, abort, p.status)) { ok = false; break; }
+        int first_neg = 1 << 30;
+        for (int w = 0; w < kProducerWarps; ++w) first_neg = min(first_neg, fneg_tab[buf * kProducerWarps + w]);
+        const int ntiles = (first_neg + kRows - 1) / kRows;
         if (!mbar_wait(&sb->q_full, (uint32_t)u_it & 1u, abort, p.status)) { ok = false; break; }
         tc_fence_after();
-        bool o_claimed = false, q_released = false;
+        bool o_claimed = false;
         int prev_stage = -1;
-        for (int t = 0;; ++t) {
-          const bool exists = tile_exists(p, row_base, row0, row_end, t);
-          if (exists) {
+        for (int t = 0; t <= ntiles; ++t) {
+          if (t < ntiles) {
             const int stage = it % kStages;
             const int sbuf = s_it & 1;
             if (!mbar_wait(&sb->c_full[stage], (uint32_t)(it / kStages) & 1u, abort, p.status)) { ok = false; break; }
             if (!mbar_wait(&sb->s_empty[sbuf], ((uint32_t)(s_it >> 1) & 1u) ^ 1u, abort, p.status)) { ok = false; break; }
+            fence_proxy_async_smem();   // the gathered rows were written by cp.async
             tc_fence_after();
             const uint32_t c_base = smem_u32(smem + Sm::kOffC + stage * Sm::kCStageBytes);
             const uint32_t d = tmem_base + s_col + (uint32_t)(sbuf * kRows);
@@ -295,14 +340,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               }
             }
             umma_commit(&sb->s_full[sbuf]);
-            if (!tile_exists(p, row_base, row0, row_end, t + 1)) {
-              umma_commit(&sb->q_empty);  // Q may be reloaded once these MMAs are done
-              q_released = true;
-            }
+            if (t + 1 == ntiles) umma_commit(&sb->q_empty);  // Q reusable once these are done
           }
           if (t > 0) {
-            // P . C for the previous tile
-            if (!mbar_wait(&sb->p_full, (uint32_t)pv_it & 1u, abort, p.status)) { ok = false; break; }
+            // O += P . C for the previous tile, with P (bf16) read straight from TMEM
+            const int pb = pv_it & 1;
+            if (!mbar_wait(&sb->p_full[pb], (uint32_t)(pv_it >> 1) & 1u, abort, p.status)) { ok = false; break; }
             if (!o_claimed) {
               if (!mbar_wait(&sb->o_empty, ((uint32_t)u_it & 1u) ^ 1u, abort, p.status)) { ok = false; break; }
               o_claimed = true;
@@ -311,22 +354,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const uint32_t c_base = smem_u32(smem + Sm::kOffC + prev_stage * Sm::kCStageBytes);
 #pragma unroll
             for (int ks = 0; ks < kRows / 16; ++ks) {
-              const uint64_t ad = umma_smem_desc(p_base + ks * 32, 16, 1024, umma_layout_type(128));
               const uint64_t bd = umma_smem_desc(c_base + ks * 16 * Lay::kLatKbw, Sm::kCLatBytes,
                                                  8 * Lay::kLatKbw, umma_layout_type(Lay::kLatKbw));
-              umma_f16(tmem_base + o_col, ad, bd, idesc_pv, (t > 1) || ks > 0);
+              umma_f16_ts(tmem_base + o_col, tmem_base + p_col + (uint32_t)(pb * (kRows / 2) + ks * 8), bd,
+                          idesc_pv, (t > 1) || ks > 0);
             }
             umma_commit(&sb->c_empty[prev_stage]);
-            umma_commit(&sb->p_empty);
+            umma_commit(&sb->p_empty[pb]);
             ++pv_it;
           }
-          if (!exists) break;
-          prev_stage = it % kStages;
-          ++it;
-          ++s_it;
+          if (t < ntiles) {
+            prev_stage = it % kStages;
+            ++it;
+            ++s_it;
+          }
         }
         if (!ok) break;
-        if (!q_released) umma_commit(&sb->q_empty);
+        if (ntiles == 0) umma_commit(&sb->q_empty);
         if (!o_claimed) {
           if (!mbar_wait(&sb->o_empty, ((uint32_t)u_it & 1u) ^ 1u, abort, p.status)) { ok = false; break; }
         }
@@ -338,94 +382,108 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- softmax + epilogue
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
     const int quad = warp & 3;
     const int h = quad * 32 + lane;   // head = TMEM lane
     const uint32_t lane_addr = tmem_base + ((uint32_t)(quad * 32) << 16);
-    float* sx = reinterpret_cast<float*>(smem + Sm::kOffSx);
-    const uint32_t sx_peer = mapa_cluster(sx, peer);
-    const uint32_t p_row = smem_u32(smem + Sm::kOffP);
+    const uint32_t sx = smem_u32(smem + Sm::kOffSx);
+    const uint32_t sx_peer = mapa_shared(sx, peer);
     int s_it = 0, pv_it = 0, u_it = 0;
     bool ok = true;
+
+    // Own partial logits of the next tile: read them from TMEM, free the TMEM buffer, round to
+    // fp16 (both CTAs then add the same two fp16 values, so their softmax inputs agree bit for
+    // bit) and push them to the peer's buffer Sx[row/8][head][row%8].
+    auto load_and_send = [&](uint32_t (&own)[kRows / 2]) -> bool {
+      const int sbuf = s_it & 1;
+      if (!mbar_wait(&sb->s_full[sbuf], (uint32_t)(s_it >> 1) & 1u, abort, p.status)) return false;
+      tc_fence_after();
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {   // 32 columns at a time keeps register use low
+        uint32_t r[2][16];
+        tmem_ld16(lane_addr + s_col + sbuf * kRows + half * 32, r[0]);
+        tmem_ld16(lane_addr + s_col + sbuf * kRows + half * 32 + 16, r[1]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            own[half * 16 + c * 8 + i] = pack_f16x2(__uint_as_float(r[c][2 * i]) * p.scale_log2,
+                                                    __uint_as_float(r[c][2 * i + 1]) * p.scale_log2);
+      }
+      tc_fence_before();
+      mbar_arrive(&sb->s_empty[sbuf]);
+      if (!mbar_wait<true>(&sb->sx_free, ((uint32_t)s_it & 1u) ^ 1u, abort, p.status)) return false;
+#pragma unroll
+      for (int g = 0; g < kRows / 8; ++g)
+        asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sx_peer + (uint32_t)((g * 128 + h) * 16)),
+                     "r"(own[4 * g]), "r"(own[4 * g + 1]), "r"(own[4 * g + 2]), "r"(own[4 * g + 3])
+                     : "memory");
+      mbar_arrive_cluster(&sb->sx_ready, peer);
+      return true;
+    };
+
     for (int u = cluster_id; u < p.units && ok; u += n_clusters, ++u_it) {
       const int bj = u / p.splits, split = u - bj * p.splits;
-      const int b = bj / p.J;
-      const int L = p.seq_lens[b];
-      const long long row_base = (long long)bj * p.K;
-      const int row0 = split * p.rows_per_split;
-      const int row_end = min(p.K, row0 + p.rows_per_split);
+      const int buf = u_it & 1;
+      if (!mbar_wait(&sb->tab_full[buf], (uint32_t)(u_it >> 1) & 1u, abort, p.status)) { ok = false; break; }
+      int first_neg = 1 << 30;
+      for (int w = 0; w < kProducerWarps; ++w) first_neg = min(first_neg, fneg_tab[buf * kProducerWarps + w]);
+      const int ntiles = (first_neg + kRows - 1) / kRows;
+      const uint32_t* mt = mask_tab + buf * (kAttnMaxSplitRows / 32);
       float m = -INFINITY, l = 0.0f;
-      int t = 0;
-      for (; tile_exists(p, row_base, row0, row_end, t); ++t, ++s_it, ++pv_it) {
-        // which of the tile's 64 rows are real positions
-        const int r_lo = row0 + t * kRows + lane, r_hi = r_lo + 32;
-        const int i_lo = r_lo < row_end ? p.topk[row_base + r_lo] : -1;
-        const int i_hi = r_hi < row_end ? p.topk[row_base + r_hi] : -1;
-        const uint32_t v_lo = __ballot_sync(0xffffffffu, phys_row(p, b, i_lo, L, false) >= 0);
-        const uint32_t v_hi = __ballot_sync(0xffffffffu, phys_row(p, b, i_hi, L, false) >= 0);
-        const uint64_t valid = ((uint64_t)v_hi << 32) | v_lo;
-
-        const int sbuf = s_it & 1;
-        if (!mbar_wait(&sb->s_full[sbuf], (uint32_t)(s_it >> 1) & 1u, abort, p.status)) { ok = false; break; }
-        tc_fence_after();
-        float s[kRows];
-        {
-          uint32_t r[4][16];
-#pragma unroll
-          for (int c = 0; c < 4; ++c) tmem_ld16(lane_addr + s_col + sbuf * kRows + c * 16, r[c]);
-          tmem_wait_ld();
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-#pragma unroll
-            for (int i = 0; i < 16; ++i) s[c * 16 + i] = __uint_as_float(r[c][i]);
-        }
-        tc_fence_before();
-        mbar_arrive(&sb->s_empty[sbuf]);
-
-        // exchange partial scores with the peer CTA: Sx[row/4][head][row%4]
-        if (!mbar_wait<true>(&sb->sx_free, ((uint32_t)s_it & 1u) ^ 1u, abort, p.status)) { ok = false; break; }
-#pragma unroll
-        for (int g = 0; g < kRows / 4; ++g)
-          st_cluster_v4(sx_peer + (uint32_t)((g * 128 + h) * 16), s[4 * g], s[4 * g + 1], s[4 * g + 2], s[4 * g + 3]);
-        mbar_arrive_cluster(&sb->sx_ready, peer);
+      float s[kRows];
+      uint32_t own[kRows / 2];
+      if (ntiles > 0 && !load_and_send(own)) { ok = false; break; }
+      for (int t = 0; t < ntiles; ++t, ++pv_it) {
+        // the peer's partial of tile t completes the logits (already scaled to base 2)
         if (!mbar_wait<true>(&sb->sx_ready, (uint32_t)s_it & 1u, abort, p.status)) { ok = false; break; }
 #pragma unroll
-        for (int g = 0; g < kRows / 4; ++g) {
-          const float4 v = *reinterpret_cast<const float4*>(sx + (g * 128 + h) * 4);
-          s[4 * g] += v.x;
-          s[4 * g + 1] += v.y;
-          s[4 * g + 2] += v.z;
-          s[4 * g + 3] += v.w;
+        for (int g = 0; g < kRows / 8; ++g) {
+          const uint4 v = *reinterpret_cast<const uint4*>(smem + Sm::kOffSx + (g * 128 + h) * 16);
+          const uint32_t pv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 a = unpack_f16x2(own[4 * g + i]), c = unpack_f16x2(pv[i]);
+            s[8 * g + 2 * i] = a.x + c.x;
+            s[8 * g + 2 * i + 1] = a.y + c.y;
+          }
         }
         mbar_arrive_cluster(&sb->sx_free, peer);
+        ++s_it;
+        // start the exchange of tile t+1 before the softmax of tile t
+        if (t + 1 < ntiles && !load_and_send(own)) { ok = false; break; }
+        uint64_t valid = ((uint64_t)mt[2 * t + 1] << 32) | mt[2 * t];
+        const int live = first_neg - t * kRows;            // rows past the first -1 are padding
+        if (live < kRows) valid &= (1ull << live) - 1ull;
 
         // online softmax (base 2), lazy rescale
-        float mt = -INFINITY;
+        float mt_ = -INFINITY;
 #pragma unroll
         for (int i = 0; i < kRows; ++i) {
-          s[i] = (valid >> i & 1ull) ? s[i] * p.scale_log2 : -INFINITY;
-          mt = fmaxf(mt, s[i]);
+          s[i] = (valid >> i & 1ull) ? s[i] : -INFINITY;
+          mt_ = fmaxf(mt_, s[i]);
         }
         float alpha = 1.0f;
-        const bool need = mt > m + 8.0f;
+        const bool need = mt_ > m + 8.0f;
         if (need) {
-          alpha = fast_exp2(m - mt);   // 0 when m is -inf
-          m = mt;
+          alpha = fast_exp2(m - mt_);   // 0 when m is -inf
+          m = mt_;
         }
         float psum = 0.0f;
-        uint32_t pk[kRows / 2];
 #pragma unroll
-        for (int i = 0; i < kRows; i += 2) {
-          const float p0 = (valid >> i & 1ull) ? fast_exp2(s[i] - m) : 0.0f;
-          const float p1 = (valid >> (i + 1) & 1ull) ? fast_exp2(s[i + 1] - m) : 0.0f;
-          psum += p0 + p1;
-          pk[i / 2] = pack_bf16x2(p0, p1);
+        for (int i = 0; i < kRows; ++i) {
+          s[i] = (valid >> i & 1ull) ? fast_exp2(s[i] - m) : 0.0f;
+          psum += s[i];
         }
         l = l * alpha + psum;
 
-        // P . C of the previous tile must be done before O is rescaled or P overwritten
-        if (!mbar_wait(&sb->p_empty, ((uint32_t)pv_it & 1u) ^ 1u, abort, p.status)) { ok = false; break; }
-        tc_fence_after();
+        const int pb = pv_it & 1;
         if (__any_sync(0xffffffffu, need && t > 0)) {
+          // O holds tiles < t of this unit once P . C of tile t-1 is done: rescale it
+          const int prev = pv_it - 1;
+          if (!mbar_wait(&sb->p_empty[prev & 1], (uint32_t)(prev >> 1) & 1u, abort, p.status)) { ok = false; break; }
+          tc_fence_after();
 #pragma unroll 1
           for (int c = 0; c < Lay::kPvN; c += 16) {
             uint32_t r[16];
@@ -437,19 +495,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
           tmem_wait_st();
         }
+        // the P buffer of tile t-2 must have been consumed by its P . C
+        if (!mbar_wait(&sb->p_empty[pb], ((uint32_t)(pv_it >> 1) & 1u) ^ 1u, abort, p.status)) { ok = false; break; }
+        tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-          st_shared_v4(p_row + swizzled_offset((uint32_t)h, (uint32_t)(c * 16), 128), pk[4 * c],
-                       pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-        fence_proxy_async_smem();
+        for (int half = 0; half < 2; ++half) {
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(s[32 * half + 2 * i], s[32 * half + 2 * i + 1]);
+          tmem_st16(lane_addr + p_col + pb * (kRows / 2) + 16 * half, w);
+        }
+        tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&sb->p_full);
+        mbar_arrive(&sb->p_full[pb]);
       }
       if (!ok) break;
+      mbar_arrive(&sb->tab_free[buf]);
       // ---- unit epilogue: normalise O and write it out
       if (!mbar_wait(&sb->o_full, (uint32_t)u_it & 1u, abort, p.status)) { ok = false; break; }
       tc_fence_after();
-      const bool any = t > 0 && l > 0.0f;
+      const bool any = ntiles > 0 && l > 0.0f;
       const float inv = any ? 1.0f / l : 0.0f;
       const float lse = any ? (m + log2f(l)) * 0.69314718055994530942f : -INFINITY;
       const bool real_head = h < p.H;
@@ -458,14 +523,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll 1
         for (int c = 0; c < Lay::kPvN; c += 16) {
           uint32_t r[16];
-          if (t > 0) {
+          if (ntiles > 0) {
             tmem_ld16(lane_addr + o_col + c, r);
             tmem_wait_ld();
           }
           uint32_t w[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i)
-            w[i] = t > 0 ? pack_bf16x2(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv) : 0u;
+            w[i] = ntiles > 0 ? pack_bf16x2(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv) : 0u;
           if (real_head) {
             uint4* dst = reinterpret_cast<uint4*>(orow + c);
             dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
@@ -478,7 +543,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll 1
         for (int c = 0; c < Lay::kPvN; c += 16) {
           uint32_t r[16];
-          if (t > 0) {
+          if (ntiles > 0) {
             tmem_ld16(lane_addr + o_col + c, r);
             tmem_wait_ld();
           }
@@ -486,9 +551,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             float4* dst = reinterpret_cast<float4*>(orow + c);
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-              dst[i] = t > 0 ? make_float4(__uint_as_float(r[4 * i]) * inv, __uint_as_float(r[4 * i + 1]) * inv,
-                                           __uint_as_float(r[4 * i + 2]) * inv, __uint_as_float(r[4 * i + 3]) * inv)
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
+              dst[i] = ntiles > 0 ? make_float4(__uint_as_float(r[4 * i]) * inv, __uint_as_float(r[4 * i + 1]) * inv,
+                                                __uint_as_float(r[4 * i + 2]) * inv, __uint_as_float(r[4 * i + 3]) * inv)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
           }
         }
         if (real_head && rank == 0) p.part_lse[((long long)split * p.B * p.J + bj) * p.H + h] = lse;
@@ -501,28 +566,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_before();
   __syncthreads();
   cluster_sync();  // the peer no longer writes into our shared memory or arrives on our barriers
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem_base, Lay::kTmemCols);
   }
 }
 
-// Log-sum-exp merge of the per-split partial results of one query row.
-__global__ void __launch_bounds__(256) combine_kernel(const CombineKernelParams p) {
+// Log-sum-exp merge of the per-split partial results: one CTA per (query row, head), each
+// thread 4 output dims.
+__global__ void __launch_bounds__(128) combine_kernel(const CombineKernelParams p) {
   pdl_wait_primary();
-  const int bj = blockIdx.x;
-  const int per_head = p.DL / 4;
-  for (int i = threadIdx.x; i < p.H * per_head; i += blockDim.x) {
-    const int h = i / per_head, d4 = (i - h * per_head) * 4;
+  const long long bjh = blockIdx.x;            // = bj * H + h
+  const int d4 = threadIdx.x * 4;
+  if (d4 < p.DL) {
+    const long long stride_lse = (long long)p.BJ * p.H;
     float mx = -INFINITY;
-    for (int s = 0; s < p.splits; ++s)
-      mx = fmaxf(mx, p.part_lse[((long long)s * p.BJ + bj) * p.H + h]);
+    for (int s = 0; s < p.splits; ++s) mx = fmaxf(mx, p.part_lse[s * stride_lse + bjh]);
     float wsum = 0.0f, o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
     if (mx != -INFINITY) {
       for (int s = 0; s < p.splits; ++s) {
-        const float ls = p.part_lse[((long long)s * p.BJ + bj) * p.H + h];
+        const float ls = p.part_lse[s * stride_lse + bjh];
         const float wgt = ls == -INFINITY ? 0.0f : expf(ls - mx);
-        const float4 v = *reinterpret_cast<const float4*>(p.part_o + (((long long)s * p.BJ + bj) * p.H + h) * p.DL + d4);
+        const float4 v = *reinterpret_cast<const float4*>(p.part_o + (s * stride_lse + bjh) * p.DL + d4);
         o0 += wgt * v.x;
         o1 += wgt * v.y;
         o2 += wgt * v.z;
@@ -531,10 +596,9 @@ __global__ void __launch_bounds__(256) combine_kernel(const CombineKernelParams 
       }
     }
     const float inv = wsum > 0.0f ? 1.0f / wsum : 0.0f;
-    uint16_t* dst = p.out + ((long long)bj * p.H + h) * p.DL + d4;
-    const uint32_t a = pack_bf16x2(o0 * inv, o1 * inv), c = pack_bf16x2(o2 * inv, o3 * inv);
-    *reinterpret_cast<uint2*>(dst) = make_uint2(a, c);
-    if (d4 == 0 && p.lse) p.lse[(long long)bj * p.H + h] = wsum > 0.0f ? mx + logf(wsum) : -INFINITY;
+    uint16_t* dst = p.out + bjh * p.DL + d4;
+    *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(o0 * inv, o1 * inv), pack_bf16x2(o2 * inv, o3 * inv));
+    if (d4 == 0 && p.lse) p.lse[bjh] = wsum > 0.0f ? mx + logf(wsum) : -INFINITY;
   }
   pdl_launch_dependents();
 }
@@ -593,8 +657,8 @@ cudaError_t launch_sparse_attend(const AttnKernelParams& p, const CUtensorMap* m
 cudaError_t launch_combine(const CombineKernelParams& p, bool pdl, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
-  cfg.gridDim = dim3((unsigned)p.BJ, 1, 1);
-  cfg.blockDim = dim3(256, 1, 1);
+  cfg.gridDim = dim3((unsigned)((long long)p.BJ * p.H), 1, 1);
+  cfg.blockDim = dim3(128, 1, 1);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
   int na = 0;

@@ -122,17 +122,25 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkKernelP
     // make every CTA's histogram visible cluster-wide, then sum them
     cluster_sync();
     // each thread owns 4 consecutive bins; count of keys in bins above, found by a suffix scan
-    const int per = kBins / kTopkThreads;
-    uint32_t cnt[kBins / kTopkThreads];
-    int mine = 0;
+    constexpr int per = kBins / kTopkThreads;   // 4 consecutive bins: one 16-byte load per CTA
+    static_assert(per == 4, "one v4 load per cluster CTA");
+    uint32_t cnt[per] = {0u, 0u, 0u, 0u};
+    {
+      uint4 v[16];
+      const uint32_t local = smem_u32(&h[tid * per]);
 #pragma unroll
-    for (int q = 0; q < per; ++q) {
-      const int bin = tid * per + q;
-      uint32_t c = 0;
-      for (int r = 0; r < C; ++r) c += ld_cluster_u32(mapa_cluster(&h[bin], (uint32_t)r));
-      cnt[q] = c;
-      mine += (int)c;
+      for (int r = 0; r < 16; ++r)
+        if (r < C) v[r] = ld_cluster_v4(mapa_shared(local, (uint32_t)r));
+#pragma unroll
+      for (int r = 0; r < 16; ++r)
+        if (r < C) {
+          cnt[0] += v[r].x;
+          cnt[1] += v[r].y;
+          cnt[2] += v[r].z;
+          cnt[3] += v[r].w;
+        }
     }
+    const int mine = (int)(cnt[0] + cnt[1] + cnt[2] + cnt[3]);
     // suffix sum over threads in descending bin order: scan with reversed thread index
     int ex_a, ex_b, tot_a, tot_b;
     // thread t's position in descending order is (kTopkThreads-1-t); compute the exclusive
@@ -201,9 +209,171 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkKernelP
   cluster_sync();  // no CTA leaves while a peer may still read its shared memory
 }
 
+
+// ---------------------------------------------------------------------------------------------
+// Rows of at most kRowKeys positions: one CTA of 1024 threads per query row, each thread holding
+// 16 consecutive keys in registers (its share is contiguous, so thread order is position order).
+constexpr int kRowThreads = 1024;
+constexpr int kRowPer = 16;
+constexpr int kRowKeys = kRowThreads * kRowPer;
+
+struct RowShared {
+  uint32_t hist[kBins];
+  int warp_a[kRowThreads / 32];
+  int warp_b[kRowThreads / 32];
+  uint32_t sel_prefix;
+  int sel_krem;
+};
+
+// Exclusive prefix sums of (a, b) over the CTA's threads in thread order, and their totals.
+__device__ __forceinline__ void row_scan2(int a, int b, int& ea, int& eb, int& ta, int& tb, RowShared* sh) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int ia = a, ib = b;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int va = __shfl_up_sync(0xffffffffu, ia, o), vb = __shfl_up_sync(0xffffffffu, ib, o);
+    if (lane >= o) { ia += va; ib += vb; }
+  }
+  if (lane == 31) { sh->warp_a[warp] = ia; sh->warp_b[warp] = ib; }
+  __syncthreads();
+  if (warp == 0) {
+    int xa = sh->warp_a[lane], xb = sh->warp_b[lane];
+    int sa = xa, sb_ = xb;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int va = __shfl_up_sync(0xffffffffu, sa, o), vb = __shfl_up_sync(0xffffffffu, sb_, o);
+      if (lane >= o) { sa += va; sb_ += vb; }
+    }
+    sh->warp_a[lane] = sa - xa;   // exclusive warp offsets
+    sh->warp_b[lane] = sb_ - xb;
+    if (lane == 31) { sh->sel_prefix = (uint32_t)sa; sh->sel_krem = sb_; }   // totals (scratch)
+  }
+  __syncthreads();
+  ea = sh->warp_a[warp] + ia - a;
+  eb = sh->warp_b[warp] + ib - b;
+  ta = (int)sh->sel_prefix;
+  tb = sh->sel_krem;
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kRowThreads, 1) topk_row_kernel(const TopkKernelParams p) {
+  __shared__ RowShared shm;
+  RowShared* sh = &shm;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const long long row = blockIdx.x;
+  const int b = (int)(row / p.J), j = (int)(row - (long long)b * p.J);
+  int32_t* out = p.topk + row * p.K;
+
+  pdl_wait_primary();  // scores come from the previous kernel on the stream
+
+  bool bad = false;
+  const int pos = query_position(p.seq_lens, p.q_pos, p.J, b, j, p.Lpad, &bad);
+  if (bad && tid == 0) report(p.status, SIA_DEV_BAD_POSITION);
+  const int n = pos + 1;
+  if (n <= p.K) {
+    for (int i = tid; i < p.K; i += kRowThreads) out[i] = i < n ? i : -1;
+    pdl_launch_dependents();
+    return;
+  }
+  // this thread's keys: positions [tid*16, tid*16+16) of the visible range
+  const int base = tid * kRowPer;
+  uint32_t key[kRowPer];
+  const float* src = p.scores + row * p.Lpad + base;
+  if (base + kRowPer <= n) {
+#pragma unroll
+    for (int q = 0; q < kRowPer / 4; ++q) {
+      const float4 v = reinterpret_cast<const float4*>(src)[q];
+      key[4 * q] = order_key(v.x);
+      key[4 * q + 1] = order_key(v.y);
+      key[4 * q + 2] = order_key(v.z);
+      key[4 * q + 3] = order_key(v.w);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < kRowPer; ++i) key[i] = base + i < n ? order_key(src[i]) : 0u;
+  }
+  const int nmine = max(0, min(kRowPer, n - base));
+
+  uint32_t prefix = 0;
+  int krem = p.K;
+  const int shifts[3] = {21, 10, 0};
+  const int widths[3] = {11, 11, 10};
+#pragma unroll 1
+  for (int pass = 0; pass < 3; ++pass) {
+    for (int i = tid; i < kBins; i += kRowThreads) sh->hist[i] = 0;
+    __syncthreads();
+    const int sh_ = shifts[pass], hi_shift = sh_ + widths[pass];
+    const uint32_t dmask = (1u << widths[pass]) - 1u;
+#pragma unroll
+    for (int i = 0; i < kRowPer; ++i) {
+      uint32_t digit = 0xffffffffu;
+      if (i < nmine && (pass == 0 || (key[i] >> hi_shift) == prefix)) digit = (key[i] >> sh_) & dmask;
+      const unsigned same = __match_any_sync(0xffffffffu, digit);
+      if (digit != 0xffffffffu && lane == __ffs(same) - 1) atomicAdd(&sh->hist[digit], (uint32_t)__popc(same));
+    }
+    __syncthreads();
+    // thread t owns bins 2t, 2t+1; "above" = keys in higher bins, via a scan in reversed order
+    const int hi_bin = kBins - 2 - 2 * tid;        // reversed: thread 0 owns the two top bins
+    const int c1 = (int)sh->hist[hi_bin + 1], c0 = (int)sh->hist[hi_bin];
+    int ex, dummy, tot, tot2;
+    row_scan2(c0 + c1, 0, ex, dummy, tot, tot2, sh);
+    if (ex < krem && krem <= ex + c1) {
+      sh->sel_prefix = (prefix << widths[pass]) | (uint32_t)(hi_bin + 1);
+      sh->sel_krem = krem - ex;
+    } else if (ex + c1 < krem && krem <= ex + c1 + c0) {
+      sh->sel_prefix = (prefix << widths[pass]) | (uint32_t)hi_bin;
+      sh->sel_krem = krem - ex - c1;
+    }
+    __syncthreads();
+    prefix = sh->sel_prefix;
+    krem = sh->sel_krem;
+    __syncthreads();
+  }
+  const uint32_t T = prefix;
+
+  int gt = 0, eq = 0;
+#pragma unroll
+  for (int i = 0; i < kRowPer; ++i) {
+    gt += (i < nmine && key[i] > T);
+    eq += (i < nmine && key[i] == T);
+  }
+  int ex_gt, ex_eq, tot_gt, tot_eq;
+  row_scan2(gt, eq, ex_gt, ex_eq, tot_gt, tot_eq, sh);
+  int gt_before = ex_gt, eq_before = ex_eq;
+#pragma unroll
+  for (int i = 0; i < kRowPer; ++i) {
+    if (i >= nmine) break;
+    if (key[i] > T) {
+      out[gt_before + min(eq_before, krem)] = base + i;
+      ++gt_before;
+    } else if (key[i] == T) {
+      if (eq_before < krem) out[gt_before + eq_before] = base + i;
+      ++eq_before;
+    }
+  }
+  pdl_launch_dependents();
+}
+
 }  // namespace
 
 cudaError_t launch_topk(const TopkKernelParams& p, bool pdl, cudaStream_t stream) {
+  if (p.Lpad <= kRowKeys) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    cfg.gridDim = dim3((unsigned)((long long)p.B * p.J), 1, 1);
+    cfg.blockDim = dim3(kRowThreads, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    int na = 0;
+    if (pdl) {
+      attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[na].val.programmaticStreamSerializationAllowed = 1;
+      ++na;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = na;
+    return cudaLaunchKernelEx(&cfg, topk_row_kernel, p);
+  }
   const size_t smem = sizeof(TopkShared) + (size_t)p.slice * sizeof(uint32_t);
   cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
