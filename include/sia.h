@@ -139,6 +139,20 @@ sia_status sia_sparse_index_topk(const sia_index_args* a, void* workspace, size_
 sia_status sia_sparse_mla_attend(const sia_attend_args* a, void* workspace, size_t ws_bytes,
                                  int32_t* dev_status, void* stream);
 
+/* Stage 1 for callers that cannot allocate device memory while they run (a serving loop with a
+ * fixed preallocated arena, a C runtime without a device allocator, a loop that must not stall
+ * on cudaMalloc/cudaFree): same operation and arguments as sia_sparse_index_topk, but the
+ * per-position scores live in a 16 MiB array inside the library, so no workspace is passed and
+ * nothing is allocated.  The pages describing the method have no counterpart of this call.
+ *   - limit: batch * n_q * max_pages_per_seq * page_size * 4 bytes <= 16 MiB, else
+ *     SIA_ERR_WORKSPACE before any launch (ignored when scores_out is given);
+ *   - the array is shared by every call in the process: calls whose kernels may overlap on the
+ *     GPU (other streams, other host threads) race on it and must be serialised by the caller;
+ *   - the first call on each device looks up the array's device address (cudaGetSymbolAddress);
+ *     make that first call before any stream capture;
+ *   - every GPU that loads the library keeps the 16 MiB until the process exits. */
+sia_status sia_sparse_index_topk_noalloc(const sia_index_args* a, int32_t* dev_status, void* stream);
+
 /* Both stages back to back on one stream (programmatic dependent launch between kernels, no
  * host synchronisation; capturable in a CUDA graph).  The two argument sets must describe the
  * same sequences: equal batch, n_q, page_size, max_pages_per_seq, top_k, page_table and

@@ -80,6 +80,8 @@ def load_library(path: str = LIB_PATH):
     lib.sia_workspace_size.argtypes = [ctypes.POINTER(IndexArgs), ctypes.POINTER(AttendArgs)]
     lib.sia_sparse_index_topk.restype = ctypes.c_int
     lib.sia_sparse_index_topk.argtypes = [ctypes.POINTER(IndexArgs), P, ctypes.c_size_t, P, P]
+    lib.sia_sparse_index_topk_noalloc.restype = ctypes.c_int
+    lib.sia_sparse_index_topk_noalloc.argtypes = [ctypes.POINTER(IndexArgs), P, P]
     lib.sia_sparse_mla_attend.restype = ctypes.c_int
     lib.sia_sparse_mla_attend.argtypes = [ctypes.POINTER(AttendArgs), P, ctypes.c_size_t, P, P]
     lib.sia_fused_decode.restype = ctypes.c_int
@@ -223,6 +225,17 @@ def sparse_index_topk(q, w, k_cache, page_table, seq_lens, *, top_k, q_scale=Non
     ws = _workspace(lib.sia_index_workspace_size(ctypes.byref(a)), q.device, workspace)
     wp, wn = _ws_ptr(ws)
     _check(lib.sia_sparse_index_topk(ctypes.byref(a), wp, wn, _ptr(dev_status), _stream_ptr(stream)))
+    return topk_out
+
+
+def sparse_index_topk_noalloc(q, w, k_cache, page_table, seq_lens, *, top_k, topk_out, q_scale=None,
+                              k_scale=None, q_pos=None, dev_status=None, stream=None):
+    """Stage 1 through the entry point that allocates nothing (its score scratch is a fixed
+    16 MiB array inside the library, shared by every call).  `topk_out` must be given."""
+    lib = load_library()
+    a = index_args(q, w, k_cache, page_table, seq_lens, top_k=top_k, q_scale=q_scale,
+                   k_scale=k_scale, q_pos=q_pos, topk_out=topk_out)
+    _check(lib.sia_sparse_index_topk_noalloc(ctypes.byref(a), _ptr(dev_status), _stream_ptr(stream)))
     return topk_out
 
 
