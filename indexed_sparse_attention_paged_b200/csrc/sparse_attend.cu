@@ -25,6 +25,8 @@
 // combine_kernel merges by log-sum-exp.
 #include <cuda.h>
 #include <cuda_fp16.h>
+
+#include <type_traits>
 #include <cuda_runtime.h>
 
 #include "sia_internal.h"
@@ -34,13 +36,22 @@ namespace sia {
 namespace {
 
 constexpr int kProducerWarps = 4;   // cp.async gather (+ TMA for q)
-constexpr int kFirstProducerWarp = 4;
-constexpr int kMmaWarp = 8;
-constexpr int kAttnThreads = 288;   // warps 0-3 softmax/epilogue, 4-7 gather, 8 MMA
-// Registers per thread after the split (launch gives 168 x 288): the softmax warpgroup holds a
-// tile of fp32 logits plus the next tile's fp16 partials, the gather warpgroup needs little.
-constexpr int kSoftmaxRegs = 232;
-constexpr int kGatherRegs = 96;
+constexpr int kFirstExchangeWarp = 4;
+constexpr int kFirstProducerWarp = 8;
+constexpr int kMmaWarp = 12;
+// warps 0-3 softmax + epilogue, 4-7 partial-logit exchange, 8-11 gather, 12 MMA
+constexpr int kAttnThreads = 416;
+// Registers per thread after the split.  The block is launched with 128 x 416 registers
+// (ptxas' allocation for 416 threads); the softmax warpgroup takes 168 (a tile of fp32 logits),
+// the gather warpgroup gives back down to 88, the exchange warpgroup and the MMA warp keep 128:
+// 128*168 + 128*88 + 128*128 + 32*128 = 53248 = 416*128, so setmaxnreg.inc never waits for
+// registers that are not there.
+constexpr int kLaunchRegs = 128;
+constexpr int kSoftmaxRegs = 168;
+constexpr int kGatherRegs = 88;
+static_assert(128 * kSoftmaxRegs + 128 * kGatherRegs + 128 * kLaunchRegs + 32 * kLaunchRegs <=
+                  kAttnThreads * kLaunchRegs,
+              "register split exceeds the launch allocation");
 constexpr int kStages = 3;          // latent-row tiles in flight per CTA
 constexpr int kRows = kAttnTileRows;
 
@@ -59,7 +70,7 @@ struct AttnLayout<512, 64> {
   __device__ static bool has_rope(int) { return true; }
   __device__ static int lat_x(int r, int i) { return 256 * r + 64 * i; }   // q columns (elements)
   __device__ static int rope_x(int r) { return 512 + 32 * r; }
-  __device__ static int chunks(int) { return 36; }                        // 16-byte pieces per row
+  static constexpr int kChunks0 = 36, kChunks1 = 36;                      // 16-byte pieces per row
   __device__ static int chunk_src(int r, int k) { return k < 32 ? 512 * r + 16 * k : 1024 + 64 * r + 16 * (k - 32); }
   __device__ static uint32_t chunk_dst(int row, int k) {
     return k < 32 ? (uint32_t)(k >> 3) * (kAttnTileRows * 128) + swizzled_offset(row, (k & 7) * 16, 128)
@@ -77,7 +88,7 @@ struct AttnLayout<64, 16> {
   __device__ static bool has_rope(int r) { return r == 0; }
   __device__ static int lat_x(int r, int) { return 32 * r; }
   __device__ static int rope_x(int) { return 64; }
-  __device__ static int chunks(int r) { return r == 0 ? 6 : 4; }
+  static constexpr int kChunks0 = 6, kChunks1 = 4;
   __device__ static int chunk_src(int r, int k) { return k < 4 ? 64 * r + 16 * k : 128 + 16 * (k - 4); }
   __device__ static uint32_t chunk_dst(int row, int k) {
     return k < 4 ? swizzled_offset(row, k * 16, 64) : (uint32_t)(kAttnTileRows * 64) + swizzled_offset(row, (k - 4) * 16, 32);
@@ -109,7 +120,7 @@ struct AttnSmem {
 
 struct AttnBarriers {
   uint64_t c_full[kStages], c_empty[kStages];
-  uint64_t s_full[2], s_empty[2];
+  uint64_t s_full[2], s_comb[2], s_empty[2];
   uint64_t p_full[2], p_empty[2];
   uint64_t q_full, q_empty;
   uint64_t o_full, o_empty;
@@ -144,6 +155,7 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
 template <int DL, int DR>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     sparse_attend_kernel(const __grid_constant__ AttnMaps maps, const AttnKernelParams p) {
+  static_assert(kAttnThreads == 416, "role layout assumes 13 warps");
   using Lay = AttnLayout<DL, DR>;
   using Sm = AttnSmem<Lay>;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -170,6 +182,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sb->s_full[s], 1);
+      mbar_init(&sb->s_comb[s], 128);
       mbar_init(&sb->s_empty[s], 128);
       mbar_init(&sb->p_full[s], 128);
       mbar_init(&sb->p_empty[s], 1);
@@ -207,7 +220,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int ptid = threadIdx.x - kFirstProducerWarp * 32;   // 0..127
     const int pwarp = warp - kFirstProducerWarp;
     const uint8_t* kv = static_cast<const uint8_t*>(p.kv);
-    const int nch = Lay::chunks((int)rank);
+    // one tile of gathers: consecutive threads take consecutive 16-byte pieces of a row, so a
+    // warp reads whole 512-byte runs of a latent row at a time
+    auto gather_tile = [&](auto nch_c, uint32_t cst, const int32_t* rows) {
+      constexpr int NCH = decltype(nch_c)::value;
+#pragma unroll 4
+      for (int i = ptid; i < kRows * NCH; i += kProducerWarps * 32) {
+        const int row = i / NCH, k = i - row * NCH;
+        cp_async16(cst + Lay::chunk_dst(row, k), kv + (size_t)(uint32_t)rows[row] * (DC * 2) + Lay::chunk_src((int)rank, k));
+      }
+    };
     int it = 0, u_it = 0;
     bool ok = true;
     for (int u = cluster_id; u < p.units && ok; u += n_clusters, ++u_it) {
@@ -280,10 +302,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (!mbar_wait(&sb->c_empty[stage], ((uint32_t)(it / kStages) & 1u) ^ 1u, abort, p.status)) { ok = false; break; }
         const uint32_t cst = smem_u32(smem + Sm::kOffC + stage * Sm::kCStageBytes);
         const int32_t* rows = rt + t * kRows;
-        for (int i = ptid; i < kRows * nch; i += kProducerWarps * 32) {
-          const int row = i / nch, k = i - row * nch;
-          cp_async16(cst + Lay::chunk_dst(row, k), kv + (size_t)(uint32_t)rows[row] * (DC * 2) + Lay::chunk_src((int)rank, k));
-        }
+        if (rank == 0) gather_tile(std::integral_constant<int, Lay::kChunks0>{}, cst, rows);
+        else gather_tile(std::integral_constant<int, Lay::kChunks1>{}, cst, rows);
         asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(&sb->c_full[stage])) : "memory");
       }
     }
@@ -380,48 +400,84 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_wait(&sb->mma_done, 0, abort, p.status);
     }
     __syncwarp();
+  } else if (warp >= kFirstExchangeWarp && warp < kFirstExchangeWarp + 4) {
+    // ---------------------------------------------------------------- partial-logit exchange
+    // Reads this CTA's partial logits of a tile from TMEM, rounds them to fp16 (scaled to base
+    // 2), pushes them to the peer CTA, adds the peer's partials and writes the complete logits
+    // back into the same TMEM columns for the softmax warps.  Both CTAs add the same two fp16
+    // values, so their softmax inputs agree bit for bit.
+    const int quad = warp & 3;
+    const int h = quad * 32 + lane;
+    const uint32_t lane_addr = tmem_base + ((uint32_t)(quad * 32) << 16);
+    const uint32_t sx_peer = mapa_shared(smem_u32(smem + Sm::kOffSx), peer);
+    int s_it = 0, u_it = 0;
+    bool ok = true;
+    for (int u = cluster_id; u < p.units && ok; u += n_clusters, ++u_it) {
+      const int buf = u_it & 1;
+      if (!mbar_wait(&sb->tab_full[buf], (uint32_t)(u_it >> 1) & 1u, abort, p.status)) { ok = false; break; }
+      int first_neg = 1 << 30;
+      for (int w = 0; w < kProducerWarps; ++w) first_neg = min(first_neg, fneg_tab[buf * kProducerWarps + w]);
+      const int ntiles = (first_neg + kRows - 1) / kRows;
+      for (int t = 0; t < ntiles; ++t, ++s_it) {
+        const int sbuf = s_it & 1;
+        const uint32_t scol = lane_addr + s_col + sbuf * kRows;
+        if (!mbar_wait(&sb->s_full[sbuf], (uint32_t)(s_it >> 1) & 1u, abort, p.status)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t own[kRows / 2];
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t r[2][16];
+          tmem_ld16(scol + half * 32, r[0]);
+          tmem_ld16(scol + half * 32 + 16, r[1]);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 2; ++c)
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              own[half * 16 + c * 8 + i] = pack_f16x2(__uint_as_float(r[c][2 * i]) * p.scale_log2,
+                                                      __uint_as_float(r[c][2 * i + 1]) * p.scale_log2);
+        }
+        if (!mbar_wait<true>(&sb->sx_free, ((uint32_t)s_it & 1u) ^ 1u, abort, p.status)) { ok = false; break; }
+#pragma unroll
+        for (int g = 0; g < kRows / 8; ++g)
+          asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sx_peer + (uint32_t)((g * 128 + h) * 16)),
+                       "r"(own[4 * g]), "r"(own[4 * g + 1]), "r"(own[4 * g + 2]), "r"(own[4 * g + 3])
+                       : "memory");
+        mbar_arrive_cluster(&sb->sx_ready, peer);
+        if (!mbar_wait<true>(&sb->sx_ready, (uint32_t)s_it & 1u, abort, p.status)) { ok = false; break; }
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t w[2][16];
+#pragma unroll
+          for (int g2 = 0; g2 < 4; ++g2) {
+            const int g = half * 4 + g2;
+            const uint4 v = *reinterpret_cast<const uint4*>(smem + Sm::kOffSx + (g * 128 + h) * 16);
+            const uint32_t pv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float2 a = unpack_f16x2(own[4 * g + i]), c = unpack_f16x2(pv[i]);
+              const int col = g2 * 8 + 2 * i;
+              w[col >> 4][col & 15] = __float_as_uint(a.x + c.x);
+              w[col >> 4][(col & 15) + 1] = __float_as_uint(a.y + c.y);
+            }
+          }
+          tmem_st16(scol + half * 32, w[0]);
+          tmem_st16(scol + half * 32 + 16, w[1]);
+        }
+        mbar_arrive_cluster(&sb->sx_free, peer);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&sb->s_comb[sbuf]);
+      }
+    }
   } else {
     // ---------------------------------------------------------------- softmax + epilogue
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
     const int quad = warp & 3;
     const int h = quad * 32 + lane;   // head = TMEM lane
     const uint32_t lane_addr = tmem_base + ((uint32_t)(quad * 32) << 16);
-    const uint32_t sx = smem_u32(smem + Sm::kOffSx);
-    const uint32_t sx_peer = mapa_shared(sx, peer);
     int s_it = 0, pv_it = 0, u_it = 0;
     bool ok = true;
-
-    // Own partial logits of the next tile: read them from TMEM, free the TMEM buffer, round to
-    // fp16 (both CTAs then add the same two fp16 values, so their softmax inputs agree bit for
-    // bit) and push them to the peer's buffer Sx[row/8][head][row%8].
-    auto load_and_send = [&](uint32_t (&own)[kRows / 2]) -> bool {
-      const int sbuf = s_it & 1;
-      if (!mbar_wait(&sb->s_full[sbuf], (uint32_t)(s_it >> 1) & 1u, abort, p.status)) return false;
-      tc_fence_after();
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {   // 32 columns at a time keeps register use low
-        uint32_t r[2][16];
-        tmem_ld16(lane_addr + s_col + sbuf * kRows + half * 32, r[0]);
-        tmem_ld16(lane_addr + s_col + sbuf * kRows + half * 32 + 16, r[1]);
-        tmem_wait_ld();
-#pragma unroll
-        for (int c = 0; c < 2; ++c)
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            own[half * 16 + c * 8 + i] = pack_f16x2(__uint_as_float(r[c][2 * i]) * p.scale_log2,
-                                                    __uint_as_float(r[c][2 * i + 1]) * p.scale_log2);
-      }
-      tc_fence_before();
-      mbar_arrive(&sb->s_empty[sbuf]);
-      if (!mbar_wait<true>(&sb->sx_free, ((uint32_t)s_it & 1u) ^ 1u, abort, p.status)) return false;
-#pragma unroll
-      for (int g = 0; g < kRows / 8; ++g)
-        asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sx_peer + (uint32_t)((g * 128 + h) * 16)),
-                     "r"(own[4 * g]), "r"(own[4 * g + 1]), "r"(own[4 * g + 2]), "r"(own[4 * g + 3])
-                     : "memory");
-      mbar_arrive_cluster(&sb->sx_ready, peer);
-      return true;
-    };
 
     for (int u = cluster_id; u < p.units && ok; u += n_clusters, ++u_it) {
       const int bj = u / p.splits, split = u - bj * p.splits;
@@ -433,26 +489,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint32_t* mt = mask_tab + buf * (kAttnMaxSplitRows / 32);
       float m = -INFINITY, l = 0.0f;
       float s[kRows];
-      uint32_t own[kRows / 2];
-      if (ntiles > 0 && !load_and_send(own)) { ok = false; break; }
       for (int t = 0; t < ntiles; ++t, ++pv_it) {
-        // the peer's partial of tile t completes the logits (already scaled to base 2)
-        if (!mbar_wait<true>(&sb->sx_ready, (uint32_t)s_it & 1u, abort, p.status)) { ok = false; break; }
+        // complete logits of tile t (base 2), assembled in TMEM by the exchange warps
+        const int sbuf = s_it & 1;
+        if (!mbar_wait(&sb->s_comb[sbuf], (uint32_t)(s_it >> 1) & 1u, abort, p.status)) { ok = false; break; }
+        tc_fence_after();
+        {
+          uint32_t r[4][16];
 #pragma unroll
-        for (int g = 0; g < kRows / 8; ++g) {
-          const uint4 v = *reinterpret_cast<const uint4*>(smem + Sm::kOffSx + (g * 128 + h) * 16);
-          const uint32_t pv[4] = {v.x, v.y, v.z, v.w};
+          for (int c = 0; c < 4; ++c) tmem_ld16(lane_addr + s_col + sbuf * kRows + c * 16, r[c]);
+          tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float2 a = unpack_f16x2(own[4 * g + i]), c = unpack_f16x2(pv[i]);
-            s[8 * g + 2 * i] = a.x + c.x;
-            s[8 * g + 2 * i + 1] = a.y + c.y;
-          }
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int i = 0; i < 16; ++i) s[c * 16 + i] = __uint_as_float(r[c][i]);
         }
-        mbar_arrive_cluster(&sb->sx_free, peer);
+        tc_fence_before();
+        mbar_arrive(&sb->s_empty[sbuf]);
         ++s_it;
-        // start the exchange of tile t+1 before the softmax of tile t
-        if (t + 1 < ntiles && !load_and_send(own)) { ok = false; break; }
         uint64_t valid = ((uint64_t)mt[2 * t + 1] << 32) | mt[2 * t];
         const int live = first_neg - t * kRows;            // rows past the first -1 are padding
         if (live < kRows) valid &= (1ull << live) - 1ull;
@@ -607,6 +661,13 @@ template <int DL, int DR>
 cudaError_t launch_attend_impl(const AttnKernelParams& p, const CUtensorMap* maps, int n_clusters,
                                bool pdl, cudaStream_t stream) {
   using Sm = AttnSmem<AttnLayout<DL, DR>>;
+  {
+    // the warpgroup register split assumes the launch allocation kLaunchRegs per thread
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, sparse_attend_kernel<DL, DR>);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
+  }
   // at most two CTAs per SM may share the 512 TMEM columns (kTmemCols each <= 256 when two fit)
   const size_t smem = Sm::kBytes < 100 * 1024 ? 100 * 1024 : Sm::kBytes;
   cudaError_t e = cudaFuncSetAttribute(sparse_attend_kernel<DL, DR>,
