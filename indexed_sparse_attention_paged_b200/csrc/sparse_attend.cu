@@ -35,21 +35,20 @@
 namespace sia {
 namespace {
 
-constexpr int kProducerWarps = 4;   // cp.async gather (+ TMA for q)
+constexpr int kProducerWarps = 8;   // cp.async gather (+ TMA for q)
 constexpr int kFirstExchangeWarp = 4;
 constexpr int kFirstProducerWarp = 8;
-constexpr int kMmaWarp = 12;
-// warps 0-3 softmax + epilogue, 4-7 partial-logit exchange, 8-11 gather, 12 MMA
-constexpr int kAttnThreads = 416;
-// Registers per thread after the split.  The block is launched with 128 x 416 registers
-// (ptxas' allocation for 416 threads); the softmax warpgroup takes 168 (a tile of fp32 logits),
-// the gather warpgroup gives back down to 88, the exchange warpgroup and the MMA warp keep 128:
-// 128*168 + 128*88 + 128*128 + 32*128 = 53248 = 416*128, so setmaxnreg.inc never waits for
-// registers that are not there.
-constexpr int kLaunchRegs = 128;
+constexpr int kMmaWarp = 16;
+// warps 0-3 softmax + epilogue, 4-7 partial-logit exchange, 8-15 gather, 16 MMA
+constexpr int kAttnThreads = 544;
+// Registers per thread after the split.  The block is launched with kLaunchRegs x 544
+// registers (ptxas' allocation for 544 threads); the softmax warpgroup takes 168 (a tile of
+// fp32 logits), the two gather warpgroups give back down to 56, the exchange warpgroup and the
+// MMA warp keep the launch value, so setmaxnreg.inc never waits for registers that are not there.
+constexpr int kLaunchRegs = 96;
 constexpr int kSoftmaxRegs = 168;
-constexpr int kGatherRegs = 88;
-static_assert(128 * kSoftmaxRegs + 128 * kGatherRegs + 128 * kLaunchRegs + 32 * kLaunchRegs <=
+constexpr int kGatherRegs = 56;
+static_assert(128 * kSoftmaxRegs + 256 * kGatherRegs + 128 * kLaunchRegs + 32 * kLaunchRegs <=
                   kAttnThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
 constexpr int kStages = 3;          // latent-row tiles in flight per CTA
@@ -120,7 +119,7 @@ struct AttnSmem {
 
 struct AttnBarriers {
   uint64_t c_full[kStages], c_empty[kStages];
-  uint64_t s_full[2], s_comb[2], s_empty[2];
+  uint64_t s_full[2], s_empty[2];
   uint64_t p_full[2], p_empty[2];
   uint64_t q_full, q_empty;
   uint64_t o_full, o_empty;
@@ -155,7 +154,7 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
 template <int DL, int DR>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     sparse_attend_kernel(const __grid_constant__ AttnMaps maps, const AttnKernelParams p) {
-  static_assert(kAttnThreads == 416, "role layout assumes 13 warps");
+  static_assert(kAttnThreads == 544, "role layout assumes 17 warps");
   using Lay = AttnLayout<DL, DR>;
   using Sm = AttnSmem<Lay>;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -182,7 +181,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sb->s_full[s], 1);
-      mbar_init(&sb->s_comb[s], 128);
       mbar_init(&sb->s_empty[s], 128);
       mbar_init(&sb->p_full[s], 128);
       mbar_init(&sb->p_empty[s], 1);
@@ -217,7 +215,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (warp >= kFirstProducerWarp && warp < kFirstProducerWarp + kProducerWarps) {
     // ---------------------------------------------------------------- gather (4 warps)
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kGatherRegs));
-    const int ptid = threadIdx.x - kFirstProducerWarp * 32;   // 0..127
+    const int ptid = threadIdx.x - kFirstProducerWarp * 32;   // 0..255
     const int pwarp = warp - kFirstProducerWarp;
     const uint8_t* kv = static_cast<const uint8_t*>(p.kv);
     // one tile of gathers: consecutive threads take consecutive 16-byte pieces of a row, so a
@@ -403,9 +401,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   } else if (warp >= kFirstExchangeWarp && warp < kFirstExchangeWarp + 4) {
     // ---------------------------------------------------------------- partial-logit exchange
     // Reads this CTA's partial logits of a tile from TMEM, rounds them to fp16 (scaled to base
-    // 2), pushes them to the peer CTA, adds the peer's partials and writes the complete logits
-    // back into the same TMEM columns for the softmax warps.  Both CTAs add the same two fp16
-    // values, so their softmax inputs agree bit for bit.
+    // 2) and pushes them into the peer CTA's exchange buffer; the peer's softmax warps add them
+    // to their own partials.  Both CTAs add the same two fp16 values, so their softmax inputs
+    // agree bit for bit.
     const int quad = warp & 3;
     const int h = quad * 32 + lane;
     const uint32_t lane_addr = tmem_base + ((uint32_t)(quad * 32) << 16);
@@ -444,30 +442,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                        "r"(own[4 * g]), "r"(own[4 * g + 1]), "r"(own[4 * g + 2]), "r"(own[4 * g + 3])
                        : "memory");
         mbar_arrive_cluster(&sb->sx_ready, peer);
-        if (!mbar_wait<true>(&sb->sx_ready, (uint32_t)s_it & 1u, abort, p.status)) { ok = false; break; }
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t w[2][16];
-#pragma unroll
-          for (int g2 = 0; g2 < 4; ++g2) {
-            const int g = half * 4 + g2;
-            const uint4 v = *reinterpret_cast<const uint4*>(smem + Sm::kOffSx + (g * 128 + h) * 16);
-            const uint32_t pv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const float2 a = unpack_f16x2(own[4 * g + i]), c = unpack_f16x2(pv[i]);
-              const int col = g2 * 8 + 2 * i;
-              w[col >> 4][col & 15] = __float_as_uint(a.x + c.x);
-              w[col >> 4][(col & 15) + 1] = __float_as_uint(a.y + c.y);
-            }
-          }
-          tmem_st16(scol + half * 32, w[0]);
-          tmem_st16(scol + half * 32 + 16, w[1]);
-        }
-        mbar_arrive_cluster(&sb->sx_free, peer);
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(&sb->s_comb[sbuf]);
       }
     }
   } else {
@@ -490,22 +464,37 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       float m = -INFINITY, l = 0.0f;
       float s[kRows];
       for (int t = 0; t < ntiles; ++t, ++pv_it) {
-        // complete logits of tile t (base 2), assembled in TMEM by the exchange warps
+        // logits of tile t (base 2) = own partial (TMEM) + the peer's partial (exchange buffer),
+        // each rounded to fp16 exactly as the exchange warps of both CTAs round them
         const int sbuf = s_it & 1;
-        if (!mbar_wait(&sb->s_comb[sbuf], (uint32_t)(s_it >> 1) & 1u, abort, p.status)) { ok = false; break; }
+        if (!mbar_wait(&sb->s_full[sbuf], (uint32_t)(s_it >> 1) & 1u, abort, p.status)) { ok = false; break; }
+        if (!mbar_wait<true>(&sb->sx_ready, (uint32_t)s_it & 1u, abort, p.status)) { ok = false; break; }
         tc_fence_after();
-        {
-          uint32_t r[4][16];
 #pragma unroll
-          for (int c = 0; c < 4; ++c) tmem_ld16(lane_addr + s_col + sbuf * kRows + c * 16, r[c]);
+        for (int half = 0; half < 2; ++half) {
+          uint32_t r[2][16];
+          tmem_ld16(lane_addr + s_col + sbuf * kRows + half * 32, r[0]);
+          tmem_ld16(lane_addr + s_col + sbuf * kRows + half * 32 + 16, r[1]);
           tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
+          for (int g2 = 0; g2 < 4; ++g2) {
+            const int g = half * 4 + g2;
+            const uint4 v = *reinterpret_cast<const uint4*>(smem + Sm::kOffSx + (g * 128 + h) * 16);
+            const uint32_t pv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-            for (int i = 0; i < 16; ++i) s[c * 16 + i] = __uint_as_float(r[c][i]);
+            for (int i = 0; i < 4; ++i) {
+              const int col = g2 * 8 + 2 * i;
+              const float2 a = unpack_f16x2(pack_f16x2(__uint_as_float(r[col >> 4][col & 15]) * p.scale_log2,
+                                                       __uint_as_float(r[col >> 4][(col & 15) + 1]) * p.scale_log2));
+              const float2 c = unpack_f16x2(pv[i]);
+              s[8 * g + 2 * i] = a.x + c.x;
+              s[8 * g + 2 * i + 1] = a.y + c.y;
+            }
+          }
         }
         tc_fence_before();
         mbar_arrive(&sb->s_empty[sbuf]);
+        mbar_arrive_cluster(&sb->sx_free, peer);
         ++s_it;
         uint64_t valid = ((uint64_t)mt[2 * t + 1] << 32) | mt[2 * t];
         const int live = first_neg - t * kRows;            // rows past the first -1 are padding
