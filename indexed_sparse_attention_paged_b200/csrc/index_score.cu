@@ -175,38 +175,37 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
         go = __shfl_sync(0xffffffffu, go, 0);
         if (!go) { ok = false; break; }
         uint8_t* kst = smem + p.off_k + stage * p.k_stage_bytes;
-        const int chunks = kIndexTileRows / p.box_rows;
-        // page ids of this tile's chunks, read 32 logical pages at a time by the whole warp
-        uint32_t valid_mask = 0;
-        int pages_of_chunk[16];
-#pragma unroll 1
-        for (int c = 0; c < chunks; ++c) {
-          const int pos = t * kIndexTileRows + c * p.box_rows;
-          const int lp = pos / p.P;
-          if (lp < cached_base || lp >= cached_base + 32) {
-            cached_base = lp;
-            cached_page = (lp + lane < p.max_pages) ? pt_row[lp + lane] : -1;
-          }
-          const int page = __shfl_sync(0xffffffffu, cached_page, lp - cached_base);
-          pages_of_chunk[c] = page;
-          if (pos <= gi.max_pos) {
-            if (page >= 0 && page < p.num_pages) valid_mask |= 1u << c;
-            else if (lane == 0) report(p.status, SIA_DEV_BAD_PAGE);
-          }
+        const int chunks = kIndexTileRows / p.box_rows;   // 1..16 boxes of whole-page rows
+        // lane c < chunks resolves chunk c's page id through the warp's window of 32 cached
+        // page-table entries (registers only: one shuffle per lane)
+        const int tile_pos0 = t * kIndexTileRows;
+        const int lp_first = tile_pos0 / p.P;
+        const int lp_last = (tile_pos0 + (chunks - 1) * p.box_rows) / p.P;
+        if (lp_first < cached_base || lp_last >= cached_base + 32) {   // warp-uniform
+          cached_base = lp_first;
+          cached_page = (lp_first + lane < p.max_pages) ? pt_row[lp_first + lane] : -1;
         }
+        const int my_pos = tile_pos0 + lane * p.box_rows;
+        const int my_lp = lane < chunks ? my_pos / p.P : lp_first;
+        const int my_page = __shfl_sync(0xffffffffu, cached_page, my_lp - cached_base);
+        const bool in_range = lane < chunks && my_pos <= gi.max_pos;
+        const bool page_ok = my_page >= 0 && my_page < p.num_pages;
+        if (in_range && !page_ok) report(p.status, SIA_DEV_BAD_PAGE);
+        const uint32_t valid_mask = __ballot_sync(0xffffffffu, in_range && page_ok);
+        uint8_t* info = smem + p.off_kinfo + stage * kStageInfoBytes;
+        const uint32_t scale_bytes = p.k_scale ? (uint32_t)p.box_rows * 4u : 0u;
         if (lane == 0) {
           // per-stage info read by the epilogue: which chunks hold real pages, and (FP8) the
           // per-token key scales of the tile, copied next to the K tile
-          uint8_t* info = smem + p.off_kinfo + stage * kStageInfoBytes;
           *reinterpret_cast<uint32_t*>(info) = valid_mask;
-          const uint32_t scale_bytes = p.k_scale ? (uint32_t)p.box_rows * 4u : 0u;
           const uint32_t bytes =
               (uint32_t)__popc(valid_mask) * (p.n_kblocks * p.box_rows * p.kbw + scale_bytes);
           mbar_arrive_expect_tx(&sb->k_full[stage], bytes);
-          for (int c = 0; c < chunks; ++c) {
-            if (!(valid_mask >> c & 1u)) continue;
-            const int pos = t * kIndexTileRows + c * p.box_rows;
-            const int y = pages_of_chunk[c] * p.P + (pos % p.P);
+        }
+        for (int c = 0; c < chunks; ++c) {   // warp-uniform trip count
+          const int page = __shfl_sync(0xffffffffu, my_page, c);
+          if (lane == 0 && (valid_mask >> c & 1u)) {
+            const int y = page * p.P + ((tile_pos0 + c * p.box_rows) % p.P);
             for (int kb = 0; kb < p.n_kblocks; ++kb)
               tma_load_2d(kst + kb * p.k_kblock_bytes + c * p.box_rows * p.kbw, &kmap,
                           &sb->k_full[stage], kb * p.kbw / (p.fp8 ? 1 : 2), y);

@@ -299,6 +299,7 @@ sia_status plan_attend(const sia_attend_args* a, AttendPlan* pl, bool make_maps)
   k.rows_per_split = best_rows;
   if (bj * best_s > 0x7fffffffll) return fail(SIA_ERR_UNSUPPORTED, "too many attention work units");
   k.units = (int)(bj * best_s);
+  k.q = a->q;
   k.kv = a->kv_cache;
   k.page_table = a->page_table;
   k.seq_lens = a->seq_lens;
@@ -308,7 +309,7 @@ sia_status plan_attend(const sia_attend_args* a, AttendPlan* pl, bool make_maps)
   pl->n_clusters = (int)std::min<long long>(k.units, pairs);
   pl->ws_part = 0;
   if (k.splits > 1) {
-    const size_t o = round_up((size_t)k.splits * bj * a->n_heads * a->d_latent * 4, 256);
+    const size_t o = round_up((size_t)k.splits * bj * a->n_heads * a->d_latent * 2, 256);
     const size_t l = round_up((size_t)k.splits * bj * a->n_heads * 4, 256);
     pl->ws_part = o + l;
   }
@@ -348,8 +349,8 @@ sia_status run_attend(AttendPlan* pl, void* ws, size_t ws_bytes, int32_t* dev_st
     if (ws_bytes < pl->ws_part) return fail(SIA_ERR_WORKSPACE, "workspace too small: %zu < %zu", ws_bytes, pl->ws_part);
     if (!aligned(ws, 256)) return fail(SIA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
     const long long bj = (long long)pl->ap.B * pl->ap.J;
-    float* o = static_cast<float*>(ws);
-    const size_t ob = round_up((size_t)pl->ap.splits * bj * pl->ap.H * pl->ap.DL * 4, 256);
+    uint16_t* o = static_cast<uint16_t*>(ws);
+    const size_t ob = round_up((size_t)pl->ap.splits * bj * pl->ap.H * pl->ap.DL * 2, 256);
     pl->ap.part_o = o;
     pl->ap.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + ob);
     pl->cp.part_o = pl->ap.part_o;

@@ -75,20 +75,21 @@ struct AttnKernelParams {
   int splits;                 // Top-K splits per query (>1 -> partials + combine)
   int rows_per_split;         // multiple of kAttnTileRows
   int units;                  // B * J * splits
+  const void* q;              // bf16 [B*J, H, DL + DR]
   const void* kv;             // bf16 [num_pages * P, DL + DR]
   const int32_t* page_table;
   const int32_t* seq_lens;
   const int32_t* topk;
   uint16_t* out;              // bf16 bits
   float* lse;
-  float* part_o;              // [splits][B*J][H][DL] fp32 (splits > 1)
+  uint16_t* part_o;           // [splits][B*J][H][DL] bf16, normalised (splits > 1)
   float* part_lse;            // [splits][B*J][H]
   int32_t* status;
 };
 
 struct CombineKernelParams {
   int BJ, H, DL, splits;
-  const float* part_o;
+  const uint16_t* part_o;
   const float* part_lse;
   uint16_t* out;
   float* lse;

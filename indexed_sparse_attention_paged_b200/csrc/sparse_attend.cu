@@ -14,15 +14,19 @@
 // OF TWO CTAs shares one (query, Top-K split):
 //   - CTA r owns output dims [r*DL/2, (r+1)*DL/2) and gathers only its half of each latent row
 //     (plus half of the rope dims), so together the pair reads each 1152-byte row once;
-//   - each CTA computes a partial S = Q_r . C_r^T over its own dims, the two partials are
-//     exchanged through distributed shared memory and summed (fp32 addition is commutative,
-//     so both CTAs hold bit-identical S and take identical softmax decisions);
-//   - each CTA runs the online softmax and accumulates O_r += P . C_r[:, its dims] in TMEM.
-// Rows are gathered by TMA tile::gather4 (4 rows per instruction) into 128B/64B/32B-swizzled
-// K-major tiles; the same tile serves as the K-major B operand of Q.C^T and as the MN-major B
-// operand of P.C.  Rescaling of O is lazy: only when a head's running max grows by more than
-// 2^8.  Splits of the Top-K list (to fill the GPU at small batch) write fp32 partials that
-// combine_kernel merges by log-sum-exp.
+//   - each CTA computes a partial S = Q_r . C_r^T over its own dims, with its latent half of Q
+//     held in TMEM (the A operand of the MMA) and only the rope part of Q in shared memory;
+//   - the partials are exchanged through distributed shared memory as fp16 (scaled to base
+//     2): each CTA adds the peer's fp16 partial to its own fp32 partial and runs its own online
+//     softmax.  The two CTAs' logits differ only by the fp16 rounding of one partial, and each
+//     CTA's (max, sum, O) triple is self-consistent, so each half of the output is normalised
+//     by the sum that produced it;
+//   - P (bf16) overwrites its own logits in TMEM and is the A operand of O_r += P . C_r.
+// Rows are gathered with 16-byte cp.async from a per-unit table of physical cache rows into
+// 128B/64B/32B-swizzled K-major tiles; the same tile serves as the K-major B operand of
+// Q.C^T and as the MN-major B operand of P.C.  Rescaling of O is lazy: only when a head's
+// running max grows by more than 2^8.  Splits of the Top-K list (to fill the GPU at small
+// batch) write fp32 partials that combine_kernel merges by log-sum-exp.
 #include <cuda.h>
 #include <cuda_fp16.h>
 
@@ -35,23 +39,25 @@
 namespace sia {
 namespace {
 
-constexpr int kProducerWarps = 8;   // cp.async gather (+ TMA for q)
+constexpr int kProducerWarps = 8;   // cp.async gather (+ TMA for the rope part of q)
 constexpr int kFirstExchangeWarp = 4;
 constexpr int kFirstProducerWarp = 8;
 constexpr int kMmaWarp = 16;
-// warps 0-3 softmax + epilogue, 4-7 partial-logit exchange, 8-15 gather, 16 MMA
+// warps 0-3 softmax + epilogue, 4-7 q loader + partial-logit exchange, 8-15 gather, 16 MMA
 constexpr int kAttnThreads = 544;
 // Registers per thread after the split.  The block is launched with kLaunchRegs x 544
 // registers (ptxas' allocation for 544 threads); the softmax warpgroup takes 168 (a tile of
-// fp32 logits), the two gather warpgroups give back down to 56, the exchange warpgroup and the
-// MMA warp keep the launch value, so setmaxnreg.inc never waits for registers that are not there.
+// fp32 logits), the exchange warpgroup 104, the two gather warpgroups give back down to 56 and
+// the MMA warp keeps the launch value.  The sum stays within the launch allocation, so
+// setmaxnreg.inc never waits for registers that are not there.
 constexpr int kLaunchRegs = 96;
 constexpr int kSoftmaxRegs = 168;
+constexpr int kExchangeRegs = 104;
 constexpr int kGatherRegs = 56;
-static_assert(128 * kSoftmaxRegs + 256 * kGatherRegs + 128 * kLaunchRegs + 32 * kLaunchRegs <=
+static_assert(128 * kSoftmaxRegs + 256 * kGatherRegs + 128 * kExchangeRegs + 32 * kLaunchRegs <=
                   kAttnThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
-constexpr int kStages = 3;          // latent-row tiles in flight per CTA
+constexpr int kStages = 4;          // latent-row tiles in flight per CTA
 constexpr int kRows = kAttnTileRows;
 
 template <int DL, int DR>
@@ -61,13 +67,13 @@ struct AttnLayout;
 // Q.C^T and P.C) and a share of the rope dims (used by Q.C^T only).
 template <>
 struct AttnLayout<512, 64> {
+  static constexpr int kLatDims = 256;    // latent dims per CTA (q part held in TMEM)
   static constexpr int kLatBlocks = 4;    // 4 x 64 latent dims per CTA, 128-byte swizzled rows
   static constexpr int kLatKbw = 128;
   static constexpr int kRopeKbw = 64;     // 32 rope dims per CTA, 64-byte swizzled rows
   static constexpr int kPvN = 256;
   static constexpr uint32_t kTmemCols = 512;
   __device__ static bool has_rope(int) { return true; }
-  __device__ static int lat_x(int r, int i) { return 256 * r + 64 * i; }   // q columns (elements)
   __device__ static int rope_x(int r) { return 512 + 32 * r; }
   static constexpr int kChunks0 = 36, kChunks1 = 36;                      // 16-byte pieces per row
   __device__ static int chunk_src(int r, int k) { return k < 32 ? 512 * r + 16 * k : 1024 + 64 * r + 16 * (k - 32); }
@@ -79,13 +85,13 @@ struct AttnLayout<512, 64> {
 
 template <>
 struct AttnLayout<64, 16> {
+  static constexpr int kLatDims = 32;
   static constexpr int kLatBlocks = 1;    // 32 latent dims per CTA, 64-byte swizzled rows
   static constexpr int kLatKbw = 64;
   static constexpr int kRopeKbw = 32;     // all 16 rope dims on CTA 0, 32-byte swizzled rows
   static constexpr int kPvN = 32;
   static constexpr uint32_t kTmemCols = 256;
   __device__ static bool has_rope(int r) { return r == 0; }
-  __device__ static int lat_x(int r, int) { return 32 * r; }
   __device__ static int rope_x(int) { return 64; }
   static constexpr int kChunks0 = 6, kChunks1 = 4;
   __device__ static int chunk_src(int r, int k) { return k < 4 ? 64 * r + 16 * k : 128 + 16 * (k - 4); }
@@ -94,20 +100,31 @@ struct AttnLayout<64, 16> {
   }
 };
 
+// TMEM columns: O [0, kPvN), two logit buffers of kRows fp32 columns, then the CTA's latent
+// half of q as bf16 pairs (the A operand of Q . C^T).
+template <class Lay>
+struct AttnTmem {
+  static constexpr uint32_t kO = 0;
+  static constexpr uint32_t kS = Lay::kPvN;
+  static constexpr uint32_t kQ = kS + 2 * kRows;
+  static_assert(kQ + Lay::kLatDims / 2 <= Lay::kTmemCols, "TMEM columns overflow");
+};
+
 struct AttnMaps {
-  CUtensorMap q_lat, q_rope, kv_lat, kv_rope;
+  CUtensorMap q_rope;
 };
 
 template <class Lay>
 struct AttnSmem {
-  static constexpr uint32_t kQLatBytes = 128 * Lay::kLatKbw;
   static constexpr uint32_t kQRopeBytes = 128 * Lay::kRopeKbw;
   static constexpr uint32_t kCLatBytes = kRows * Lay::kLatKbw;
   static constexpr uint32_t kCRopeBytes = kRows * Lay::kRopeKbw;
   static constexpr uint32_t kCStageBytes = Lay::kLatBlocks * kCLatBytes + kCRopeBytes;
-  static constexpr uint32_t kOffQ = 0;
-  static constexpr uint32_t kOffC = kOffQ + Lay::kLatBlocks * kQLatBytes + kQRopeBytes;
-  static constexpr uint32_t kOffSx = kOffC + kStages * kCStageBytes;   // peer logits, fp16
+  static constexpr uint32_t kOffQ = 0;                                  // rope part of q only
+  static constexpr uint32_t kOffC = (kOffQ + kQRopeBytes + 1023u) & ~1023u;
+  // P (bf16, 128 heads x kRows, 128B-swizzled K-major): the A operand of P . C
+  static constexpr uint32_t kOffP = kOffC + kStages * kCStageBytes;
+  static constexpr uint32_t kOffSx = kOffP + 128 * kRows * 2;          // peer logits, fp16
   static constexpr uint32_t kOffRows = kOffSx + kRows * 128 * 2;
   // per unit (double-buffered): physical cache row of each Top-K entry, validity bits, and
   // each gather warp's lowest position of a -1 entry
@@ -115,14 +132,17 @@ struct AttnSmem {
   static constexpr uint32_t kOffFirstNeg = kOffMask + 2 * (kAttnMaxSplitRows / 8);
   static constexpr uint32_t kOffBar = kOffFirstNeg + 2 * kProducerWarps * 4;
   static constexpr uint32_t kBytes = kOffBar + 256;
+  static_assert(kOffP % 1024 == 0, "P must sit on a 1024-byte swizzle atom");
 };
 
 struct AttnBarriers {
   uint64_t c_full[kStages], c_empty[kStages];
-  uint64_t s_full[2], s_empty[2];
-  uint64_t p_full[2], p_empty[2];
+  uint64_t s_full[2], s_empty[2];   // logits ready / read by the softmax and exchange warps
+  uint64_t p_full;                  // all softmax threads wrote P (waited by the P . C issuer)
+  uint64_t p_empty;                 // P . C of the previous tile done (P buffer and O free)
+  uint64_t epi_sync;                // all softmax threads are past the unit's last tile
   uint64_t q_full, q_empty;
-  uint64_t o_full, o_empty;
+  uint64_t o_full;
   uint64_t sx_ready, sx_free;
   uint64_t tab_full[2], tab_free[2];
   uint64_t mma_done;
@@ -142,13 +162,26 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   return r;
 }
 
-__device__ __forceinline__ float2 unpack_f16x2(uint32_t v) {
-  __half2 h = *reinterpret_cast<__half2*>(&v);
-  return __half22float2(h);
+// a + (fp32) the two fp16 halves of h: {a_lo + lo(h), a_hi + hi(h)}, one rounding each
+__device__ __forceinline__ void add_f16x2_to_f32(uint32_t h, float& lo, float& hi) {
+  asm("{\n\t.reg .b16 l16, h16;\n\t"
+      "mov.b32 {l16, h16}, %2;\n\t"
+      "add.rn.f32.f16 %0, l16, %0;\n\t"
+      "add.rn.f32.f16 %1, h16, %1;\n\t}"
+      : "+f"(lo), "+f"(hi)
+      : "r"(h));
 }
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
 }
 
 template <int DL, int DR>
@@ -157,6 +190,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   static_assert(kAttnThreads == 544, "role layout assumes 17 warps");
   using Lay = AttnLayout<DL, DR>;
   using Sm = AttnSmem<Lay>;
+  using Tm = AttnTmem<Lay>;
   extern __shared__ __align__(1024) uint8_t smem[];
   AttnBarriers* sb = reinterpret_cast<AttnBarriers*>(smem + Sm::kOffBar);
   int32_t* rows_tab = reinterpret_cast<int32_t*>(smem + Sm::kOffRows);        // [2][max rows]
@@ -181,22 +215,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sb->s_full[s], 1);
-      mbar_init(&sb->s_empty[s], 128);
-      mbar_init(&sb->p_full[s], 128);
-      mbar_init(&sb->p_empty[s], 1);
+      mbar_init(&sb->s_empty[s], 128 + 128);   // softmax and exchange threads
       mbar_init(&sb->tab_full[s], kProducerWarps * 32);
-      mbar_init(&sb->tab_free[s], 128);
+      mbar_init(&sb->tab_free[s], 128 + 128 + 1);   // softmax, exchange and MMA threads
     }
-    mbar_init(&sb->q_full, 1);
+    mbar_init(&sb->p_full, 128);
+    mbar_init(&sb->p_empty, 1);
+    mbar_init(&sb->epi_sync, 128);
+    mbar_init(&sb->q_full, 128 + 1);   // 128 TMEM writers + the rope TMA
     mbar_init(&sb->q_empty, 1);
     mbar_init(&sb->o_full, 1);
-    mbar_init(&sb->o_empty, 128);
-    mbar_init(&sb->sx_ready, 128);   // arrived by the peer's 128 softmax threads
-    mbar_init(&sb->sx_free, 128);
+    mbar_init(&sb->sx_ready, 128);   // arrived by the peer's 128 exchange threads
+    mbar_init(&sb->sx_free, 128);    // arrived by the peer's 128 softmax threads
     mbar_init(&sb->mma_done, 1);
     sb->abort = 0;
     fence_mbarrier_init();
-    tma_prefetch_desc(&maps.q_lat);
     tma_prefetch_desc(&maps.q_rope);
   }
   if (warp == kMmaWarp) {
@@ -208,12 +241,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = sb->tmem_base;
   volatile int* abort = &sb->abort;
-  const uint32_t o_col = 0, s_col = Lay::kPvN, p_col = Lay::kPvN + 2 * kRows;
 
-  pdl_wait_primary();  // the Top-K lists come from the previous kernel on the stream
+  // Only the gather warps read what the previous kernel on the stream (Top-K) writes; they wait
+  // for it below.  The query rows are inputs written before the previous kernels were launched.
+
+  // number of 64-row tiles of unit buffer `buf`: rows up to the first -1 entry of the list
+  auto unit_tiles = [&](int buf) {
+    int first_neg = 1 << 30;
+#pragma unroll
+    for (int w = 0; w < kProducerWarps; ++w) first_neg = min(first_neg, fneg_tab[buf * kProducerWarps + w]);
+    return first_neg;
+  };
 
   if (warp >= kFirstProducerWarp && warp < kFirstProducerWarp + kProducerWarps) {
-    // ---------------------------------------------------------------- gather (4 warps)
+    // ---------------------------------------------------------------- gather (8 warps)
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kGatherRegs));
     const int ptid = threadIdx.x - kFirstProducerWarp * 32;   // 0..255
     const int pwarp = warp - kFirstProducerWarp;
@@ -230,6 +271,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     };
     int it = 0, u_it = 0;
     bool ok = true;
+    bool waited = false;
+    if (cluster_id < p.units) {
+      // While the previous kernel still runs: touch every cache page of the first unit's
+      // sequence (address translation and the page-table row warm up before the gather)
+      const int b = (cluster_id / p.splits) / p.J;
+      const int L = p.seq_lens[b];
+      const int npages = min(p.max_pages, (L + p.P - 1) / p.P);
+      const int32_t* pt_row = p.page_table + (long long)b * p.max_pages;
+      const uint8_t* kv = static_cast<const uint8_t*>(p.kv);
+      for (int i = ptid; i < npages; i += kProducerWarps * 32) {
+        const int pg = pt_row[i];
+        if (pg >= 0 && pg < p.num_pages)
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(kv + ((size_t)pg * p.P * DC + (size_t)rank * (p.DL / 2)) * 2));
+      }
+    }
     for (int u = cluster_id; u < p.units && ok; u += n_clusters, ++u_it) {
       const int bj = u / p.splits, split = u - bj * p.splits;
       const int b = bj / p.J;
@@ -239,20 +295,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int nrows = min(p.K, row0 + p.rows_per_split) - row0;
       const int nrows_pad = (nrows + kRows - 1) / kRows * kRows;
       const int buf = u_it & 1;
-      // query rows of all heads (TMA; independent of the Top-K list)
+      // rope part of the query rows of all heads (TMA; independent of the Top-K list)
       if (ptid == 0) {
         if (mbar_wait(&sb->q_empty, ((uint32_t)u_it & 1u) ^ 1u, abort, p.status)) {
-          const uint32_t qbytes = Lay::kLatBlocks * Sm::kQLatBytes + (rope ? Sm::kQRopeBytes : 0);
-          mbar_arrive_expect_tx(&sb->q_full, qbytes);
-          const int y = bj * p.H;
-          for (int i = 0; i < Lay::kLatBlocks; ++i)
-            tma_load_2d(smem + Sm::kOffQ + i * Sm::kQLatBytes, &maps.q_lat, &sb->q_full, Lay::lat_x((int)rank, i), y);
-          if (rope)
-            tma_load_2d(smem + Sm::kOffQ + Lay::kLatBlocks * Sm::kQLatBytes, &maps.q_rope, &sb->q_full,
-                        Lay::rope_x((int)rank), y);
+          if (rope) {
+            mbar_arrive_expect_tx(&sb->q_full, Sm::kQRopeBytes);
+            tma_load_2d(smem + Sm::kOffQ, &maps.q_rope, &sb->q_full, Lay::rope_x((int)rank), bj * p.H);
+          } else {
+            mbar_arrive(&sb->q_full);
+          }
         }
       }
-      // resolve this unit's Top-K entries to physical cache rows: 16 entries per thread, all
+      if (!waited) {
+        pdl_wait_primary();  // the Top-K lists come from the previous kernel on the stream
+        waited = true;
+      }
+      // resolve this unit's Top-K entries to physical cache rows: 8 entries per thread, all
       // loads of a thread in flight at once
       if (!mbar_wait(&sb->tab_free[buf], ((uint32_t)(u_it >> 1) & 1u) ^ 1u, abort, p.status)) { ok = false; break; }
       int32_t* rt = rows_tab + buf * kAttnMaxSplitRows;
@@ -291,10 +349,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (lane == 0) fneg_tab[buf * kProducerWarps + pwarp] = fneg;
       mbar_arrive(&sb->tab_full[buf]);
       if (!mbar_wait(&sb->tab_full[buf], (uint32_t)(u_it >> 1) & 1u, abort, p.status)) { ok = false; break; }
-      int first_neg = nrows;
-#pragma unroll
-      for (int w = 0; w < kProducerWarps; ++w) first_neg = min(first_neg, fneg_tab[buf * kProducerWarps + w]);
-      const int ntiles = (first_neg + kRows - 1) / kRows;
+      const int ntiles = (unit_tiles(buf) + kRows - 1) / kRows;
       for (int t = 0; t < ntiles; ++t, ++it) {
         const int stage = it % kStages;
         if (!mbar_wait(&sb->c_empty[stage], ((uint32_t)(it / kStages) & 1u) ^ 1u, abort, p.status)) { ok = false; break; }
@@ -309,101 +364,128 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (ptid == 0 && u_it > 0) mbar_wait(&sb->q_full, (uint32_t)(u_it - 1) & 1u, abort, p.status);
   } else if (warp == kMmaWarp) {
     // ---------------------------------------------------------------- MMA issuer
+    // Two cursors over the same sequence of (unit, tile): S = Q . C^T of a tile can start as
+    // soon as its rows have landed and a logit buffer is free, O += P . C as soon as the
+    // softmax has written P.  The issuer polls both and issues whichever is ready, so neither
+    // product waits behind the other's inputs.
     if (lane == 0) {
       const uint32_t idesc_qk = umma_idesc(1, 1, false, false, kRows, 128);
       const uint32_t idesc_pv = umma_idesc(1, 1, false, true, Lay::kPvN, 128);
-      const uint32_t q_base = smem_u32(smem + Sm::kOffQ);
-      int it = 0, s_it = 0, pv_it = 0, u_it = 0;
+      const uint32_t qr_base = smem_u32(smem + Sm::kOffQ);
+      const uint32_t p_base = smem_u32(smem + Sm::kOffP);
+      int nt_ring[4];                       // tile counts of units the S cursor has opened
+      // S cursor: 0 = needs the unit's table, 1 = needs q, 2 = issuing tiles
+      int q_u = cluster_id, q_uit = 0, q_state = 0, q_nt = 0, q_t = 0, q_it = 0;
+      // P cursor
+      int p_u = cluster_id, p_uit = 0, p_t = 0, p_it = 0;
       bool ok = true;
-      for (int u = cluster_id; u < p.units && ok; u += n_clusters, ++u_it) {
-        const int buf = u_it & 1;
-        if (!mbar_wait(&sb->tab_full[buf], (uint32_t)(u_it >> 1) & 1u, abort, p.status)) { ok = false; break; }
-        int first_neg = 1 << 30;
-        for (int w = 0; w < kProducerWarps; ++w) first_neg = min(first_neg, fneg_tab[buf * kProducerWarps + w]);
-        const int ntiles = (first_neg + kRows - 1) / kRows;
-        if (!mbar_wait(&sb->q_full, (uint32_t)u_it & 1u, abort, p.status)) { ok = false; break; }
-        tc_fence_after();
-        bool o_claimed = false;
-        int prev_stage = -1;
-        for (int t = 0; t <= ntiles; ++t) {
-          if (t < ntiles) {
-            const int stage = it % kStages;
-            const int sbuf = s_it & 1;
-            if (!mbar_wait(&sb->c_full[stage], (uint32_t)(it / kStages) & 1u, abort, p.status)) { ok = false; break; }
-            if (!mbar_wait(&sb->s_empty[sbuf], ((uint32_t)(s_it >> 1) & 1u) ^ 1u, abort, p.status)) { ok = false; break; }
-            fence_proxy_async_smem();   // the gathered rows were written by cp.async
-            tc_fence_after();
-            const uint32_t c_base = smem_u32(smem + Sm::kOffC + stage * Sm::kCStageBytes);
-            const uint32_t d = tmem_base + s_col + (uint32_t)(sbuf * kRows);
-            bool acc = false;
-#pragma unroll
-            for (int i = 0; i < Lay::kLatBlocks; ++i)
-#pragma unroll
-              for (int ks = 0; ks < Lay::kLatKbw / 32; ++ks) {
-                const uint64_t ad = umma_smem_desc(q_base + i * Sm::kQLatBytes + ks * 32, 16,
-                                                   8 * Lay::kLatKbw, umma_layout_type(Lay::kLatKbw));
-                const uint64_t bd = umma_smem_desc(c_base + i * Sm::kCLatBytes + ks * 32, 16,
-                                                   8 * Lay::kLatKbw, umma_layout_type(Lay::kLatKbw));
-                umma_f16(d, ad, bd, idesc_qk, acc);
-                acc = true;
-              }
-            if (rope) {
-#pragma unroll
-              for (int ks = 0; ks < Lay::kRopeKbw / 32; ++ks) {
-                const uint64_t ad = umma_smem_desc(q_base + Lay::kLatBlocks * Sm::kQLatBytes + ks * 32, 16,
-                                                   8 * Lay::kRopeKbw, umma_layout_type(Lay::kRopeKbw));
-                const uint64_t bd = umma_smem_desc(c_base + Lay::kLatBlocks * Sm::kCLatBytes + ks * 32, 16,
-                                                   8 * Lay::kRopeKbw, umma_layout_type(Lay::kRopeKbw));
-                umma_f16(d, ad, bd, idesc_qk, true);
-              }
-            }
-            umma_commit(&sb->s_full[sbuf]);
-            if (t + 1 == ntiles) umma_commit(&sb->q_empty);  // Q reusable once these are done
+      uint64_t last = globaltimer_ns();
+      while (ok && (q_u < p.units || p_u < p.units)) {
+        bool progress = false;
+        if (q_u < p.units) {
+          const int buf = q_uit & 1;
+          if (q_state == 0 && mbar_test(&sb->tab_full[buf], (uint32_t)(q_uit >> 1) & 1u)) {
+            q_nt = (unit_tiles(buf) + kRows - 1) / kRows;
+            nt_ring[q_uit & 3] = q_nt;
+            mbar_arrive(&sb->tab_free[buf]);
+            q_state = 1;
+            progress = true;
           }
-          if (t > 0) {
-            // O += P . C for the previous tile, with P (bf16) read straight from TMEM
-            const int pb = pv_it & 1;
-            if (!mbar_wait(&sb->p_full[pb], (uint32_t)(pv_it >> 1) & 1u, abort, p.status)) { ok = false; break; }
-            if (!o_claimed) {
-              if (!mbar_wait(&sb->o_empty, ((uint32_t)u_it & 1u) ^ 1u, abort, p.status)) { ok = false; break; }
-              o_claimed = true;
-            }
+          if (q_state == 1 && mbar_test(&sb->q_full, (uint32_t)q_uit & 1u)) {
             tc_fence_after();
-            const uint32_t c_base = smem_u32(smem + Sm::kOffC + prev_stage * Sm::kCStageBytes);
+            q_state = 2;
+            q_t = 0;
+            progress = true;
+          }
+          if (q_state == 2 && q_t < q_nt) {
+            const int stage = q_it % kStages;
+            const int sbuf = q_it & 1;
+            if (mbar_test(&sb->c_full[stage], (uint32_t)(q_it / kStages) & 1u) &&
+                mbar_test(&sb->s_empty[sbuf], ((uint32_t)(q_it >> 1) & 1u) ^ 1u)) {
+              fence_proxy_async_smem();   // the gathered rows were written by cp.async
+              tc_fence_after();
+              const uint32_t c_base = smem_u32(smem + Sm::kOffC + stage * Sm::kCStageBytes);
+              const uint32_t d = tmem_base + Tm::kS + (uint32_t)(sbuf * kRows);
+              constexpr int kSub = Lay::kLatKbw / 32;   // 16-element K steps per swizzled block
+#pragma unroll
+              for (int g = 0; g < Lay::kLatDims / 16; ++g) {
+                const uint64_t bd = umma_smem_desc(c_base + (g / kSub) * Sm::kCLatBytes + (g % kSub) * 32, 16,
+                                                   8 * Lay::kLatKbw, umma_layout_type(Lay::kLatKbw));
+                umma_f16_ts(d, tmem_base + Tm::kQ + (uint32_t)(8 * g), bd, idesc_qk, g > 0);
+              }
+              if (rope) {
+#pragma unroll
+                for (int ks = 0; ks < Lay::kRopeKbw / 32; ++ks) {
+                  const uint64_t ad = umma_smem_desc(qr_base + ks * 32, 16, 8 * Lay::kRopeKbw, umma_layout_type(Lay::kRopeKbw));
+                  const uint64_t bd = umma_smem_desc(c_base + Lay::kLatBlocks * Sm::kCLatBytes + ks * 32, 16,
+                                                     8 * Lay::kRopeKbw, umma_layout_type(Lay::kRopeKbw));
+                  umma_f16(d, ad, bd, idesc_qk, true);
+                }
+              }
+              umma_commit(&sb->s_full[sbuf]);
+              ++q_it;
+              ++q_t;
+              progress = true;
+            }
+          }
+          if (q_state == 2 && q_t == q_nt) {
+            umma_commit(&sb->q_empty);  // q reusable once this unit's products are done
+            q_u += n_clusters;
+            ++q_uit;
+            q_state = 0;
+            progress = true;
+          }
+        }
+        if (p_u < p.units && p_uit < q_uit + (q_state > 0 ? 1 : 0)) {
+          const int nt = nt_ring[p_uit & 3];
+          if (p_t < nt && mbar_test(&sb->p_full, (uint32_t)p_it & 1u)) {
+            fence_proxy_async_smem();   // the row stage (cp.async) and P (st.shared)
+            tc_fence_after();
+            const int stage = p_it % kStages;
+            const uint32_t c_base = smem_u32(smem + Sm::kOffC + stage * Sm::kCStageBytes);
 #pragma unroll
             for (int ks = 0; ks < kRows / 16; ++ks) {
+              const uint64_t ad = umma_smem_desc(p_base + ks * 32, 16, 1024, umma_layout_type(128));
               const uint64_t bd = umma_smem_desc(c_base + ks * 16 * Lay::kLatKbw, Sm::kCLatBytes,
                                                  8 * Lay::kLatKbw, umma_layout_type(Lay::kLatKbw));
-              umma_f16_ts(tmem_base + o_col, tmem_base + p_col + (uint32_t)(pb * (kRows / 2) + ks * 8), bd,
-                          idesc_pv, (t > 1) || ks > 0);
+              umma_f16(tmem_base + Tm::kO, ad, bd, idesc_pv, p_t > 0 || ks > 0);
             }
-            umma_commit(&sb->c_empty[prev_stage]);
-            umma_commit(&sb->p_empty[pb]);
-            ++pv_it;
+            umma_commit(&sb->c_empty[stage]);
+            umma_commit(&sb->p_empty);
+            ++p_it;
+            ++p_t;
+            if (p_t == nt) umma_commit(&sb->o_full);
+            progress = true;
           }
-          if (t < ntiles) {
-            prev_stage = it % kStages;
-            ++it;
-            ++s_it;
+          if (p_t == nt) {
+            p_u += n_clusters;
+            ++p_uit;
+            p_t = 0;
+            progress = true;
           }
         }
-        if (!ok) break;
-        if (ntiles == 0) umma_commit(&sb->q_empty);
-        if (!o_claimed) {
-          if (!mbar_wait(&sb->o_empty, ((uint32_t)u_it & 1u) ^ 1u, abort, p.status)) { ok = false; break; }
+        if (progress) {
+          last = globaltimer_ns();
+        } else {
+          if (*abort) { ok = false; break; }
+          if (globaltimer_ns() - last > kWaitTimeoutNs) {
+            *abort = 1;
+            report(p.status, SIA_DEV_TIMEOUT);
+            ok = false;
+            break;
+          }
         }
-        umma_commit(&sb->o_full);
       }
       umma_commit(&sb->mma_done);
       mbar_wait(&sb->mma_done, 0, abort, p.status);
     }
     __syncwarp();
   } else if (warp >= kFirstExchangeWarp && warp < kFirstExchangeWarp + 4) {
-    // ---------------------------------------------------------------- partial-logit exchange
-    // Reads this CTA's partial logits of a tile from TMEM, rounds them to fp16 (scaled to base
-    // 2) and pushes them into the peer CTA's exchange buffer; the peer's softmax warps add them
-    // to their own partials.  Both CTAs add the same two fp16 values, so their softmax inputs
-    // agree bit for bit.
+    // ---------------------------------------------------------------- q loader + exchange
+    // Per unit: writes this CTA's latent half of every head's query row into TMEM (the A
+    // operand of Q . C^T).  Per tile: reads this CTA's partial logits from TMEM, rounds them
+    // to fp16 (scaled to base 2) and pushes them into the peer CTA's exchange buffer.
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kExchangeRegs));
     const int quad = warp & 3;
     const int h = quad * 32 + lane;
     const uint32_t lane_addr = tmem_base + ((uint32_t)(quad * 32) << 16);
@@ -411,14 +493,39 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     int s_it = 0, u_it = 0;
     bool ok = true;
     for (int u = cluster_id; u < p.units && ok; u += n_clusters, ++u_it) {
+      const int bj = u / p.splits;
       const int buf = u_it & 1;
+      {
+        // q: head h's dims [rank * kLatDims, +kLatDims) as bf16 pairs, 16 columns per store
+        if (!mbar_wait(&sb->q_empty, ((uint32_t)u_it & 1u) ^ 1u, abort, p.status)) { ok = false; break; }
+        const bool real = h < p.H;
+        const uint8_t* qrow = static_cast<const uint8_t*>(p.q) + ((long long)bj * p.H + (real ? h : 0)) * (DC * 2) +
+                              (size_t)rank * Lay::kLatDims * 2;
+        constexpr int kGroups = Lay::kLatDims / 32;   // 64 bytes = 16 columns each
+        tc_fence_after();
+#pragma unroll 1
+        for (int g = 0; g < kGroups; ++g) {
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint4 v = real ? ld_nc_v4(qrow + g * 64 + 16 * i) : make_uint4(0, 0, 0, 0);
+            w[4 * i] = v.x;
+            w[4 * i + 1] = v.y;
+            w[4 * i + 2] = v.z;
+            w[4 * i + 3] = v.w;
+          }
+          tmem_st16(lane_addr + Tm::kQ + (uint32_t)(16 * g), w);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&sb->q_full);
+      }
       if (!mbar_wait(&sb->tab_full[buf], (uint32_t)(u_it >> 1) & 1u, abort, p.status)) { ok = false; break; }
-      int first_neg = 1 << 30;
-      for (int w = 0; w < kProducerWarps; ++w) first_neg = min(first_neg, fneg_tab[buf * kProducerWarps + w]);
-      const int ntiles = (first_neg + kRows - 1) / kRows;
+      const int ntiles = (unit_tiles(buf) + kRows - 1) / kRows;
+      mbar_arrive(&sb->tab_free[buf]);
       for (int t = 0; t < ntiles; ++t, ++s_it) {
         const int sbuf = s_it & 1;
-        const uint32_t scol = lane_addr + s_col + sbuf * kRows;
+        const uint32_t scol = lane_addr + Tm::kS + sbuf * kRows;
         if (!mbar_wait(&sb->s_full[sbuf], (uint32_t)(s_it >> 1) & 1u, abort, p.status)) { ok = false; break; }
         tc_fence_after();
         uint32_t own[kRows / 2];
@@ -435,6 +542,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               own[half * 16 + c * 8 + i] = pack_f16x2(__uint_as_float(r[c][2 * i]) * p.scale_log2,
                                                       __uint_as_float(r[c][2 * i + 1]) * p.scale_log2);
         }
+        tc_fence_before();
+        mbar_arrive(&sb->s_empty[sbuf]);   // our reads of these logits are done
         if (!mbar_wait<true>(&sb->sx_free, ((uint32_t)s_it & 1u) ^ 1u, abort, p.status)) { ok = false; break; }
 #pragma unroll
         for (int g = 0; g < kRows / 8; ++g)
@@ -450,31 +559,33 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int quad = warp & 3;
     const int h = quad * 32 + lane;   // head = TMEM lane
     const uint32_t lane_addr = tmem_base + ((uint32_t)(quad * 32) << 16);
-    int s_it = 0, pv_it = 0, u_it = 0;
+    int s_it = 0, u_it = 0, o_it = 0, e_it = 0;
     bool ok = true;
 
     for (int u = cluster_id; u < p.units && ok; u += n_clusters, ++u_it) {
       const int bj = u / p.splits, split = u - bj * p.splits;
       const int buf = u_it & 1;
       if (!mbar_wait(&sb->tab_full[buf], (uint32_t)(u_it >> 1) & 1u, abort, p.status)) { ok = false; break; }
-      int first_neg = 1 << 30;
-      for (int w = 0; w < kProducerWarps; ++w) first_neg = min(first_neg, fneg_tab[buf * kProducerWarps + w]);
+      const int first_neg = unit_tiles(buf);
       const int ntiles = (first_neg + kRows - 1) / kRows;
       const uint32_t* mt = mask_tab + buf * (kAttnMaxSplitRows / 32);
       float m = -INFINITY, l = 0.0f;
       float s[kRows];
-      for (int t = 0; t < ntiles; ++t, ++pv_it) {
-        // logits of tile t (base 2) = own partial (TMEM) + the peer's partial (exchange buffer),
-        // each rounded to fp16 exactly as the exchange warps of both CTAs round them
+      for (int t = 0; t < ntiles; ++t, ++s_it) {
+        // logits of tile t (base 2) = own fp32 partial (TMEM) + the peer's fp16 partial
         const int sbuf = s_it & 1;
+        const uint32_t scol = lane_addr + Tm::kS + sbuf * kRows;
+        uint64_t valid = ((uint64_t)mt[2 * t + 1] << 32) | mt[2 * t];
+        const int live = first_neg - t * kRows;            // rows past the first -1 are padding
+        if (live < kRows) valid &= (1ull << live) - 1ull;
         if (!mbar_wait(&sb->s_full[sbuf], (uint32_t)(s_it >> 1) & 1u, abort, p.status)) { ok = false; break; }
         if (!mbar_wait<true>(&sb->sx_ready, (uint32_t)s_it & 1u, abort, p.status)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           uint32_t r[2][16];
-          tmem_ld16(lane_addr + s_col + sbuf * kRows + half * 32, r[0]);
-          tmem_ld16(lane_addr + s_col + sbuf * kRows + half * 32 + 16, r[1]);
+          tmem_ld16(scol + half * 32, r[0]);
+          tmem_ld16(scol + half * 32 + 16, r[1]);
           tmem_wait_ld();
 #pragma unroll
           for (int g2 = 0; g2 < 4; ++g2) {
@@ -484,125 +595,143 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const int col = g2 * 8 + 2 * i;
-              const float2 a = unpack_f16x2(pack_f16x2(__uint_as_float(r[col >> 4][col & 15]) * p.scale_log2,
-                                                       __uint_as_float(r[col >> 4][(col & 15) + 1]) * p.scale_log2));
-              const float2 c = unpack_f16x2(pv[i]);
-              s[8 * g + 2 * i] = a.x + c.x;
-              s[8 * g + 2 * i + 1] = a.y + c.y;
+              float lo = __uint_as_float(r[col >> 4][col & 15]) * p.scale_log2;
+              float hi = __uint_as_float(r[col >> 4][(col & 15) + 1]) * p.scale_log2;
+              add_f16x2_to_f32(pv[i], lo, hi);
+              s[8 * g + 2 * i] = lo;
+              s[8 * g + 2 * i + 1] = hi;
             }
           }
         }
         tc_fence_before();
         mbar_arrive(&sb->s_empty[sbuf]);
-        mbar_arrive_cluster(&sb->sx_free, peer);
-        ++s_it;
-        uint64_t valid = ((uint64_t)mt[2 * t + 1] << 32) | mt[2 * t];
-        const int live = first_neg - t * kRows;            // rows past the first -1 are padding
-        if (live < kRows) valid &= (1ull << live) - 1ull;
+        // the peer may refill the exchange buffer (the logit values read above are already in
+        // registers); after the unit's last tile the buffer first serves the epilogue
+        if (t + 1 < ntiles) mbar_arrive_cluster_relaxed(&sb->sx_free, peer);
 
         // online softmax (base 2), lazy rescale
-        float mt_ = -INFINITY;
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        if (valid == ~0ull) {
 #pragma unroll
-        for (int i = 0; i < kRows; ++i) {
-          s[i] = (valid >> i & 1ull) ? s[i] : -INFINITY;
-          mt_ = fmaxf(mt_, s[i]);
+          for (int i = 0; i < kRows; ++i) mx[i & 3] = fmaxf(mx[i & 3], s[i]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < kRows; ++i) {
+            s[i] = (valid >> i & 1ull) ? s[i] : -INFINITY;
+            mx[i & 3] = fmaxf(mx[i & 3], s[i]);
+          }
         }
+        const float mt_ = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
         float alpha = 1.0f;
         const bool need = mt_ > m + 8.0f;
         if (need) {
           alpha = fast_exp2(m - mt_);   // 0 when m is -inf
           m = mt_;
         }
-        float psum = 0.0f;
+        float ps[4] = {0.f, 0.f, 0.f, 0.f};
+        if (m != -INFINITY) {
+          // masked logits are -inf and m is finite: their exp2 is exactly 0
 #pragma unroll
-        for (int i = 0; i < kRows; ++i) {
-          s[i] = (valid >> i & 1ull) ? fast_exp2(s[i] - m) : 0.0f;
-          psum += s[i];
+          for (int i = 0; i < kRows; ++i) {
+            s[i] = fast_exp2(s[i] - m);
+            ps[i & 3] += s[i];
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < kRows; ++i) s[i] = 0.0f;
         }
-        l = l * alpha + psum;
+        l = l * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
 
-        const int pb = pv_it & 1;
+        // P . C of the previous tile must be done: it reads the P buffer, and O is rescaled
+        if (!mbar_wait(&sb->p_empty, ((uint32_t)s_it & 1u) ^ 1u, abort, p.status)) { ok = false; break; }
+        tc_fence_after();
         if (__any_sync(0xffffffffu, need && t > 0)) {
-          // O holds tiles < t of this unit once P . C of tile t-1 is done: rescale it
-          const int prev = pv_it - 1;
-          if (!mbar_wait(&sb->p_empty[prev & 1], (uint32_t)(prev >> 1) & 1u, abort, p.status)) { ok = false; break; }
-          tc_fence_after();
+          // O holds the tiles < t of this unit: rescale it
 #pragma unroll 1
           for (int c = 0; c < Lay::kPvN; c += 16) {
             uint32_t r[16];
-            tmem_ld16(lane_addr + o_col + c, r);
+            tmem_ld16(lane_addr + Tm::kO + c, r);
             tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-            tmem_st16(lane_addr + o_col + c, r);
+            tmem_st16(lane_addr + Tm::kO + c, r);
           }
           tmem_wait_st();
         }
-        // the P buffer of tile t-2 must have been consumed by its P . C
-        if (!mbar_wait(&sb->p_empty[pb], ((uint32_t)(pv_it >> 1) & 1u) ^ 1u, abort, p.status)) { ok = false; break; }
-        tc_fence_after();
+        // P (bf16) into shared memory: this head's row of kRows values, 128B-swizzled
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t w[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(s[32 * half + 2 * i], s[32 * half + 2 * i + 1]);
-          tmem_st16(lane_addr + p_col + pb * (kRows / 2) + 16 * half, w);
-        }
-        tmem_wait_st();
+        for (int k = 0; k < kRows / 8; ++k)
+          st_shared_v4(smem_u32(smem + Sm::kOffP + swizzled_offset((uint32_t)h, (uint32_t)k * 16, 128)),
+                       pack_bf16x2(s[8 * k], s[8 * k + 1]), pack_bf16x2(s[8 * k + 2], s[8 * k + 3]),
+                       pack_bf16x2(s[8 * k + 4], s[8 * k + 5]), pack_bf16x2(s[8 * k + 6], s[8 * k + 7]));
+        fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(&sb->p_full[pb]);
+        mbar_arrive(&sb->p_full);   // P written (and O rescaled) by this thread
       }
       if (!ok) break;
       mbar_arrive(&sb->tab_free[buf]);
       // ---- unit epilogue: normalise O and write it out
-      if (!mbar_wait(&sb->o_full, (uint32_t)u_it & 1u, abort, p.status)) { ok = false; break; }
+      if (ntiles > 0) {
+        if (!mbar_wait(&sb->o_full, (uint32_t)o_it & 1u, abort, p.status)) { ok = false; break; }
+        ++o_it;
+      }
       tc_fence_after();
       const bool any = ntiles > 0 && l > 0.0f;
       const float inv = any ? 1.0f / l : 0.0f;
       const float lse = any ? (m + log2f(l)) * 0.69314718055994530942f : -INFINITY;
       const bool real_head = h < p.H;
-      if (p.splits == 1) {
-        uint16_t* orow = p.out + ((long long)bj * p.H + h) * p.DL + rank * Lay::kPvN;
+      // O rows (bf16: the output, or a split's normalised partial) go out through the exchange
+      // buffer (free until the deferred sx_free below): each warp stages 32 heads x 128 bytes
+      // per round in a 128B-swizzled 4 KB slice, then writes whole 128-byte runs of 4 heads per
+      // instruction
+      uint16_t* obase = (p.splits > 1 ? p.part_o + ((long long)split * p.B * p.J + bj) * p.H * p.DL
+                                      : p.out + (long long)bj * p.H * p.DL) + rank * Lay::kPvN;
+      if (ntiles > 0) {
+        // every softmax warp has read the last tile's peer logits before any slice is reused
+        mbar_arrive(&sb->epi_sync);
+        if (!mbar_wait(&sb->epi_sync, (uint32_t)e_it & 1u, abort, p.status)) { ok = false; break; }
+        ++e_it;
+        uint8_t* slice = smem + Sm::kOffSx + quad * 4096;
 #pragma unroll 1
-        for (int c = 0; c < Lay::kPvN; c += 16) {
-          uint32_t r[16];
-          if (ntiles > 0) {
-            tmem_ld16(lane_addr + o_col + c, r);
-            tmem_wait_ld();
-          }
-          uint32_t w[8];
+        for (int c = 0; c < Lay::kPvN; c += 64) {
+          uint32_t w[32];
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            w[i] = ntiles > 0 ? pack_bf16x2(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv) : 0u;
-          if (real_head) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + c);
-            dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-            dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+          for (int q = 0; q < 4; ++q) {
+            uint32_t r[16];
+            tmem_ld16(lane_addr + Tm::kO + c + 16 * q, r);   // past kPvN: other columns, not stored
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              w[8 * q + i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
+          }
+          __syncwarp();
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            st_shared_v4(smem_u32(slice + lane * 128 + ((k ^ (lane & 7)) * 16)), w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+          __syncwarp();
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const int r = 4 * k + (lane >> 3), blk = lane & 7;
+            const int head = quad * 32 + r;
+            const uint4 v = *reinterpret_cast<const uint4*>(slice + r * 128 + ((blk ^ (r & 7)) * 16));
+            if (head < p.H && c + 8 * blk < Lay::kPvN)
+              *reinterpret_cast<uint4*>(obase + (long long)head * p.DL + c + 8 * blk) = v;
           }
         }
-        if (real_head && rank == 0 && p.lse) p.lse[(long long)bj * p.H + h] = lse;
-      } else {
-        float* orow = p.part_o + (((long long)split * p.B * p.J + bj) * p.H + h) * p.DL + rank * Lay::kPvN;
-#pragma unroll 1
-        for (int c = 0; c < Lay::kPvN; c += 16) {
-          uint32_t r[16];
-          if (ntiles > 0) {
-            tmem_ld16(lane_addr + o_col + c, r);
-            tmem_wait_ld();
-          }
-          if (real_head) {
-            float4* dst = reinterpret_cast<float4*>(orow + c);
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-              dst[i] = ntiles > 0 ? make_float4(__uint_as_float(r[4 * i]) * inv, __uint_as_float(r[4 * i + 1]) * inv,
-                                                __uint_as_float(r[4 * i + 2]) * inv, __uint_as_float(r[4 * i + 3]) * inv)
-                                  : make_float4(0.f, 0.f, 0.f, 0.f);
-          }
-        }
-        if (real_head && rank == 0) p.part_lse[((long long)split * p.B * p.J + bj) * p.H + h] = lse;
+      } else if (real_head) {
+        // empty list: zeros (the exchange buffer may already hold the peer's next logits)
+        for (int c = 0; c < Lay::kPvN; c += 8)
+          *reinterpret_cast<uint4*>(obase + (long long)h * p.DL + c) = make_uint4(0, 0, 0, 0);
       }
-      tc_fence_before();
-      mbar_arrive(&sb->o_empty);
+      if (real_head && rank == 0) {
+        if (p.splits > 1) p.part_lse[((long long)split * p.B * p.J + bj) * p.H + h] = lse;
+        else if (p.lse) p.lse[(long long)bj * p.H + h] = lse;
+      }
+      if (ntiles > 0) {
+        __syncwarp();
+        mbar_arrive_cluster_relaxed(&sb->sx_free, peer);   // deferred from the unit's last tile
+      }
+      tc_fence_before();   // our reads of O come before the next unit's first P . C
     }
   }
   pdl_launch_dependents();
@@ -630,11 +759,11 @@ __global__ void __launch_bounds__(128) combine_kernel(const CombineKernelParams 
       for (int s = 0; s < p.splits; ++s) {
         const float ls = p.part_lse[s * stride_lse + bjh];
         const float wgt = ls == -INFINITY ? 0.0f : expf(ls - mx);
-        const float4 v = *reinterpret_cast<const float4*>(p.part_o + (s * stride_lse + bjh) * p.DL + d4);
-        o0 += wgt * v.x;
-        o1 += wgt * v.y;
-        o2 += wgt * v.z;
-        o3 += wgt * v.w;
+        const uint2 v = *reinterpret_cast<const uint2*>(p.part_o + (s * stride_lse + bjh) * p.DL + d4);
+        o0 += wgt * __uint_as_float(v.x << 16);
+        o1 += wgt * __uint_as_float(v.x & 0xffff0000u);
+        o2 += wgt * __uint_as_float(v.y << 16);
+        o3 += wgt * __uint_as_float(v.y & 0xffff0000u);
         wsum += wgt;
       }
     }
@@ -663,10 +792,7 @@ cudaError_t launch_attend_impl(const AttnKernelParams& p, const CUtensorMap* map
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   AttnMaps m;
-  m.q_lat = maps[0];
   m.q_rope = maps[1];
-  m.kv_lat = maps[2];
-  m.kv_rope = maps[3];
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[2];
   cfg.gridDim = dim3(2 * n_clusters, 1, 1);

@@ -265,6 +265,9 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_row_kernel(const TopkKern
   int32_t* out = p.topk + row * p.K;
 
   pdl_wait_primary();  // scores come from the previous kernel on the stream
+  // the next kernel (attention) may be scheduled now: it only reads our output after its own
+  // griddepcontrol.wait, which waits for this whole grid to finish
+  pdl_launch_dependents();
 
   bool bad = false;
   const int pos = query_position(p.seq_lens, p.q_pos, p.J, b, j, p.Lpad, &bad);
@@ -272,7 +275,6 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_row_kernel(const TopkKern
   const int n = pos + 1;
   if (n <= p.K) {
     for (int i = tid; i < p.K; i += kRowThreads) out[i] = i < n ? i : -1;
-    pdl_launch_dependents();
     return;
   }
   // this thread's keys: positions [tid*16, tid*16+16) of the visible range
@@ -351,7 +353,6 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_row_kernel(const TopkKern
       ++eq_before;
     }
   }
-  pdl_launch_dependents();
 }
 
 }  // namespace
