@@ -69,7 +69,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkKernelP
   extern __shared__ __align__(16) uint8_t smem[];
   TopkShared* sh = reinterpret_cast<TopkShared*>(smem);
   uint32_t* keys = reinterpret_cast<uint32_t*>(smem + sizeof(TopkShared));
-  const int tid = threadIdx.x, lane = tid & 31;
+  const int tid = threadIdx.x;
   const uint32_t rank = cluster_ctarank();
   const int C = p.cluster;
   const long long row = blockIdx.x / C;
@@ -110,14 +110,13 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkKernelP
     const int rounds = (len + kTopkThreads - 1) / kTopkThreads;
     for (int r = 0; r < rounds; ++r) {
       const int i = r * kTopkThreads + tid;
-      uint32_t digit = 0xffffffffu;
       if (i < len) {
+        // plain shared-memory atomics: on sm_100a they absorb same-bin conflicts far faster
+        // than a warp-level __match_any_sync aggregation (measured 1.9k vs 8k-33k cycles per
+        // 16k-key pass, growing with the number of distinct bins)
         const uint32_t k = keys[i];
-        const bool match = pass == 0 || (k >> hi_shift) == prefix;
-        if (match) digit = (k >> sh_) & dmask;
+        if (pass == 0 || (k >> hi_shift) == prefix) atomicAdd(&h[(k >> sh_) & dmask], 1u);
       }
-      const unsigned same = __match_any_sync(0xffffffffu, digit);
-      if (digit != 0xffffffffu && lane == __ffs(same) - 1) atomicAdd(&h[digit], (uint32_t)__popc(same));
     }
     // make every CTA's histogram visible cluster-wide, then sum them
     cluster_sync();
@@ -259,7 +258,7 @@ __device__ __forceinline__ void row_scan2(int a, int b, int& ea, int& eb, int& t
 __global__ void __launch_bounds__(kRowThreads, 1) topk_row_kernel(const TopkKernelParams p) {
   __shared__ RowShared shm;
   RowShared* sh = &shm;
-  const int tid = threadIdx.x, lane = tid & 31;
+  const int tid = threadIdx.x;
   const long long row = blockIdx.x;
   const int b = (int)(row / p.J), j = (int)(row - (long long)b * p.J);
   int32_t* out = p.topk + row * p.K;
@@ -307,12 +306,8 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_row_kernel(const TopkKern
     const int sh_ = shifts[pass], hi_shift = sh_ + widths[pass];
     const uint32_t dmask = (1u << widths[pass]) - 1u;
 #pragma unroll
-    for (int i = 0; i < kRowPer; ++i) {
-      uint32_t digit = 0xffffffffu;
-      if (i < nmine && (pass == 0 || (key[i] >> hi_shift) == prefix)) digit = (key[i] >> sh_) & dmask;
-      const unsigned same = __match_any_sync(0xffffffffu, digit);
-      if (digit != 0xffffffffu && lane == __ffs(same) - 1) atomicAdd(&sh->hist[digit], (uint32_t)__popc(same));
-    }
+    for (int i = 0; i < kRowPer; ++i)
+      if (i < nmine && (pass == 0 || (key[i] >> hi_shift) == prefix)) atomicAdd(&sh->hist[(key[i] >> sh_) & dmask], 1u);
     __syncthreads();
     // thread t owns bins 2t, 2t+1; "above" = keys in higher bins, via a scan in reversed order
     const int hi_bin = kBins - 2 - 2 * tid;        // reversed: thread 0 owns the two top bins
