@@ -113,7 +113,10 @@ __device__ void locate_start(const IndexKernelParams& p, IndexBarriers* sb) {
   }
 }
 
-template <int NSUB>
+// KBW (64 or 128 bytes per K-block row), NKB (K blocks per row) and FP8 are compile-time so
+// that the MMA issue loop is fully unrolled with constant descriptors: with runtime trip counts
+// each tcgen05.mma took about three times longer to issue.
+template <int NSUB, int KBW, int NKB, bool FP8>
 __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
     index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexKernelParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -199,16 +202,17 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
           // per-token key scales of the tile, copied next to the K tile
           *reinterpret_cast<uint32_t*>(info) = valid_mask;
           const uint32_t bytes =
-              (uint32_t)__popc(valid_mask) * (p.n_kblocks * p.box_rows * p.kbw + scale_bytes);
+              (uint32_t)__popc(valid_mask) * (NKB * p.box_rows * KBW + scale_bytes);
           mbar_arrive_expect_tx(&sb->k_full[stage], bytes);
         }
         for (int c = 0; c < chunks; ++c) {   // warp-uniform trip count
           const int page = __shfl_sync(0xffffffffu, my_page, c);
           if (lane == 0 && (valid_mask >> c & 1u)) {
             const int y = page * p.P + ((tile_pos0 + c * p.box_rows) % p.P);
-            for (int kb = 0; kb < p.n_kblocks; ++kb)
-              tma_load_2d(kst + kb * p.k_kblock_bytes + c * p.box_rows * p.kbw, &kmap,
-                          &sb->k_full[stage], kb * p.kbw / (p.fp8 ? 1 : 2), y);
+#pragma unroll
+            for (int kb = 0; kb < NKB; ++kb)
+              tma_load_2d(kst + kb * p.k_kblock_bytes + c * p.box_rows * KBW, &kmap,
+                          &sb->k_full[stage], kb * KBW / (FP8 ? 1 : 2), y);
             if (p.k_scale)
               bulk_load(info + 16 + c * p.box_rows * 4, p.k_scale + (long long)y, scale_bytes,
                         &sb->k_full[stage]);
@@ -229,10 +233,11 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = p.fp8 ? umma_idesc(0, 0, false, false, p.n_cols, 128)
-                                   : umma_idesc(1, 1, false, false, p.n_cols, 128);
-      const uint32_t layout = umma_layout_type(p.kbw);
-      const uint32_t sbo = 8 * p.kbw;
+      const uint32_t idesc = FP8 ? umma_idesc(0, 0, false, false, p.n_cols, 128)
+                                 : umma_idesc(1, 1, false, false, p.n_cols, 128);
+      constexpr uint32_t layout = umma_layout_type(KBW);
+      constexpr uint32_t sbo = 8 * KBW;
+      constexpr uint32_t a_kblock = kIndexTileRows * KBW;
       int it = 0, acc_it = 0, seg = 0;
       int item = start_item, t0 = start_tile, remaining = my_count;
       bool ok = true;
@@ -257,15 +262,15 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
               tc_fence_after();
               const uint32_t d_tmem = tmem_base + (uint32_t)((as * NSUB + sub) * p.n_cols);
               const uint32_t b_base = smem_u32(smem + p.off_q + sub * p.q_sub_bytes);
-              for (int kb = 0; kb < p.n_kblocks; ++kb)
-                for (int ks = 0; ks < p.ksteps_per_block; ++ks) {
-                  const uint64_t ad =
-                      umma_smem_desc(a_base + kb * p.k_kblock_bytes + ks * 32, 16, sbo, layout);
-                  const uint64_t bd =
-                      umma_smem_desc(b_base + kb * p.q_kblock_bytes + ks * 32, 16, sbo, layout);
-                  const bool acc = (kb | ks) != 0;
-                  if (p.fp8) umma_f8(d_tmem, ad, bd, idesc, acc);
-                  else umma_f16(d_tmem, ad, bd, idesc, acc);
+              const uint32_t q_kblock = p.q_kblock_bytes;
+#pragma unroll
+              for (int kb = 0; kb < NKB; ++kb)
+#pragma unroll
+                for (int ks = 0; ks < KBW / 32; ++ks) {
+                  const uint64_t ad = umma_smem_desc(a_base + kb * a_kblock + ks * 32, 16, sbo, layout);
+                  const uint64_t bd = umma_smem_desc(b_base + kb * q_kblock + ks * 32, 16, sbo, layout);
+                  if (FP8) umma_f8(d_tmem, ad, bd, idesc, (kb | ks) != 0);
+                  else umma_f16(d_tmem, ad, bd, idesc, (kb | ks) != 0);
                 }
               umma_commit(&sb->acc_full[as][sub]);
             }
@@ -305,23 +310,23 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
         float* w_s = reinterpret_cast<float*>(smem + p.off_w) + (seg & 1) * w_words;
         int* info_pos = reinterpret_cast<int*>(smem + p.off_info) + (seg & 1) * 16;
         float* info_qs = reinterpret_cast<float*>(smem + p.off_info + 128) + (seg & 1) * 16;
-        const int chunks16 = p.kbw / 16;
-        const int total16 = NSUB * p.n_kblocks * p.n_cols * chunks16;
+        constexpr int chunks16 = KBW / 16;
+        const int total16 = NSUB * NKB * p.n_cols * chunks16;
         for (int i = et; i < total16; i += kEpiThreads) {
           const int c16 = i % chunks16;
           int r = i / chunks16;
           const int rr = r % p.n_cols;
           r /= p.n_cols;
-          const int kb = r % p.n_kblocks;
-          const int sb_ = r / p.n_kblocks;
+          const int kb = r % NKB;
+          const int sb_ = r / NKB;
           const int ql = rr / p.HP, h = rr - ql * p.HP;
           const int j = gi.g * p.qg + sb_ * p.nq_sub + ql;
           uint4 v = make_uint4(0u, 0u, 0u, 0u);
           if (j < p.J && h < p.H)
             v = *reinterpret_cast<const uint4*>(p.q + (((long long)gi.b * p.J + j) * p.H + h) * p.d_bytes +
-                                                kb * p.kbw + c16 * 16);
+                                                kb * KBW + c16 * 16);
           const uint32_t dst = smem_u32(smem + p.off_q + sb_ * p.q_sub_bytes + kb * p.q_kblock_bytes) +
-                               swizzled_offset(rr, c16 * 16, p.kbw);
+                               swizzled_offset(rr, c16 * 16, KBW);
           st_shared_v4(dst, v.x, v.y, v.z, v.w);
         }
         for (int i = et; i < p.qg * p.HP; i += kEpiThreads) {
@@ -359,8 +364,9 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
           const uint32_t col0 = (uint32_t)((as * NSUB + sub) * p.n_cols);
           for (int ql = 0; ql < p.nq_sub; ++ql) {
             const int qloc = sub * p.nq_sub + ql;
-            const float* wq = w_s + qloc * p.HP;
-            float acc = 0.0f;
+            const float4* wq = reinterpret_cast<const float4*>(w_s + qloc * p.HP);
+            // four independent partial sums over the heads (w from shared memory, 4 per load)
+            float a4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
             for (int hc = 0; hc * 16 < p.H; hc += 2) {
               uint32_t v0[16], v1[16];
               const uint32_t ta = tmem_addr(tmem_base, quad * 32, col0 + ql * p.HP + hc * 16);
@@ -369,14 +375,25 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
               if (two) tmem_ld16(ta + 16, v1);
               tmem_wait_ld();
 #pragma unroll
-              for (int i = 0; i < 16; ++i)
-                acc = fmaf(wq[hc * 16 + i], fmaxf(__uint_as_float(v0[i]), 0.0f), acc);
+              for (int i = 0; i < 4; ++i) {
+                const float4 wv = wq[hc * 4 + i];
+                a4[0] = fmaf(wv.x, fmaxf(__uint_as_float(v0[4 * i]), 0.0f), a4[0]);
+                a4[1] = fmaf(wv.y, fmaxf(__uint_as_float(v0[4 * i + 1]), 0.0f), a4[1]);
+                a4[2] = fmaf(wv.z, fmaxf(__uint_as_float(v0[4 * i + 2]), 0.0f), a4[2]);
+                a4[3] = fmaf(wv.w, fmaxf(__uint_as_float(v0[4 * i + 3]), 0.0f), a4[3]);
+              }
               if (two) {
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
-                  acc = fmaf(wq[hc * 16 + 16 + i], fmaxf(__uint_as_float(v1[i]), 0.0f), acc);
+                for (int i = 0; i < 4; ++i) {
+                  const float4 wv = wq[hc * 4 + 4 + i];
+                  a4[0] = fmaf(wv.x, fmaxf(__uint_as_float(v1[4 * i]), 0.0f), a4[0]);
+                  a4[1] = fmaf(wv.y, fmaxf(__uint_as_float(v1[4 * i + 1]), 0.0f), a4[1]);
+                  a4[2] = fmaf(wv.z, fmaxf(__uint_as_float(v1[4 * i + 2]), 0.0f), a4[2]);
+                  a4[3] = fmaf(wv.w, fmaxf(__uint_as_float(v1[4 * i + 3]), 0.0f), a4[3]);
+                }
               }
             }
+            const float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
             const int pos = info_pos[qloc];
             if (s <= pos) {
               const int j = gi.g * p.qg + qloc;
@@ -423,17 +440,24 @@ cudaError_t launch_index_score(const IndexKernelParams& p, const CUtensorMap& km
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  cudaError_t e;
-  if (p.n_sub == 2) {
-    e = cudaFuncSetAttribute(index_score_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)p.smem_bytes);
+  auto go = [&](auto kernel) -> cudaError_t {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem_bytes);
     if (e != cudaSuccess) return e;
-    return cudaLaunchKernelEx(&cfg, index_score_kernel<2>, kmap, p);
-  }
-  e = cudaFuncSetAttribute(index_score_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)p.smem_bytes);
-  if (e != cudaSuccess) return e;
-  return cudaLaunchKernelEx(&cfg, index_score_kernel<1>, kmap, p);
+    return cudaLaunchKernelEx(&cfg, kernel, kmap, p);
+  };
+  // (K-block width, K blocks) from the row size: 64 B -> (64, 1), 128 B -> (128, 1), 256 B -> (128, 2)
+  const int shape = p.kbw == 64 ? 0 : (p.n_kblocks == 1 ? 1 : 2);
+#define SIA_INDEX_CASE(NS, SH, KB, NK)                                                            \
+  if (p.n_sub == NS && shape == SH) return p.fp8 ? go(index_score_kernel<NS, KB, NK, true>)      \
+                                                 : go(index_score_kernel<NS, KB, NK, false>);
+  SIA_INDEX_CASE(1, 0, 64, 1)
+  SIA_INDEX_CASE(1, 1, 128, 1)
+  SIA_INDEX_CASE(1, 2, 128, 2)
+  SIA_INDEX_CASE(2, 0, 64, 1)
+  SIA_INDEX_CASE(2, 1, 128, 1)
+  SIA_INDEX_CASE(2, 2, 128, 2)
+#undef SIA_INDEX_CASE
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace sia
