@@ -205,18 +205,18 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
               (uint32_t)__popc(valid_mask) * (NKB * p.box_rows * KBW + scale_bytes);
           mbar_arrive_expect_tx(&sb->k_full[stage], bytes);
         }
-        for (int c = 0; c < chunks; ++c) {   // warp-uniform trip count
-          const int page = __shfl_sync(0xffffffffu, my_page, c);
-          if (lane == 0 && (valid_mask >> c & 1u)) {
-            const int y = page * p.P + ((tile_pos0 + c * p.box_rows) % p.P);
+        __syncwarp();
+        // lane c issues chunk c's boxes: a TMA instruction blocks its issuing thread for a few
+        // hundred cycles, so several issuing lanes move a tile's bytes sooner than one
+        if (valid_mask >> lane & 1u) {
+          const int y = my_page * p.P + (my_pos % p.P);
 #pragma unroll
-            for (int kb = 0; kb < NKB; ++kb)
-              tma_load_2d(kst + kb * p.k_kblock_bytes + c * p.box_rows * KBW, &kmap,
-                          &sb->k_full[stage], kb * KBW / (FP8 ? 1 : 2), y);
-            if (p.k_scale)
-              bulk_load(info + 16 + c * p.box_rows * 4, p.k_scale + (long long)y, scale_bytes,
-                        &sb->k_full[stage]);
-          }
+          for (int kb = 0; kb < NKB; ++kb)
+            tma_load_2d(kst + kb * p.k_kblock_bytes + lane * p.box_rows * KBW, &kmap,
+                        &sb->k_full[stage], kb * KBW / (FP8 ? 1 : 2), y);
+          if (p.k_scale)
+            bulk_load(info + 16 + lane * p.box_rows * 4, p.k_scale + (long long)y, scale_bytes,
+                      &sb->k_full[stage]);
         }
         __syncwarp();
       }
@@ -321,13 +321,16 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
           const int sb_ = r / NKB;
           const int ql = rr / p.HP, h = rr - ql * p.HP;
           const int j = gi.g * p.qg + sb_ * p.nq_sub + ql;
-          uint4 v = make_uint4(0u, 0u, 0u, 0u);
-          if (j < p.J && h < p.H)
-            v = *reinterpret_cast<const uint4*>(p.q + (((long long)gi.b * p.J + j) * p.H + h) * p.d_bytes +
-                                                kb * KBW + c16 * 16);
           const uint32_t dst = smem_u32(smem + p.off_q + sb_ * p.q_sub_bytes + kb * p.q_kblock_bytes) +
                                swizzled_offset(rr, c16 * 16, KBW);
-          st_shared_v4(dst, v.x, v.y, v.z, v.w);
+          // cp.async keeps every piece of the group in flight at once (a load -> store loop
+          // would wait one memory latency per piece)
+          if (j < p.J && h < p.H)
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst),
+                         "l"(p.q + (((long long)gi.b * p.J + j) * p.H + h) * p.d_bytes + kb * KBW + c16 * 16)
+                         : "memory");
+          else
+            st_shared_v4(dst, 0u, 0u, 0u, 0u);
         }
         for (int i = et; i < p.qg * p.HP; i += kEpiThreads) {
           const int ql = i / p.HP, h = i - ql * p.HP;
@@ -339,6 +342,7 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
           info_pos[et] = j < p.J ? query_position(p.seq_lens, p.q_pos, p.J, gi.b, j, p.Lpad) : -1;
           info_qs[et] = (j < p.J && p.q_scale) ? p.q_scale[(long long)gi.b * p.J + j] : 1.0f;
         }
+        asm volatile("cp.async.wait_all;" ::: "memory");
         fence_proxy_async_smem();
         mbar_arrive(&sb->q_full);
         // every epilogue thread has staged its share (w_s / info are visible after this)

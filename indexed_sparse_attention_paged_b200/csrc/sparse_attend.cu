@@ -502,6 +502,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const uint8_t* qrow = static_cast<const uint8_t*>(p.q) + ((long long)bj * p.H + (real ? h : 0)) * (DC * 2) +
                               (size_t)rank * Lay::kLatDims * 2;
         constexpr int kGroups = Lay::kLatDims / 32;   // 64 bytes = 16 columns each
+        // pull the whole row share into L2 first, so the grouped loads below wait on L2, not DRAM
+        if (real) {
+#pragma unroll
+          for (int g = 0; g < kGroups; g += 2)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(qrow + g * 64));
+        }
         tc_fence_after();
 #pragma unroll 1
         for (int g = 0; g < kGroups; ++g) {
