@@ -750,33 +750,39 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
 }
 
-// Log-sum-exp merge of the per-split partial results: one CTA per (query row, head), each
-// thread 4 output dims.
-__global__ void __launch_bounds__(128) combine_kernel(const CombineKernelParams p) {
+// Log-sum-exp merge of the per-split partial results: 256 threads per CTA, 8 output dims per
+// thread (16-byte loads of the bf16 partials), DL/8 threads per (query row, head).
+constexpr int kCombineThreads = 256;
+
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineKernelParams p) {
   pdl_wait_primary();
-  const long long bjh = blockIdx.x;            // = bj * H + h
-  const int d4 = threadIdx.x * 4;
-  if (d4 < p.DL) {
-    const long long stride_lse = (long long)p.BJ * p.H;
+  const int tph = p.DL / 8;                               // threads per (row, head)
+  const long long bjh = (long long)blockIdx.x * (kCombineThreads / tph) + threadIdx.x / tph;
+  const int d8 = (threadIdx.x % tph) * 8;
+  const long long n_bjh = (long long)p.BJ * p.H;
+  if (bjh < n_bjh) {
     float mx = -INFINITY;
-    for (int s = 0; s < p.splits; ++s) mx = fmaxf(mx, p.part_lse[s * stride_lse + bjh]);
-    float wsum = 0.0f, o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
+    for (int s = 0; s < p.splits; ++s) mx = fmaxf(mx, p.part_lse[s * n_bjh + bjh]);
+    float wsum = 0.0f, o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     if (mx != -INFINITY) {
       for (int s = 0; s < p.splits; ++s) {
-        const float ls = p.part_lse[s * stride_lse + bjh];
+        const float ls = p.part_lse[s * n_bjh + bjh];
         const float wgt = ls == -INFINITY ? 0.0f : expf(ls - mx);
-        const uint2 v = *reinterpret_cast<const uint2*>(p.part_o + (s * stride_lse + bjh) * p.DL + d4);
-        o0 += wgt * __uint_as_float(v.x << 16);
-        o1 += wgt * __uint_as_float(v.x & 0xffff0000u);
-        o2 += wgt * __uint_as_float(v.y << 16);
-        o3 += wgt * __uint_as_float(v.y & 0xffff0000u);
+        const uint4 v = *reinterpret_cast<const uint4*>(p.part_o + (s * n_bjh + bjh) * p.DL + d8);
+        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          o[2 * i] += wgt * __uint_as_float(w4[i] << 16);
+          o[2 * i + 1] += wgt * __uint_as_float(w4[i] & 0xffff0000u);
+        }
         wsum += wgt;
       }
     }
     const float inv = wsum > 0.0f ? 1.0f / wsum : 0.0f;
-    uint16_t* dst = p.out + bjh * p.DL + d4;
-    *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(o0 * inv, o1 * inv), pack_bf16x2(o2 * inv, o3 * inv));
-    if (d4 == 0 && p.lse) p.lse[bjh] = wsum > 0.0f ? mx + logf(wsum) : -INFINITY;
+    *reinterpret_cast<uint4*>(p.out + bjh * p.DL + d8) =
+        make_uint4(pack_bf16x2(o[0] * inv, o[1] * inv), pack_bf16x2(o[2] * inv, o[3] * inv),
+                   pack_bf16x2(o[4] * inv, o[5] * inv), pack_bf16x2(o[6] * inv, o[7] * inv));
+    if (d8 == 0 && p.lse) p.lse[bjh] = wsum > 0.0f ? mx + logf(wsum) : -INFINITY;
   }
   pdl_launch_dependents();
 }
@@ -839,8 +845,9 @@ cudaError_t launch_sparse_attend(const AttnKernelParams& p, const CUtensorMap* m
 cudaError_t launch_combine(const CombineKernelParams& p, bool pdl, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
-  cfg.gridDim = dim3((unsigned)((long long)p.BJ * p.H), 1, 1);
-  cfg.blockDim = dim3(128, 1, 1);
+  const long long per_cta = kCombineThreads / (p.DL / 8);
+  cfg.gridDim = dim3((unsigned)(((long long)p.BJ * p.H + per_cta - 1) / per_cta), 1, 1);
+  cfg.blockDim = dim3(kCombineThreads, 1, 1);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
   int na = 0;
