@@ -33,6 +33,7 @@ sys.path.insert(0, ROOT)
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 L2_BYTES = 126 * 1024 * 1024
 
 
@@ -42,7 +43,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", type=int, default=2, choices=[2, 3, 5])
+    ap.add_argument("--workload", type=int, default=2, choices=[2, 3, 4, 5],
+                    help="2, 3, 5: fused decode (queries/s); 4: prefill indexer scoring (TFLOP/s)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
 
@@ -143,9 +145,9 @@ def peaks() -> dict:
     try:
         with open(PEAKS_FILE) as f:
             p = json.load(f)
-        return {"hbm_gbs": float(p["hbm_gbs"]), "source": "measured"}
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]), "source": "measured"}
     except (OSError, KeyError, ValueError):
-        return {"hbm_gbs": FALLBACK_HBM_GBS, "source": "fallback"}
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS, "source": "fallback"}
 
 
 # What each stage-level roofline entry times: one C-ABI call, i.e. both kernels of the stage.
@@ -225,6 +227,83 @@ def config_of(wl, inputs, l2):
             "l2": l2, "parallelism": "replicas"}
 
 
+def prefill_scoring_flops(seq_lens, n_q, heads, dim) -> int:
+    """FLOPs of the causal q.k contraction: 2 * D * H per (query, visible position)."""
+    total = 0
+    for L in seq_lens:
+        first = int(L) - n_q                 # query j sits at position L - n_q + j and sees 0..pos
+        total += sum(first + j + 1 for j in range(n_q))
+    return 2 * heads * dim * total
+
+
+def run_prefill_scoring(args, rank, world, dev, wl):
+    """Prefill chunk (T = 16384 causal): the indexer's scoring step alone (sia_index_scores),
+    in TFLOP/s of the causal q.k contraction against the measured bf16 tensor peak."""
+    import torch
+    import torch.distributed as dist
+    import indexed_sparse_attention_paged_b200 as sia
+    from indexed_sparse_attention_paged_b200 import workloads
+
+    host = workloads.make_inputs(wl, seed=1000 + wl.number + 7919 * rank)
+    d = workloads.to_device(host, dev)
+    B, J = host["batch"], host["n_q"]
+    Lpad = host["max_pages"] * wl.page_size
+    scores = torch.empty((B, J, Lpad), dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        sia.index_scores(d["q_idx"], d["w"], d["k_cache"], d["page_table"], d["seq_lens"],
+                         k_scale=d["k_scale"], scores_out=scores, dev_status=status, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    steps = max(1, min(args.steps, 50))
+    sampler = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
+    sampler.start()
+    time.sleep(0.25)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    clocks = sampler.stop()
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    if int(status.item()) != 0:
+        raise RuntimeError("device status %d" % int(status.item()))
+    flops = prefill_scoring_flops(host["seq_lens"].tolist(), J, wl.idx_heads, wl.idx_dim)
+    tflops = flops / (ms / 1000.0) / 1e12
+    pk = peaks()
+    if rank == 0:
+        print(json.dumps({
+            "metric": "prefill indexer scoring TFLOP/s @T=%d causal, %dx%d bf16" % (J, wl.idx_heads, wl.idx_dim),
+            "value": world * tflops, "unit": "TFLOP/s", "n_gpus": world, "steps": steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl.name, "tokens": J, "idx_heads": wl.idx_heads, "idx_dim": wl.idx_dim,
+                       "l2": "the 16384 x 256 B index keys (4 MB) are L2-resident by design: the "
+                             "contraction reuses each key tile for every query group",
+                       "parallelism": "replicas"},
+            "roofline": {"bound": "tensor", "kernel": "index_score_kernel (one sia_index_scores call)",
+                         "achieved": tflops, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": tflops / pk["bf16_tflops"], "peak_source": pk["source"] + " burst",
+                         "traffic": None, "flops_per_launch": flops},
+            "gpu_launches": steps, "clocks": clocks,
+        }), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     args = parse()
     rank = int(os.environ.get("RANK", "0"))
@@ -246,6 +325,8 @@ def main():
         dist.init_process_group("nccl", device_id=dev, timeout=__import__("datetime").timedelta(seconds=120))
 
     wl = workloads.WORKLOADS[args.workload]
+    if wl.number == 4:
+        return run_prefill_scoring(args, rank, world, dev, wl)
     host = workloads.make_inputs(wl, seed=1000 + wl.number + 7919 * rank)
     # Several independent input sets, used round-robin: together they are far larger than the
     # 126 MB L2, so every timed step reads its index keys and latent rows from HBM (no flush

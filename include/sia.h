@@ -135,6 +135,15 @@ size_t sia_workspace_size(const sia_index_args* ia, const sia_attend_args* aa);
 sia_status sia_sparse_index_topk(const sia_index_args* a, void* workspace, size_t ws_bytes,
                                  int32_t* dev_status, void* stream);
 
+/* The scoring step of stage 1 alone: writes I[t,s] for every causal position s <= p(t) of
+ * every query into a->scores_out (required; positions past p(t) are left untouched) and no
+ * Top-K list ("Day 0 Inference Adaptation and Performance Optimization for Hybrid Sparse
+ * Attention LLMs", section "Operator Fusion and Multi-Stream Scheduling", the score-and-
+ * aggregate steps before the selection).  For a prefill chunk this is the dense causal q.k
+ * contraction on the tensor cores.  a->topk_out and a->top_k are ignored; a->scores_out NULL
+ * -> SIA_ERR_INVALID_ARGUMENT. */
+sia_status sia_index_scores(const sia_index_args* a, int32_t* dev_status, void* stream);
+
 /* Stage 2: sparse MLA attention over a Top-K list. */
 sia_status sia_sparse_mla_attend(const sia_attend_args* a, void* workspace, size_t ws_bytes,
                                  int32_t* dev_status, void* stream);

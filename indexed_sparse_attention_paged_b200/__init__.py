@@ -80,6 +80,8 @@ def load_library(path: str = LIB_PATH):
     lib.sia_workspace_size.argtypes = [ctypes.POINTER(IndexArgs), ctypes.POINTER(AttendArgs)]
     lib.sia_sparse_index_topk.restype = ctypes.c_int
     lib.sia_sparse_index_topk.argtypes = [ctypes.POINTER(IndexArgs), P, ctypes.c_size_t, P, P]
+    lib.sia_index_scores.restype = ctypes.c_int
+    lib.sia_index_scores.argtypes = [ctypes.POINTER(IndexArgs), P, P]
     lib.sia_sparse_index_topk_noalloc.restype = ctypes.c_int
     lib.sia_sparse_index_topk_noalloc.argtypes = [ctypes.POINTER(IndexArgs), P, P]
     lib.sia_sparse_mla_attend.restype = ctypes.c_int
@@ -226,6 +228,17 @@ def sparse_index_topk(q, w, k_cache, page_table, seq_lens, *, top_k, q_scale=Non
     wp, wn = _ws_ptr(ws)
     _check(lib.sia_sparse_index_topk(ctypes.byref(a), wp, wn, _ptr(dev_status), _stream_ptr(stream)))
     return topk_out
+
+
+def index_scores(q, w, k_cache, page_table, seq_lens, *, scores_out, q_scale=None, k_scale=None,
+                 q_pos=None, dev_status=None, stream=None):
+    """The scoring step alone: I[t, s] for every causal position into `scores_out`
+    (fp32 [B, J, max_pages_per_seq * page_size]; positions past a query's own are untouched)."""
+    lib = load_library()
+    a = index_args(q, w, k_cache, page_table, seq_lens, top_k=1, q_scale=q_scale, k_scale=k_scale,
+                   q_pos=q_pos, topk_out=None, scores_out=scores_out)
+    _check(lib.sia_index_scores(ctypes.byref(a), _ptr(dev_status), _stream_ptr(stream)))
+    return scores_out
 
 
 def sparse_index_topk_noalloc(q, w, k_cache, page_table, seq_lens, *, top_k, topk_out, q_scale=None,

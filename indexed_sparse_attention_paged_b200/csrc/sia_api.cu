@@ -98,11 +98,11 @@ struct IndexPlan {
   int grid;
 };
 
-sia_status check_index(const sia_index_args* a) {
+sia_status check_index(const sia_index_args* a, bool with_topk) {
   if (!a) return fail(SIA_ERR_INVALID_ARGUMENT, "index args are NULL");
-  if (a->batch < 1 || a->n_q < 1 || a->top_k < 1 || a->max_pages_per_seq < 1 || a->num_pages < 1)
+  if (a->batch < 1 || a->n_q < 1 || (with_topk && a->top_k < 1) || a->max_pages_per_seq < 1 || a->num_pages < 1)
     return fail(SIA_ERR_INVALID_ARGUMENT, "batch, n_q, top_k, max_pages_per_seq and num_pages must be >= 1");
-  if (!a->q || !a->w || !a->k_cache || !a->page_table || !a->seq_lens || !a->topk_out)
+  if (!a->q || !a->w || !a->k_cache || !a->page_table || !a->seq_lens || (with_topk && !a->topk_out))
     return fail(SIA_ERR_INVALID_ARGUMENT, "q, w, k_cache, page_table, seq_lens and topk_out must be set");
   if (a->dtype != SIA_BF16 && a->dtype != SIA_FP8_E4M3) return fail(SIA_ERR_UNSUPPORTED, "unknown dtype %d", (int)a->dtype);
   if (a->n_heads < 1 || a->n_heads > 64) return fail(SIA_ERR_UNSUPPORTED, "n_heads must be 1..64 (got %d)", a->n_heads);
@@ -122,8 +122,8 @@ sia_status check_index(const sia_index_args* a) {
   return SIA_OK;
 }
 
-sia_status plan_index(const sia_index_args* a, IndexPlan* pl, bool make_maps) {
-  sia_status st = check_index(a);
+sia_status plan_index(const sia_index_args* a, IndexPlan* pl, bool make_maps, bool with_topk = true) {
+  sia_status st = check_index(a, with_topk);
   if (st != SIA_OK) return st;
   IndexKernelParams& k = pl->kp;
   memset(&k, 0, sizeof k);
@@ -196,7 +196,8 @@ sia_status plan_index(const sia_index_args* a, IndexPlan* pl, bool make_maps) {
   t.Lpad = k.Lpad;
   int cs = 1;
   while ((k.Lpad + cs - 1) / cs > kTopkSliceMax) cs <<= 1;
-  if (cs > 16) return fail(SIA_ERR_UNSUPPORTED, "context too long for the Top-K kernel (max %d)", 16 * kTopkSliceMax);
+  if (with_topk && cs > 16)
+    return fail(SIA_ERR_UNSUPPORTED, "context too long for the Top-K kernel (max %d)", 16 * kTopkSliceMax);
   const long long rows = (long long)a->batch * a->n_q;
   // rows of up to 16384 positions take one CTA each (no cluster); longer rows split across a
   // cluster, widened while that still leaves SMs idle
@@ -204,7 +205,7 @@ sia_status plan_index(const sia_index_args* a, IndexPlan* pl, bool make_maps) {
     while (cs < 8 && rows * cs * 2 <= 2ll * pl->grid) cs <<= 1;
   t.cluster = cs;
   t.slice = (int)round_up((size_t)((k.Lpad + cs - 1) / cs), 32);
-  if (rows * cs > 0x7fffffffll) return fail(SIA_ERR_UNSUPPORTED, "too many query rows");
+  if (with_topk && rows * cs > 0x7fffffffll) return fail(SIA_ERR_UNSUPPORTED, "too many query rows");
   t.seq_lens = a->seq_lens;
   t.q_pos = a->q_pos;
   t.topk = a->topk_out;
@@ -396,6 +397,19 @@ sia_status sia_sparse_index_topk(const sia_index_args* a, void* workspace, size_
   sia_status st = plan_index(a, &pl, true);
   if (st != SIA_OK) return st;
   return run_index(&pl, workspace, ws_bytes, dev_status, static_cast<cudaStream_t>(stream), false);
+}
+
+sia_status sia_index_scores(const sia_index_args* a, int32_t* dev_status, void* stream) {
+  g_last_error[0] = 0;
+  if (a && !a->scores_out) return fail(SIA_ERR_INVALID_ARGUMENT, "scores_out is required");
+  IndexPlan pl;
+  sia_status st = plan_index(a, &pl, true, false);
+  if (st != SIA_OK) return st;
+  pl.kp.scores = a->scores_out;
+  pl.kp.status = dev_status;
+  cudaError_t e = launch_index_score(pl.kp, pl.kmap, pl.grid, false, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "index scoring launch");
+  return SIA_OK;
 }
 
 sia_status sia_sparse_mla_attend(const sia_attend_args* a, void* workspace, size_t ws_bytes, int32_t* dev_status,

@@ -93,6 +93,18 @@ def test_index_arguments_refused_on_the_host(lib, kw, status):
 
 
 @pytest.mark.parametrize("kw,status", [
+    ({}, sia.SIA_ERR_INVALID_ARGUMENT),                      # scores_out is required
+    (dict(scores_out=8192, q=None), sia.SIA_ERR_INVALID_ARGUMENT),
+    (dict(scores_out=8192, head_dim=48), sia.SIA_ERR_UNSUPPORTED),
+    (dict(scores_out=8200), sia.SIA_ERR_INVALID_ARGUMENT),    # misaligned scores_out
+])
+def test_scoring_only_arguments_refused_on_the_host(lib, kw, status):
+    a = _index_args(**kw)
+    assert lib.sia_index_scores(ctypes.byref(a), None, None) == status
+    assert lib.sia_last_error() != b""
+
+
+@pytest.mark.parametrize("kw,status", [
     (dict(out=None), sia.SIA_ERR_INVALID_ARGUMENT),
     (dict(d_latent=256), sia.SIA_ERR_UNSUPPORTED),
     (dict(n_heads=129), sia.SIA_ERR_UNSUPPORTED),

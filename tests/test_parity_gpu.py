@@ -175,6 +175,30 @@ def test_index_bad_page_id_sets_status_without_fault():
     assert np.array_equal(topk[0, 0], ref[0, 0])      # the untouched sequence is still exact
 
 
+@pytest.mark.parametrize("num,kw", [(4, dict(seq_lens=[300], n_q=300)), (2, dict(seq_lens=[700, 33]))])
+def test_scoring_only_call_matches_oracle(num, kw):
+    """sia_index_scores: every visible score bit-exact, positions past each query untouched."""
+    h = workloads.make_inputs(workloads.WORKLOADS[num], **kw)
+    d = workloads.to_device(h, DEV)
+    B, J = h["batch"], h["n_q"]
+    Lpad = h["max_pages"] * h["workload"].page_size
+    scores = torch.full((B, J, Lpad), 12345.0, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    sia.index_scores(d["q_idx"], d["w"], d["k_cache"], d["page_table"], d["seq_lens"],
+                     k_scale=d["k_scale"], scores_out=scores, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    got = scores.cpu().numpy()
+    _, ref, _ = oracle_index(h, 1)
+    nv = []
+    for b in range(B):
+        for j in range(J):
+            n = int(np.sum(~np.isnan(ref[b, j])))
+            nv.append(((b, j), n))
+            assert np.all(got[b, j, n:] == 12345.0), "row (%d,%d) written past its position" % (b, j)
+    assert_scores_equal(got, ref, nv)
+
+
 # ------------------------------------------------------------------ stage 2: sparse attention
 
 def _random_topk(h, top_k, seed, fill=1.0):
