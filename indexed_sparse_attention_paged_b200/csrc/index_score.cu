@@ -118,7 +118,8 @@ __device__ void locate_start(const IndexKernelParams& p, IndexBarriers* sb) {
 // each tcgen05.mma took about three times longer to issue.
 template <int NSUB, int KBW, int NKB, bool FP8>
 __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
-    index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexKernelParams p) {
+    index_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
+                       const IndexKernelParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   IndexBarriers* sb = reinterpret_cast<IndexBarriers*>(smem + p.off_bar);
   const int warp = threadIdx.x >> 5;
@@ -145,6 +146,7 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
     sb->abort = 0;
     fence_mbarrier_init();
     tma_prefetch_desc(&kmap);
+    tma_prefetch_desc(&qmap);
   }
   if (warp == 0) locate_start(p, sb);
   if (warp == 1) {
@@ -310,27 +312,16 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
         float* w_s = reinterpret_cast<float*>(smem + p.off_w) + (seg & 1) * w_words;
         int* info_pos = reinterpret_cast<int*>(smem + p.off_info) + (seg & 1) * 16;
         float* info_qs = reinterpret_cast<float*>(smem + p.off_info + 128) + (seg & 1) * 16;
-        constexpr int chunks16 = KBW / 16;
-        const int total16 = NSUB * NKB * p.n_cols * chunks16;
-        for (int i = et; i < total16; i += kEpiThreads) {
-          const int c16 = i % chunks16;
-          int r = i / chunks16;
-          const int rr = r % p.n_cols;
-          r /= p.n_cols;
-          const int kb = r % NKB;
-          const int sb_ = r / NKB;
-          const int ql = rr / p.HP, h = rr - ql * p.HP;
-          const int j = gi.g * p.qg + sb_ * p.nq_sub + ql;
-          const uint32_t dst = smem_u32(smem + p.off_q + sb_ * p.q_sub_bytes + kb * p.q_kblock_bytes) +
-                               swizzled_offset(rr, c16 * 16, KBW);
-          // cp.async keeps every piece of the group in flight at once (a load -> store loop
-          // would wait one memory latency per piece)
-          if (j < p.J && h < p.H)
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst),
-                         "l"(p.q + (((long long)gi.b * p.J + j) * p.H + h) * p.d_bytes + kb * KBW + c16 * 16)
-                         : "memory");
-          else
-            st_shared_v4(dst, 0u, 0u, 0u, 0u);
+        if (et == 0) {
+          // q of the group: one 3-D TMA box (nq_sub queries x HP heads x one K block, heads
+          // past H and queries past the batch zero-filled) per (sub-block, K block)
+          mbar_arrive_expect_tx(&sb->q_full, (uint32_t)(NSUB * NKB) * p.q_kblock_bytes);
+#pragma unroll
+          for (int sb_ = 0; sb_ < NSUB; ++sb_)
+#pragma unroll
+            for (int kb = 0; kb < NKB; ++kb)
+              tma_load_3d(smem + p.off_q + sb_ * p.q_sub_bytes + kb * p.q_kblock_bytes, &qmap, &sb->q_full,
+                          kb * KBW / (FP8 ? 1 : 2), 0, gi.b * p.J + gi.g * p.qg + sb_ * p.nq_sub);
         }
         for (int i = et; i < p.qg * p.HP; i += kEpiThreads) {
           const int ql = i / p.HP, h = i - ql * p.HP;
@@ -342,9 +333,7 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
           info_pos[et] = j < p.J ? query_position(p.seq_lens, p.q_pos, p.J, gi.b, j, p.Lpad) : -1;
           info_qs[et] = (j < p.J && p.q_scale) ? p.q_scale[(long long)gi.b * p.J + j] : 1.0f;
         }
-        asm volatile("cp.async.wait_all;" ::: "memory");
-        fence_proxy_async_smem();
-        mbar_arrive(&sb->q_full);
+        if (et != 0) mbar_arrive(&sb->q_full);
         // every epilogue thread has staged its share (w_s / info are visible after this)
         if (!mbar_wait(&sb->q_full, (uint32_t)seg & 1u, abort, p.status)) { ok = false; break; }
         const long long out_row0 = (long long)gi.b * p.J;
@@ -366,43 +355,45 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
           else if (p.k_scale)
             ks = reinterpret_cast<const float*>(info + 16)[row];
           const uint32_t col0 = (uint32_t)((as * NSUB + sub) * p.n_cols);
-          for (int ql = 0; ql < p.nq_sub; ++ql) {
-            const int qloc = sub * p.nq_sub + ql;
-            const float4* wq = reinterpret_cast<const float4*>(w_s + qloc * p.HP);
-            // four independent partial sums over the heads (w from shared memory, 4 per load)
-            float a4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-            for (int hc = 0; hc * 16 < p.H; hc += 2) {
-              uint32_t v0[16], v1[16];
-              const uint32_t ta = tmem_addr(tmem_base, quad * 32, col0 + ql * p.HP + hc * 16);
-              tmem_ld16(ta, v0);
-              const bool two = (hc + 1) * 16 < p.H;
-              if (two) tmem_ld16(ta + 16, v1);
-              tmem_wait_ld();
+          // QB queries' columns (up to QB x 64 heads) per TMEM wait: the loads of a batch are in
+          // flight together, so each tile pays the TMEM latency once per batch (QB = 1 with two
+          // sub-blocks, to stay within the registers of 320 threads)
+          constexpr int QB = NSUB == 1 ? 2 : 1;
+          for (int q0 = 0; q0 < p.nq_sub; q0 += QB) {
+            uint32_t v[QB][4][16];
 #pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const float4 wv = wq[hc * 4 + i];
-                a4[0] = fmaf(wv.x, fmaxf(__uint_as_float(v0[4 * i]), 0.0f), a4[0]);
-                a4[1] = fmaf(wv.y, fmaxf(__uint_as_float(v0[4 * i + 1]), 0.0f), a4[1]);
-                a4[2] = fmaf(wv.z, fmaxf(__uint_as_float(v0[4 * i + 2]), 0.0f), a4[2]);
-                a4[3] = fmaf(wv.w, fmaxf(__uint_as_float(v0[4 * i + 3]), 0.0f), a4[3]);
-              }
-              if (two) {
+            for (int qq = 0; qq < QB; ++qq)
+#pragma unroll
+              for (int hc = 0; hc < 4; ++hc)
+                if (q0 + qq < p.nq_sub && hc * 16 < p.H)   // warp-uniform
+                  tmem_ld16(tmem_addr(tmem_base, quad * 32, col0 + (q0 + qq) * p.HP + hc * 16), v[qq][hc]);
+            tmem_wait_ld();
+#pragma unroll
+            for (int qq = 0; qq < QB; ++qq) {
+              if (q0 + qq >= p.nq_sub) break;
+              const int qloc = sub * p.nq_sub + q0 + qq;
+              const float4* wq = reinterpret_cast<const float4*>(w_s + qloc * p.HP);
+              // four independent partial sums over the heads (w from shared memory, 4 per load)
+              float a4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+              for (int hc = 0; hc < 4; ++hc) {
+                if (hc * 16 >= p.H) break;
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                  const float4 wv = wq[hc * 4 + 4 + i];
-                  a4[0] = fmaf(wv.x, fmaxf(__uint_as_float(v1[4 * i]), 0.0f), a4[0]);
-                  a4[1] = fmaf(wv.y, fmaxf(__uint_as_float(v1[4 * i + 1]), 0.0f), a4[1]);
-                  a4[2] = fmaf(wv.z, fmaxf(__uint_as_float(v1[4 * i + 2]), 0.0f), a4[2]);
-                  a4[3] = fmaf(wv.w, fmaxf(__uint_as_float(v1[4 * i + 3]), 0.0f), a4[3]);
+                  const float4 wv = wq[hc * 4 + i];
+                  a4[0] = fmaf(wv.x, fmaxf(__uint_as_float(v[qq][hc][4 * i]), 0.0f), a4[0]);
+                  a4[1] = fmaf(wv.y, fmaxf(__uint_as_float(v[qq][hc][4 * i + 1]), 0.0f), a4[1]);
+                  a4[2] = fmaf(wv.z, fmaxf(__uint_as_float(v[qq][hc][4 * i + 2]), 0.0f), a4[2]);
+                  a4[3] = fmaf(wv.w, fmaxf(__uint_as_float(v[qq][hc][4 * i + 3]), 0.0f), a4[3]);
                 }
               }
-            }
-            const float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
-            const int pos = info_pos[qloc];
-            if (s <= pos) {
-              const int j = gi.g * p.qg + qloc;
-              const float v = isinf(ks) ? ks : acc * ks * info_qs[qloc];
-              p.scores[(out_row0 + j) * p.Lpad + s] = v;
+              const float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+              const int pos = info_pos[qloc];
+              if (s <= pos) {
+                const int j = gi.g * p.qg + qloc;
+                const float val = isinf(ks) ? ks : acc * ks * info_qs[qloc];
+                p.scores[(out_row0 + j) * p.Lpad + s] = val;
+              }
             }
           }
           tc_fence_before();
@@ -428,7 +419,7 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
 
 }  // namespace
 
-cudaError_t launch_index_score(const IndexKernelParams& p, const CUtensorMap& kmap, int grid,
+cudaError_t launch_index_score(const IndexKernelParams& p, const CUtensorMap& kmap, const CUtensorMap& qmap, int grid,
                                bool pdl, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
@@ -447,7 +438,7 @@ cudaError_t launch_index_score(const IndexKernelParams& p, const CUtensorMap& km
   auto go = [&](auto kernel) -> cudaError_t {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem_bytes);
     if (e != cudaSuccess) return e;
-    return cudaLaunchKernelEx(&cfg, kernel, kmap, p);
+    return cudaLaunchKernelEx(&cfg, kernel, kmap, qmap, p);
   };
   // (K-block width, K blocks) from the row size: 64 B -> (64, 1), 128 B -> (128, 1), 256 B -> (128, 2)
   const int shape = p.kbw == 64 ? 0 : (p.n_kblocks == 1 ? 1 : 2);

@@ -89,11 +89,28 @@ sia_status make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt,
   return SIA_OK;
 }
 
+// 3-D map over a [d2, d1, d0] array (d0 innermost) with a [b2, b1, b0] box.
+sia_status make_map_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes, uint64_t d0,
+                       uint64_t d1, uint64_t d2, uint32_t b0, uint32_t b1, uint32_t b2, int row_bytes_in_smem,
+                       CUtensorMapL2promotion l2) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(SIA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {d0 * (uint64_t)elem_bytes, d0 * d1 * (uint64_t)elem_bytes};
+  cuuint32_t box[3] = {b0, b1, b2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle_for(row_bytes_in_smem), l2, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SIA_ERR_CUDA, "cuTensorMapEncodeTiled (3-D) failed (%d)", (int)r);
+  return SIA_OK;
+}
+
 // ---------------------------------------------------------------- stage 1 plan
 struct IndexPlan {
   IndexKernelParams kp;
   TopkKernelParams tp;
   CUtensorMap kmap;
+  CUtensorMap qmap;   // q as [B*J queries, H heads, D]: one box = one query sub-block's K block
   size_t ws_scores;   // workspace bytes for the scores (0 when scores_out is given)
   int grid;
 };
@@ -141,8 +158,10 @@ sia_status plan_index(const sia_index_args* a, IndexPlan* pl, bool make_maps, bo
   k.n_kblocks = k.d_bytes / k.kbw;
   k.ksteps_per_block = k.kbw / 32;
   k.fp8 = a->dtype == SIA_FP8_E4M3;
-  // queries sharing one A tile: up to 256 columns per MMA, two MMAs for long prefill chunks
-  k.nq_sub = std::max(1, std::min(a->n_q, 256 / k.HP));
+  // queries sharing one A tile: up to 128 accumulator columns per MMA and two MMAs per tile
+  // for a prefill chunk, so that two accumulator stages fit in TMEM (the MMA of the next tile
+  // overlaps the epilogue of this one)
+  k.nq_sub = std::max(1, std::min(a->n_q, 128 / k.HP));
   k.n_sub = (a->n_q > k.nq_sub) ? 2 : 1;
   k.qg = k.nq_sub * k.n_sub;
   k.n_cols = k.nq_sub * k.HP;
@@ -215,6 +234,11 @@ sia_status plan_index(const sia_index_args* a, IndexPlan* pl, bool make_maps, bo
                      eb, (uint64_t)a->num_pages * a->page_size, (uint64_t)a->head_dim, (uint32_t)k.box_rows,
                      (uint32_t)(k.kbw / eb), k.kbw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
     if (st != SIA_OK) return st;
+    st = make_map_3d(&pl->qmap, a->q, k.fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, eb,
+                     (uint64_t)a->head_dim, (uint64_t)a->n_heads, (uint64_t)a->batch * a->n_q,
+                     (uint32_t)(k.kbw / eb), (uint32_t)k.HP, (uint32_t)k.nq_sub, k.kbw,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
+    if (st != SIA_OK) return st;
   }
   return SIA_OK;
 }
@@ -229,7 +253,7 @@ sia_status run_index(IndexPlan* pl, void* ws, size_t ws_bytes, int32_t* dev_stat
   pl->kp.status = dev_status;
   pl->tp.scores = pl->kp.scores;
   pl->tp.status = dev_status;
-  cudaError_t e = launch_index_score(pl->kp, pl->kmap, pl->grid, pdl_first, stream);
+  cudaError_t e = launch_index_score(pl->kp, pl->kmap, pl->qmap, pl->grid, pdl_first, stream);
   if (e != cudaSuccess) return cuda_fail(e, "index scoring launch");
   e = launch_topk(pl->tp, true, stream);
   if (e != cudaSuccess) return cuda_fail(e, "top-k launch");
@@ -407,7 +431,7 @@ sia_status sia_index_scores(const sia_index_args* a, int32_t* dev_status, void* 
   if (st != SIA_OK) return st;
   pl.kp.scores = a->scores_out;
   pl.kp.status = dev_status;
-  cudaError_t e = launch_index_score(pl.kp, pl.kmap, pl.grid, false, static_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_index_score(pl.kp, pl.kmap, pl.qmap, pl.grid, false, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "index scoring launch");
   return SIA_OK;
 }

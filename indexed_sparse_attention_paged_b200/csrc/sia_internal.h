@@ -97,7 +97,7 @@ struct CombineKernelParams {
 
 // Launchers (each returns cudaSuccess or the launch error).  `pdl` asks for programmatic
 // dependent launch on the previous kernel of the stream.
-cudaError_t launch_index_score(const IndexKernelParams& p, const CUtensorMap& kmap, int grid,
+cudaError_t launch_index_score(const IndexKernelParams& p, const CUtensorMap& kmap, const CUtensorMap& qmap, int grid,
                                bool pdl, cudaStream_t stream);
 cudaError_t launch_topk(const TopkKernelParams& p, bool pdl, cudaStream_t stream);
 cudaError_t launch_sparse_attend(const AttnKernelParams& p, const CUtensorMap* maps,
