@@ -70,46 +70,69 @@ __device__ __forceinline__ GroupInfo group_info(const IndexKernelParams& p, int 
   return gi;
 }
 
-// Warp 0 finds where this CTA's share of the flat tile list starts.
+// Work per (query group, tile) list entry, in tile units: a group also costs about two tiles of
+// set-up (its q and w staged, the pipeline drained and refilled), which matters for the short
+// groups at the start of a causal prefill chunk.
+constexpr long long kGroupCost = 2;
+
+// Warp 0 finds this CTA's share of the flat tile list: the weighted work (tiles + kGroupCost per
+// group) is split evenly between CTAs; the share is returned as (first group, first tile, tile
+// count).
 __device__ void locate_start(const IndexKernelParams& p, IndexBarriers* sb) {
   const int lane = threadIdx.x & 31;
   const int items = p.B * p.groups_per_seq;
   long long total = 0;
   for (int base = 0; base < items; base += 32) {
     const int it = base + lane;
-    long long t = it < items ? group_info(p, it).n_tiles : 0;
+    const int nt = it < items ? group_info(p, it).n_tiles : 0;
+    long long t = nt > 0 ? nt + kGroupCost : 0;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
     total += t;
   }
+  // (item, tile) and tiles-before of a weighted position: inside a group the set-up comes first
+  auto find = [&](long long pos, int& item_out, int& tile_out, long long& tiles_before) {
+    long long wbefore = 0, tbefore = 0;
+    item_out = items;
+    tile_out = 0;
+    tiles_before = 0;
+    for (int base = 0; base < items; base += 32) {
+      const int it = base + lane;
+      const int nt = it < items ? group_info(p, it).n_tiles : 0;
+      const long long w = nt > 0 ? nt + kGroupCost : 0;
+      long long wi = w, ti = nt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const long long vw = __shfl_up_sync(0xffffffffu, wi, o);
+        const long long vt = __shfl_up_sync(0xffffffffu, ti, o);
+        if (lane >= o) { wi += vw; ti += vt; }
+      }
+      const long long wex = wbefore + wi - w, tex = tbefore + ti - nt;
+      const bool here = w > 0 && pos >= wex && pos < wex + w;
+      const unsigned m = __ballot_sync(0xffffffffu, here);
+      if (m) {
+        const int src = __ffs(m) - 1;
+        item_out = __shfl_sync(0xffffffffu, it, src);
+        const long long off = pos - __shfl_sync(0xffffffffu, wex, src);
+        tile_out = (int)(off > kGroupCost ? off - kGroupCost : 0);
+        tiles_before = __shfl_sync(0xffffffffu, tex, src) + tile_out;
+        return;
+      }
+      wbefore += __shfl_sync(0xffffffffu, wi, 31);
+      tbefore += __shfl_sync(0xffffffffu, ti, 31);
+    }
+    tiles_before = tbefore;   // past the end: every tile is before
+  };
   const long long begin = total * blockIdx.x / gridDim.x;
   const long long end = total * (blockIdx.x + 1) / gridDim.x;
-  int start_item = items, start_tile = 0;
-  long long before = 0;
-  for (int base = 0; base < items; base += 32) {
-    const int it = base + lane;
-    const long long t = it < items ? group_info(p, it).n_tiles : 0;
-    long long incl = t;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const long long v = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += v;
-    }
-    const long long excl = before + incl - t;
-    const bool here = t > 0 && begin >= excl && begin < excl + t;
-    const unsigned m = __ballot_sync(0xffffffffu, here);
-    if (m) {
-      const int src = __ffs(m) - 1;
-      start_item = __shfl_sync(0xffffffffu, it, src);
-      start_tile = (int)(begin - __shfl_sync(0xffffffffu, excl, src));
-      break;
-    }
-    before += __shfl_sync(0xffffffffu, incl, 31);
-  }
+  int start_item, start_tile, end_item, end_tile;
+  long long tb_begin, tb_end;
+  find(begin, start_item, start_tile, tb_begin);
+  find(end, end_item, end_tile, tb_end);
   if (lane == 0) {
     sb->start_item = start_item;
     sb->start_tile = start_tile;
-    sb->count = (int)(end - begin);
+    sb->count = (int)(tb_end - tb_begin);
   }
 }
 
