@@ -42,22 +42,24 @@ namespace {
 constexpr int kProducerWarps = 8;   // cp.async gather (+ TMA for the rope part of q)
 constexpr int kFirstExchangeWarp = 4;
 constexpr int kFirstProducerWarp = 8;
-constexpr int kMmaWarp = 16;
+constexpr int kMmaWarp = 16;    // S = Q . C^T issuer (and TMEM owner)
+constexpr int kPvWarp = 17;     // O += P . C issuer
 // warps 0-3 softmax + epilogue, 4-7 q loader + partial-logit exchange, 8-15 gather, 16 MMA
-constexpr int kAttnThreads = 544;
-// Registers per thread after the split.  The block is launched with kLaunchRegs x 544
-// registers (ptxas' allocation for 544 threads); the softmax warpgroup takes 168 (a tile of
-// fp32 logits), the exchange warpgroup 104, the two gather warpgroups give back down to 56 and
-// the MMA warp keeps the launch value.  The sum stays within the launch allocation, so
+constexpr int kAttnThreads = 576;
+// Registers per thread after the split.  The block is launched with kLaunchRegs x 576
+// registers (ptxas' allocation for 576 threads); the softmax warpgroup takes 152 (a tile of
+// fp32 logits), the exchange warpgroup 104, the two gather warpgroups give back down to 64 and
+// the two MMA warps keep the launch value.  The sum stays within the launch allocation, so
 // setmaxnreg.inc never waits for registers that are not there.
 constexpr int kLaunchRegs = 96;
-constexpr int kSoftmaxRegs = 168;
+constexpr int kSoftmaxRegs = 152;
 constexpr int kExchangeRegs = 104;
-constexpr int kGatherRegs = 56;
-static_assert(128 * kSoftmaxRegs + 256 * kGatherRegs + 128 * kExchangeRegs + 32 * kLaunchRegs <=
+constexpr int kGatherRegs = 64;
+static_assert(128 * kSoftmaxRegs + 256 * kGatherRegs + 128 * kExchangeRegs + 64 * kLaunchRegs <=
                   kAttnThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
-constexpr int kStages = 4;          // latent-row tiles in flight per CTA
+constexpr int kStages = 5;          // latent-row tiles in flight per CTA
+constexpr int kRopeSlots = 2;       // their rope parts (read by S = Q . C^T only) in flight
 constexpr int kRows = kAttnTileRows;
 
 template <int DL, int DR>
@@ -76,10 +78,12 @@ struct AttnLayout<512, 64> {
   __device__ static bool has_rope(int) { return true; }
   __device__ static int rope_x(int r) { return 512 + 32 * r; }
   static constexpr int kChunks0 = 36, kChunks1 = 36;                      // 16-byte pieces per row
+  static constexpr int kLatChunks = 32;                                   // the first 32 are latent
   __device__ static int chunk_src(int r, int k) { return k < 32 ? 512 * r + 16 * k : 1024 + 64 * r + 16 * (k - 32); }
+  // offset inside the latent stage (k < kLatChunks) or inside the rope slot
   __device__ static uint32_t chunk_dst(int row, int k) {
     return k < 32 ? (uint32_t)(k >> 3) * (kAttnTileRows * 128) + swizzled_offset(row, (k & 7) * 16, 128)
-                  : 4u * (kAttnTileRows * 128) + swizzled_offset(row, (k - 32) * 16, 64);
+                  : swizzled_offset(row, (k - 32) * 16, 64);
   }
 };
 
@@ -94,9 +98,10 @@ struct AttnLayout<64, 16> {
   __device__ static bool has_rope(int r) { return r == 0; }
   __device__ static int rope_x(int) { return 64; }
   static constexpr int kChunks0 = 6, kChunks1 = 4;
+  static constexpr int kLatChunks = 4;
   __device__ static int chunk_src(int r, int k) { return k < 4 ? 64 * r + 16 * k : 128 + 16 * (k - 4); }
   __device__ static uint32_t chunk_dst(int row, int k) {
-    return k < 4 ? swizzled_offset(row, k * 16, 64) : (uint32_t)(kAttnTileRows * 64) + swizzled_offset(row, (k - 4) * 16, 32);
+    return k < 4 ? swizzled_offset(row, k * 16, 64) : swizzled_offset(row, (k - 4) * 16, 32);
   }
 };
 
@@ -117,13 +122,14 @@ struct AttnMaps {
 template <class Lay>
 struct AttnSmem {
   static constexpr uint32_t kQRopeBytes = 128 * Lay::kRopeKbw;
-  static constexpr uint32_t kCLatBytes = kRows * Lay::kLatKbw;
-  static constexpr uint32_t kCRopeBytes = kRows * Lay::kRopeKbw;
-  static constexpr uint32_t kCStageBytes = Lay::kLatBlocks * kCLatBytes + kCRopeBytes;
+  static constexpr uint32_t kCLatBytes = kRows * Lay::kLatKbw;       // one latent block of a tile
+  static constexpr uint32_t kCStageBytes = Lay::kLatBlocks * kCLatBytes;
+  static constexpr uint32_t kCRopeBytes = kRows * Lay::kRopeKbw;     // one rope slot
   static constexpr uint32_t kOffQ = 0;                                  // rope part of q only
   static constexpr uint32_t kOffC = (kOffQ + kQRopeBytes + 1023u) & ~1023u;
+  static constexpr uint32_t kOffR = kOffC + kStages * kCStageBytes;
   // P (bf16, 128 heads x kRows, 128B-swizzled K-major): the A operand of P . C
-  static constexpr uint32_t kOffP = kOffC + kStages * kCStageBytes;
+  static constexpr uint32_t kOffP = (kOffR + kRopeSlots * kCRopeBytes + 1023u) & ~1023u;
   static constexpr uint32_t kOffSx = kOffP + 128 * kRows * 2;          // peer logits, fp16
   static constexpr uint32_t kOffRows = kOffSx + kRows * 128 * 2;
   // per unit (double-buffered): physical cache row of each Top-K entry, validity bits, and
@@ -133,10 +139,12 @@ struct AttnSmem {
   static constexpr uint32_t kOffBar = kOffFirstNeg + 2 * kProducerWarps * 4;
   static constexpr uint32_t kBytes = kOffBar + 256;
   static_assert(kOffP % 1024 == 0, "P must sit on a 1024-byte swizzle atom");
+  static_assert(kBytes <= 232448, "shared memory over the 227 KB a CTA may opt into");
 };
 
 struct AttnBarriers {
-  uint64_t c_full[kStages], c_empty[kStages];
+  uint64_t c_full[kStages], c_empty[kStages];   // a tile's rows landed / latent stage free
+  uint64_t r_empty[kRopeSlots];                 // rope slot free (its S = Q . C^T done)
   uint64_t s_full[2], s_empty[2];   // logits ready / read by the softmax and exchange warps
   uint64_t p_full;                  // all softmax threads wrote P (waited by the P . C issuer)
   uint64_t p_empty;                 // P . C of the previous tile done (P buffer and O free)
@@ -145,7 +153,7 @@ struct AttnBarriers {
   uint64_t o_full;
   uint64_t sx_ready, sx_free;
   uint64_t tab_full[2], tab_free[2];
-  uint64_t mma_done;
+  uint64_t mma_done, pv_done;
   uint32_t tmem_base;
   int abort;
 };
@@ -187,7 +195,7 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
 template <int DL, int DR>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     sparse_attend_kernel(const __grid_constant__ AttnMaps maps, const AttnKernelParams p) {
-  static_assert(kAttnThreads == 544, "role layout assumes 17 warps");
+  static_assert(kAttnThreads == 576, "role layout assumes 18 warps");
   using Lay = AttnLayout<DL, DR>;
   using Sm = AttnSmem<Lay>;
   using Tm = AttnTmem<Lay>;
@@ -213,11 +221,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(&sb->c_full[s], kProducerWarps * 32);  // one cp.async completion per gather thread
       mbar_init(&sb->c_empty[s], 1);
     }
+    for (int s = 0; s < kRopeSlots; ++s) mbar_init(&sb->r_empty[s], 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sb->s_full[s], 1);
       mbar_init(&sb->s_empty[s], 128 + 128);   // softmax and exchange threads
       mbar_init(&sb->tab_full[s], kProducerWarps * 32);
-      mbar_init(&sb->tab_free[s], 128 + 128 + 1);   // softmax, exchange and MMA threads
+      mbar_init(&sb->tab_free[s], 128 + 128 + 2);   // softmax, exchange and both MMA threads
     }
     mbar_init(&sb->p_full, 128);
     mbar_init(&sb->p_empty, 1);
@@ -228,6 +237,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     mbar_init(&sb->sx_ready, 128);   // arrived by the peer's 128 exchange threads
     mbar_init(&sb->sx_free, 128);    // arrived by the peer's 128 softmax threads
     mbar_init(&sb->mma_done, 1);
+    mbar_init(&sb->pv_done, 1);
     sb->abort = 0;
     fence_mbarrier_init();
     tma_prefetch_desc(&maps.q_rope);
@@ -259,14 +269,35 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int ptid = threadIdx.x - kFirstProducerWarp * 32;   // 0..255
     const int pwarp = warp - kFirstProducerWarp;
     const uint8_t* kv = static_cast<const uint8_t*>(p.kv);
-    // one tile of gathers: consecutive threads take consecutive 16-byte pieces of a row, so a
-    // warp reads whole 512-byte runs of a latent row at a time
-    auto gather_tile = [&](auto nch_c, uint32_t cst, const int32_t* rows) {
-      constexpr int NCH = decltype(nch_c)::value;
-#pragma unroll 4
-      for (int i = ptid; i < kRows * NCH; i += kProducerWarps * 32) {
-        const int row = i / NCH, k = i - row * NCH;
-        cp_async16(cst + Lay::chunk_dst(row, k), kv + (size_t)(uint32_t)rows[row] * (DC * 2) + Lay::chunk_src((int)rank, k));
+    // One tile of gathers: consecutive threads take consecutive 16-byte pieces of a row, so a
+    // warp reads whole 512-byte runs of a latent row at a time.  A thread's pieces are the same
+    // for every tile, so their row, source offset and destination (latent stage or rope slot)
+    // are packed once: row [0,6), source/16 [6,13), rope flag 13, destination/16 [14,26), and
+    // bit 26 when the piece exists.
+    const int nch = rank == 0 ? Lay::kChunks0 : Lay::kChunks1;
+    constexpr int kPer = (kRows * (Lay::kChunks0 > Lay::kChunks1 ? Lay::kChunks0 : Lay::kChunks1) +
+                          kProducerWarps * 32 - 1) / (kProducerWarps * 32);
+    uint32_t piece[kPer];
+    auto make_pieces = [&]() {
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) {
+        const int i = ptid + j * kProducerWarps * 32;
+        const int row = i / nch, k = i - row * nch;
+        const bool lat = k < Lay::kLatChunks;
+        piece[j] = i < kRows * nch
+                       ? (uint32_t)row | ((uint32_t)Lay::chunk_src((int)rank, k) / 16u) << 6 | (lat ? 0u : 1u) << 13 |
+                             (Lay::chunk_dst(row, k) / 16u) << 14 | 1u << 26
+                       : 0u;
+      }
+    };
+    auto gather_tile = [&](uint32_t lat_base, uint32_t rope_base, const int32_t* rows) {
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) {
+        const uint32_t pc = piece[j];
+        if (pc >> 26) {
+          const uint8_t* src = kv + (size_t)(uint32_t)rows[pc & 63u] * (DC * 2) + ((pc >> 6) & 127u) * 16u;
+          cp_async16(((pc >> 13) & 1u ? rope_base : lat_base) + ((pc >> 14) & 4095u) * 16u, src);
+        }
       }
     };
     int it = 0, u_it = 0;
@@ -350,134 +381,102 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_arrive(&sb->tab_full[buf]);
       if (!mbar_wait(&sb->tab_full[buf], (uint32_t)(u_it >> 1) & 1u, abort, p.status)) { ok = false; break; }
       const int ntiles = (unit_tiles(buf) + kRows - 1) / kRows;
+      make_pieces();   // (after the table: the two never hold registers at the same time)
       for (int t = 0; t < ntiles; ++t, ++it) {
-        const int stage = it % kStages;
+        const int stage = it % kStages, rslot = it % kRopeSlots;
         if (!mbar_wait(&sb->c_empty[stage], ((uint32_t)(it / kStages) & 1u) ^ 1u, abort, p.status)) { ok = false; break; }
-        const uint32_t cst = smem_u32(smem + Sm::kOffC + stage * Sm::kCStageBytes);
-        const int32_t* rows = rt + t * kRows;
-        if (rank == 0) gather_tile(std::integral_constant<int, Lay::kChunks0>{}, cst, rows);
-        else gather_tile(std::integral_constant<int, Lay::kChunks1>{}, cst, rows);
+        if (!mbar_wait(&sb->r_empty[rslot], ((uint32_t)(it / kRopeSlots) & 1u) ^ 1u, abort, p.status)) { ok = false; break; }
+        gather_tile(smem_u32(smem + Sm::kOffC + stage * Sm::kCStageBytes),
+                    smem_u32(smem + Sm::kOffR + rslot * Sm::kCRopeBytes), rt + t * kRows);
         asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(&sb->c_full[stage])) : "memory");
       }
     }
     asm volatile("cp.async.wait_all;" ::: "memory");  // our copies have landed before we may leave
     if (ptid == 0 && u_it > 0) mbar_wait(&sb->q_full, (uint32_t)(u_it - 1) & 1u, abort, p.status);
   } else if (warp == kMmaWarp) {
-    // ---------------------------------------------------------------- MMA issuer
-    // Two cursors over the same sequence of (unit, tile): S = Q . C^T of a tile can start as
-    // soon as its rows have landed and a logit buffer is free, O += P . C as soon as the
-    // softmax has written P.  The issuer polls both and issues whichever is ready, so neither
-    // product waits behind the other's inputs.
+    // ---------------------------------------------------------------- S = Q . C^T issuer
+    // (O += P . C has its own issuing warp, so a logit tile never waits for P of an earlier
+    // tile and P never waits for a logit tile being issued)
     if (lane == 0) {
       const uint32_t idesc_qk = umma_idesc(1, 1, false, false, kRows, 128);
-      const uint32_t idesc_pv = umma_idesc(1, 1, false, true, Lay::kPvN, 128);
       const uint32_t qr_base = smem_u32(smem + Sm::kOffQ);
-      const uint32_t p_base = smem_u32(smem + Sm::kOffP);
-      int nt_ring[4];                       // tile counts of units the S cursor has opened
-      // S cursor: 0 = needs the unit's table, 1 = needs q, 2 = issuing tiles
-      int q_u = cluster_id, q_uit = 0, q_state = 0, q_nt = 0, q_t = 0, q_it = 0;
-      // P cursor
-      int p_u = cluster_id, p_uit = 0, p_t = 0, p_it = 0;
+      int it = 0, u_it = 0;
       bool ok = true;
-      uint64_t last = globaltimer_ns();
-      while (ok && (q_u < p.units || p_u < p.units)) {
-        bool progress = false;
-        if (q_u < p.units) {
-          const int buf = q_uit & 1;
-          if (q_state == 0 && mbar_test(&sb->tab_full[buf], (uint32_t)(q_uit >> 1) & 1u)) {
-            q_nt = (unit_tiles(buf) + kRows - 1) / kRows;
-            nt_ring[q_uit & 3] = q_nt;
-            mbar_arrive(&sb->tab_free[buf]);
-            q_state = 1;
-            progress = true;
-          }
-          if (q_state == 1 && mbar_test(&sb->q_full, (uint32_t)q_uit & 1u)) {
-            tc_fence_after();
-            q_state = 2;
-            q_t = 0;
-            progress = true;
-          }
-          if (q_state == 2 && q_t < q_nt) {
-            const int stage = q_it % kStages;
-            const int sbuf = q_it & 1;
-            if (mbar_test(&sb->c_full[stage], (uint32_t)(q_it / kStages) & 1u) &&
-                mbar_test(&sb->s_empty[sbuf], ((uint32_t)(q_it >> 1) & 1u) ^ 1u)) {
-              fence_proxy_async_smem();   // the gathered rows were written by cp.async
-              tc_fence_after();
-              const uint32_t c_base = smem_u32(smem + Sm::kOffC + stage * Sm::kCStageBytes);
-              const uint32_t d = tmem_base + Tm::kS + (uint32_t)(sbuf * kRows);
-              constexpr int kSub = Lay::kLatKbw / 32;   // 16-element K steps per swizzled block
+      for (int u = cluster_id; u < p.units && ok; u += n_clusters, ++u_it) {
+        const int buf = u_it & 1;
+        if (!mbar_wait(&sb->tab_full[buf], (uint32_t)(u_it >> 1) & 1u, abort, p.status)) { ok = false; break; }
+        const int ntiles = (unit_tiles(buf) + kRows - 1) / kRows;
+        mbar_arrive(&sb->tab_free[buf]);
+        if (!mbar_wait(&sb->q_full, (uint32_t)u_it & 1u, abort, p.status)) { ok = false; break; }
+        tc_fence_after();
+        for (int t = 0; t < ntiles; ++t, ++it) {
+          const int stage = it % kStages;
+          const int sbuf = it & 1;
+          if (!mbar_wait(&sb->c_full[stage], (uint32_t)(it / kStages) & 1u, abort, p.status)) { ok = false; break; }
+          if (!mbar_wait(&sb->s_empty[sbuf], ((uint32_t)(it >> 1) & 1u) ^ 1u, abort, p.status)) { ok = false; break; }
+          fence_proxy_async_smem();   // the gathered rows were written by cp.async
+          tc_fence_after();
+          const uint32_t c_base = smem_u32(smem + Sm::kOffC + stage * Sm::kCStageBytes);
+          const uint32_t d = tmem_base + Tm::kS + (uint32_t)(sbuf * kRows);
+          constexpr int kSub = Lay::kLatKbw / 32;   // 16-element K steps per swizzled block
 #pragma unroll
-              for (int g = 0; g < Lay::kLatDims / 16; ++g) {
-                const uint64_t bd = umma_smem_desc(c_base + (g / kSub) * Sm::kCLatBytes + (g % kSub) * 32, 16,
-                                                   8 * Lay::kLatKbw, umma_layout_type(Lay::kLatKbw));
-                umma_f16_ts(d, tmem_base + Tm::kQ + (uint32_t)(8 * g), bd, idesc_qk, g > 0);
-              }
-              if (rope) {
+          for (int g = 0; g < Lay::kLatDims / 16; ++g) {
+            const uint64_t bd = umma_smem_desc(c_base + (g / kSub) * Sm::kCLatBytes + (g % kSub) * 32, 16,
+                                               8 * Lay::kLatKbw, umma_layout_type(Lay::kLatKbw));
+            umma_f16_ts(d, tmem_base + Tm::kQ + (uint32_t)(8 * g), bd, idesc_qk, g > 0);
+          }
+          const int rslot = it % kRopeSlots;
+          if (rope) {
+            const uint32_t r_base = smem_u32(smem + Sm::kOffR + rslot * Sm::kCRopeBytes);
 #pragma unroll
-                for (int ks = 0; ks < Lay::kRopeKbw / 32; ++ks) {
-                  const uint64_t ad = umma_smem_desc(qr_base + ks * 32, 16, 8 * Lay::kRopeKbw, umma_layout_type(Lay::kRopeKbw));
-                  const uint64_t bd = umma_smem_desc(c_base + Lay::kLatBlocks * Sm::kCLatBytes + ks * 32, 16,
-                                                     8 * Lay::kRopeKbw, umma_layout_type(Lay::kRopeKbw));
-                  umma_f16(d, ad, bd, idesc_qk, true);
-                }
-              }
-              umma_commit(&sb->s_full[sbuf]);
-              ++q_it;
-              ++q_t;
-              progress = true;
+            for (int ks = 0; ks < Lay::kRopeKbw / 32; ++ks) {
+              const uint64_t ad = umma_smem_desc(qr_base + ks * 32, 16, 8 * Lay::kRopeKbw, umma_layout_type(Lay::kRopeKbw));
+              const uint64_t bd = umma_smem_desc(r_base + ks * 32, 16, 8 * Lay::kRopeKbw, umma_layout_type(Lay::kRopeKbw));
+              umma_f16(d, ad, bd, idesc_qk, true);
             }
           }
-          if (q_state == 2 && q_t == q_nt) {
-            umma_commit(&sb->q_empty);  // q reusable once this unit's products are done
-            q_u += n_clusters;
-            ++q_uit;
-            q_state = 0;
-            progress = true;
-          }
+          umma_commit(&sb->s_full[sbuf]);
+          umma_commit(&sb->r_empty[rslot]);
         }
-        if (p_u < p.units && p_uit < q_uit + (q_state > 0 ? 1 : 0)) {
-          const int nt = nt_ring[p_uit & 3];
-          if (p_t < nt && mbar_test(&sb->p_full, (uint32_t)p_it & 1u)) {
-            fence_proxy_async_smem();   // the row stage (cp.async) and P (st.shared)
-            tc_fence_after();
-            const int stage = p_it % kStages;
-            const uint32_t c_base = smem_u32(smem + Sm::kOffC + stage * Sm::kCStageBytes);
-#pragma unroll
-            for (int ks = 0; ks < kRows / 16; ++ks) {
-              const uint64_t ad = umma_smem_desc(p_base + ks * 32, 16, 1024, umma_layout_type(128));
-              const uint64_t bd = umma_smem_desc(c_base + ks * 16 * Lay::kLatKbw, Sm::kCLatBytes,
-                                                 8 * Lay::kLatKbw, umma_layout_type(Lay::kLatKbw));
-              umma_f16(tmem_base + Tm::kO, ad, bd, idesc_pv, p_t > 0 || ks > 0);
-            }
-            umma_commit(&sb->c_empty[stage]);
-            umma_commit(&sb->p_empty);
-            ++p_it;
-            ++p_t;
-            if (p_t == nt) umma_commit(&sb->o_full);
-            progress = true;
-          }
-          if (p_t == nt) {
-            p_u += n_clusters;
-            ++p_uit;
-            p_t = 0;
-            progress = true;
-          }
-        }
-        if (progress) {
-          last = globaltimer_ns();
-        } else {
-          if (*abort) { ok = false; break; }
-          if (globaltimer_ns() - last > kWaitTimeoutNs) {
-            *abort = 1;
-            report(p.status, SIA_DEV_TIMEOUT);
-            ok = false;
-            break;
-          }
-        }
+        if (!ok) break;
+        umma_commit(&sb->q_empty);  // q reusable once this unit's products are done
       }
       umma_commit(&sb->mma_done);
       mbar_wait(&sb->mma_done, 0, abort, p.status);
+    }
+    __syncwarp();
+  } else if (warp == kPvWarp) {
+    // ---------------------------------------------------------------- O += P . C issuer
+    if (lane == 0) {
+      const uint32_t idesc_pv = umma_idesc(1, 1, false, true, Lay::kPvN, 128);
+      const uint32_t p_base = smem_u32(smem + Sm::kOffP);
+      int it = 0, u_it = 0;
+      bool ok = true;
+      for (int u = cluster_id; u < p.units && ok; u += n_clusters, ++u_it) {
+        const int buf = u_it & 1;
+        if (!mbar_wait(&sb->tab_full[buf], (uint32_t)(u_it >> 1) & 1u, abort, p.status)) { ok = false; break; }
+        const int ntiles = (unit_tiles(buf) + kRows - 1) / kRows;
+        mbar_arrive(&sb->tab_free[buf]);
+        for (int t = 0; t < ntiles; ++t, ++it) {
+          if (!mbar_wait(&sb->p_full, (uint32_t)it & 1u, abort, p.status)) { ok = false; break; }
+          fence_proxy_async_smem();   // the row stage (cp.async) and P (st.shared)
+          tc_fence_after();
+          const int stage = it % kStages;
+          const uint32_t c_base = smem_u32(smem + Sm::kOffC + stage * Sm::kCStageBytes);
+#pragma unroll
+          for (int ks = 0; ks < kRows / 16; ++ks) {
+            const uint64_t ad = umma_smem_desc(p_base + ks * 32, 16, 1024, umma_layout_type(128));
+            const uint64_t bd = umma_smem_desc(c_base + ks * 16 * Lay::kLatKbw, Sm::kCLatBytes,
+                                               8 * Lay::kLatKbw, umma_layout_type(Lay::kLatKbw));
+            umma_f16(tmem_base + Tm::kO, ad, bd, idesc_pv, t > 0 || ks > 0);
+          }
+          umma_commit(&sb->c_empty[stage]);
+          umma_commit(&sb->p_empty);
+          if (t + 1 == ntiles) umma_commit(&sb->o_full);
+        }
+      }
+      umma_commit(&sb->pv_done);
+      mbar_wait(&sb->pv_done, 0, abort, p.status);
     }
     __syncwarp();
   } else if (warp >= kFirstExchangeWarp && warp < kFirstExchangeWarp + 4) {
