@@ -58,7 +58,7 @@ constexpr int kGatherRegs = 64;
 static_assert(128 * kSoftmaxRegs + 256 * kGatherRegs + 128 * kExchangeRegs + 64 * kLaunchRegs <=
                   kAttnThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
-constexpr int kStages = 5;          // latent-row tiles in flight per CTA
+constexpr int kStages = 4;          // latent-row tiles in flight per CTA
 constexpr int kRopeSlots = 2;       // their rope parts (read by S = Q . C^T only) in flight
 constexpr int kRows = kAttnTileRows;
 
@@ -131,13 +131,17 @@ struct AttnSmem {
   // P (bf16, 128 heads x kRows, 128B-swizzled K-major): the A operand of P . C
   static constexpr uint32_t kOffP = (kOffR + kRopeSlots * kCRopeBytes + 1023u) & ~1023u;
   static constexpr uint32_t kOffSx = kOffP + 128 * kRows * 2;          // peer logits, fp16
-  static constexpr uint32_t kOffRows = kOffSx + kRows * 128 * 2;
+  // this CTA's own logits, fp16, two tiles: the exchange warps copy them out of TMEM so that a
+  // logit buffer is free for the next product as soon as they have read it
+  static constexpr uint32_t kOffStash = kOffSx + kRows * 128 * 2;
+  static constexpr uint32_t kOffRows = kOffStash + 2 * kRows * 128 * 2;
   // per unit (double-buffered): physical cache row of each Top-K entry, validity bits, and
   // each gather warp's lowest position of a -1 entry
   static constexpr uint32_t kOffMask = kOffRows + 2 * kAttnMaxSplitRows * 4;
   static constexpr uint32_t kOffFirstNeg = kOffMask + 2 * (kAttnMaxSplitRows / 8);
   static constexpr uint32_t kOffBar = kOffFirstNeg + 2 * kProducerWarps * 4;
-  static constexpr uint32_t kBytes = kOffBar + 256;
+  static constexpr uint32_t kBarBytes = 512;
+  static constexpr uint32_t kBytes = kOffBar + kBarBytes;
   static_assert(kOffP % 1024 == 0, "P must sit on a 1024-byte swizzle atom");
   static_assert(kBytes <= 232448, "shared memory over the 227 KB a CTA may opt into");
 };
@@ -145,7 +149,8 @@ struct AttnSmem {
 struct AttnBarriers {
   uint64_t c_full[kStages], c_empty[kStages];   // a tile's rows landed / latent stage free
   uint64_t r_empty[kRopeSlots];                 // rope slot free (its S = Q . C^T done)
-  uint64_t s_full[2], s_empty[2];   // logits ready / read by the softmax and exchange warps
+  uint64_t s_full[2], s_empty[2];   // logits ready in TMEM / read by the exchange warps
+  uint64_t own_ready[2], own_free[2];   // own fp16 logits stashed / read by the softmax
   uint64_t p_full;                  // all softmax threads wrote P (waited by the P . C issuer)
   uint64_t p_empty;                 // P . C of the previous tile done (P buffer and O free)
   uint64_t epi_sync;                // all softmax threads are past the unit's last tile
@@ -157,6 +162,8 @@ struct AttnBarriers {
   uint32_t tmem_base;
   int abort;
 };
+
+static_assert(sizeof(AttnBarriers) <= 512, "barrier block outgrew its shared-memory slot");
 
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
@@ -224,7 +231,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     for (int s = 0; s < kRopeSlots; ++s) mbar_init(&sb->r_empty[s], 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sb->s_full[s], 1);
-      mbar_init(&sb->s_empty[s], 128 + 128);   // softmax and exchange threads
+      mbar_init(&sb->s_empty[s], 128);         // exchange threads
+      mbar_init(&sb->own_ready[s], 128);
+      mbar_init(&sb->own_free[s], 128);
       mbar_init(&sb->tab_full[s], kProducerWarps * 32);
       mbar_init(&sb->tab_free[s], 128 + 128 + 2);   // softmax, exchange and both MMA threads
     }
@@ -549,6 +558,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         tc_fence_before();
         mbar_arrive(&sb->s_empty[sbuf]);   // our reads of these logits are done
+        // own fp16 logits for our softmax (the same values the peer receives)
+        if (!mbar_wait(&sb->own_free[sbuf], ((uint32_t)(s_it >> 1) & 1u) ^ 1u, abort, p.status)) { ok = false; break; }
+#pragma unroll
+        for (int g = 0; g < kRows / 8; ++g)
+          st_shared_v4(smem_u32(smem + Sm::kOffStash + sbuf * (kRows * 128 * 2) + (g * 128 + h) * 16),
+                       own[4 * g], own[4 * g + 1], own[4 * g + 2], own[4 * g + 3]);
+        mbar_arrive(&sb->own_ready[sbuf]);
         if (!mbar_wait<true>(&sb->sx_free, ((uint32_t)s_it & 1u) ^ 1u, abort, p.status)) { ok = false; break; }
 #pragma unroll
         for (int g = 0; g < kRows / 8; ++g)
@@ -577,39 +593,30 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       float m = -INFINITY, l = 0.0f;
       float s[kRows];
       for (int t = 0; t < ntiles; ++t, ++s_it) {
-        // logits of tile t (base 2) = own fp32 partial (TMEM) + the peer's fp16 partial
         const int sbuf = s_it & 1;
-        const uint32_t scol = lane_addr + Tm::kS + sbuf * kRows;
         uint64_t valid = ((uint64_t)mt[2 * t + 1] << 32) | mt[2 * t];
         const int live = first_neg - t * kRows;            // rows past the first -1 are padding
         if (live < kRows) valid &= (1ull << live) - 1ull;
-        if (!mbar_wait(&sb->s_full[sbuf], (uint32_t)(s_it >> 1) & 1u, abort, p.status)) { ok = false; break; }
+        if (!mbar_wait(&sb->own_ready[sbuf], (uint32_t)(s_it >> 1) & 1u, abort, p.status)) { ok = false; break; }
         if (!mbar_wait<true>(&sb->sx_ready, (uint32_t)s_it & 1u, abort, p.status)) { ok = false; break; }
-        tc_fence_after();
+        // logits of tile t (base 2) = own fp16 partial + the peer's fp16 partial: both CTAs add
+        // the same two values, so their logits agree bit for bit
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t r[2][16];
-          tmem_ld16(scol + half * 32, r[0]);
-          tmem_ld16(scol + half * 32 + 16, r[1]);
-          tmem_wait_ld();
+        for (int g = 0; g < kRows / 8; ++g) {
+          const uint4 ov = *reinterpret_cast<const uint4*>(smem + Sm::kOffStash + sbuf * (kRows * 128 * 2) + (g * 128 + h) * 16);
+          const uint4 pv4 = *reinterpret_cast<const uint4*>(smem + Sm::kOffSx + (g * 128 + h) * 16);
+          const uint32_t o4[4] = {ov.x, ov.y, ov.z, ov.w};
+          const uint32_t q4[4] = {pv4.x, pv4.y, pv4.z, pv4.w};
 #pragma unroll
-          for (int g2 = 0; g2 < 4; ++g2) {
-            const int g = half * 4 + g2;
-            const uint4 v = *reinterpret_cast<const uint4*>(smem + Sm::kOffSx + (g * 128 + h) * 16);
-            const uint32_t pv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int col = g2 * 8 + 2 * i;
-              float lo = __uint_as_float(r[col >> 4][col & 15]) * p.scale_log2;
-              float hi = __uint_as_float(r[col >> 4][(col & 15) + 1]) * p.scale_log2;
-              add_f16x2_to_f32(pv[i], lo, hi);
-              s[8 * g + 2 * i] = lo;
-              s[8 * g + 2 * i + 1] = hi;
-            }
+          for (int i = 0; i < 4; ++i) {
+            float lo = 0.0f, hi = 0.0f;
+            add_f16x2_to_f32(o4[i], lo, hi);   // exact: fp16 -> fp32
+            add_f16x2_to_f32(q4[i], lo, hi);   // one rounding
+            s[8 * g + 2 * i] = lo;
+            s[8 * g + 2 * i + 1] = hi;
           }
         }
-        tc_fence_before();
-        mbar_arrive(&sb->s_empty[sbuf]);
+        mbar_arrive(&sb->own_free[sbuf]);
         // the peer may refill the exchange buffer (the logit values read above are already in
         // registers); after the unit's last tile the buffer first serves the epilogue
         if (t + 1 < ntiles) mbar_arrive_cluster_relaxed(&sb->sx_free, peer);
