@@ -213,6 +213,23 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def max_over_ranks(values, device):
+    """Each value's maximum over the ranks of the job (device times: a job is as slow as its
+    slowest rank).  One all-reduce; identity when there is no process group."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def job_rate(world, units_per_rank, ms):
+    """Whole-job throughput: every rank processed units_per_rank in (at most) ms."""
+    return world * units_per_rank / (ms / 1000.0)
+
+
 def metric_name(wl):
     return "fused sparse-attn decode queries/s @B=%d ctx=%s; achieved HBM GB/s %% of peak" % (
         wl.batch, "8K" if wl.context == 8192 else str(wl.context or "1k-32k"))
@@ -274,10 +291,7 @@ def run_prefill_scoring(args, rank, world, dev, wl):
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / steps
     clocks = sampler.stop()
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    (ms,) = max_over_ranks([ms], dev)
     if int(status.item()) != 0:
         raise RuntimeError("device status %d" % int(status.item()))
     flops = prefill_scoring_flops(host["seq_lens"].tolist(), J, wl.idx_heads, wl.idx_dim)
@@ -396,10 +410,7 @@ def main():
     if bad:
         raise RuntimeError("device status %#x during the benchmark" % bad[0])
 
-    if world > 1:
-        t = torch.tensor([mean_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        mean_ms = float(t.item())
+    mean_ms, s1, s2 = max_over_ranks([mean_ms, s1, s2], dev)
 
     # ---------------- end-to-end through the C ABI with host buffers
     pin = {k: host[k].pin_memory() for k in ("q_idx", "w", "q_attn", "page_table", "seq_lens")}
@@ -421,13 +432,10 @@ def main():
         e2e_step()
     torch.cuda.synchronize()
     e2e_ms = timed([e2e_step], max(10, args.steps // 4))
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    (e2e_ms,) = max_over_ranks([e2e_ms], dev)
 
     queries = host["batch"] * host["n_q"]
-    value = world * queries / (mean_ms / 1000.0)
+    value = job_rate(world, queries, mean_ms)
     ab = algorithmic_bytes(host)
     pk = peaks()
     dominant = "sparse_attend" if s2 >= s1 else "index_topk"
@@ -453,7 +461,7 @@ def main():
                    "index_topk_gbs": ab["stage1"] / (s1 / 1000.0) / 1e9,
                    "sparse_attend_gbs": ab["stage2"] / (s2 / 1000.0) / 1e9,
                    "step_algorithmic_bytes": ab["total"]},
-        "e2e": {"value": world * queries / (e2e_ms / 1000.0), "unit": "queries/s",
+        "e2e": {"value": job_rate(world, queries, e2e_ms), "unit": "queries/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": kernels_per_step * args.steps,
         "clocks": clocks,
