@@ -190,6 +190,7 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
     int it = 0;
     int item = start_item, t0 = start_tile, remaining = my_count;
     bool ok = true;
+    const uint64_t stream_policy = l2_evict_first_policy();   // keys are read once per call
     while (remaining > 0 && ok) {
       const GroupInfo gi = group_info(p, item);
       const int t1 = min(gi.n_tiles, t0 + remaining);
@@ -237,8 +238,8 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
           const int y = my_page * p.P + (my_pos % p.P);
 #pragma unroll
           for (int kb = 0; kb < NKB; ++kb)
-            tma_load_2d(kst + kb * p.k_kblock_bytes + lane * p.box_rows * KBW, &kmap,
-                        &sb->k_full[stage], kb * KBW / (FP8 ? 1 : 2), y);
+            tma_load_2d_hint(kst + kb * p.k_kblock_bytes + lane * p.box_rows * KBW, &kmap,
+                             &sb->k_full[stage], kb * KBW / (FP8 ? 1 : 2), y, stream_policy);
           if (p.k_scale)
             bulk_load(info + 16 + lane * p.box_rows * 4, p.k_scale + (long long)y, scale_bytes,
                       &sb->k_full[stage]);

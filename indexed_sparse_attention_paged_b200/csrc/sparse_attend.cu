@@ -187,8 +187,9 @@ __device__ __forceinline__ void add_f16x2_to_f32(uint32_t h, float& lo, float& h
       : "r"(h));
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+__device__ __forceinline__ void cp_async16_hint(uint32_t dst, const void* src, uint64_t policy) {
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "l"(policy)
+               : "memory");
 }
 
 __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
@@ -283,6 +284,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // for every tile, so their row, source offset and destination (latent stage or rope slot)
     // are packed once: row [0,6), source/16 [6,13), rope flag 13, destination/16 [14,26), and
     // bit 26 when the piece exists.
+    // latent rows are read once per call: evict them first, so the split partials this kernel
+    // writes stay in L2 for the merge
+    const uint64_t stream_policy = l2_evict_first_policy();
     const int nch = rank == 0 ? Lay::kChunks0 : Lay::kChunks1;
     constexpr int kPer = (kRows * (Lay::kChunks0 > Lay::kChunks1 ? Lay::kChunks0 : Lay::kChunks1) +
                           kProducerWarps * 32 - 1) / (kProducerWarps * 32);
@@ -305,7 +309,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const uint32_t pc = piece[j];
         if (pc >> 26) {
           const uint8_t* src = kv + (size_t)(uint32_t)rows[pc & 63u] * (DC * 2) + ((pc >> 6) & 127u) * 16u;
-          cp_async16(((pc >> 13) & 1u ? rope_base : lat_base) + ((pc >> 14) & 4095u) * 16u, src);
+          cp_async16_hint(((pc >> 13) & 1u ? rope_base : lat_base) + ((pc >> 14) & 4095u) * 16u, src, stream_policy);
         }
       }
     };
