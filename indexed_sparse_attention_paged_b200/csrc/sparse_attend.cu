@@ -547,18 +547,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (!mbar_wait(&sb->s_full[sbuf], (uint32_t)(s_it >> 1) & 1u, abort, p.status)) { ok = false; break; }
         tc_fence_after();
         uint32_t own[kRows / 2];
+        {
+          uint32_t r[4][16];   // the whole tile's row in one TMEM wait
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t r[2][16];
-          tmem_ld16(scol + half * 32, r[0]);
-          tmem_ld16(scol + half * 32 + 16, r[1]);
+          for (int c = 0; c < 4; ++c) tmem_ld16(scol + c * 16, r[c]);
           tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 2; ++c)
+          for (int c = 0; c < 4; ++c)
 #pragma unroll
             for (int i = 0; i < 8; ++i)
-              own[half * 16 + c * 8 + i] = pack_f16x2(__uint_as_float(r[c][2 * i]) * p.scale_log2,
-                                                      __uint_as_float(r[c][2 * i + 1]) * p.scale_log2);
+              own[c * 8 + i] = pack_f16x2(__uint_as_float(r[c][2 * i]) * p.scale_log2,
+                                          __uint_as_float(r[c][2 * i + 1]) * p.scale_log2);
         }
         tc_fence_before();
         mbar_arrive(&sb->s_empty[sbuf]);   // our reads of these logits are done
@@ -711,14 +710,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll 1
         for (int c = 0; c < Lay::kPvN; c += 64) {
           uint32_t w[32];
+          {
+            // four loads in flight per TMEM wait (a wait per load made the epilogue latency bound)
+            uint32_t r[4][16];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint32_t r[16];
-            tmem_ld16(lane_addr + Tm::kO + c + 16 * q, r);   // past kPvN: other columns, not stored
+            for (int q = 0; q < 4; ++q) tmem_ld16(lane_addr + Tm::kO + c + 16 * q, r[q]);   // past kPvN: not stored
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-              w[8 * q + i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
+            for (int q = 0; q < 4; ++q)
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                w[8 * q + i] = pack_bf16x2(__uint_as_float(r[q][2 * i]) * inv, __uint_as_float(r[q][2 * i + 1]) * inv);
           }
           __syncwarp();
 #pragma unroll
