@@ -217,7 +217,8 @@ constexpr int kRowPer = 16;
 constexpr int kRowKeys = kRowThreads * kRowPer;
 
 struct RowShared {
-  uint32_t hist[kBins];
+  uint32_t hist[2][kBins];          // alternate passes use alternate histograms
+  int wtot[kRowThreads / 32];       // per-warp totals of the bin scan
   int warp_a[kRowThreads / 32];
   int warp_b[kRowThreads / 32];
   uint32_t sel_prefix;
@@ -299,21 +300,35 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_row_kernel(const TopkKern
   int krem = p.K;
   const int shifts[3] = {21, 10, 0};
   const int widths[3] = {11, 11, 10};
+  for (int i = tid; i < kBins; i += kRowThreads) sh->hist[0][i] = 0;
+  __syncthreads();
 #pragma unroll 1
   for (int pass = 0; pass < 3; ++pass) {
-    for (int i = tid; i < kBins; i += kRowThreads) sh->hist[i] = 0;
-    __syncthreads();
+    uint32_t* hist = sh->hist[pass & 1];
+    // the other histogram is cleared for the next pass (nobody reads it in this one)
+    for (int i = tid; i < kBins; i += kRowThreads) sh->hist[(pass + 1) & 1][i] = 0;
     const int sh_ = shifts[pass], hi_shift = sh_ + widths[pass];
     const uint32_t dmask = (1u << widths[pass]) - 1u;
 #pragma unroll
     for (int i = 0; i < kRowPer; ++i)
-      if (i < nmine && (pass == 0 || (key[i] >> hi_shift) == prefix)) atomicAdd(&sh->hist[(key[i] >> sh_) & dmask], 1u);
+      if (i < nmine && (pass == 0 || (key[i] >> hi_shift) == prefix)) atomicAdd(&hist[(key[i] >> sh_) & dmask], 1u);
     __syncthreads();
-    // thread t owns bins 2t, 2t+1; "above" = keys in higher bins, via a scan in reversed order
+    // thread t owns bins 2t, 2t+1 counted from the top; "above" = keys in higher bins, by a warp
+    // scan plus the totals of the warps before (each warp adds those up itself)
+    const int lane = tid & 31, wid = tid >> 5;
     const int hi_bin = kBins - 2 - 2 * tid;        // reversed: thread 0 owns the two top bins
-    const int c1 = (int)sh->hist[hi_bin + 1], c0 = (int)sh->hist[hi_bin];
-    int ex, dummy, tot, tot2;
-    row_scan2(c0 + c1, 0, ex, dummy, tot, tot2, sh);
+    const int c1 = (int)hist[hi_bin + 1], c0 = (int)hist[hi_bin];
+    int incl = c0 + c1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) sh->wtot[wid] = incl;
+    __syncthreads();
+    int before = 0;
+    for (int w = 0; w < wid; ++w) before += sh->wtot[w];
+    const int ex = before + incl - (c0 + c1);
     if (ex < krem && krem <= ex + c1) {
       sh->sel_prefix = (prefix << widths[pass]) | (uint32_t)(hi_bin + 1);
       sh->sel_krem = krem - ex;
@@ -324,7 +339,6 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_row_kernel(const TopkKern
     __syncthreads();
     prefix = sh->sel_prefix;
     krem = sh->sel_krem;
-    __syncthreads();
   }
   const uint32_t T = prefix;
 
