@@ -163,7 +163,10 @@ sia_status sia_sparse_mla_attend(const sia_attend_args* a, void* workspace, size
 sia_status sia_sparse_index_topk_noalloc(const sia_index_args* a, int32_t* dev_status, void* stream);
 
 /* Both stages back to back on one stream (programmatic dependent launch between kernels, no
- * host synchronisation; capturable in a CUDA graph).  The two argument sets must describe the
+ * host synchronisation; capturable in a CUDA graph).  Stream order is kept: the first kernel of
+ * this call (and of sia_sparse_index_topk and sia_index_scores) may be scheduled while the
+ * previous kernel on the stream drains, but it reads and writes no global memory before that
+ * kernel has completed.  The two argument sets must describe the
  * same sequences: equal batch, n_q, page_size, max_pages_per_seq, top_k, page_table and
  * seq_lens, with aa->topk == ia->topk_out. */
 sia_status sia_fused_decode(const sia_index_args* ia, const sia_attend_args* aa,

@@ -150,9 +150,13 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
   constexpr int kEpiThreads = 128 * NSUB;
 
   if ((smem_u32(smem) & 1023u) != 0) {  // the swizzled layouts need a 1024-byte aligned base
+    pdl_wait_primary();
     if (threadIdx.x == 0) report(p.status, SIA_DEV_TIMEOUT);
     return;
   }
+  // The next kernel on the stream may be scheduled as soon as every CTA of this grid runs: it
+  // waits for this grid's completion itself, so only its launch and set-up overlap this grid.
+  pdl_launch_dependents();
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.k_stages; ++s) {
       mbar_init(&sb->k_full[s], 1);
@@ -171,6 +175,9 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
     tma_prefetch_desc(&kmap);
     tma_prefetch_desc(&qmap);
   }
+  // Launched as a programmatic dependent of the previous kernel on the stream: nothing in global
+  // memory (inputs, workspace, status) is touched before that grid has completed.
+  pdl_wait_primary();
   if (warp == 0) locate_start(p, sb);
   if (warp == 1) {
     tmem_alloc(&sb->tmem_base, p.tmem_cols);
@@ -432,7 +439,6 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
       t0 = 0;
     }
   }
-  pdl_launch_dependents();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

@@ -420,7 +420,7 @@ sia_status sia_sparse_index_topk(const sia_index_args* a, void* workspace, size_
   IndexPlan pl;
   sia_status st = plan_index(a, &pl, true);
   if (st != SIA_OK) return st;
-  return run_index(&pl, workspace, ws_bytes, dev_status, static_cast<cudaStream_t>(stream), false);
+  return run_index(&pl, workspace, ws_bytes, dev_status, static_cast<cudaStream_t>(stream), true);
 }
 
 sia_status sia_index_scores(const sia_index_args* a, int32_t* dev_status, void* stream) {
@@ -431,7 +431,7 @@ sia_status sia_index_scores(const sia_index_args* a, int32_t* dev_status, void* 
   if (st != SIA_OK) return st;
   pl.kp.scores = a->scores_out;
   pl.kp.status = dev_status;
-  cudaError_t e = launch_index_score(pl.kp, pl.kmap, pl.qmap, pl.grid, false, static_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_index_score(pl.kp, pl.kmap, pl.qmap, pl.grid, true, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "index scoring launch");
   return SIA_OK;
 }
@@ -464,7 +464,7 @@ sia_status sia_fused_decode(const sia_index_args* ia, const sia_attend_args* aa,
   if (need && (!workspace || ws_bytes < need || !aligned(workspace, 256)))
     return fail(SIA_ERR_WORKSPACE, "the fused call needs a 256-byte aligned workspace of %zu bytes", need);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  st = run_index(&ip, workspace, ip.ws_scores, dev_status, s, false);
+  st = run_index(&ip, workspace, ip.ws_scores, dev_status, s, true);
   if (st != SIA_OK) return st;
   void* ws2 = ap.ws_part ? static_cast<uint8_t*>(workspace) + round_up(ip.ws_scores, 256) : nullptr;
   return run_attend(&ap, ws2, ap.ws_part, dev_status, s, true);

@@ -261,6 +261,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = sb->tmem_base;
   volatile int* abort = &sb->abort;
+  // The next kernel (the split merge, or the next call's first kernel) waits for this grid's
+  // completion before its loads, so it may be scheduled now and only its launch overlaps ours.
+  pdl_launch_dependents();
 
   // Only the gather warps read what the previous kernel on the stream (Top-K) writes; they wait
   // for it below.  The query rows are inputs written before the previous kernels were launched.
@@ -752,7 +755,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       tc_fence_before();   // our reads of O come before the next unit's first P . C
     }
   }
-  pdl_launch_dependents();
   tc_fence_before();
   __syncthreads();
   cluster_sync();  // the peer no longer writes into our shared memory or arrives on our barriers
@@ -767,28 +769,46 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 constexpr int kCombineThreads = 256;
 
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineKernelParams p) {
+  pdl_launch_dependents();  // the dependent waits for this grid's completion before its loads
   pdl_wait_primary();
   const int tph = p.DL / 8;                               // threads per (row, head)
   const long long bjh = (long long)blockIdx.x * (kCombineThreads / tph) + threadIdx.x / tph;
   const int d8 = (threadIdx.x % tph) * 8;
   const long long n_bjh = (long long)p.BJ * p.H;
   if (bjh < n_bjh) {
-    float mx = -INFINITY;
-    for (int s = 0; s < p.splits; ++s) mx = fmaxf(mx, p.part_lse[s * n_bjh + bjh]);
-    float wsum = 0.0f, o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    if (mx != -INFINITY) {
-      for (int s = 0; s < p.splits; ++s) {
-        const float ls = p.part_lse[s * n_bjh + bjh];
-        const float wgt = ls == -INFINITY ? 0.0f : expf(ls - mx);
-        const uint4 v = *reinterpret_cast<const uint4*>(p.part_o + (s * n_bjh + bjh) * p.DL + d8);
-        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+    // Splits are merged four at a time: the four log-sum-exps and partial vectors are loaded
+    // together, so a merge of up to four splits waits for one memory latency.
+    float mx = -INFINITY, wsum = 0.0f, o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int s0 = 0; s0 < p.splits; s0 += 4) {
+      float ls[4];
+      uint4 v[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          o[2 * i] += wgt * __uint_as_float(w4[i] << 16);
-          o[2 * i + 1] += wgt * __uint_as_float(w4[i] & 0xffff0000u);
+      for (int i = 0; i < 4; ++i) {
+        const bool in = s0 + i < p.splits;
+        const long long e = (long long)(s0 + i) * n_bjh + bjh;
+        ls[i] = in ? p.part_lse[e] : -INFINITY;
+        v[i] = in ? ld_nc_v4(p.part_o + e * p.DL + d8) : make_uint4(0, 0, 0, 0);
+      }
+      float m_new = mx;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) m_new = fmaxf(m_new, ls[i]);
+      if (m_new == -INFINITY) continue;   // every split so far is empty
+      const float c = mx == -INFINITY ? 0.0f : expf(mx - m_new);
+      wsum *= c;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) o[j] *= c;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float wgt = ls[i] == -INFINITY ? 0.0f : expf(ls[i] - m_new);
+        const uint32_t w4[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          o[2 * k] += wgt * __uint_as_float(w4[k] << 16);
+          o[2 * k + 1] += wgt * __uint_as_float(w4[k] & 0xffff0000u);
         }
         wsum += wgt;
       }
+      mx = m_new;
     }
     const float inv = wsum > 0.0f ? 1.0f / wsum : 0.0f;
     *reinterpret_cast<uint4*>(p.out + bjh * p.DL + d8) =
@@ -796,7 +816,6 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineK
                    pack_bf16x2(o[4] * inv, o[5] * inv), pack_bf16x2(o[6] * inv, o[7] * inv));
     if (d8 == 0 && p.lse) p.lse[bjh] = wsum > 0.0f ? mx + logf(wsum) : -INFINITY;
   }
-  pdl_launch_dependents();
 }
 
 template <int DL, int DR>

@@ -126,6 +126,10 @@ INDEX_CASES = {
     "fp8_ragged": (3, dict(seq_lens=[513, 2000, 64]), 256),
     "fp8_j2": (5, dict(seq_lens=[1500, 777], n_q=2), 300),
     "prefill_chunk_300": (4, dict(seq_lens=[300], n_q=300), 64),
+    # an odd number of rows that all need ranking
+    "bf16_odd_rows": (2, dict(seq_lens=[700, 900, 1100]), 128),
+    # rows past 8192 positions: every thread of the row Top-K holds a full 16 keys
+    "bf16_long_rows": (2, dict(seq_lens=[12000, 9000]), 2048),
 }
 
 
