@@ -329,6 +329,46 @@ def test_attention_special_cases():
     assert np.all(o == 0) and np.all(np.isneginf(l))
 
 
+def test_attention_identical_rows_shift_and_list_order():
+    q, kv, pt, sl, topk = _attn_case(303)
+    DL = 8
+    kvn = kv.to(torch.float64).numpy()
+    ref_o, ref_l, st = oracle.sparse_attend(q, kv, pt, sl, topk, page_size=4, d_latent=DL, scale=0.3)
+    assert st == 0
+    # the list is a set: its order does not matter
+    perm = topk.copy()
+    for b in range(2):
+        for j in range(2):
+            n = int(np.sum(topk[b, j] >= 0))
+            perm[b, j, :n] = topk[b, j, :n][::-1]
+    o, l, _ = oracle.sparse_attend(q, kv, pt, sl, perm, page_size=4, d_latent=DL, scale=0.3)
+    np.testing.assert_allclose(o, ref_o, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(l, ref_l, rtol=0, atol=1e-12)
+    # a constant added to every logit: give every cache row the same first rope value 1 and
+    # raise that query component by 1, so each logit grows by exactly the scale; the output
+    # (latent part only) is unchanged and the log-sum-exp moves by the scale
+    kv1 = kv.clone()
+    kv1[:, :, DL] = 1.0
+    o0, l0, _ = oracle.sparse_attend(q, kv1, pt, sl, topk, page_size=4, d_latent=DL, scale=0.3)
+    q1 = q.clone()
+    q1[..., DL] = (q1[..., DL].float() + 1.0).to(torch.bfloat16)
+    shifted = (q1[..., DL].double() - q[..., DL].double()).numpy()     # 1, up to bf16 rounding
+    o1, l1, _ = oracle.sparse_attend(q1, kv1, pt, sl, topk, page_size=4, d_latent=DL, scale=0.3)
+    np.testing.assert_allclose(o1, o0, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(l1, l0 + 0.3 * shifted, rtol=0, atol=1e-12)
+    # every selected position holds the same row: the output is that row, lse = z + log(n)
+    kv2 = kv.clone()
+    kv2[:, :, :] = kv[pt[0, 0], 0]
+    o2, l2, _ = oracle.sparse_attend(q, kv2, pt, sl, topk, page_size=4, d_latent=DL, scale=0.3)
+    row = kvn[pt[0, 0], 0]
+    for b in range(2):
+        for j in range(2):
+            n = int(np.sum(topk[b, j] >= 0))
+            np.testing.assert_allclose(o2[b, j], np.broadcast_to(row[:DL], o2[b, j].shape), rtol=0, atol=1e-12)
+            z = 0.3 * q[b, j].to(torch.float64).numpy() @ row
+            np.testing.assert_allclose(l2[b, j], z + math.log(n), rtol=0, atol=1e-12)
+
+
 # ---------------------------------------------------------------- generators
 
 def test_workload_generator_is_deterministic_and_shaped():
