@@ -264,7 +264,7 @@ sia_status run_index(IndexPlan* pl, void* ws, size_t ws_bytes, int32_t* dev_stat
 struct AttendPlan {
   AttnKernelParams ap;
   CombineKernelParams cp;
-  CUtensorMap maps[4];
+  CUtensorMap q_rope;   // the query rows' rope slices (the only TMA load of the attention)
   size_t ws_part;
   int n_clusters;
 };
@@ -348,21 +348,10 @@ sia_status plan_attend(const sia_attend_args* a, AttendPlan* pl, bool make_maps)
 
   if (make_maps) {
     const int dc = a->d_latent + a->d_rope;
-    const bool big = a->d_latent == 512;
-    const int lat_kbw = big ? 128 : 64, rope_kbw = big ? 64 : 32;
+    const int rope_kbw = a->d_latent == 512 ? 64 : 32;
     const uint64_t q_rows = (uint64_t)bj * a->n_heads;
-    const uint64_t kv_rows = (uint64_t)a->num_pages * a->page_size;
-    st = make_map_2d(&pl->maps[0], a->q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q_rows, dc, 128, lat_kbw / 2, lat_kbw,
+    st = make_map_2d(&pl->q_rope, a->q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q_rows, dc, 128, rope_kbw / 2, rope_kbw,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
-    if (st != SIA_OK) return st;
-    st = make_map_2d(&pl->maps[1], a->q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q_rows, dc, 128, rope_kbw / 2, rope_kbw,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
-    if (st != SIA_OK) return st;
-    st = make_map_2d(&pl->maps[2], a->kv_cache, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kv_rows, dc, 1, lat_kbw / 2,
-                     lat_kbw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B);
-    if (st != SIA_OK) return st;
-    st = make_map_2d(&pl->maps[3], a->kv_cache, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kv_rows, dc, 1, rope_kbw / 2,
-                     rope_kbw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B);
     if (st != SIA_OK) return st;
   }
   return SIA_OK;
@@ -382,7 +371,7 @@ sia_status run_attend(AttendPlan* pl, void* ws, size_t ws_bytes, int32_t* dev_st
     pl->cp.part_lse = pl->ap.part_lse;
   }
   pl->ap.status = dev_status;
-  cudaError_t e = launch_sparse_attend(pl->ap, pl->maps, pl->n_clusters, pdl_first, stream);
+  cudaError_t e = launch_sparse_attend(pl->ap, pl->q_rope, pl->n_clusters, pdl_first, stream);
   if (e != cudaSuccess) return cuda_fail(e, "sparse attention launch");
   if (pl->ap.splits > 1) {
     e = launch_combine(pl->cp, true, stream);

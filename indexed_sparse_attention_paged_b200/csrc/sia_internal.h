@@ -100,7 +100,8 @@ struct CombineKernelParams {
 cudaError_t launch_index_score(const IndexKernelParams& p, const CUtensorMap& kmap, const CUtensorMap& qmap, int grid,
                                bool pdl, cudaStream_t stream);
 cudaError_t launch_topk(const TopkKernelParams& p, bool pdl, cudaStream_t stream);
-cudaError_t launch_sparse_attend(const AttnKernelParams& p, const CUtensorMap* maps,
+// q_rope: 2-D map over the query rows [B*J*H, DL+DR] whose box is one CTA's rope slice of 128 heads
+cudaError_t launch_sparse_attend(const AttnKernelParams& p, const CUtensorMap& q_rope,
                                  int n_clusters, bool pdl, cudaStream_t stream);
 cudaError_t launch_combine(const CombineKernelParams& p, bool pdl, cudaStream_t stream);
 

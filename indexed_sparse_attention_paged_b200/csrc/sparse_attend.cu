@@ -819,7 +819,7 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineK
 }
 
 template <int DL, int DR>
-cudaError_t launch_attend_impl(const AttnKernelParams& p, const CUtensorMap* maps, int n_clusters,
+cudaError_t launch_attend_impl(const AttnKernelParams& p, const CUtensorMap& q_rope, int n_clusters,
                                bool pdl, cudaStream_t stream) {
   using Sm = AttnSmem<AttnLayout<DL, DR>>;
   {
@@ -835,7 +835,7 @@ cudaError_t launch_attend_impl(const AttnKernelParams& p, const CUtensorMap* map
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   AttnMaps m;
-  m.q_rope = maps[1];
+  m.q_rope = q_rope;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[2];
   cfg.gridDim = dim3(2 * n_clusters, 1, 1);
@@ -866,10 +866,10 @@ size_t attend_smem_bytes(int dl, int dr) {
   return 0;
 }
 
-cudaError_t launch_sparse_attend(const AttnKernelParams& p, const CUtensorMap* maps,
+cudaError_t launch_sparse_attend(const AttnKernelParams& p, const CUtensorMap& q_rope,
                                  int n_clusters, bool pdl, cudaStream_t stream) {
-  if (p.DL == 512 && p.DR == 64) return launch_attend_impl<512, 64>(p, maps, n_clusters, pdl, stream);
-  if (p.DL == 64 && p.DR == 16) return launch_attend_impl<64, 16>(p, maps, n_clusters, pdl, stream);
+  if (p.DL == 512 && p.DR == 64) return launch_attend_impl<512, 64>(p, q_rope, n_clusters, pdl, stream);
+  if (p.DL == 64 && p.DR == 16) return launch_attend_impl<64, 16>(p, q_rope, n_clusters, pdl, stream);
   return cudaErrorInvalidValue;
 }
 
