@@ -57,6 +57,9 @@ def _load():
             lib.oracle_sparse_attend.restype = I
             lib.oracle_sparse_attend.argtypes = [I, I, I, I, I, I, I, I, ctypes.c_double, P, P,
                                                  P, P, P, I, P, I, P, P]
+            lib.oracle_sparse_attend_fp8kv.restype = I
+            lib.oracle_sparse_attend_fp8kv.argtypes = [I, I, I, I, I, I, I, I, ctypes.c_double, P,
+                                                       P, P, P, P, P, I, P, I, P, P]
             lib.oracle_dense_masked_attend.restype = I
             lib.oracle_dense_masked_attend.argtypes = [I, I, I, I, I, I, I, I, ctypes.c_double,
                                                        P, P, P, P, P, P, P, P]
@@ -169,26 +172,40 @@ def index_topk(q, w, k_cache, page_table, seq_lens, *, page_size, top_k, fp8=Fal
 
 
 def sparse_attend(q, kv_cache, page_table, seq_lens, topk_idx, *, page_size, d_latent, scale,
-                  rows=None):
+                  rows=None, kv_scale=None):
     """Steps 4-5: gather the selected latent rows and attend (fp64).
 
-    q [B,J,H,DL+DR] bf16, kv_cache [num_pages,P,DL+DR] bf16, topk [B,J,K] int32.
+    q [B,J,H,DL+DR] bf16, kv_cache [num_pages,P,DL+DR] bf16, topk [B,J,K] int32.  With
+    kv_scale (fp32 [num_pages,P,ceil((DL+DR)/128)]) the cache holds e4m3 codes instead and each
+    element is its decoded code times the scale of its 128-element block of the token's row.
     Returns (out fp64 [B,J,H,DL], lse fp64 [B,J,H], status).
     """
     B, J, H, DC = q.shape
     DL = int(d_latent)
     DR = DC - DL
     K = topk_idx.shape[-1]
-    qa, kva = _raw16(q), _raw16(kv_cache)
+    qa = _raw16(q)
     pt, sl = _c(page_table, np.int32), _c(seq_lens, np.int32)
     tk = _c(topk_idx, np.int32)
     r, nr = _rows_arg(rows)
     out = np.zeros((B, J, H, DL), dtype=np.float64)
     lse = np.full((B, J, H), np.nan, dtype=np.float64)
-    st = _load().oracle_sparse_attend(B, J, H, DL, DR, page_size, page_table.shape[1],
-                                      kv_cache.shape[0], float(scale), _ptr(qa), _ptr(kva),
-                                      _ptr(pt), _ptr(sl), _ptr(tk), K, _ptr(r), nr, _ptr(out),
-                                      _ptr(lse))
+    if kv_scale is None:
+        kva = _raw16(kv_cache)
+        st = _load().oracle_sparse_attend(B, J, H, DL, DR, page_size, page_table.shape[1],
+                                          kv_cache.shape[0], float(scale), _ptr(qa), _ptr(kva),
+                                          _ptr(pt), _ptr(sl), _ptr(tk), K, _ptr(r), nr, _ptr(out),
+                                          _ptr(lse))
+    else:
+        kva = _raw8(kv_cache)
+        nblk = (DC + 127) // 128
+        ks = _c(kv_scale, np.float32)
+        if ks.shape != (kv_cache.shape[0], kv_cache.shape[1], nblk):
+            raise ValueError("kv_scale must be [num_pages, P, %d]" % nblk)
+        st = _load().oracle_sparse_attend_fp8kv(B, J, H, DL, DR, page_size, page_table.shape[1],
+                                                kv_cache.shape[0], float(scale), _ptr(qa),
+                                                _ptr(kva), _ptr(ks), _ptr(pt), _ptr(sl), _ptr(tk), K,
+                                                _ptr(r), nr, _ptr(out), _ptr(lse))
     return out, lse, st
 
 

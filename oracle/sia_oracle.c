@@ -178,16 +178,33 @@ int oracle_topk(const double* scores, const int32_t* n_visible, long Lpad, int K
 
 /* ---- steps a6-a7: gather the selected latent rows, softmax attention --------------------- */
 
+/* Elements of one token's main-cache row that share a scale in the FP8 cache: "Rapid
+ * Adaptation and Inference Optimization" (tiered quantization table) and "Day 0 Inference
+ * Adaptation..." (section 5.2) quantize the main KV cache in blocks of 128 elements per token
+ * and head.  The MLA row (DL latent + DR rope elements, one KV head) is read as consecutive
+ * blocks [0,128), [128,256), ...; the last block may be shorter (the 64 rope elements). */
+#define KV_QUANT_BLOCK 128
+
+/* Element d of physical main-cache row `row`: a bf16 value, or (fp8) the e4m3 code decoded
+ * exactly times the fp32 scale of its block -- dequantise, then compute in fp64. */
+static double kv_value(const void* kv, const float* kv_scale, int fp8, int DC, long row, int d) {
+    if (!fp8) return oracle_bf16_value(((const uint16_t*)kv)[row * DC + d]);
+    int nblk = (DC + KV_QUANT_BLOCK - 1) / KV_QUANT_BLOCK;
+    return oracle_e4m3_value(((const uint8_t*)kv)[row * DC + d]) *
+           (double)kv_scale[row * nblk + d / KV_QUANT_BLOCK];
+}
+
 /*
- * q   bf16 [B, J, H, DL+DR];  kv bf16 [num_pages, P, DL+DR];  topk int32 [B, J, K] (-1 = none)
+ * q   bf16 [B, J, H, DL+DR];  kv [num_pages, P, DL+DR] (see kv_value);  topk int32 [B, J, K]
+ * (-1 = none)
  * out [B, J, H, DL] = sum_s softmax_s(z) * c[s][0:DL],  z_s = scale * q[h] . c[s]
  * lse [B, J, H]     = log sum_s exp(z_s)  (-inf and out = 0 when the list is empty)
  */
-int oracle_sparse_attend(int B, int J, int H, int DL, int DR, int P, int max_pages,
-                         int num_pages, double scale, const uint16_t* q, const uint16_t* kv,
-                         const int32_t* page_table, const int32_t* seq_lens,
-                         const int32_t* topk, int K, const int32_t* rows, int n_rows,
-                         double* out, double* lse) {
+static int sparse_attend_rows(int B, int J, int H, int DL, int DR, int P, int max_pages,
+                              int num_pages, double scale, const uint16_t* q, const void* kv,
+                              const float* kv_scale, int kv_fp8, const int32_t* page_table,
+                              const int32_t* seq_lens, const int32_t* topk, int K,
+                              const int32_t* rows, int n_rows, double* out, double* lse) {
     int DC = DL + DR;
     int total = rows ? n_rows : B * J;
     int bad = 0;
@@ -212,9 +229,9 @@ int oracle_sparse_attend(int B, int J, int H, int DL, int DR, int P, int max_pag
             double* oh = out + ((long)bj * H + h) * DL;
             double m = -INFINITY;
             for (int i = 0; i < n; ++i) {
-                const uint16_t* c = kv + phys[i] * DC;
                 double dot = 0.0;
-                for (int d = 0; d < DC; ++d) dot += oracle_bf16_value(qh[d]) * oracle_bf16_value(c[d]);
+                for (int d = 0; d < DC; ++d)
+                    dot += oracle_bf16_value(qh[d]) * kv_value(kv, kv_scale, kv_fp8, DC, phys[i], d);
                 z[i] = scale * dot;
                 if (z[i] > m) m = z[i];
             }
@@ -222,7 +239,7 @@ int oracle_sparse_attend(int B, int J, int H, int DL, int DR, int P, int max_pag
             for (int i = 0; i < n; ++i) denom += exp(z[i] - m);
             for (int d = 0; d < DL; ++d) {
                 double acc = 0.0;
-                for (int i = 0; i < n; ++i) acc += exp(z[i] - m) * oracle_bf16_value(kv[phys[i] * DC + d]);
+                for (int i = 0; i < n; ++i) acc += exp(z[i] - m) * kv_value(kv, kv_scale, kv_fp8, DC, phys[i], d);
                 oh[d] = n > 0 ? acc / denom : 0.0;
             }
             lse[(long)bj * H + h] = n > 0 ? m + log(denom) : -INFINITY;
@@ -231,6 +248,27 @@ int oracle_sparse_attend(int B, int J, int H, int DL, int DR, int P, int max_pag
         free(z);
     }
     return bad ? ORACLE_BAD_INPUT : ORACLE_OK;
+}
+
+/* bf16 main cache. */
+int oracle_sparse_attend(int B, int J, int H, int DL, int DR, int P, int max_pages,
+                         int num_pages, double scale, const uint16_t* q, const uint16_t* kv,
+                         const int32_t* page_table, const int32_t* seq_lens,
+                         const int32_t* topk, int K, const int32_t* rows, int n_rows,
+                         double* out, double* lse) {
+    return sparse_attend_rows(B, J, H, DL, DR, P, max_pages, num_pages, scale, q, kv, NULL, 0,
+                              page_table, seq_lens, topk, K, rows, n_rows, out, lse);
+}
+
+/* FP8 main cache: kv holds e4m3 codes [num_pages, P, DL+DR]; kv_scale fp32
+ * [num_pages, P, ceil((DL+DR) / 128)], one scale per block of the token's row. */
+int oracle_sparse_attend_fp8kv(int B, int J, int H, int DL, int DR, int P, int max_pages,
+                               int num_pages, double scale, const uint16_t* q, const uint8_t* kv,
+                               const float* kv_scale, const int32_t* page_table,
+                               const int32_t* seq_lens, const int32_t* topk, int K,
+                               const int32_t* rows, int n_rows, double* out, double* lse) {
+    return sparse_attend_rows(B, J, H, DL, DR, P, max_pages, num_pages, scale, q, kv, kv_scale, 1,
+                              page_table, seq_lens, topk, K, rows, n_rows, out, lse);
 }
 
 /*

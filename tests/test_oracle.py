@@ -369,6 +369,75 @@ def test_attention_identical_rows_shift_and_list_order():
             np.testing.assert_allclose(l2[b, j], z + math.log(n), rtol=0, atol=1e-12)
 
 
+# ---------------------------------------------------------------- FP8 main cache (NEXT row)
+
+def _fp8_case(seed, B=2, J=1, H=3, DL=512, DR=64, P=4, L=11):
+    """e4m3 codes of a random cache, torch's decode of them (float64), the page table."""
+    r = rng(seed)
+    pages = (L + P - 1) // P
+    num_pages = B * pages
+    pt = r.permutation(num_pages).astype(np.int32).reshape(B, pages)
+    codes = torch.tensor(r.uniform(-3, 3, (num_pages, P, DL + DR)).astype(np.float32)).to(torch.float8_e4m3fn)
+    decoded = codes.to(torch.float32).double().numpy()
+    q = bf16(r.standard_normal((B, J, H, DL + DR)))
+    sl = np.full(B, L, dtype=np.int32)
+    return q, codes, decoded, pt, sl
+
+
+def test_fp8_main_cache_single_row_gives_the_dequantised_row():
+    """One selected row: out is that row's latent part, dequantised block by block (scales that
+    differ per token and per 128-element block, not powers of two), and lse its logit, whose
+    last block is the 64 rope elements."""
+    q, codes, decoded, pt, sl = _fp8_case(401)
+    DC, DL, P = 576, 512, 4
+    nblk = 5
+    r = rng(402)
+    kv_scale = r.uniform(0.01, 2.0, (codes.shape[0], P, nblk)).astype(np.float32)
+    topk = np.full((2, 1, 4), -1, dtype=np.int32)
+    topk[:, 0, 0] = [6, 9]
+    out, lse, st = oracle.sparse_attend(q, codes, pt, sl, topk, page_size=P, d_latent=DL,
+                                        scale=0.05, kv_scale=kv_scale)
+    assert st == 0
+    blk = np.arange(DC) // 128
+    for b, s in enumerate((6, 9)):
+        page, off = pt[b, s // P], s % P
+        deq = decoded[page, off] * kv_scale[page, off][blk].astype(np.float64)
+        for h in range(3):
+            np.testing.assert_array_equal(out[b, 0, h], deq[:DL])
+            z = 0.05 * float(np.dot(q[b, 0, h].to(torch.float64).numpy(), deq))
+            np.testing.assert_allclose(lse[b, 0, h], z, rtol=0, atol=1e-12)
+
+
+def test_fp8_main_cache_with_power_of_two_scales_equals_the_bf16_cache_of_its_values():
+    """Power-of-two block scales keep every dequantised element exact in bf16, so the FP8 path
+    must give exactly what the bf16 path gives on a bf16 cache holding those values."""
+    q, codes, decoded, pt, sl = _fp8_case(403, J=2, L=13)
+    P, DL = 4, 512
+    r = rng(404)
+    kv_scale = np.power(2.0, r.integers(-3, 4, (codes.shape[0], P, 5))).astype(np.float32)
+    deq = decoded * np.repeat(kv_scale.astype(np.float64), 128, axis=2)[:, :, :576]
+    kv_bf16 = torch.tensor(deq.astype(np.float32)).to(torch.bfloat16)
+    assert np.array_equal(kv_bf16.double().numpy(), deq)          # exact in bf16
+    topk = np.full((2, 2, 6), -1, dtype=np.int32)
+    for b in range(2):
+        for j in range(2):
+            topk[b, j, :5] = np.sort(r.choice(13 - 2 + j + 1, 5, replace=False))
+    o8, l8, s8 = oracle.sparse_attend(q, codes, pt, sl, topk, page_size=P, d_latent=DL,
+                                      scale=0.05, kv_scale=kv_scale)
+    ob, lb, sb = oracle.sparse_attend(q, kv_bf16, pt, sl, topk, page_size=P, d_latent=DL, scale=0.05)
+    assert s8 == 0 and sb == 0
+    np.testing.assert_array_equal(o8, ob)
+    np.testing.assert_array_equal(l8, lb)
+
+
+def test_fp8_main_cache_refuses_a_scale_array_of_the_wrong_shape():
+    q, codes, _, pt, sl = _fp8_case(405)
+    topk = np.zeros((2, 1, 1), dtype=np.int32)
+    with pytest.raises(ValueError):
+        oracle.sparse_attend(q, codes, pt, sl, topk, page_size=4, d_latent=512, scale=0.05,
+                             kv_scale=np.ones((codes.shape[0], 4, 4), np.float32))
+
+
 # ---------------------------------------------------------------- generators
 
 def test_workload_generator_is_deterministic_and_shaped():
