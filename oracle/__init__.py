@@ -47,6 +47,11 @@ def _load():
             lib.oracle_bf16_value.argtypes = [ctypes.c_uint16]
             lib.oracle_e4m3_value.restype = ctypes.c_double
             lib.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+            lib.oracle_e8m0_value.restype = ctypes.c_double
+            lib.oracle_e8m0_value.argtypes = [ctypes.c_uint8]
+            lib.oracle_index_scores_mx.restype = I
+            lib.oracle_index_scores_mx.argtypes = [I, I, I, I, I, I, I, P, P, P, P, P, P, P, P, P,
+                                                   I, P, P]
             lib.oracle_index_scores.restype = I
             lib.oracle_index_scores.argtypes = [I, I, I, I, I, I, I, I, P, P, P, P, P, P, P, P,
                                                 P, I, P, P]
@@ -109,6 +114,10 @@ def e4m3_value(code: int) -> float:
     return _load().oracle_e4m3_value(int(code))
 
 
+def e8m0_value(code: int) -> float:
+    return _load().oracle_e8m0_value(int(code))
+
+
 def _rows_arg(rows):
     if rows is None:
         return None, 0
@@ -160,6 +169,33 @@ def topk(scores, n_visible, k, rows=None):
     out = np.full((B, J, k), -1, dtype=np.int32)
     _load().oracle_topk(_ptr(s), _ptr(nv), Lpad, int(k), _ptr(r), nr, B * J, _ptr(out))
     return out
+
+
+def index_scores_mx(q, q_mx, w, k_cache, k_mx, page_table, seq_lens, *, page_size, q_pos=None,
+                    rows=None):
+    """Steps 1-2 on the MXFP8 index path: e4m3 codes with one E8M0 scale per 32 elements.
+
+    q [B,J,H,D] e4m3, q_mx [B,J,H,D/32] E8M0 (uint8 codes or torch float8_e8m0fnu), w [B,J,H]
+    fp32, k_cache [num_pages,P,D] e4m3, k_mx [num_pages,P,D/32] E8M0.  Returns (scores fp64
+    [B,J,Lpad] with NaN past the query position, n_visible int32 [B,J], status).
+    """
+    B, J, H, D = q.shape
+    num_pages = k_cache.shape[0]
+    max_pages = page_table.shape[1]
+    qa, ka, qm, km = _raw8(q), _raw8(k_cache), _raw8(q_mx), _raw8(k_mx)
+    if qm.shape != (B, J, H, D // 32) or km.shape != (num_pages, k_cache.shape[1], D // 32):
+        raise ValueError("one E8M0 scale per 32 elements of q and of each key is expected")
+    wa = _c(w, np.float32)
+    pt, sl = _c(page_table, np.int32), _c(seq_lens, np.int32)
+    qp = _c(q_pos, np.int32)
+    r, nr = _rows_arg(rows)
+    Lpad = max_pages * page_size
+    scores = np.full((B, J, Lpad), np.nan, dtype=np.float64)
+    nvis = np.zeros((B, J), dtype=np.int32)
+    st = _load().oracle_index_scores_mx(B, J, H, D, page_size, max_pages, num_pages, _ptr(qa),
+                                        _ptr(qm), _ptr(wa), _ptr(ka), _ptr(km), _ptr(pt), _ptr(sl),
+                                        _ptr(qp), _ptr(r), nr, _ptr(scores), _ptr(nvis))
+    return scores, nvis, st
 
 
 def index_topk(q, w, k_cache, page_table, seq_lens, *, page_size, top_k, fp8=False,

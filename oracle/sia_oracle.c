@@ -59,6 +59,13 @@ double oracle_e4m3_value(uint8_t bits) {
     return sign ? -mag : mag;
 }
 
+/* OCP Microscaling (MX) E8M0 shared scale: an 8-bit exponent with bias 127, value 2^(e-127);
+ * the code 0xFF is NaN.  No sign, no mantissa. */
+double oracle_e8m0_value(uint8_t bits) {
+    if (bits == 0xFF) return NAN;
+    return ldexp(1.0, (int)bits - 127);
+}
+
 static double elem_value(const void* base, long idx, int fp8) {
     if (fp8) return oracle_e4m3_value(((const uint8_t*)base)[idx]);
     return oracle_bf16_value(((const uint16_t*)base)[idx]);
@@ -116,6 +123,60 @@ int oracle_index_scores(int B, int J, int H, int D, int P, int max_pages, int nu
                 for (int d = 0; d < D; ++d) {
                     double qv = elem_value(q, ((long)bj * H + h) * D + d, fp8) * qs;
                     double kv = elem_value(k_cache, row * D + d, fp8) * ks;
+                    dot += qv * kv;
+                }
+                double relu = dot > 0.0 ? dot : 0.0;
+                total_score += (double)w[(long)bj * H + h] * relu;
+            }
+            out[s] = total_score;
+        }
+    }
+    return bad ? ORACLE_BAD_INPUT : ORACLE_OK;
+}
+
+/*
+ * MXFP8 index path (NEXT row; oracle only so far): "Rapid Adaptation and Inference
+ * Optimization" (tiered quantization table: index Q/K in MXFP8, per group of 32) and "Day 0
+ * Inference Adaptation..." (section 5.1: every 32 elements share one scaling factor).  q holds
+ * e4m3 codes [B, J, H, D] with one E8M0 scale per 32 consecutive elements of each head vector
+ * (q_mx [B, J, H, D/32]); the key cache holds e4m3 codes [num_pages, P, D] with one E8M0
+ * scale per 32 consecutive elements of each key (k_mx [num_pages, P, D/32]).  Each element is
+ * dequantised (code times its group's scale) and the score is then the one above:
+ *      I[t,s] = sum_h w[t,h] * ReLU(sum_d q[t,h,d] k[s,d]).
+ * D must be a multiple of 32.  Output as for oracle_index_scores.
+ */
+#define MX_GROUP 32
+int oracle_index_scores_mx(int B, int J, int H, int D, int P, int max_pages, int num_pages,
+                           const uint8_t* q, const uint8_t* q_mx, const float* w,
+                           const uint8_t* k_cache, const uint8_t* k_mx,
+                           const int32_t* page_table, const int32_t* seq_lens,
+                           const int32_t* q_pos, const int32_t* rows, int n_rows,
+                           double* scores, int32_t* n_visible) {
+    if (D % MX_GROUP != 0) return ORACLE_BAD_INPUT;
+    int G = D / MX_GROUP;
+    long Lpad = (long)max_pages * P;
+    int total = rows ? n_rows : B * J;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (int r = 0; r < total; ++r) {
+        int bj = rows ? rows[r] : r;
+        int b = bj / J, j = bj % J;
+        int p = query_position(seq_lens, q_pos, J, b, j);
+        double* out = scores + (long)bj * Lpad;
+        for (long s = 0; s < Lpad; ++s) out[s] = NAN;
+        if (p >= seq_lens[b] || p >= Lpad) { bad = 1; n_visible[bj] = 0; continue; }
+        n_visible[bj] = p + 1 > 0 ? p + 1 : 0;
+        for (int s = 0; s <= p; ++s) {
+            long row = physical_row(page_table, max_pages, P, num_pages, b, s);
+            if (row < 0) { bad = 1; continue; }
+            double total_score = 0.0;
+            for (int h = 0; h < H; ++h) {
+                long qh = (long)bj * H + h;
+                double dot = 0.0;
+                for (int d = 0; d < D; ++d) {
+                    double qv = oracle_e4m3_value(q[qh * D + d]) * oracle_e8m0_value(q_mx[qh * G + d / MX_GROUP]);
+                    double kv = oracle_e4m3_value(k_cache[row * D + d]) *
+                                oracle_e8m0_value(k_mx[row * G + d / MX_GROUP]);
                     dot += qv * kv;
                 }
                 double relu = dot > 0.0 ? dot : 0.0;

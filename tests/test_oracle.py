@@ -438,6 +438,68 @@ def test_fp8_main_cache_refuses_a_scale_array_of_the_wrong_shape():
                              kv_scale=np.ones((codes.shape[0], 4, 4), np.float32))
 
 
+# ---------------------------------------------------------------- MXFP8 index path (NEXT row)
+
+def test_e8m0_decode_matches_torch_for_every_code():
+    ref = torch.arange(256, dtype=torch.uint8).view(torch.float8_e8m0fnu).to(torch.float32).double().numpy()
+    got = np.array([oracle.e8m0_value(c) for c in range(256)])
+    nan = np.isnan(ref)
+    assert nan.sum() == 1 and np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+
+
+def _mx_case(seed, B=2, J=2, H=4, D=128, P=4, L=11):
+    """Integer-valued e4m3 codes in [-8, 8] and E8M0 scales 2^-4..2^4: every product and sum
+    of the score is exact in fp64, so any summation order gives the same value."""
+    r = rng(seed)
+    pages = (L + P - 1) // P
+    num_pages = B * pages
+    pt = r.permutation(num_pages).astype(np.int32).reshape(B, pages)
+    q = torch.tensor(r.integers(-8, 9, (B, J, H, D)).astype(np.float32)).to(torch.float8_e4m3fn)
+    k = torch.tensor(r.integers(-8, 9, (num_pages, P, D)).astype(np.float32)).to(torch.float8_e4m3fn)
+    q_mx = r.integers(123, 132, (B, J, H, D // 32)).astype(np.uint8)
+    k_mx = r.integers(123, 132, (num_pages, P, D // 32)).astype(np.uint8)
+    w = r.integers(-2, 3, (B, J, H)).astype(np.float32)
+    sl = np.full(B, L, dtype=np.int32)
+    return q, q_mx, w, k, k_mx, pt, sl
+
+
+def test_mx_scores_with_unit_scales_equal_the_fp8_path():
+    q, q_mx, w, k, k_mx, pt, sl = _mx_case(501)
+    ones_q, ones_k = np.full_like(q_mx, 127), np.full_like(k_mx, 127)
+    mx, nv1, s1 = oracle.index_scores_mx(q, ones_q, w, k, ones_k, pt, sl, page_size=4)
+    f8, nv2, s2 = oracle.index_scores(q, w, k, pt, sl, page_size=4, fp8=True)
+    assert s1 == 0 and s2 == 0 and np.array_equal(nv1, nv2)
+    assert np.array_equal(mx, f8, equal_nan=True)
+
+
+def test_mx_scores_match_the_closed_form_with_group_scales():
+    """I[t,s] = sum_h w ReLU(sum_d (q_d 2^(eq[d/32]-127)) (k_d 2^(ek[d/32]-127))), with the codes
+    and scales decoded by torch, against the oracle's own decoding and loop."""
+    q, q_mx, w, k, k_mx, pt, sl = _mx_case(502)
+    B, J, H, D = q.shape
+    got, nv, st = oracle.index_scores_mx(q, q_mx, w, k, k_mx, pt, sl, page_size=4)
+    assert st == 0
+    e8 = lambda a: torch.tensor(a).view(torch.float8_e8m0fnu).to(torch.float32).double().numpy()
+    qd = q.to(torch.float32).double().numpy() * np.repeat(e8(q_mx), 32, axis=-1)
+    kd = k.to(torch.float32).double().numpy() * np.repeat(e8(k_mx), 32, axis=-1)
+    for b in range(B):
+        for j in range(J):
+            p = 11 - J + j
+            assert nv[b, j] == p + 1
+            for s in range(p + 1):
+                key = kd[pt[b, s // 4], s % 4]
+                want = float(np.sum(w[b, j].astype(np.float64) * np.maximum(qd[b, j] @ key, 0.0)))
+                assert got[b, j, s] == want, (b, j, s)
+            assert np.all(np.isnan(got[b, j, p + 1:]))
+
+
+def test_mx_scores_refuse_scale_arrays_of_the_wrong_shape():
+    q, q_mx, w, k, k_mx, pt, sl = _mx_case(503)
+    with pytest.raises(ValueError):
+        oracle.index_scores_mx(q, q_mx[..., :2], w, k, k_mx, pt, sl, page_size=4)
+
+
 # ---------------------------------------------------------------- generators
 
 def test_workload_generator_is_deterministic_and_shaped():
