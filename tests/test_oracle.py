@@ -514,3 +514,36 @@ def test_workload_generator_is_deterministic_and_shaped():
     assert a["q_idx"].shape == (1, 1, 4, 32) and a["kv_cache"].shape == (16, 16, 80)
     v = a["q_idx"].float()
     assert v.min() >= -3 and v.max() <= 3 and torch.equal(v, v.round())
+
+
+# ---------------------------------------------------------------- Zigzag prefill pairing (NEXT row)
+
+def test_zigzag_assignment_matches_the_printed_example():
+    from oracle import zigzag
+    with open(os.path.join(GOLDEN, "zigzag_example.json")) as f:
+        g = json.load(f)
+    assert zigzag.assignment(g["cards"]) == g["assignment"]
+    assert sorted(s for pair in g["assignment"] for s in pair) == list(range(g["shards"]))
+
+
+@pytest.mark.parametrize("cards,shard_len", [(1, 5), (2, 3), (4, 16), (8, 7)])
+def test_zigzag_balances_causal_load_exactly_when_the_shards_are_equal(cards, shard_len):
+    """Shard i covers [iL, (i+1)L): its causal load is L*i*L + L(L+1)/2, so shards i and S-1-i
+    together carry L*L*(S-1) + L(L+1) on every card, against a naive split that grows with i."""
+    from oracle import zigzag
+    T, S = 2 * cards * shard_len, 2 * cards
+    loads = [zigzag.causal_load(p) for p in zigzag.card_positions(T, cards)]
+    L = shard_len
+    assert loads == [L * L * (S - 1) + L * (L + 1)] * cards
+    assert sum(loads) == T * (T + 1) // 2
+    naive = [zigzag.causal_load(range(i * T // cards, (i + 1) * T // cards)) for i in range(cards)]
+    assert cards == 1 or naive[-1] > naive[0]
+
+
+@pytest.mark.parametrize("tokens,cards", [(0, 2), (5, 2), (17, 4), (64, 8), (1000, 3)])
+def test_zigzag_restore_inverts_the_assignment(tokens, cards):
+    from oracle import zigzag
+    pos = zigzag.card_positions(tokens, cards)
+    assert sorted(t for p in pos for t in p) == list(range(tokens))
+    per_card = [[("tok", t) for t in p] for p in pos]
+    assert zigzag.restore(per_card, tokens, cards) == [("tok", t) for t in range(tokens)]
