@@ -68,6 +68,10 @@ def _load():
             lib.oracle_dense_masked_attend.restype = I
             lib.oracle_dense_masked_attend.argtypes = [I, I, I, I, I, I, I, I, ctypes.c_double,
                                                        P, P, P, P, P, P, P, P]
+            lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+            lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+            lib.oracle_cache_append.restype = I
+            lib.oracle_cache_append.argtypes = [I, I, I, I, I, I, I, P, P, P, I, P, P, P, I, P, P]
             lib.oracle_num_threads.restype = I
             lib.oracle_set_num_threads.argtypes = [I]
             _lib = lib
@@ -112,6 +116,40 @@ def bf16_value(bits: int) -> float:
 
 def e4m3_value(code: int) -> float:
     return _load().oracle_e4m3_value(int(code))
+
+
+def e4m3_encode(x: float) -> int:
+    """e4m3 code of an fp32 value: nearest grid value, ties to even, saturating at 448."""
+    return _load().oracle_e4m3_encode(float(x))
+
+
+def cache_append(new_k, new_kv, page_table, seq_lens, k_cache, kv_cache, *, page_size,
+                 k_mode="bf16", k_scale=None, kv_scale=None):
+    """The step before scoring: write the J new tokens of every sequence into the paged caches
+    (token j of sequence b at position seq_lens[b] - J + j), in place.
+
+    new_k [B,J,D] and new_kv [B,J,DC] are float values (fp32, or bf16 tensors).  k_mode:
+    "bf16" (k_cache uint16 bits), "fp8" (e4m3 codes + per-token power-of-two fp32 scale in
+    k_scale [pages,P]) or "mx" (e4m3 codes + E8M0 codes in k_scale uint8 [pages,P,D/32]).
+    kv_scale None: kv_cache holds bf16 bits; else e4m3 codes + fp32 scale per 128-element
+    block (kv_scale [pages,P,ceil(DC/128)]).  Every array is a contiguous numpy array, updated
+    in place.  Returns the status.
+    """
+    nk = np.ascontiguousarray(np.asarray(new_k.float() if hasattr(new_k, "float") else new_k,
+                                         dtype=np.float32))
+    nv = np.ascontiguousarray(np.asarray(new_kv.float() if hasattr(new_kv, "float") else new_kv,
+                                         dtype=np.float32))
+    B, J, D = nk.shape
+    DC = nv.shape[2]
+    mode = {"bf16": 0, "fp8": 1, "mx": 2}[k_mode]
+    for a in (k_cache, kv_cache, k_scale, kv_scale):
+        if a is not None and not (isinstance(a, np.ndarray) and a.flags.c_contiguous):
+            raise ValueError("caches and scales must be contiguous numpy arrays")
+    pt, sl = _c(page_table, np.int32), _c(seq_lens, np.int32)
+    return _load().oracle_cache_append(B, J, D, DC, page_size, pt.shape[1], k_cache.shape[0],
+                                       _ptr(pt), _ptr(sl), _ptr(nk), mode, _ptr(k_cache),
+                                       _ptr(k_scale), _ptr(nv), 0 if kv_scale is None else 1,
+                                       _ptr(kv_cache), _ptr(kv_scale))
 
 
 def e8m0_value(code: int) -> float:

@@ -387,6 +387,139 @@ int oracle_dense_masked_attend(int B, int J, int H, int DL, int DR, int P, int m
     return bad ? ORACLE_BAD_INPUT : ORACLE_OK;
 }
 
+/* ---- paged cache append (NEXT row; oracle only so far) ---------------------------------- */
+
+/* e4m3 encoding of an fp32 value, from the format definition: round to the nearest value of
+ * the e4m3 grid (3 mantissa bits; below 2^-6 the subnormal step 2^-9), ties to the even
+ * code; magnitudes at or above 448 give +-448 (saturation); NaN gives 0x7F. */
+uint8_t oracle_e4m3_encode(float x) {
+    if (isnan(x)) return 0x7F;
+    uint8_t sign = signbit(x) ? 0x80 : 0x00;
+    double v = fabs((double)x);
+    if (v >= 448.0) return sign | 0x7E;
+    int e = v > 0.0 ? (int)floor(log2(v)) : -6;
+    if (e < -6) e = -6;                       /* subnormal range: fixed step 2^-9 */
+    while (ldexp(1.0, e) > v && e > -6) --e;  /* guard log2 rounding at binade edges */
+    while (ldexp(1.0, e + 1) <= v) ++e;
+    double step = ldexp(1.0, e - 3);
+    double r = rint(v / step) * step;          /* v / step is exact; rint rounds half to even */
+    if (r == 0.0) return sign;
+    int re = (int)floor(log2(r));
+    while (ldexp(1.0, re) > r) --re;
+    while (ldexp(1.0, re + 1) <= r) ++re;
+    if (re < -6) return sign | (uint8_t)(r / ldexp(1.0, -9));             /* subnormal code */
+    return sign | (uint8_t)((re + 7) << 3) | (uint8_t)(r / ldexp(1.0, re - 3) - 8.0);
+}
+
+static float absmax_f(const float* x, int n) {
+    float m = 0.0f;
+    for (int i = 0; i < n; ++i) if (fabsf(x[i]) > m) m = fabsf(x[i]);
+    return m;
+}
+
+/* Per-token FP8 index key: scale = the smallest power of two s with amax <= 448 s (1 for an
+ * all-zero key); codes = e4m3(x / s), the division being exact. */
+static float quantise_key_pow2(const float* x, int n, uint8_t* codes) {
+    float amax = absmax_f(x, n);
+    int e = 0;
+    if (amax > 0.0f) {
+        e = -160;
+        while ((double)amax > 448.0 * ldexp(1.0, e)) ++e;
+    }
+    float s = (float)ldexp(1.0, e);
+    for (int i = 0; i < n; ++i) codes[i] = oracle_e4m3_encode((float)ldexp((double)x[i], -e));
+    return s;
+}
+
+/* FP8 main-cache block: scale = fp32(amax / 448) (1 for an all-zero block); codes =
+ * e4m3(fp32(x / scale)), both divisions rounded to fp32 as a GPU computes them. */
+static float quantise_block_amax(const float* x, int n, uint8_t* codes) {
+    float amax = absmax_f(x, n);
+    volatile float s = amax > 0.0f ? amax / 448.0f : 1.0f;
+    for (int i = 0; i < n; ++i) {
+        volatile float y = x[i] / s;
+        codes[i] = oracle_e4m3_encode(y);
+    }
+    return s;
+}
+
+/* MX group (OCP Microscaling): shared exponent E = floor(log2 amax) - 8 (8 = the largest
+ * e4m3 exponent), clamped to the E8M0 range [-127, 127]; scale code E + 127 (127 for an
+ * all-zero group); codes = e4m3(x / 2^E), saturating. */
+static uint8_t quantise_group_mx(const float* x, int n, uint8_t* codes) {
+    float amax = absmax_f(x, n);
+    int E = 0;
+    if (amax > 0.0f) {
+        int f = (int)floor(log2((double)amax));
+        while (ldexp(1.0, f) > (double)amax) --f;
+        while (ldexp(1.0, f + 1) <= (double)amax) ++f;
+        E = f - 8;
+        if (E < -127) E = -127;
+        if (E > 127) E = 127;
+    }
+    for (int i = 0; i < n; ++i) codes[i] = oracle_e4m3_encode((float)ldexp((double)x[i], -E));
+    return (uint8_t)(E + 127);
+}
+
+/*
+ * Write the J new tokens of every sequence into the paged caches: token j of sequence b sits
+ * at position p = seq_lens[b] - J + j (seq_lens counts the new tokens) and goes to row p % P
+ * of page page_table[b][p / P].
+ *   new_k  fp32 [B, J, D]      -> index cache, by k_mode:
+ *          0: bf16 bits (k_cache uint16 [pages, P, D]; the input must already be bf16 values)
+ *          1: e4m3 codes + per-token power-of-two scale (k_cache uint8, k_scale fp32 [pages, P])
+ *          2: MXFP8 codes + one E8M0 code per 32 elements (k_scale read as uint8 [pages, P, D/32])
+ *   new_kv fp32 [B, J, DC]     -> main cache, by kv_mode:
+ *          0: bf16 bits (kv_cache uint16 [pages, P, DC])
+ *          1: e4m3 codes + fp32 scale per 128-element block (kv_scale [pages, P, ceil(DC/128)])
+ * Rows not written keep their contents.  A page id outside the pool skips the token and
+ * reports ORACLE_BAD_INPUT.
+ */
+int oracle_cache_append(int B, int J, int D, int DC, int P, int max_pages, int num_pages,
+                        const int32_t* page_table, const int32_t* seq_lens,
+                        const float* new_k, int k_mode, void* k_cache, void* k_scale,
+                        const float* new_kv, int kv_mode, void* kv_cache, float* kv_scale) {
+    int bad = 0;
+    int nblk = (DC + KV_QUANT_BLOCK - 1) / KV_QUANT_BLOCK;
+    if (k_mode == 2 && D % MX_GROUP != 0) return ORACLE_BAD_INPUT;
+    for (int b = 0; b < B; ++b) {
+        for (int j = 0; j < J; ++j) {
+            int p = seq_lens[b] - J + j;
+            if (p < 0 || p >= max_pages * P) { bad = 1; continue; }
+            long row = physical_row(page_table, max_pages, P, num_pages, b, p);
+            if (row < 0) { bad = 1; continue; }
+            const float* xk = new_k + ((long)b * J + j) * D;
+            if (k_mode == 0) {
+                for (int d = 0; d < D; ++d) {
+                    uint32_t u;
+                    memcpy(&u, &xk[d], sizeof u);
+                    ((uint16_t*)k_cache)[row * D + d] = (uint16_t)(u >> 16);
+                }
+            } else if (k_mode == 1) {
+                ((float*)k_scale)[row] = quantise_key_pow2(xk, D, (uint8_t*)k_cache + row * D);
+            } else {
+                for (int g = 0; g < D / MX_GROUP; ++g)
+                    ((uint8_t*)k_scale)[row * (D / MX_GROUP) + g] =
+                        quantise_group_mx(xk + g * MX_GROUP, MX_GROUP, (uint8_t*)k_cache + row * D + g * MX_GROUP);
+            }
+            const float* xv = new_kv + ((long)b * J + j) * DC;
+            if (kv_mode == 0) {
+                for (int d = 0; d < DC; ++d) {
+                    uint32_t u;
+                    memcpy(&u, &xv[d], sizeof u);
+                    ((uint16_t*)kv_cache)[row * DC + d] = (uint16_t)(u >> 16);
+                }
+            } else {
+                for (int g = 0; g < nblk; ++g) {
+                    int lo = g * KV_QUANT_BLOCK, n = DC - lo < KV_QUANT_BLOCK ? DC - lo : KV_QUANT_BLOCK;
+                    kv_scale[row * nblk + g] = quantise_block_amax(xv + lo, n, (uint8_t*)kv_cache + row * DC + lo);
+                }
+            }
+        }
+    }
+    return bad ? ORACLE_BAD_INPUT : ORACLE_OK;
+}
+
 /* Number of threads the OpenMP runtime uses for the loops above (1 without OpenMP). */
 #ifdef _OPENMP
 #include <omp.h>

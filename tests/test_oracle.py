@@ -547,3 +547,114 @@ def test_zigzag_restore_inverts_the_assignment(tokens, cards):
     assert sorted(t for p in pos for t in p) == list(range(tokens))
     per_card = [[("tok", t) for t in p] for p in pos]
     assert zigzag.restore(per_card, tokens, cards) == [("tok", t) for t in range(tokens)]
+
+
+# ---------------------------------------------------------------- paged cache append (NEXT row)
+
+def _torch_e4m3(x):
+    return torch.tensor(np.asarray(x, dtype=np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def test_e4m3_encode_matches_torch_on_the_grid_on_ties_and_below_overflow():
+    grid = [c for c in range(256) if not np.isnan(oracle.e4m3_value(c))]
+    for c in grid:                                   # every finite code round-trips
+        assert oracle.e4m3_encode(oracle.e4m3_value(c)) == c
+    pos = sorted({oracle.e4m3_value(c) for c in grid if oracle.e4m3_value(c) > 0})
+    ties = np.array([(a + b) / 2 for a, b in zip([0.0] + pos[:-1], pos)], dtype=np.float32)
+    ties = np.concatenate([ties, -ties])             # exact midpoints: ties go to the even code
+    r = rng(601)
+    rand = np.concatenate([r.uniform(-463, 463, 4000), r.uniform(-0.05, 0.05, 4000)]).astype(np.float32)
+    band = np.linspace(448.0, 463.9, 50, dtype=np.float32)   # rounds down to 448 in both
+    for x in (ties, rand, band, -band):
+        assert np.array_equal(np.array([oracle.e4m3_encode(v) for v in x], np.uint8), _torch_e4m3(x))
+    assert oracle.e4m3_encode(1e6) == 0x7E and oracle.e4m3_encode(-500.0) == 0xFE   # saturation
+
+
+def _append_case(seed, B=3, J=2, D=64, DC=576, P=4, pages_per_seq=3):
+    r = rng(seed)
+    num_pages = B * pages_per_seq + 2                # two pages no sequence uses
+    pt = r.permutation(num_pages)[:B * pages_per_seq].astype(np.int32).reshape(B, pages_per_seq)
+    sl = r.integers(J, pages_per_seq * P + 1, B).astype(np.int32)
+    new_k = r.standard_normal((B, J, D)).astype(np.float32) * r.uniform(0.01, 100, (B, J, 1)).astype(np.float32)
+    new_kv = r.standard_normal((B, J, DC)).astype(np.float32) * r.uniform(0.01, 10, (B, J, 1)).astype(np.float32)
+    return pt, sl, new_k, new_kv, num_pages
+
+
+def _written_rows(pt, sl, J, P):
+    return {(b, j): (pt[b, (int(sl[b]) - J + j) // P], (int(sl[b]) - J + j) % P)
+            for b in range(pt.shape[0]) for j in range(J)}
+
+
+def test_cache_append_bf16_writes_exactly_the_new_rows():
+    pt, sl, new_k, new_kv, num_pages = _append_case(602)
+    B, J, D = new_k.shape
+    DC, P = new_kv.shape[2], 4
+    nk, nv = bf16(new_k), bf16(new_kv)               # bf16 values, as a bf16 cache holds them
+    r = rng(603)
+    k_cache = r.integers(0, 65536, (num_pages, P, D)).astype(np.uint16)
+    kv_cache = r.integers(0, 65536, (num_pages, P, DC)).astype(np.uint16)
+    k0, kv0 = k_cache.copy(), kv_cache.copy()
+    assert oracle.cache_append(nk, nv, pt, sl, k_cache, kv_cache, page_size=P) == 0
+    bits = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)
+    touched = np.zeros((num_pages, P), bool)
+    for (b, j), (page, off) in _written_rows(pt, sl, J, P).items():
+        assert np.array_equal(k_cache[page, off], bits(nk[b, j]))
+        assert np.array_equal(kv_cache[page, off], bits(nv[b, j]))
+        touched[page, off] = True
+    assert np.array_equal(k_cache[~touched], k0[~touched])
+    assert np.array_equal(kv_cache[~touched], kv0[~touched])
+
+
+def test_cache_append_fp8_scale_rules_and_codes():
+    pt, sl, new_k, new_kv, num_pages = _append_case(604)
+    B, J, D = new_k.shape
+    DC, P = new_kv.shape[2], 4
+    new_k[0, 0] = 0.0                                 # an all-zero key: scale 1, codes 0
+    k_cache = np.zeros((num_pages, P, D), np.uint8)
+    k_scale = np.zeros((num_pages, P), np.float32)
+    kv_cache = np.zeros((num_pages, P, DC), np.uint8)
+    kv_scale = np.zeros((num_pages, P, 5), np.float32)
+    assert oracle.cache_append(new_k, new_kv, pt, sl, k_cache, kv_cache, page_size=P, k_mode="fp8",
+                               k_scale=k_scale, kv_scale=kv_scale) == 0
+    for (b, j), (page, off) in _written_rows(pt, sl, J, P).items():
+        # index key: the smallest power of two s with amax <= 448 s, codes of x / s
+        x = new_k[b, j]
+        amax = float(np.abs(x).max())
+        s = k_scale[page, off]
+        if amax == 0.0:
+            assert s == 1.0 and not k_cache[page, off].any()
+        else:
+            e = int(np.log2(s))
+            assert s == 2.0 ** e and amax <= 448 * s and amax > 224 * s
+            assert np.array_equal(k_cache[page, off], _torch_e4m3(x / np.float32(s)))
+        # main cache: per 128-element block, scale = fp32(amax / 448), codes of fp32(x / scale)
+        v = new_kv[b, j]
+        for g in range(5):
+            blk = v[128 * g:128 * g + 128]
+            sc = np.float32(np.abs(blk).max()) / np.float32(448.0)
+            assert kv_scale[page, off, g] == sc
+            assert np.array_equal(kv_cache[page, off, 128 * g:128 * g + 128], _torch_e4m3(blk / sc))
+        # dequantised, every element is within half an e4m3 step of its input
+        deq = np.array([oracle.e4m3_value(c) for c in kv_cache[page, off]]) * np.repeat(kv_scale[page, off], 128)[:DC]
+        step = np.maximum(2.0 ** (np.floor(np.log2(np.maximum(np.abs(v / np.repeat(kv_scale[page, off], 128)[:DC]), 2.0 ** -6))) - 3), 2.0 ** -9)
+        assert np.all(np.abs(deq - v) <= 0.5 * step * np.repeat(kv_scale[page, off], 128)[:DC] * (1 + 1e-6))
+
+
+def test_cache_append_mx_groups():
+    pt, sl, new_k, new_kv, num_pages = _append_case(605, D=128)
+    B, J, D = new_k.shape
+    P = 4
+    k_cache = np.zeros((num_pages, P, D), np.uint8)
+    k_mx = np.zeros((num_pages, P, D // 32), np.uint8)
+    kv_cache = np.zeros((num_pages, P, new_kv.shape[2]), np.uint16)
+    assert oracle.cache_append(bf16(new_k), bf16(new_kv), pt, sl, k_cache, kv_cache, page_size=P,
+                               k_mode="mx", k_scale=k_mx) == 0
+    xk = bf16(new_k).float().numpy()
+    for (b, j), (page, off) in _written_rows(pt, sl, J, P).items():
+        for g in range(D // 32):
+            x = xk[b, j, 32 * g:32 * g + 32]
+            E = int(np.floor(np.log2(np.abs(x).max()))) - 8     # OCP MX shared exponent
+            assert k_mx[page, off, g] == E + 127
+            y = (x * np.float32(2.0 ** -E)).astype(np.float32)
+            want = _torch_e4m3(np.clip(y, -448, 448))           # saturating above 448
+            assert np.array_equal(k_cache[page, off, 32 * g:32 * g + 32], want)
