@@ -49,13 +49,39 @@ def parse():
     return ap.parse_args()
 
 
+def _code_only(text: str) -> str:
+    """C/C++/CUDA source with comments removed and whitespace runs collapsed, string and
+    character literals kept as they are."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            i = text.find("\n", i)
+            i = n if i < 0 else i
+        elif text.startswith("/*", i):
+            i = text.find("*/", i + 2)
+            i = n if i < 0 else i + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def source_sha() -> str:
-    """Hash of the CUDA sources, to tell whether recorded ncu counters are still current."""
+    """Hash of the CUDA sources' code (comments and layout ignored), to tell whether recorded
+    ncu counters are still current."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "indexed_sparse_attention_paged_b200", "csrc")
     for f in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, f), "rb") as fh:
-            h.update(f.encode() + fh.read())
+        with open(os.path.join(csrc, f), encoding="utf-8") as fh:
+            h.update(f.encode() + _code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

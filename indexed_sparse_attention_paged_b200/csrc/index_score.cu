@@ -10,13 +10,16 @@
 // the pages ask of the fused indexer.
 //
 // Design (B200): one tcgen05 MMA per (128-position tile, query sub-block):
-//   A = K tile   [128 positions x D]   (TMA, K-major, swizzled; M = 128 = TMEM lanes)
-//   B = Q group  [nq_sub*HP rows x D]  (threads, K-major, swizzled; N = queries x heads)
-//   D = TMEM     [128 lanes x N fp32 columns]
+//   A = K tile   [128 positions x D]   (TMA from the paged cache, K-major, swizzled; M = 128)
+//   B = Q group  [nq_sub*HP rows x D]  (one 3-D TMA box per K block, K-major, swizzled;
+//                                       N = queries x heads)
+//   D = TMEM     [128 lanes x N fp32 columns], two accumulator stages
 // so that in the epilogue each thread owns one position and reduces sum_h w*ReLU(d) over its
 // own registers, without shuffles.  The grid is persistent (one CTA per SM); the flat list of
-// (query group, tile) work is split evenly between CTAs, which balances ragged context lengths
-// and the causal "light at the start, heavy at the end" prefill load.
+// (query group, tile) work is split between CTAs by a weight of tiles plus a per-group set-up
+// cost, which balances ragged context lengths and the causal "light at the start, heavy at the
+// end" prefill load.  The kernel is a programmatic dependent of the previous kernel on the
+// stream: it touches no global memory before that grid has completed.
 //
 // Exactness: for integer-valued q, k, w (the tests' inputs) every product and every partial
 // sum is an integer below 2^24, so the fp32 result equals the exact score whatever order the

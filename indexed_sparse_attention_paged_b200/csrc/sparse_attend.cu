@@ -16,17 +16,21 @@
 //     (plus half of the rope dims), so together the pair reads each 1152-byte row once;
 //   - each CTA computes a partial S = Q_r . C_r^T over its own dims, with its latent half of Q
 //     held in TMEM (the A operand of the MMA) and only the rope part of Q in shared memory;
-//   - the partials are exchanged through distributed shared memory as fp16 (scaled to base
-//     2): each CTA adds the peer's fp16 partial to its own fp32 partial and runs its own online
-//     softmax.  The two CTAs' logits differ only by the fp16 rounding of one partial, and each
-//     CTA's (max, sum, O) triple is self-consistent, so each half of the output is normalised
-//     by the sum that produced it;
-//   - P (bf16) overwrites its own logits in TMEM and is the A operand of O_r += P . C_r.
-// Rows are gathered with 16-byte cp.async from a per-unit table of physical cache rows into
-// 128B/64B/32B-swizzled K-major tiles; the same tile serves as the K-major B operand of
-// Q.C^T and as the MN-major B operand of P.C.  Rescaling of O is lazy: only when a head's
-// running max grows by more than 2^8.  Splits of the Top-K list (to fill the GPU at small
-// batch) write fp32 partials that combine_kernel merges by log-sum-exp.
+//   - the partials are rounded to fp16 (scaled to base 2); each CTA keeps its own in a shared
+//     stash and sends it to the peer through distributed shared memory, and each softmax adds
+//     the same two fp16 values, so both CTAs see bit-identical logits and take the same
+//     decisions;
+//   - P (bf16) is written to a 128B-swizzled shared buffer and is the A operand of
+//     O_r += P . C_r.
+// Warp roles (576 threads): softmax + epilogue (warps 0-3), TMEM q loading and the logit
+// exchange (4-7), the row gather (8-15), the S = Q C^T issuer (16) and the P . C issuer (17);
+// setmaxnreg splits the registers between them.  Rows are gathered with 16-byte cp.async from a
+// per-unit table of physical cache rows into swizzled K-major tiles (four latent stages, a
+// separate two-slot rope ring); the same tile serves as the K-major B operand of Q.C^T and as
+// the MN-major B operand of P.C.  Rescaling of O is lazy: only when a head's running max grows
+// by more than 2^8.  Splits of the Top-K list (to fill the GPU at small batch) write normalised
+// bf16 partials and an fp32 log-sum-exp per split that combine_kernel merges.  Every pipeline
+// wait is an mbarrier wait with a bounded spin.
 #include <cuda.h>
 #include <cuda_fp16.h>
 

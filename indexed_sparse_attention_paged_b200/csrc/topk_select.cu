@@ -7,13 +7,16 @@
 // operator outputs only these indices, "Rapid Adaptation and Inference Optimization",
 // section IV.4.1).
 //
-// Design: one thread-block cluster of `cluster` CTAs per query row; each CTA keeps a slice of
-// the row's keys in shared memory.  Keys are the scores mapped to order-preserving uint32
-// (-0.0 folded onto +0.0).  Three MSB-first radix passes (11, 11, 10 bits) find the exact K-th
-// largest key T; the per-CTA digit histograms are summed across the cluster through
-// distributed shared memory.  The selection is then every key > T plus the lowest-positioned
-// keys == T, compacted in position order with block- and cluster-level prefix sums, which
-// makes the output ascending without a sort.
+// Design: keys are the scores mapped to order-preserving uint32 (-0.0 folded onto +0.0).
+// Three MSB-first radix passes (11, 11, 10 bits) find the exact K-th largest key T; the
+// selection is then every key > T plus the lowest-positioned keys == T, compacted in position
+// order with prefix sums, which makes the output ascending without a sort.
+//   - Rows of up to 16384 positions (topk_row_kernel): one CTA of 1024 threads per row, 16
+//     consecutive keys per thread in registers, shared-memory histograms with plain atomics,
+//     three barriers per pass.
+//   - Longer rows (topk_kernel): a thread-block cluster of 2-16 CTAs per row, each keeping a
+//     slice of the keys in shared memory; the per-CTA digit histograms are summed across the
+//     cluster through distributed shared memory.
 #include <cuda_runtime.h>
 
 #include "sia_common.cuh"
