@@ -30,8 +30,11 @@
  *     position or Top-K entry at or past seq_len) never trap: the kernel ORs a SIA_DEV_* bit
  *     into *dev_status (when dev_status is not NULL), treats the offending row as absent and
  *     carries on; the caller reads *dev_status after synchronising;
- *   - every wait inside a kernel is bounded (about two seconds); a wait that gives up sets
- *     SIA_DEV_TIMEOUT and the kernel returns early, leaving its outputs undefined;
+ *   - every wait inside a kernel is bounded (two seconds unless sia_set_wait_limit_ns says
+ *     otherwise); a wait that gives up sets SIA_DEV_TIMEOUT and the kernel returns early,
+ *     leaving its outputs undefined (before it returns, every CTA still waits, with a bound of
+ *     its own, for the asynchronous copies and tensor-core operations it issued); when
+ *     SIA_DEV_TIMEOUT or SIA_DEV_INTERNAL is set, every output of the call is undefined;
  *   - layout: row-major, innermost dimension last, no padding between rows.
  */
 #ifndef SIA_H
@@ -56,6 +59,8 @@ typedef enum {
 #define SIA_DEV_BAD_PAGE 0x1      /* a page-table entry used by the call is outside the pool  */
 #define SIA_DEV_BAD_POSITION 0x2  /* a query position or Top-K entry is >= seq_len          */
 #define SIA_DEV_TIMEOUT 0x4       /* a bounded in-kernel wait gave up                         */
+#define SIA_DEV_INTERNAL 0x8      /* a kernel could not set itself up (its shared-memory base
+                                     was not 1024-byte aligned) and returned at once           */
 
 typedef enum {
     SIA_BF16 = 0,                 /* bfloat16                                                 */
@@ -157,9 +162,11 @@ sia_status sia_sparse_mla_attend(const sia_attend_args* a, void* workspace, size
  *     SIA_ERR_WORKSPACE before any launch (ignored when scores_out is given);
  *   - the array is shared by every call in the process: calls whose kernels may overlap on the
  *     GPU (other streams, other host threads) race on it and must be serialised by the caller;
- *   - the first call on each device looks up the array's device address (cudaGetSymbolAddress);
- *     make that first call before any stream capture;
- *   - every GPU that loads the library keeps the 16 MiB until the process exits. */
+ *   - the first call on each device (and the first after that device's context was reset)
+ *     loads the array's module -- which is when the 16 MiB are reserved on the device -- and
+ *     looks up the array's device address (cudaGetSymbolAddress); make that first call at
+ *     start-up, before carving a memory arena out of the device and before any stream capture;
+ *   - once reserved, the 16 MiB stay reserved on that device until the process exits. */
 sia_status sia_sparse_index_topk_noalloc(const sia_index_args* a, int32_t* dev_status, void* stream);
 
 /* Both stages back to back on one stream (programmatic dependent launch between kernels, no
@@ -171,6 +178,13 @@ sia_status sia_sparse_index_topk_noalloc(const sia_index_args* a, int32_t* dev_s
  * seq_lens, with aa->topk == ia->topk_out. */
 sia_status sia_fused_decode(const sia_index_args* ia, const sia_attend_args* aa,
                             void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream);
+
+/* The bound of every pipeline wait inside the kernels of calls made after this one, from any
+ * host thread, in nanoseconds of the GPU's global timer; 0 restores the default of two seconds.
+ * Returns the previous bound.  For testing the timeout path (a tiny bound makes the first wait
+ * that does not succeed at once give up and report SIA_DEV_TIMEOUT); a serving caller leaves it
+ * alone.  Not a counterpart of anything in the pages describing the method. */
+uint64_t sia_set_wait_limit_ns(uint64_t ns);
 
 /* Static description of a status code. */
 const char* sia_status_string(sia_status s);

@@ -26,7 +26,7 @@ LIB_PATH = os.path.join(_PKG, "libsia.so")
 HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "sia.h")
 
 SIA_OK, SIA_ERR_INVALID_ARGUMENT, SIA_ERR_UNSUPPORTED, SIA_ERR_CUDA, SIA_ERR_WORKSPACE = range(5)
-SIA_DEV_BAD_PAGE, SIA_DEV_BAD_POSITION, SIA_DEV_TIMEOUT = 0x1, 0x2, 0x4
+SIA_DEV_BAD_PAGE, SIA_DEV_BAD_POSITION, SIA_DEV_TIMEOUT, SIA_DEV_INTERNAL = 0x1, 0x2, 0x4, 0x8
 SIA_BF16, SIA_FP8_E4M3 = 0, 1
 
 
@@ -93,6 +93,8 @@ def load_library(path: str = LIB_PATH):
     lib.sia_status_string.argtypes = [ctypes.c_int]
     lib.sia_last_error.restype = ctypes.c_char_p
     lib.sia_version.restype = ctypes.c_int32
+    lib.sia_set_wait_limit_ns.restype = ctypes.c_uint64
+    lib.sia_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
     _lib = lib
     return lib
 
@@ -102,6 +104,12 @@ def header_functions(path: str = HEADER_PATH):
     with open(path) as f:
         text = f.read()
     return sorted(set(re.findall(r"^\s*[A-Za-z_][\w\s\*]*?\b(sia_\w+)\s*\(", text, re.M)))
+
+
+def set_wait_limit_ns(ns: int) -> int:
+    """Bound of every in-kernel wait of later calls (0 = the default two seconds); returns the
+    previous bound.  Only for testing the timeout path."""
+    return int(load_library().sia_set_wait_limit_ns(int(ns)))
 
 
 def _check(status: int):

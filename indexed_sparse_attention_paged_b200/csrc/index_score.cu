@@ -42,13 +42,16 @@ struct IndexBarriers {
   uint64_t k_empty[8];
   uint64_t acc_full[2][2];
   uint64_t acc_empty[2][2];
-  uint64_t q_full;
+  uint64_t q_full;    // every epilogue thread staged the group's w and positions
+  uint64_t q_tma;     // the group's q boxes landed (TMA bytes only)
   uint64_t q_empty;
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort;
   int start_item, start_tile, count;
 };
+// the host reserves 256 bytes for the barrier block (bar_bytes in the stage-1 plan)
+static_assert(sizeof(IndexBarriers) <= 256, "barrier block outgrew its shared-memory slot");
 
 struct GroupInfo {
   int b, g;         // sequence, query group
@@ -154,7 +157,7 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
 
   if ((smem_u32(smem) & 1023u) != 0) {  // the swizzled layouts need a 1024-byte aligned base
     pdl_wait_primary();
-    if (threadIdx.x == 0) report(p.status, SIA_DEV_TIMEOUT);
+    if (threadIdx.x == 0) report(p.status, SIA_DEV_INTERNAL);
     return;
   }
   // The next kernel on the stream may be scheduled as soon as every CTA of this grid runs: it
@@ -171,6 +174,7 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
         mbar_init(&sb->acc_empty[a][s], 128);
       }
     mbar_init(&sb->q_full, kEpiThreads);
+    mbar_init(&sb->q_tma, 1);
     mbar_init(&sb->q_empty, 1);
     mbar_init(&sb->mma_done, 1);
     sb->abort = 0;
@@ -191,6 +195,7 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
   tc_fence_after();
   const uint32_t tmem_base = sb->tmem_base;
   volatile int* abort = &sb->abort;
+  const WaitCtl wc{abort, p.status, p.wait_ns};
   const int start_item = sb->start_item;
   const int start_tile = sb->start_tile;
   const int my_count = sb->count;
@@ -210,7 +215,7 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
         const int stage = it % p.k_stages;
         const uint32_t phase = (uint32_t)(it / p.k_stages) & 1u;
         int go = 1;
-        if (lane == 0) go = mbar_wait(&sb->k_empty[stage], phase ^ 1u, abort, p.status);
+        if (lane == 0) go = mbar_wait(&sb->k_empty[stage], phase ^ 1u, wc);
         go = __shfl_sync(0xffffffffu, go, 0);
         if (!go) { ok = false; break; }
         uint8_t* kst = smem + p.off_k + stage * p.k_stage_bytes;
@@ -260,11 +265,13 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
       ++item;
       t0 = 0;
     }
-    // do not leave while loads into our shared memory may still be landing
+    // do not leave while loads into our shared memory may still be landing: the last k_stages
+    // tiles issued (earlier ones were consumed before their stage was refilled) are drained
+    // whether or not the CTA is aborting
     if (lane == 0 && it > 0) {
       const int first = it > p.k_stages ? it - p.k_stages : 0;
       for (int i = first; i < it; ++i)
-        mbar_wait(&sb->k_full[i % p.k_stages], (uint32_t)(i / p.k_stages) & 1u, abort, p.status);
+        mbar_drain(&sb->k_full[i % p.k_stages], (uint32_t)(i / p.k_stages) & 1u, p.status);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
@@ -281,11 +288,12 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
         const GroupInfo gi = group_info(p, item);
         const int t1 = min(gi.n_tiles, t0 + remaining);
         if (t1 > t0) {
-          if (!mbar_wait(&sb->q_full, (uint32_t)seg & 1u, abort, p.status)) { ok = false; break; }
+          if (!mbar_wait(&sb->q_full, (uint32_t)seg & 1u, wc)) { ok = false; break; }
+          if (!mbar_wait(&sb->q_tma, (uint32_t)seg & 1u, wc)) { ok = false; break; }
           tc_fence_after();
           for (int t = t0; t < t1; ++t, ++it, ++acc_it) {
             const int stage = it % p.k_stages;
-            if (!mbar_wait(&sb->k_full[stage], (uint32_t)(it / p.k_stages) & 1u, abort, p.status)) {
+            if (!mbar_wait(&sb->k_full[stage], (uint32_t)(it / p.k_stages) & 1u, wc)) {
               ok = false;
               break;
             }
@@ -294,7 +302,7 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
             const uint32_t aph = (uint32_t)(acc_it / p.acc_stages) & 1u;
             const uint32_t a_base = smem_u32(smem + p.off_k + stage * p.k_stage_bytes);
             for (int sub = 0; sub < NSUB; ++sub) {
-              if (!mbar_wait(&sb->acc_empty[as][sub], aph ^ 1u, abort, p.status)) { ok = false; break; }
+              if (!mbar_wait(&sb->acc_empty[as][sub], aph ^ 1u, wc)) { ok = false; break; }
               tc_fence_after();
               const uint32_t d_tmem = tmem_base + (uint32_t)((as * NSUB + sub) * p.n_cols);
               const uint32_t b_base = smem_u32(smem + p.off_q + sub * p.q_sub_bytes);
@@ -321,7 +329,7 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
         t0 = 0;
       }
       umma_commit(&sb->mma_done);
-      mbar_wait(&sb->mma_done, 0, abort, p.status);
+      mbar_drain(&sb->mma_done, 0, p.status);   // every MMA (reading shared memory, writing TMEM) done
     }
     __syncwarp();
   } else {
@@ -334,7 +342,7 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
     // the next group while another still reads the current one (it cannot get two groups ahead,
     // since every epilogue thread must stage a group before its MMAs can run)
     const int w_words = p.qg * p.HP;
-    int acc_it = 0, seg = 0;
+    int acc_it = 0, seg = 0, q_issued = 0;
     int item = start_item, t0 = start_tile, remaining = my_count;
     bool ok = true;
     while (remaining > 0 && ok) {
@@ -342,20 +350,21 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
       const int t1 = min(gi.n_tiles, t0 + remaining);
       if (t1 > t0) {
         // -- stage this group's q (swizzled, zero-padded) and head weights
-        if (seg > 0 && !mbar_wait(&sb->q_empty, (uint32_t)(seg - 1) & 1u, abort, p.status)) { ok = false; break; }
+        if (seg > 0 && !mbar_wait_warp(&sb->q_empty, (uint32_t)(seg - 1) & 1u, wc)) { ok = false; break; }
         float* w_s = reinterpret_cast<float*>(smem + p.off_w) + (seg & 1) * w_words;
         int* info_pos = reinterpret_cast<int*>(smem + p.off_info) + (seg & 1) * 16;
         float* info_qs = reinterpret_cast<float*>(smem + p.off_info + 128) + (seg & 1) * 16;
         if (et == 0) {
           // q of the group: one 3-D TMA box (nq_sub queries x HP heads x one K block, heads
           // past H and queries past the batch zero-filled) per (sub-block, K block)
-          mbar_arrive_expect_tx(&sb->q_full, (uint32_t)(NSUB * NKB) * p.q_kblock_bytes);
+          mbar_arrive_expect_tx(&sb->q_tma, (uint32_t)(NSUB * NKB) * p.q_kblock_bytes);
 #pragma unroll
           for (int sb_ = 0; sb_ < NSUB; ++sb_)
 #pragma unroll
             for (int kb = 0; kb < NKB; ++kb)
-              tma_load_3d(smem + p.off_q + sb_ * p.q_sub_bytes + kb * p.q_kblock_bytes, &qmap, &sb->q_full,
+              tma_load_3d(smem + p.off_q + sb_ * p.q_sub_bytes + kb * p.q_kblock_bytes, &qmap, &sb->q_tma,
                           kb * KBW / (FP8 ? 1 : 2), 0, gi.b * p.J + gi.g * p.qg + sb_ * p.nq_sub);
+          ++q_issued;
         }
         for (int i = et; i < p.qg * p.HP; i += kEpiThreads) {
           const int ql = i / p.HP, h = i - ql * p.HP;
@@ -367,19 +376,19 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
           info_pos[et] = j < p.J ? query_position(p.seq_lens, p.q_pos, p.J, gi.b, j, p.Lpad) : -1;
           info_qs[et] = (j < p.J && p.q_scale) ? p.q_scale[(long long)gi.b * p.J + j] : 1.0f;
         }
-        if (et != 0) mbar_arrive(&sb->q_full);
+        mbar_arrive(&sb->q_full);
         // every epilogue thread has staged its share (w_s / info are visible after this)
-        if (!mbar_wait(&sb->q_full, (uint32_t)seg & 1u, abort, p.status)) { ok = false; break; }
+        if (!mbar_wait_warp(&sb->q_full, (uint32_t)seg & 1u, wc)) { ok = false; break; }
         const long long out_row0 = (long long)gi.b * p.J;
         for (int t = t0; t < t1; ++t, ++acc_it) {
           const int as = acc_it % p.acc_stages;
           const uint32_t aph = (uint32_t)(acc_it / p.acc_stages) & 1u;
           const int kstage = acc_it % p.k_stages;
           const int s = t * kIndexTileRows + row;
-          if (!mbar_wait(&sb->acc_full[as][sub], aph, abort, p.status)) { ok = false; break; }
+          if (!mbar_wait_warp(&sb->acc_full[as][sub], aph, wc)) { ok = false; break; }
           // the K stage of this tile is still held (k_empty also waits for us): its loads have
           // landed, and waiting on k_full makes the scales and the chunk mask visible here
-          if (!mbar_wait(&sb->k_full[kstage], (uint32_t)(acc_it / p.k_stages) & 1u, abort, p.status)) { ok = false; break; }
+          if (!mbar_wait_warp(&sb->k_full[kstage], (uint32_t)(acc_it / p.k_stages) & 1u, wc)) { ok = false; break; }
           tc_fence_after();
           const uint8_t* info = smem + p.off_kinfo + kstage * kStageInfoBytes;
           // a position whose page id is outside the pool is ranked last (-inf)
@@ -441,6 +450,9 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
       ++item;
       t0 = 0;
     }
+    // the q boxes of the last group this thread issued land before the CTA may leave (one group
+    // at a time: the next group's boxes are only issued once the MMAs have read this one's)
+    if (et == 0 && q_issued > 0) mbar_drain(&sb->q_tma, (uint32_t)(q_issued - 1) & 1u, p.status);
   }
   tc_fence_before();
   __syncthreads();

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -24,6 +25,8 @@ sia_status fail(sia_status s, const char* fmt, ...) {
   va_end(ap);
   return s;
 }
+
+std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
 
 sia_status cuda_fail(cudaError_t e, const char* what) {
   return fail(SIA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
@@ -251,6 +254,7 @@ sia_status run_index(IndexPlan* pl, void* ws, size_t ws_bytes, int32_t* dev_stat
     pl->kp.scores = static_cast<float*>(ws);
   }
   pl->kp.status = dev_status;
+  pl->kp.wait_ns = wait_limit_ns();
   pl->tp.scores = pl->kp.scores;
   pl->tp.status = dev_status;
   cudaError_t e = launch_index_score(pl->kp, pl->kmap, pl->qmap, pl->grid, pdl_first, stream);
@@ -371,6 +375,7 @@ sia_status run_attend(AttendPlan* pl, void* ws, size_t ws_bytes, int32_t* dev_st
     pl->cp.part_lse = pl->ap.part_lse;
   }
   pl->ap.status = dev_status;
+  pl->ap.wait_ns = wait_limit_ns();
   cudaError_t e = launch_sparse_attend(pl->ap, pl->q_rope, pl->n_clusters, pdl_first, stream);
   if (e != cudaSuccess) return cuda_fail(e, "sparse attention launch");
   if (pl->ap.splits > 1) {
@@ -381,6 +386,17 @@ sia_status run_attend(AttendPlan* pl, void* ws, size_t ws_bytes, int32_t* dev_st
 }
 
 }  // namespace
+
+uint64_t wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed); }
+
+sia_status set_last_error(sia_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+  va_end(ap);
+  return s;
+}
+
 }  // namespace sia
 
 using namespace sia;
@@ -420,6 +436,7 @@ sia_status sia_index_scores(const sia_index_args* a, int32_t* dev_status, void* 
   if (st != SIA_OK) return st;
   pl.kp.scores = a->scores_out;
   pl.kp.status = dev_status;
+  pl.kp.wait_ns = wait_limit_ns();
   cudaError_t e = launch_index_score(pl.kp, pl.kmap, pl.qmap, pl.grid, true, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "index scoring launch");
   return SIA_OK;
@@ -471,6 +488,10 @@ const char* sia_status_string(sia_status s) {
 }
 
 const char* sia_last_error(void) { return g_last_error; }
+
+uint64_t sia_set_wait_limit_ns(uint64_t ns) {
+  return g_wait_limit_ns.exchange(ns ? ns : 2000000000ull);
+}
 
 int32_t sia_version(void) { return 100; }
 

@@ -53,6 +53,7 @@ struct IndexKernelParams {
   const int32_t* q_pos;
   float* scores;
   int32_t* status;
+  uint64_t wait_ns;           // limit of every bounded in-kernel wait
 };
 
 // -------------------------------------------------------------------------- Top-K
@@ -85,6 +86,7 @@ struct AttnKernelParams {
   uint16_t* part_o;           // [splits][B*J][H][DL] bf16, normalised (splits > 1)
   float* part_lse;            // [splits][B*J][H]
   int32_t* status;
+  uint64_t wait_ns;           // limit of every bounded in-kernel wait
 };
 
 struct CombineKernelParams {
@@ -107,5 +109,11 @@ cudaError_t launch_combine(const CombineKernelParams& p, bool pdl, cudaStream_t 
 
 // Shared memory the attention kernel needs for (d_latent, d_rope).
 size_t attend_smem_bytes(int dl, int dr);
+
+// Limit of every bounded in-kernel wait, in nanoseconds (set by sia_set_wait_limit_ns).
+uint64_t wait_limit_ns();
+
+// Records the detail message that sia_last_error() returns on this host thread; returns s.
+sia_status set_last_error(sia_status s, const char* fmt, ...);
 
 }  // namespace sia

@@ -11,8 +11,13 @@
 
 namespace sia {
 
-// A bounded wait gives up after this many nanoseconds of %globaltimer.
-constexpr uint64_t kWaitTimeoutNs = 2000000000ull;
+// Every pipeline wait is bounded: it gives up after a limit of %globaltimer nanoseconds that the
+// host passes in the launch parameters (2 s unless sia_set_wait_limit_ns changed it).  A drain --
+// the wait for this thread's own asynchronous copies or tensor-core operations before the CTA
+// leaves -- has its own fixed limit and ignores the abort flag: those operations complete by
+// themselves, and a CTA must not exit while they may still write its shared memory or TMEM.
+constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;
+constexpr uint64_t kDrainLimitNs = 2000000000ull;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -109,12 +114,19 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
   return ok != 0;
 }
 
+// What a bounded wait needs: the CTA's abort flag (set by the first wait that gives up, so that
+// every other wait of the CTA gives up at once), the caller's status word and the limit.
+struct WaitCtl {
+  volatile int* abort;
+  int32_t* status;
+  uint64_t limit_ns;
+};
+
 // Waits for the completion of the barrier phase with parity `parity`.  Gives up when *abort
-// becomes non-zero or after kWaitTimeoutNs (then it sets *abort and reports SIA_DEV_TIMEOUT).
+// becomes non-zero or after wc.limit_ns (then it sets *abort and reports SIA_DEV_TIMEOUT).
 // Returns false when it gave up.
 template <bool kClusterScope = false>
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          int32_t* status) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtl& wc) {
   auto poll = [&]() {
     return kClusterScope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
   };
@@ -124,11 +136,34 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
       if (poll()) return true;
-    if (*abort) return false;
-    if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
-      *abort = 1;
-      report(status, SIA_DEV_TIMEOUT);
+    if (*wc.abort) return false;
+    if (globaltimer_ns() - t0 > wc.limit_ns) {
+      *wc.abort = 1;
+      report(wc.status, SIA_DEV_TIMEOUT);
       return false;
+    }
+  }
+}
+
+// The same wait made by every lane of a warp at the same point: the lanes agree on the outcome
+// (a lane that saw the phase complete just after another lane gave up gives up too), so that the
+// warp-wide instructions after the wait (shuffles, votes, tcgen05.ld/st) are reached by all of
+// its lanes or by none.
+template <bool kClusterScope = false>
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, const WaitCtl& wc) {
+  const bool ok = mbar_wait<kClusterScope>(bar, parity, wc);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Drain: waits for a barrier phase that only this thread's own asynchronous operations (TMA or
+// bulk copies, tcgen05 commits) complete, ignoring the abort flag, for at most kDrainLimitNs.
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity, int32_t* status) {
+  if (mbar_try_wait(bar, parity)) return;
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kDrainLimitNs) {
+      report(status, SIA_DEV_TIMEOUT);
+      return;
     }
   }
 }

@@ -158,7 +158,8 @@ struct AttnBarriers {
   uint64_t p_full;                  // all softmax threads wrote P (waited by the P . C issuer)
   uint64_t p_empty;                 // P . C of the previous tile done (P buffer and O free)
   uint64_t epi_sync;                // all softmax threads are past the unit's last tile
-  uint64_t q_full, q_empty;
+  uint64_t q_full, q_empty;       // q in TMEM written by the 128 loader threads / q reusable
+  uint64_t q_tma;                 // the rope part of q landed (TMA bytes only)
   uint64_t o_full;
   uint64_t sx_ready, sx_free;
   uint64_t tab_full[2], tab_free[2];
@@ -225,7 +226,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int DC = p.DL + p.DR;
 
   if ((smem_u32(smem) & 1023u) != 0) {
-    if (threadIdx.x == 0) report(p.status, SIA_DEV_TIMEOUT);
+    if (threadIdx.x == 0) report(p.status, SIA_DEV_INTERNAL);
     return;  // both CTAs of the pair see the same base alignment and leave together
   }
   if (threadIdx.x == 0) {
@@ -245,7 +246,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     mbar_init(&sb->p_full, 128);
     mbar_init(&sb->p_empty, 1);
     mbar_init(&sb->epi_sync, 128);
-    mbar_init(&sb->q_full, 128 + 1);   // 128 TMEM writers + the rope TMA
+    mbar_init(&sb->q_full, 128);       // the 128 TMEM writers
+    mbar_init(&sb->q_tma, 1);          // the rope TMA (or a plain arrive when this CTA has none)
     mbar_init(&sb->q_empty, 1);
     mbar_init(&sb->o_full, 1);
     mbar_init(&sb->sx_ready, 128);   // arrived by the peer's 128 exchange threads
@@ -265,6 +267,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = sb->tmem_base;
   volatile int* abort = &sb->abort;
+  const WaitCtl wc{abort, p.status, p.wait_ns};
   // The next kernel (the split merge, or the next call's first kernel) waits for this grid's
   // completion before its loads, so it may be scheduled now and only its launch overlaps ours.
   pdl_launch_dependents();
@@ -320,7 +323,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
       }
     };
-    int it = 0, u_it = 0;
+    int it = 0, u_it = 0, q_issued = 0;
     bool ok = true;
     bool waited = false;
     if (cluster_id < p.units) {
@@ -348,13 +351,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int buf = u_it & 1;
       // rope part of the query rows of all heads (TMA; independent of the Top-K list)
       if (ptid == 0) {
-        if (mbar_wait(&sb->q_empty, ((uint32_t)u_it & 1u) ^ 1u, abort, p.status)) {
+        if (mbar_wait(&sb->q_empty, ((uint32_t)u_it & 1u) ^ 1u, wc)) {
           if (rope) {
-            mbar_arrive_expect_tx(&sb->q_full, Sm::kQRopeBytes);
-            tma_load_2d(smem + Sm::kOffQ, &maps.q_rope, &sb->q_full, Lay::rope_x((int)rank), bj * p.H);
+            mbar_arrive_expect_tx(&sb->q_tma, Sm::kQRopeBytes);
+            tma_load_2d(smem + Sm::kOffQ, &maps.q_rope, &sb->q_tma, Lay::rope_x((int)rank), bj * p.H);
           } else {
-            mbar_arrive(&sb->q_full);
+            mbar_arrive(&sb->q_tma);
           }
+          ++q_issued;
         }
       }
       if (!waited) {
@@ -363,7 +367,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       // resolve this unit's Top-K entries to physical cache rows: 8 entries per thread, all
       // loads of a thread in flight at once
-      if (!mbar_wait(&sb->tab_free[buf], ((uint32_t)(u_it >> 1) & 1u) ^ 1u, abort, p.status)) { ok = false; break; }
+      if (!mbar_wait_warp(&sb->tab_free[buf], ((uint32_t)(u_it >> 1) & 1u) ^ 1u, wc)) { ok = false; break; }
       int32_t* rt = rows_tab + buf * kAttnMaxSplitRows;
       uint32_t* mt = mask_tab + buf * (kAttnMaxSplitRows / 32);
       const int32_t* tk = p.topk + row_base + row0;
@@ -399,20 +403,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       for (int o = 16; o > 0; o >>= 1) fneg = min(fneg, __shfl_xor_sync(0xffffffffu, fneg, o));
       if (lane == 0) fneg_tab[buf * kProducerWarps + pwarp] = fneg;
       mbar_arrive(&sb->tab_full[buf]);
-      if (!mbar_wait(&sb->tab_full[buf], (uint32_t)(u_it >> 1) & 1u, abort, p.status)) { ok = false; break; }
+      if (!mbar_wait_warp(&sb->tab_full[buf], (uint32_t)(u_it >> 1) & 1u, wc)) { ok = false; break; }
       const int ntiles = (unit_tiles(buf) + kRows - 1) / kRows;
       make_pieces();   // (after the table: the two never hold registers at the same time)
       for (int t = 0; t < ntiles; ++t, ++it) {
         const int stage = it % kStages, rslot = it % kRopeSlots;
-        if (!mbar_wait(&sb->c_empty[stage], ((uint32_t)(it / kStages) & 1u) ^ 1u, abort, p.status)) { ok = false; break; }
-        if (!mbar_wait(&sb->r_empty[rslot], ((uint32_t)(it / kRopeSlots) & 1u) ^ 1u, abort, p.status)) { ok = false; break; }
+        if (!mbar_wait_warp(&sb->c_empty[stage], ((uint32_t)(it / kStages) & 1u) ^ 1u, wc)) { ok = false; break; }
+        if (!mbar_wait_warp(&sb->r_empty[rslot], ((uint32_t)(it / kRopeSlots) & 1u) ^ 1u, wc)) { ok = false; break; }
         gather_tile(smem_u32(smem + Sm::kOffC + stage * Sm::kCStageBytes),
                     smem_u32(smem + Sm::kOffR + rslot * Sm::kCRopeBytes), rt + t * kRows);
         asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(&sb->c_full[stage])) : "memory");
       }
     }
-    asm volatile("cp.async.wait_all;" ::: "memory");  // our copies have landed before we may leave
-    if (ptid == 0 && u_it > 0) mbar_wait(&sb->q_full, (uint32_t)(u_it - 1) & 1u, abort, p.status);
+    // our copies have landed before we may leave, whether or not the CTA is aborting: every
+    // cp.async of this thread, and the rope TMA of the last unit (one unit's q at a time: the
+    // next is only issued once the products of this one are done)
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    if (ptid == 0 && q_issued > 0) mbar_drain(&sb->q_tma, (uint32_t)(q_issued - 1) & 1u, p.status);
   } else if (warp == kMmaWarp) {
     // ---------------------------------------------------------------- S = Q . C^T issuer
     // (O += P . C has its own issuing warp, so a logit tile never waits for P of an earlier
@@ -424,16 +431,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       bool ok = true;
       for (int u = cluster_id; u < p.units && ok; u += n_clusters, ++u_it) {
         const int buf = u_it & 1;
-        if (!mbar_wait(&sb->tab_full[buf], (uint32_t)(u_it >> 1) & 1u, abort, p.status)) { ok = false; break; }
+        if (!mbar_wait(&sb->tab_full[buf], (uint32_t)(u_it >> 1) & 1u, wc)) { ok = false; break; }
         const int ntiles = (unit_tiles(buf) + kRows - 1) / kRows;
         mbar_arrive(&sb->tab_free[buf]);
-        if (!mbar_wait(&sb->q_full, (uint32_t)u_it & 1u, abort, p.status)) { ok = false; break; }
+        if (!mbar_wait(&sb->q_full, (uint32_t)u_it & 1u, wc)) { ok = false; break; }
+        if (!mbar_wait(&sb->q_tma, (uint32_t)u_it & 1u, wc)) { ok = false; break; }
         tc_fence_after();
         for (int t = 0; t < ntiles; ++t, ++it) {
           const int stage = it % kStages;
           const int sbuf = it & 1;
-          if (!mbar_wait(&sb->c_full[stage], (uint32_t)(it / kStages) & 1u, abort, p.status)) { ok = false; break; }
-          if (!mbar_wait(&sb->s_empty[sbuf], ((uint32_t)(it >> 1) & 1u) ^ 1u, abort, p.status)) { ok = false; break; }
+          if (!mbar_wait(&sb->c_full[stage], (uint32_t)(it / kStages) & 1u, wc)) { ok = false; break; }
+          if (!mbar_wait(&sb->s_empty[sbuf], ((uint32_t)(it >> 1) & 1u) ^ 1u, wc)) { ok = false; break; }
           fence_proxy_async_smem();   // the gathered rows were written by cp.async
           tc_fence_after();
           const uint32_t c_base = smem_u32(smem + Sm::kOffC + stage * Sm::kCStageBytes);
@@ -462,7 +470,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         umma_commit(&sb->q_empty);  // q reusable once this unit's products are done
       }
       umma_commit(&sb->mma_done);
-      mbar_wait(&sb->mma_done, 0, abort, p.status);
+      mbar_drain(&sb->mma_done, 0, p.status);   // every S = Q . C^T product done
     }
     __syncwarp();
   } else if (warp == kPvWarp) {
@@ -474,11 +482,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       bool ok = true;
       for (int u = cluster_id; u < p.units && ok; u += n_clusters, ++u_it) {
         const int buf = u_it & 1;
-        if (!mbar_wait(&sb->tab_full[buf], (uint32_t)(u_it >> 1) & 1u, abort, p.status)) { ok = false; break; }
+        if (!mbar_wait(&sb->tab_full[buf], (uint32_t)(u_it >> 1) & 1u, wc)) { ok = false; break; }
         const int ntiles = (unit_tiles(buf) + kRows - 1) / kRows;
         mbar_arrive(&sb->tab_free[buf]);
         for (int t = 0; t < ntiles; ++t, ++it) {
-          if (!mbar_wait(&sb->p_full, (uint32_t)it & 1u, abort, p.status)) { ok = false; break; }
+          if (!mbar_wait(&sb->p_full, (uint32_t)it & 1u, wc)) { ok = false; break; }
           fence_proxy_async_smem();   // the row stage (cp.async) and P (st.shared)
           tc_fence_after();
           const int stage = it % kStages;
@@ -496,7 +504,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
       }
       umma_commit(&sb->pv_done);
-      mbar_wait(&sb->pv_done, 0, abort, p.status);
+      mbar_drain(&sb->pv_done, 0, p.status);    // every O += P . C product done
     }
     __syncwarp();
   } else if (warp >= kFirstExchangeWarp && warp < kFirstExchangeWarp + 4) {
@@ -516,7 +524,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int buf = u_it & 1;
       {
         // q: head h's dims [rank * kLatDims, +kLatDims) as bf16 pairs, 16 columns per store
-        if (!mbar_wait(&sb->q_empty, ((uint32_t)u_it & 1u) ^ 1u, abort, p.status)) { ok = false; break; }
+        if (!mbar_wait_warp(&sb->q_empty, ((uint32_t)u_it & 1u) ^ 1u, wc)) { ok = false; break; }
         const bool real = h < p.H;
         const uint8_t* qrow = static_cast<const uint8_t*>(p.q) + ((long long)bj * p.H + (real ? h : 0)) * (DC * 2) +
                               (size_t)rank * Lay::kLatDims * 2;
@@ -545,13 +553,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tc_fence_before();
         mbar_arrive(&sb->q_full);
       }
-      if (!mbar_wait(&sb->tab_full[buf], (uint32_t)(u_it >> 1) & 1u, abort, p.status)) { ok = false; break; }
+      if (!mbar_wait_warp(&sb->tab_full[buf], (uint32_t)(u_it >> 1) & 1u, wc)) { ok = false; break; }
       const int ntiles = (unit_tiles(buf) + kRows - 1) / kRows;
       mbar_arrive(&sb->tab_free[buf]);
       for (int t = 0; t < ntiles; ++t, ++s_it) {
         const int sbuf = s_it & 1;
         const uint32_t scol = lane_addr + Tm::kS + sbuf * kRows;
-        if (!mbar_wait(&sb->s_full[sbuf], (uint32_t)(s_it >> 1) & 1u, abort, p.status)) { ok = false; break; }
+        if (!mbar_wait_warp(&sb->s_full[sbuf], (uint32_t)(s_it >> 1) & 1u, wc)) { ok = false; break; }
         tc_fence_after();
         uint32_t own[kRows / 2];
         {
@@ -569,13 +577,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tc_fence_before();
         mbar_arrive(&sb->s_empty[sbuf]);   // our reads of these logits are done
         // own fp16 logits for our softmax (the same values the peer receives)
-        if (!mbar_wait(&sb->own_free[sbuf], ((uint32_t)(s_it >> 1) & 1u) ^ 1u, abort, p.status)) { ok = false; break; }
+        if (!mbar_wait_warp(&sb->own_free[sbuf], ((uint32_t)(s_it >> 1) & 1u) ^ 1u, wc)) { ok = false; break; }
 #pragma unroll
         for (int g = 0; g < kRows / 8; ++g)
           st_shared_v4(smem_u32(smem + Sm::kOffStash + sbuf * (kRows * 128 * 2) + (g * 128 + h) * 16),
                        own[4 * g], own[4 * g + 1], own[4 * g + 2], own[4 * g + 3]);
         mbar_arrive(&sb->own_ready[sbuf]);
-        if (!mbar_wait<true>(&sb->sx_free, ((uint32_t)s_it & 1u) ^ 1u, abort, p.status)) { ok = false; break; }
+        if (!mbar_wait_warp<true>(&sb->sx_free, ((uint32_t)s_it & 1u) ^ 1u, wc)) { ok = false; break; }
 #pragma unroll
         for (int g = 0; g < kRows / 8; ++g)
           asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sx_peer + (uint32_t)((g * 128 + h) * 16)),
@@ -596,7 +604,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     for (int u = cluster_id; u < p.units && ok; u += n_clusters, ++u_it) {
       const int bj = u / p.splits, split = u - bj * p.splits;
       const int buf = u_it & 1;
-      if (!mbar_wait(&sb->tab_full[buf], (uint32_t)(u_it >> 1) & 1u, abort, p.status)) { ok = false; break; }
+      if (!mbar_wait_warp(&sb->tab_full[buf], (uint32_t)(u_it >> 1) & 1u, wc)) { ok = false; break; }
       const int first_neg = unit_tiles(buf);
       const int ntiles = (first_neg + kRows - 1) / kRows;
       const uint32_t* mt = mask_tab + buf * (kAttnMaxSplitRows / 32);
@@ -607,8 +615,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         uint64_t valid = ((uint64_t)mt[2 * t + 1] << 32) | mt[2 * t];
         const int live = first_neg - t * kRows;            // rows past the first -1 are padding
         if (live < kRows) valid &= (1ull << live) - 1ull;
-        if (!mbar_wait(&sb->own_ready[sbuf], (uint32_t)(s_it >> 1) & 1u, abort, p.status)) { ok = false; break; }
-        if (!mbar_wait<true>(&sb->sx_ready, (uint32_t)s_it & 1u, abort, p.status)) { ok = false; break; }
+        if (!mbar_wait_warp(&sb->own_ready[sbuf], (uint32_t)(s_it >> 1) & 1u, wc)) { ok = false; break; }
+        if (!mbar_wait_warp<true>(&sb->sx_ready, (uint32_t)s_it & 1u, wc)) { ok = false; break; }
         // logits of tile t (base 2) = own fp16 partial + the peer's fp16 partial: both CTAs add
         // the same two values, so their logits agree bit for bit
 #pragma unroll
@@ -665,7 +673,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         l = l * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
 
         // P . C of the previous tile must be done: it reads the P buffer, and O is rescaled
-        if (!mbar_wait(&sb->p_empty, ((uint32_t)s_it & 1u) ^ 1u, abort, p.status)) { ok = false; break; }
+        if (!mbar_wait_warp(&sb->p_empty, ((uint32_t)s_it & 1u) ^ 1u, wc)) { ok = false; break; }
         tc_fence_after();
         if (__any_sync(0xffffffffu, need && t > 0)) {
           // O holds the tiles < t of this unit: rescale it
@@ -694,7 +702,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_arrive(&sb->tab_free[buf]);
       // ---- unit epilogue: normalise O and write it out
       if (ntiles > 0) {
-        if (!mbar_wait(&sb->o_full, (uint32_t)o_it & 1u, abort, p.status)) { ok = false; break; }
+        if (!mbar_wait_warp(&sb->o_full, (uint32_t)o_it & 1u, wc)) { ok = false; break; }
         ++o_it;
       }
       tc_fence_after();
@@ -711,7 +719,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (ntiles > 0) {
         // every softmax warp has read the last tile's peer logits before any slice is reused
         mbar_arrive(&sb->epi_sync);
-        if (!mbar_wait(&sb->epi_sync, (uint32_t)e_it & 1u, abort, p.status)) { ok = false; break; }
+        if (!mbar_wait_warp(&sb->epi_sync, (uint32_t)e_it & 1u, wc)) { ok = false; break; }
         ++e_it;
         uint8_t* slice = smem + Sm::kOffSx + quad * 4096;
 #pragma unroll 1

@@ -4,7 +4,7 @@ This module only draws random inputs (on the CPU, with ``torch.Generator``) and 
 the method's arithmetic.  Both the CUDA path and the CPU oracle are fed from it, so they see
 identical bytes.
 
-Input recipe (also stated in the design doc):
+Input recipe:
   * index q and index k: integers drawn uniformly from [-3, 3], stored as bf16 or as FP8 E4M3
     (exact either way);
   * head weights w: integers drawn uniformly from [-2, 2], fp32;

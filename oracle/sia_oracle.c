@@ -14,7 +14,7 @@
  * (one index key per position shared by all heads), ties in Top-K go to the lower position,
  * and every floating-point value is carried in fp64.
  *
- * Readings of points the pages leave open (each one is listed in the design doc):
+ * Readings of points the pages leave open:
  *   - causal: query j of sequence b at position p sees positions 0..p (itself included);
  *   - quantised index cache: value = e4m3 code decoded exactly, times its per-token scale
  *     ("high-precision computation + low-precision cache": dequantise, then compute);

@@ -138,3 +138,17 @@ def test_binding_refuses_cpu_tensors():
     q = torch.zeros(1, 1, 4, 32, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         sia.index_args(q, q, q, q, q, top_k=4)
+
+
+def test_wait_limit_setter_returns_the_previous_bound(lib):
+    first = sia.set_wait_limit_ns(12345)
+    assert sia.set_wait_limit_ns(0) == 12345
+    assert sia.set_wait_limit_ns(first) == 2_000_000_000
+
+
+def test_noalloc_entry_point_clears_a_stale_error_message(lib):
+    bad = _index_args(batch=0)
+    assert lib.sia_sparse_index_topk(ctypes.byref(bad), None, 0, None, None) == sia.SIA_ERR_INVALID_ARGUMENT
+    assert lib.sia_last_error() != b""
+    assert lib.sia_sparse_index_topk_noalloc(None, None, None) == sia.SIA_ERR_INVALID_ARGUMENT
+    assert b"NULL" in lib.sia_last_error()
