@@ -12,8 +12,12 @@ back between two CUDA events on the launching stream; the reported time is the m
 maximum over ranks.  With N GPUs every rank runs its own independent batch (weak scaling, no
 collective on the data path).
 
-Prints one JSON line (rank 0).  `--impl reference` times the CPU oracle (the only reference
-implementation: the pages have no code) on a bounded sample of the same workload.
+Prints one JSON line (rank 0).  The headline is the B=32 decode; the same line carries, under
+`workloads`, the FP8-index decode (B=128, ragged contexts), the speculative decode (B=8, J=2,
+context 131072) and the causal prefill chunk (T=16384: scoring TFLOP/s against the tensor peak,
+and the full index + Top-K + attention path), unless --no-sub-workloads.  `--impl reference`
+times the CPU oracle (the only reference implementation: the pages have no code) on a bounded
+sample of the same workload.
 """
 from __future__ import annotations
 
@@ -34,6 +38,7 @@ PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
+FALLBACK_BF16_SUSTAINED = 1400.0
 L2_BYTES = 126 * 1024 * 1024
 
 
@@ -46,6 +51,10 @@ def parse():
     ap.add_argument("--workload", type=int, default=2, choices=[2, 3, 4, 5],
                     help="2, 3, 5: fused decode (queries/s); 4: prefill indexer scoring (TFLOP/s)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sub-workloads", action="store_true",
+                    help="only the headline workload (no configs 3, 4, 5 in the same line)")
+    ap.add_argument("--soak-s", type=float, default=1.0,
+                    help="seconds of untimed steps right before the timed region, under the clock sampler")
     return ap.parse_args()
 
 
@@ -114,6 +123,40 @@ def algorithmic_bytes(inputs) -> dict:
                 idx_k=idx_k, kv=kv)
 
 
+def algorithmic_flops(inputs) -> dict:
+    """Tensor-core work of one step: the scoring contraction over every visible (query,
+    position) pair (2 * H_i * D_i each) and the attention over every selected row of every query
+    (2 * H_a * (d_latent + d_rope) for the logits plus 2 * H_a * d_latent for the output)."""
+    wl = inputs["workload"]
+    J = inputs["n_q"]
+    lens = [int(x) for x in inputs["seq_lens"]]
+    pairs = sum(L - J + j + 1 for L in lens for j in range(J))
+    sel = sum(min(wl.top_k, L - J + j + 1) for L in lens for j in range(J))
+    stage1 = 2 * wl.idx_heads * wl.idx_dim * pairs
+    stage2 = 2 * wl.attn_heads * sel * ((wl.d_latent + wl.d_rope) + wl.d_latent)
+    return dict(stage1=stage1, stage2=stage2, total=stage1 + stage2)
+
+
+def roofline_entry(kernel, nbytes, flops, ms, pk, tensor_peak_key="bf16_tflops"):
+    """Roofline of one timed call: achieved bytes/s and FLOP/s against the measured peaks.  The
+    bound is the resource whose roofline time (bytes / bandwidth, FLOPs / tensor peak) is the
+    longer; `frac` is achieved / peak for that bound, and both fractions are given."""
+    gbs = nbytes / (ms / 1000.0) / 1e9
+    tfs = flops / (ms / 1000.0) / 1e12
+    t_hbm = nbytes / (pk["hbm_gbs"] * 1e9)
+    t_tc = flops / (pk[tensor_peak_key] * 1e12) if flops else 0.0
+    hbm = t_hbm >= t_tc
+    return {"bound": "hbm" if hbm else "tensor", "kernel": kernel,
+            "achieved": gbs if hbm else tfs, "peak": pk["hbm_gbs"] if hbm else pk[tensor_peak_key],
+            "unit": "GB/s" if hbm else "TFLOP/s",
+            "frac": gbs / pk["hbm_gbs"] if hbm else tfs / pk[tensor_peak_key],
+            "hbm_frac": gbs / pk["hbm_gbs"], "tensor_frac": tfs / pk[tensor_peak_key],
+            "achieved_gbs": gbs, "achieved_tflops": tfs,
+            "roofline_us": max(t_hbm, t_tc) * 1e6,
+            "peak_source": "%s (HBM copy; bf16 %s)" % (pk["source"], "burst" if tensor_peak_key == "bf16_tflops" else "sustained"),
+            "algorithmic_bytes_per_launch": nbytes, "flops_per_launch": flops, "ms_per_launch": ms}
+
+
 class ClockSampler:
     """nvidia-smi clocks and throttle reasons every 200 ms while the timed region runs."""
 
@@ -171,9 +214,12 @@ def peaks() -> dict:
     try:
         with open(PEAKS_FILE) as f:
             p = json.load(f)
-        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]), "source": "measured"}
+        burst = float(p["bf16_tflops"])
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": burst,
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", burst)), "source": "measured"}
     except (OSError, KeyError, ValueError):
-        return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS, "source": "fallback"}
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+                "bf16_tflops_sustained": FALLBACK_BF16_SUSTAINED, "source": "fallback"}
 
 
 # What each stage-level roofline entry times: one C-ABI call, i.e. both kernels of the stage.
@@ -231,8 +277,10 @@ def run_reference(args, rank, world):
     v = statistics.mean(x["value"] for x in vals)
     cb = dict(vals[-1])
     cb["value"] = v
+    # a step is the whole batch: its time at the sampled rate
+    queries = inputs["batch"] * inputs["n_q"]
     line = dict(impl="reference", metric=metric_name(wl), value=v, unit="queries/s", n_gpus=args.gpus,
-                steps=args.steps, warmup=args.warmup, ms_per_step=1000.0 * len(rows) / v / 1.0,
+                steps=args.steps, warmup=args.warmup, ms_per_step=1000.0 * queries / v,
                 higher_is_better=True, scaling="weak", vs_baseline=None, dtype="f64", data="synthetic",
                 config=config_of(wl, inputs, "cpu (no L2 flush)"), cpu_baseline=cb,
                 e2e={"value": v, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0})
@@ -334,11 +382,12 @@ def prefill_scoring_flops(seq_lens, n_q, heads, dim) -> int:
     return 2 * heads * dim * total
 
 
-def run_prefill_scoring(args, rank, world, dev, wl):
-    """Prefill chunk (T = 16384 causal): the indexer's scoring step alone (sia_index_scores),
-    in TFLOP/s of the causal q.k contraction against the measured bf16 tensor peak."""
+def measure_prefill(dev, wl, rank, steps, warmup, full_path):
+    """Causal prefill chunk (T = 16384): the indexer's scoring step alone (sia_index_scores), in
+    TFLOP/s of the causal q.k contraction against the measured bf16 tensor peaks; with
+    `full_path`, also the whole path for the chunk (sia_sparse_index_topk over the 1 GiB score
+    workspace, then sia_sparse_mla_attend for every query), timed once per step."""
     import torch
-    import torch.distributed as dist
     import indexed_sparse_attention_paged_b200 as sia
     from indexed_sparse_attention_paged_b200 import workloads
 
@@ -354,49 +403,198 @@ def run_prefill_scoring(args, rank, world, dev, wl):
         sia.index_scores(d["q_idx"], d["w"], d["k_cache"], d["page_table"], d["seq_lens"],
                          k_scale=d["k_scale"], scores_out=scores, dev_status=status, stream=stream)
 
-    for _ in range(max(3, args.warmup)):
+    for _ in range(max(3, warmup)):
         step()
     torch.cuda.synchronize()
-    steps = max(1, min(args.steps, 50))
-    sampler = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
-    sampler.start()
-    time.sleep(0.25)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
+    n = max(1, min(steps, 50))
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(steps):
+    for _ in range(n):
         step()
     e1.record(stream)
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / steps
-    clocks = sampler.stop()
-    (ms,) = max_over_ranks([ms], dev)
+    ms = e0.elapsed_time(e1) / n
     if int(status.item()) != 0:
         raise RuntimeError("device status %d" % int(status.item()))
     flops = prefill_scoring_flops(host["seq_lens"].tolist(), J, wl.idx_heads, wl.idx_dim)
+    out = {"ms_per_step": ms, "steps": n, "flops_per_launch": flops, "launches": n}
+    out["_ms"] = ms
+    out["_flops"] = flops
+    if full_path:
+        topk = torch.empty((B, J, wl.top_k), dtype=torch.int32, device=dev)
+        att = torch.empty((B, J, wl.attn_heads, wl.d_latent), dtype=torch.bfloat16, device=dev)
+        ws1 = torch.empty(max(256, sia.load_library().sia_index_workspace_size(__import__("ctypes").byref(
+            sia.index_args(d["q_idx"], d["w"], d["k_cache"], d["page_table"], d["seq_lens"], top_k=wl.top_k,
+                           topk_out=topk)))), dtype=torch.uint8, device=dev)
+
+        def full():
+            sia.sparse_index_topk(d["q_idx"], d["w"], d["k_cache"], d["page_table"], d["seq_lens"],
+                                  top_k=wl.top_k, k_scale=d["k_scale"], topk_out=topk, workspace=ws1,
+                                  dev_status=status, stream=stream)
+            sia.sparse_mla_attend(d["q_attn"], d["kv_cache"], d["page_table"], d["seq_lens"], topk,
+                                  d_latent=wl.d_latent, softmax_scale=wl.softmax_scale, out=att,
+                                  dev_status=status, stream=stream)
+        full()
+        torch.cuda.synchronize()
+        nf = 3
+        e0.record(stream)
+        for _ in range(nf):
+            full()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        fms = e0.elapsed_time(e1) / nf
+        if int(status.item()) != 0:
+            raise RuntimeError("device status %d" % int(status.item()))
+        ab = algorithmic_flops(host)
+        out["full_path"] = {"ms_per_step": fms, "queries_per_s": B * J / (fms / 1000.0), "steps": nf,
+                            "calls": "sia_sparse_index_topk (score workspace %.2f GiB) + sia_sparse_mla_attend"
+                                     % (B * J * Lpad * 4 / 2 ** 30),
+                            "tensor_flops": ab["total"],
+                            "achieved_tflops": ab["total"] / (fms / 1000.0) / 1e12}
+        out["launches"] += nf * 4
+        del topk, att, ws1
+    del scores, d
+    torch.cuda.empty_cache()
+    return out
+
+
+def prefill_entry(res, pk, wl):
+    ms, flops = res["_ms"], res["_flops"]
     tflops = flops / (ms / 1000.0) / 1e12
+    e = {"workload": wl.name, "metric": "prefill indexer scoring TFLOP/s @T=%d causal, %dx%d bf16"
+         % (wl.context, wl.idx_heads, wl.idx_dim),
+         "value": tflops, "unit": "TFLOP/s", "ms_per_step": ms, "steps": res["steps"],
+         "roofline": {"bound": "tensor", "kernel": "index_score_kernel (one sia_index_scores call)",
+                      "achieved": tflops, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                      "frac": tflops / pk["bf16_tflops"], "peak_source": pk["source"] + " burst",
+                      "frac_of_sustained": tflops / pk["bf16_tflops_sustained"],
+                      "traffic": None, "flops_per_launch": flops}}
+    if "full_path" in res:
+        e["full_path"] = res["full_path"]
+    return e
+
+
+def run_prefill_scoring(args, rank, world, dev, wl):
+    """`--workload 4` as the headline: the prefill scoring line."""
+    import torch.distributed as dist
+    sampler = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
+    sampler.start()
+    if world > 1:
+        dist.barrier()
+    res = measure_prefill(dev, wl, rank, args.steps, args.warmup, full_path=False)
+    clocks = sampler.stop()
+    (ms,) = max_over_ranks([res["_ms"]], dev)
+    res["_ms"] = ms
     pk = peaks()
+    e = prefill_entry(res, pk, wl)
     if rank == 0:
-        print(json.dumps({
-            "metric": "prefill indexer scoring TFLOP/s @T=%d causal, %dx%d bf16" % (J, wl.idx_heads, wl.idx_dim),
-            "value": world * tflops, "unit": "TFLOP/s", "n_gpus": world, "steps": steps,
-            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": wl.name, "tokens": J, "idx_heads": wl.idx_heads, "idx_dim": wl.idx_dim,
-                       "l2": "the 16384 x 256 B index keys (4 MB) are L2-resident by design: the "
-                             "contraction reuses each key tile for every query group",
-                       "parallelism": "replicas"},
-            "roofline": {"bound": "tensor", "kernel": "index_score_kernel (one sia_index_scores call)",
-                         "achieved": tflops, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                         "frac": tflops / pk["bf16_tflops"], "peak_source": pk["source"] + " burst",
-                         "traffic": None, "flops_per_launch": flops},
-            "gpu_launches": steps, "clocks": clocks,
-        }), flush=True)
+        line = {"metric": e["metric"], "value": world * e["value"], "unit": "TFLOP/s", "n_gpus": world,
+                "steps": res["steps"], "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": wl.name, "tokens": wl.context, "idx_heads": wl.idx_heads,
+                           "idx_dim": wl.idx_dim,
+                           "l2": "the 16384 x 256 B index keys (4 MB) are L2-resident by design: the "
+                                 "contraction reuses each key tile for every query group",
+                           "parallelism": "replicas"},
+                "roofline": e["roofline"], "gpu_launches": res["launches"], "clocks": clocks}
+        print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
     return 0
+
+
+class DecodeBench:
+    """One decode workload on this rank: input sets (round-robin, larger than L2 together),
+    one fused-decode plan per set, and the stage-only calls for the per-stage rooflines."""
+
+    def __init__(self, sia, workloads, wl, rank, dev, min_sets):
+        import ctypes
+        import torch
+        self.wl = wl
+        self.host = workloads.make_inputs(wl, seed=1000 + wl.number + 7919 * rank)
+        per_step = step_bytes(self.host)
+        self.n_sets = max(min_sets, -(-4 * L2_BYTES // max(1, per_step))) if per_step < 4 * L2_BYTES else min_sets
+        self.sets = [workloads.to_device(self.host, dev)]
+        for i in range(1, self.n_sets):
+            self.sets.append(workloads.to_device(
+                workloads.make_inputs(wl, seed=1000 + wl.number + 7919 * rank + 104729 * i), dev))
+        self.plans = [sia.FusedDecodePlan(d, dev) for d in self.sets]
+        self.stream = torch.cuda.current_stream()
+        lib = sia.load_library()
+        sp = ctypes.c_void_p(self.stream.cuda_stream)
+        self.stage1, self.stage2 = [], []
+        for pl in self.plans:
+            ws1 = torch.empty(max(256, lib.sia_index_workspace_size(ctypes.byref(pl.ia))), dtype=torch.uint8, device=dev)
+            ws2 = torch.empty(max(256, lib.sia_attend_workspace_size(ctypes.byref(pl.aa))), dtype=torch.uint8, device=dev)
+            st_ptr = ctypes.c_void_p(pl.status.data_ptr())
+
+            def f1(pl=pl, ws1=ws1, st_ptr=st_ptr):
+                sia._check(lib.sia_sparse_index_topk(ctypes.byref(pl.ia), ctypes.c_void_p(ws1.data_ptr()), ws1.numel(), st_ptr, sp))
+
+            def f2(pl=pl, ws2=ws2, st_ptr=st_ptr):
+                sia._check(lib.sia_sparse_mla_attend(ctypes.byref(pl.aa), ctypes.c_void_p(ws2.data_ptr()), ws2.numel(), st_ptr, sp))
+            self.stage1.append(f1)
+            self.stage2.append(f2)
+        self.kernels_per_step = 3 + (1 if plan_splits(lib, self.plans[0].aa) > 1 else 0)
+
+    def timed(self, fns, steps):
+        """Mean device time per call of fns[i % len(fns)], back to back, CUDA events."""
+        import torch
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(self.stream)
+        for i in range(steps):
+            fns[i % len(fns)]()
+        e.record(self.stream)
+        torch.cuda.synchronize()
+        return s.elapsed_time(e) / steps
+
+    def warm(self, n):
+        import torch
+        for i in range(n):
+            self.plans[i % self.n_sets]()
+        for f in self.stage1 + self.stage2:
+            f()
+        torch.cuda.synchronize()
+
+    def soak(self, seconds):
+        """Untimed steps back to back for about `seconds` (the clock sampler runs meanwhile)."""
+        import torch
+        t0 = time.perf_counter()
+        i = 0
+        while time.perf_counter() - t0 < seconds:
+            for _ in range(64):
+                self.plans[i % self.n_sets]()
+                i += 1
+            torch.cuda.synchronize()
+        return i
+
+    def check_status(self):
+        bad = [int(pl.status.item()) for pl in self.plans if int(pl.status.item()) != 0]
+        if bad:
+            raise RuntimeError("device status %#x during the benchmark" % bad[0])
+
+    def entry(self, step_ms, s1, s2, pk, steps):
+        host = self.host
+        queries = host["batch"] * host["n_q"]
+        ab = algorithmic_bytes(host)
+        af = algorithmic_flops(host)
+        r2 = roofline_entry(STAGE_KERNELS["sparse_attend"], ab["stage2"], af["stage2"], s2, pk)
+        r1 = roofline_entry(STAGE_KERNELS["index_topk"], ab["stage1"], af["stage1"], s1, pk)
+        dominant = "sparse_attend" if s2 >= s1 else "index_topk"
+        roof = dict(r2 if dominant == "sparse_attend" else r1)
+        roof["traffic"] = recorded_traffic(dominant)
+        return {
+            "workload": self.wl.name, "metric": metric_name(self.wl), "value": queries / (step_ms / 1000.0),
+            "unit": "queries/s", "ms_per_step": step_ms, "steps": steps,
+            "config": config_of(self.wl, host, "inputs larger than L2: %d input set(s), %.0f MB of cache bytes "
+                                "read per step" % (self.n_sets, ab["total"] / 1e6)),
+            "achieved_hbm_gbs": ab["total"] / (step_ms / 1000.0) / 1e9,
+            "hbm_frac_of_measured": ab["total"] / (step_ms / 1000.0) / 1e9 / pk["hbm_gbs"],
+            "hbm_frac_of_8tbs": ab["total"] / (step_ms / 1000.0) / 1e9 / 8000.0,
+            "roofline": roof,
+            "stages": {"index_topk_ms": s1, "sparse_attend_ms": s2, "index_topk": r1, "sparse_attend": r2,
+                       "step_algorithmic_bytes": ab["total"], "step_tensor_flops": af["total"]},
+        }
 
 
 def main():
@@ -422,75 +620,28 @@ def main():
     wl = workloads.WORKLOADS[args.workload]
     if wl.number == 4:
         return run_prefill_scoring(args, rank, world, dev, wl)
-    host = workloads.make_inputs(wl, seed=1000 + wl.number + 7919 * rank)
-    # Several independent input sets, used round-robin: together they are far larger than the
-    # 126 MB L2, so every timed step reads its index keys and latent rows from HBM (no flush
-    # kernel between steps, whose dirty lines would be written back inside the next step).
-    n_sets = max(2, -(-4 * L2_BYTES // max(1, step_bytes(host))))
-    sets = [workloads.to_device(host, dev)]
-    for i in range(1, n_sets):
-        sets.append(workloads.to_device(workloads.make_inputs(wl, seed=1000 + wl.number + 7919 * rank + 104729 * i), dev))
-    plans = [sia.FusedDecodePlan(d, dev) for d in sets]
-    d, plan = sets[0], plans[0]
-    stream = torch.cuda.current_stream()
+    db = DecodeBench(sia, workloads, wl, rank, dev, min_sets=2)
+    host, d, plan = db.host, db.sets[0], db.plans[0]
+    db.warm(max(3, args.warmup))
 
-    def timed(fns, steps):
-        """Mean device time per call of fns[i % len(fns)], back to back, CUDA events."""
-        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s.record(stream)
-        for i in range(steps):
-            fns[i % len(fns)]()
-        e.record(stream)
-        torch.cuda.synchronize()
-        return s.elapsed_time(e) / steps
-
-    # warm-up
-    for i in range(max(3, args.warmup)):
-        plans[i % n_sets]()
-    torch.cuda.synchronize()
-
-    # stage-only calls (stage 1: indexer + Top-K; stage 2: sparse attention + merge) for the
-    # per-kernel roofline, on the same rotating input sets
-    import ctypes
-    lib = sia.load_library()
-    sp = ctypes.c_void_p(stream.cuda_stream)
-    stage1, stage2 = [], []
-    for pl in plans:
-        ws1 = torch.empty(max(256, lib.sia_index_workspace_size(ctypes.byref(pl.ia))), dtype=torch.uint8, device=dev)
-        ws2 = torch.empty(max(256, lib.sia_attend_workspace_size(ctypes.byref(pl.aa))), dtype=torch.uint8, device=dev)
-        st_ptr = ctypes.c_void_p(pl.status.data_ptr())
-
-        def f1(pl=pl, ws1=ws1, st_ptr=st_ptr):
-            sia._check(lib.sia_sparse_index_topk(ctypes.byref(pl.ia), ctypes.c_void_p(ws1.data_ptr()), ws1.numel(), st_ptr, sp))
-
-        def f2(pl=pl, ws2=ws2, st_ptr=st_ptr):
-            sia._check(lib.sia_sparse_mla_attend(ctypes.byref(pl.aa), ctypes.c_void_p(ws2.data_ptr()), ws2.numel(), st_ptr, sp))
-        stage1.append(f1)
-        stage2.append(f2)
-    for f in stage1 + stage2:
-        f()
-    torch.cuda.synchronize()
-
-    # ---------------- timed region
+    # ---------------- timed region (the clock sampler runs over a soak of the same steps right
+    # before it, so that its median rests on many samples under load, and over the region itself)
     sampler = ClockSampler(local)
     sampler.start()
-    time.sleep(0.25)
+    db.soak(args.soak_s)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     t_wall = time.perf_counter()
-    mean_ms = timed(plans, args.steps)
+    mean_ms = db.timed(db.plans, args.steps)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     wall = time.perf_counter() - t_wall
-    s1 = timed(stage1, args.steps)
-    s2 = timed(stage2, args.steps)
+    s1 = db.timed(db.stage1, args.steps)
+    s2 = db.timed(db.stage2, args.steps)
     clocks = sampler.stop()
-    bad = [int(pl.status.item()) for pl in plans if int(pl.status.item()) != 0]
-    if bad:
-        raise RuntimeError("device status %#x during the benchmark" % bad[0])
-
+    db.check_status()
     mean_ms, s1, s2 = max_over_ranks([mean_ms, s1, s2], dev)
 
     # ---------------- end-to-end through the C ABI with host buffers
@@ -513,12 +664,12 @@ def main():
     for _ in range(2):
         e2e_step()
     torch.cuda.synchronize()
-    serial_ms = timed([e2e_step], n_e2e)
+    serial_ms = db.timed([e2e_step], n_e2e)
     # The same calls as a serving loop issues them: two slots of per-step input and output
     # buffers, the host->device copies on one stream, the fused call on another, the
     # device->host copies on a third, so neighbouring steps' copies overlap the compute.
     try:
-        pipe_ms = e2e_pipelined(sia, d, plan, pin, dev, stream, n_e2e)
+        pipe_ms = e2e_pipelined(sia, d, plan, pin, dev, db.stream, n_e2e)
     except Exception as exc:  # reported below; the serial figure stands
         sys.stderr.write("pipelined end-to-end loop failed: %r\n" % (exc,))
         pipe_ms = float("inf")
@@ -527,41 +678,56 @@ def main():
     e2e_ms = pipe_ms if pipelined else serial_ms
 
     queries = host["batch"] * host["n_q"]
-    value = job_rate(world, queries, mean_ms)
-    ab = algorithmic_bytes(host)
     pk = peaks()
-    dominant = "sparse_attend" if s2 >= s1 else "index_topk"
-    dom_bytes, dom_ms = (ab["stage2"], s2) if dominant == "sparse_attend" else (ab["stage1"], s1)
-    achieved = dom_bytes / (dom_ms / 1000.0) / 1e9
-    step_gbs = ab["total"] / (mean_ms / 1000.0) / 1e9
-    kernels_per_step = 3 + (1 if plan_splits(lib, plan.aa) > 1 else 0)
-
+    head = db.entry(mean_ms, s1, s2, pk, args.steps)
     line = {
-        "metric": metric_name(wl), "value": value, "unit": "queries/s", "n_gpus": world,
+        "metric": head["metric"], "value": job_rate(world, queries, mean_ms), "unit": "queries/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": mean_ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": config_of(wl, host, "inputs larger than L2: %d independent input sets (%.0f MB) used round-robin" % (n_sets, n_sets * input_bytes(host) / 1e6)),
-        "achieved_hbm_gbs": step_gbs,
-        "hbm_frac_of_measured": step_gbs / pk["hbm_gbs"],
-        "hbm_frac_of_8tbs": step_gbs / 8000.0,
-        "roofline": {"bound": "hbm", "kernel": STAGE_KERNELS[dominant], "achieved": achieved, "peak": pk["hbm_gbs"],
-                     "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "peak_source": pk["source"],
-                     "traffic": recorded_traffic(dominant),
-                     "algorithmic_bytes_per_launch": dom_bytes, "ms_per_launch": dom_ms},
-        "stages": {"index_topk_ms": s1, "sparse_attend_ms": s2,
-                   "index_topk_gbs": ab["stage1"] / (s1 / 1000.0) / 1e9,
-                   "sparse_attend_gbs": ab["stage2"] / (s2 / 1000.0) / 1e9,
-                   "step_algorithmic_bytes": ab["total"]},
+        "config": config_of(wl, host, "inputs larger than L2: %d independent input sets (%.0f MB) used round-robin"
+                            % (db.n_sets, db.n_sets * input_bytes(host) / 1e6)),
+        "achieved_hbm_gbs": head["achieved_hbm_gbs"],
+        "hbm_frac_of_measured": head["hbm_frac_of_measured"],
+        "hbm_frac_of_8tbs": head["hbm_frac_of_8tbs"],
+        "roofline": head["roofline"],
+        "stages": head["stages"],
         "e2e": {"value": job_rate(world, queries, e2e_ms), "unit": "queries/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "loop": "pipelined: 2 buffer slots, copy-in / compute / copy-out streams" if pipelined
                         else "serial: copy-in, fused call, copy-out on one stream",
                 "serial_ms_per_step": serial_ms},
-        "gpu_launches": kernels_per_step * args.steps,
-        "clocks": clocks,
+        "gpu_launches": db.kernels_per_step * args.steps,
+        "clocks": dict(clocks, window="nvidia-smi every 200 ms over a %.1f s soak of the same steps "
+                                      "right before the timed region, the timed region and the "
+                                      "stage timings" % args.soak_s),
         "wall_s_timed_region": wall,
     }
+    # ---------------- the other configurations, in the same run (not part of the headline)
+    if not args.no_sub_workloads:
+        del db, d, plan, pin
+        torch.cuda.empty_cache()
+        subs = {}
+        for num in (3, 5):
+            w2 = workloads.WORKLOADS[num]
+            sb = DecodeBench(sia, workloads, w2, rank, dev, min_sets=1)
+            sb.warm(3)
+            n = max(10, min(args.steps, 200))
+            m = sb.timed(sb.plans, n)
+            a1 = sb.timed(sb.stage1, n)
+            a2 = sb.timed(sb.stage2, n)
+            sb.check_status()
+            m, a1, a2 = max_over_ranks([m, a1, a2], dev)
+            subs[w2.name] = sb.entry(m, a1, a2, pk, n)
+            line["gpu_launches"] += sb.kernels_per_step * n
+            del sb
+            torch.cuda.empty_cache()
+        w4 = workloads.WORKLOADS[4]
+        res = measure_prefill(dev, w4, rank, min(args.steps, 20), 3, full_path=True)
+        (res["_ms"],) = max_over_ranks([res["_ms"]], dev)
+        subs[w4.name] = prefill_entry(res, pk, w4)
+        line["gpu_launches"] += res["launches"]
+        line["workloads"] = subs
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
         n = max(4, min(16, oracle.num_threads()))

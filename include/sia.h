@@ -64,7 +64,8 @@ typedef enum {
 
 typedef enum {
     SIA_BF16 = 0,                 /* bfloat16                                                 */
-    SIA_FP8_E4M3 = 1              /* OCP FP8 E4M3 ("fn": no infinities), one byte per value   */
+    SIA_FP8_E4M3 = 1,             /* OCP FP8 E4M3 ("fn": no infinities), one byte per value   */
+    SIA_MXFP8 = 2                 /* E4M3 codes with one E8M0 scale per 32 elements (OCP MX)  */
 } sia_dtype;
 
 /*
@@ -75,6 +76,14 @@ typedef enum {
  * where k[s] is row (s % page_size) of page page_table[b][s / page_size] of k_cache, and
  * topk_out[b][j] receives the positions of the top_k largest I[s] (ties: lower s first) in
  * ascending order, padded with -1 when fewer than top_k positions are visible (p+1 < top_k).
+ *
+ * dtype SIA_MXFP8 (the pages' MXFP8 indexing path: "Rapid Adaptation and Inference
+ * Optimization", tiered quantisation table; "Day 0 Inference Adaptation and Performance
+ * Optimization for Hybrid Sparse Attention LLMs", section 5.1): q and k_cache hold E4M3 codes and
+ * every 32 consecutive elements of a q head vector or of a key share one E8M0 scale 2^(e - 127)
+ * (q_mx, k_mx; q_scale and k_scale must be NULL); elements are dequantised, then scored by the
+ * same formula.  head_dim must be 64 or 128.  Each query is scored on its own (the keys are
+ * read once per query token, so J = 2 reads them twice).
  */
 typedef struct {
     int32_t batch;              /* B >= 1                                                    */
@@ -97,6 +106,8 @@ typedef struct {
     int32_t* topk_out;          /* [B, J, K] int32 output                                    */
     float* scores_out;          /* NULL, or [B, J, max_pages_per_seq * P] fp32: receives I[s]
                                    for s <= p (other entries are left unwritten)             */
+    const uint8_t* q_mx;        /* SIA_MXFP8 only: E8M0 scale codes [B, J, H, D / 32]        */
+    const uint8_t* k_mx;        /* SIA_MXFP8 only: E8M0 scale codes [num_pages, P, D / 32]   */
 } sia_index_args;
 
 /*
@@ -107,7 +118,9 @@ typedef struct {
  *   out[b][j][h] = sum_s softmax(z)_s * c[s][0 : d_latent]     (bf16, fp32 accumulation),
  *   lse[b][j][h] = ln sum_s exp(z_s)                            (-inf if the list is empty)
  * over the positions s listed in topk[b][j] (valid entries first, -1 padding after them; the
- * list need not be sorted).
+ * list need not be sorted).  The main cache is bf16, or FP8 with block scales (kv_scale): "Rapid
+ * Adaptation and Inference Optimization", tiered quantisation table, and "Day 0 Inference
+ * Adaptation and Performance Optimization for Hybrid Sparse Attention LLMs", section 5.2.
  */
 typedef struct {
     int32_t batch;              /* B >= 1                                                    */
@@ -127,7 +140,61 @@ typedef struct {
     const int32_t* topk;        /* [B, J, K] int32                                           */
     void* out;                  /* bf16 [B, J, n_heads, d_latent] output                     */
     float* lse;                 /* NULL or fp32 [B, J, n_heads] output                       */
+    const float* kv_scale;      /* NULL: kv_cache is bf16.  Else kv_cache holds FP8 E4M3 codes
+                                   [num_pages, P, d_latent + d_rope] and kv_scale fp32
+                                   [num_pages, P, ceil((d_latent + d_rope) / 128)]: element d of
+                                   a row is its decoded code times the scale of block d / 128 of
+                                   that row (the pages' FP8 main cache, one scale per 128-element
+                                   block); it is rounded once to bf16 before the products     */
 } sia_attend_args;
+
+/*
+ * Paged cache append: the step before page-table translation.  Writes the J new tokens of every
+ * sequence into the index-K cache and the main latent cache, quantising on the way in when a
+ * cache is FP8 ("Day0 Inference Adaptation and Performance Optimization for a New
+ * Hybrid-Attention LLM Architecture", new cache structures kept in pages; "Rapid Adaptation and
+ * Inference Optimization", section IV.4.2, paged cache management; the formats are those of the
+ * pages' tiered quantisation table).  Token j of sequence b sits at position
+ * p = seq_lens[b] - n_q + j (seq_lens counts the new tokens) and goes to row p % page_size of
+ * page page_table[b][p / page_size] of both caches; no other row is written.
+ *   SIA_KEY_BF16      k_cache bf16 [num_pages, P, head_dim] (a copy), k_scale NULL;
+ *   SIA_KEY_FP8_POW2  k_cache e4m3 codes, k_scale fp32 [num_pages, P]: per token the smallest
+ *                     power of two s with max|x| <= 448 s (1 for an all-zero key), codes of x / s;
+ *   SIA_KEY_MXFP8     k_cache e4m3 codes, k_scale uint8 E8M0 [num_pages, P, head_dim / 32]: per
+ *                     group of 32 elements E = floor(log2 max|x|) - 8 clamped to [-127, 127],
+ *                     code E + 127 (127 for an all-zero group), codes of x / 2^E;
+ *   SIA_KV_BF16       kv_cache bf16 [num_pages, P, d_kv] (a copy), kv_scale NULL;
+ *   SIA_KV_FP8_BLOCK128  kv_cache e4m3 codes, kv_scale fp32 [num_pages, P, ceil(d_kv / 128)]:
+ *                     per 128-element block of the row s = fp32(max|x| / 448) (1 for an all-zero
+ *                     block), codes of fp32(x / s).
+ * e4m3 codes round to nearest, ties to even, and saturate at +-448.  A token whose position is
+ * outside [0, max_pages_per_seq * P) or whose page id is outside the pool is skipped and sets
+ * SIA_DEV_BAD_POSITION / SIA_DEV_BAD_PAGE.  No workspace.
+ */
+typedef enum { SIA_KEY_BF16 = 0, SIA_KEY_FP8_POW2 = 1, SIA_KEY_MXFP8 = 2 } sia_key_format;
+typedef enum { SIA_KV_BF16 = 0, SIA_KV_FP8_BLOCK128 = 1 } sia_kv_format;
+
+typedef struct {
+    int32_t batch;              /* B >= 1                                                    */
+    int32_t n_q;                /* new tokens per sequence J >= 1                            */
+    int32_t head_dim;           /* index key length: 32..256, a multiple of 32               */
+    int32_t d_kv;               /* main-cache row length (d_latent + d_rope): 16..1024, even */
+    int32_t page_size;          /* P >= 1                                                    */
+    int32_t max_pages_per_seq;
+    int32_t num_pages;          /* pages in each pool                                        */
+    sia_key_format key_format;
+    sia_kv_format kv_format;
+    const void* new_k;          /* bf16 [B, J, head_dim]                                     */
+    const void* new_kv;         /* bf16 [B, J, d_kv]                                         */
+    const int32_t* page_table;  /* [B, max_pages_per_seq]                                    */
+    const int32_t* seq_lens;    /* [B], including the J new tokens                          */
+    void* k_cache;              /* see key_format                                            */
+    void* k_scale;              /* see key_format                                            */
+    void* kv_cache;             /* see kv_format                                             */
+    float* kv_scale;            /* see kv_format                                             */
+} sia_append_args;
+
+sia_status sia_cache_append(const sia_append_args* a, int32_t* dev_status, void* stream);
 
 /* Workspace bytes a call needs (0 for a NULL argument).  The workspace is caller-owned device
  * memory, 256-byte aligned, whose contents need no initialisation and may be reused by the

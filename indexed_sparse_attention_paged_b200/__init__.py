@@ -27,7 +27,9 @@ HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "sia.h")
 
 SIA_OK, SIA_ERR_INVALID_ARGUMENT, SIA_ERR_UNSUPPORTED, SIA_ERR_CUDA, SIA_ERR_WORKSPACE = range(5)
 SIA_DEV_BAD_PAGE, SIA_DEV_BAD_POSITION, SIA_DEV_TIMEOUT, SIA_DEV_INTERNAL = 0x1, 0x2, 0x4, 0x8
-SIA_BF16, SIA_FP8_E4M3 = 0, 1
+SIA_BF16, SIA_FP8_E4M3, SIA_MXFP8 = 0, 1, 2
+SIA_KEY_BF16, SIA_KEY_FP8_POW2, SIA_KEY_MXFP8 = 0, 1, 2
+SIA_KV_BF16, SIA_KV_FP8_BLOCK128 = 0, 1
 
 
 class SiaError(RuntimeError):
@@ -45,7 +47,7 @@ class IndexArgs(ctypes.Structure):
                 ("k_cache", ctypes.c_void_p), ("k_scale", ctypes.c_void_p),
                 ("page_table", ctypes.c_void_p), ("seq_lens", ctypes.c_void_p),
                 ("q_pos", ctypes.c_void_p), ("topk_out", ctypes.c_void_p),
-                ("scores_out", ctypes.c_void_p)]
+                ("scores_out", ctypes.c_void_p), ("q_mx", ctypes.c_void_p), ("k_mx", ctypes.c_void_p)]
 
 
 class AttendArgs(ctypes.Structure):
@@ -56,7 +58,19 @@ class AttendArgs(ctypes.Structure):
                 ("softmax_scale", ctypes.c_float),
                 ("q", ctypes.c_void_p), ("kv_cache", ctypes.c_void_p),
                 ("page_table", ctypes.c_void_p), ("seq_lens", ctypes.c_void_p),
-                ("topk", ctypes.c_void_p), ("out", ctypes.c_void_p), ("lse", ctypes.c_void_p)]
+                ("topk", ctypes.c_void_p), ("out", ctypes.c_void_p), ("lse", ctypes.c_void_p),
+                ("kv_scale", ctypes.c_void_p)]
+
+
+class AppendArgs(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("n_q", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("d_kv", ctypes.c_int32), ("page_size", ctypes.c_int32),
+                ("max_pages_per_seq", ctypes.c_int32), ("num_pages", ctypes.c_int32),
+                ("key_format", ctypes.c_int32), ("kv_format", ctypes.c_int32),
+                ("new_k", ctypes.c_void_p), ("new_kv", ctypes.c_void_p),
+                ("page_table", ctypes.c_void_p), ("seq_lens", ctypes.c_void_p),
+                ("k_cache", ctypes.c_void_p), ("k_scale", ctypes.c_void_p),
+                ("kv_cache", ctypes.c_void_p), ("kv_scale", ctypes.c_void_p)]
 
 
 _lib = None
@@ -93,6 +107,8 @@ def load_library(path: str = LIB_PATH):
     lib.sia_status_string.argtypes = [ctypes.c_int]
     lib.sia_last_error.restype = ctypes.c_char_p
     lib.sia_version.restype = ctypes.c_int32
+    lib.sia_cache_append.restype = ctypes.c_int
+    lib.sia_cache_append.argtypes = [ctypes.POINTER(AppendArgs), P, P]
     lib.sia_set_wait_limit_ns.restype = ctypes.c_uint64
     lib.sia_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
     _lib = lib
@@ -146,8 +162,10 @@ def _need(t, name, dtype=None, dim=None, device=None):
 
 
 def index_args(q, w, k_cache, page_table, seq_lens, *, top_k, q_scale=None, k_scale=None,
-               q_pos=None, topk_out=None, scores_out=None) -> IndexArgs:
-    """Fill the stage-1 argument struct from tensors (see sia_index_args in include/sia.h)."""
+               q_pos=None, topk_out=None, scores_out=None, q_mx=None, k_mx=None) -> IndexArgs:
+    """Fill the stage-1 argument struct from tensors (see sia_index_args in include/sia.h).
+    With q_mx and k_mx (E8M0 codes, uint8 or float8_e8m0fnu, one per 32 elements) the e4m3 q and
+    k_cache are the MXFP8 index path."""
     _need(q, "q", (torch.bfloat16, torch.float8_e4m3fn), 4)
     dev = q.device
     B, J, H, D = q.shape
@@ -166,27 +184,43 @@ def index_args(q, w, k_cache, page_table, seq_lens, *, top_k, q_scale=None, k_sc
         _need(topk_out, "topk_out", torch.int32, 3, dev)
     if scores_out is not None:
         _need(scores_out, "scores_out", torch.float32, 3, dev)
+    mx = q_mx is not None or k_mx is not None
+    if mx:
+        if not fp8:
+            raise ValueError("the MXFP8 path takes e4m3 q and k_cache")
+        _need(q_mx, "q_mx", (torch.uint8, torch.float8_e8m0fnu), 4, dev)
+        _need(k_mx, "k_mx", (torch.uint8, torch.float8_e8m0fnu), 3, dev)
+        if tuple(q_mx.shape) != (B, J, H, D // 32) or tuple(k_mx.shape) != (k_cache.shape[0], k_cache.shape[1], D // 32):
+            raise ValueError("one E8M0 scale per 32 elements of q and of each key is expected")
     a = IndexArgs()
     a.batch, a.n_q, a.n_heads, a.head_dim = B, J, H, D
     a.page_size = k_cache.shape[1]
     a.max_pages_per_seq = page_table.shape[1]
     a.num_pages = k_cache.shape[0]
     a.top_k = int(top_k)
-    a.dtype = SIA_FP8_E4M3 if fp8 else SIA_BF16
+    a.dtype = SIA_MXFP8 if mx else (SIA_FP8_E4M3 if fp8 else SIA_BF16)
     a.q, a.q_scale, a.w = _ptr(q), _ptr(q_scale), _ptr(w)
     a.k_cache, a.k_scale = _ptr(k_cache), _ptr(k_scale)
     a.page_table, a.seq_lens, a.q_pos = _ptr(page_table), _ptr(seq_lens), _ptr(q_pos)
     a.topk_out, a.scores_out = _ptr(topk_out), _ptr(scores_out)
+    a.q_mx, a.k_mx = _ptr(q_mx), _ptr(k_mx)
     return a
 
 
 def attend_args(q, kv_cache, page_table, seq_lens, topk, *, d_latent, softmax_scale, out=None,
-                lse=None) -> AttendArgs:
-    """Fill the stage-2 argument struct from tensors (see sia_attend_args in include/sia.h)."""
+                lse=None, kv_scale=None) -> AttendArgs:
+    """Fill the stage-2 argument struct from tensors (see sia_attend_args in include/sia.h).
+    With kv_scale (fp32 [pages, P, ceil(DC/128)]) kv_cache holds FP8 E4M3 codes."""
     _need(q, "q", torch.bfloat16, 4)
     dev = q.device
     B, J, H, DC = q.shape
-    _need(kv_cache, "kv_cache", torch.bfloat16, 3, dev)
+    if kv_scale is None:
+        _need(kv_cache, "kv_cache", torch.bfloat16, 3, dev)
+    else:
+        _need(kv_cache, "kv_cache", (torch.float8_e4m3fn, torch.uint8), 3, dev)
+        _need(kv_scale, "kv_scale", torch.float32, 3, dev)
+        if tuple(kv_scale.shape) != (kv_cache.shape[0], kv_cache.shape[1], (DC + 127) // 128):
+            raise ValueError("kv_scale must be [num_pages, page_size, ceil(DC / 128)]")
     _need(page_table, "page_table", torch.int32, 2, dev)
     _need(seq_lens, "seq_lens", torch.int32, 1, dev)
     _need(topk, "topk", torch.int32, 3, dev)
@@ -205,6 +239,7 @@ def attend_args(q, kv_cache, page_table, seq_lens, topk, *, d_latent, softmax_sc
     a.q, a.kv_cache = _ptr(q), _ptr(kv_cache)
     a.page_table, a.seq_lens, a.topk = _ptr(page_table), _ptr(seq_lens), _ptr(topk)
     a.out, a.lse = _ptr(out), _ptr(lse)
+    a.kv_scale = _ptr(kv_scale)
     return a
 
 
@@ -224,14 +259,15 @@ def _ws_ptr(ws):
 
 def sparse_index_topk(q, w, k_cache, page_table, seq_lens, *, top_k, q_scale=None, k_scale=None,
                       q_pos=None, topk_out=None, scores_out=None, workspace=None, dev_status=None,
-                      stream=None):
+                      stream=None, q_mx=None, k_mx=None):
     """Stage 1: Top-K positions per query, int32 [B, J, top_k] (ascending, -1 padded)."""
     lib = load_library()
     B, J = q.shape[:2]
     if topk_out is None:
         topk_out = torch.empty((B, J, int(top_k)), dtype=torch.int32, device=q.device)
     a = index_args(q, w, k_cache, page_table, seq_lens, top_k=top_k, q_scale=q_scale,
-                   k_scale=k_scale, q_pos=q_pos, topk_out=topk_out, scores_out=scores_out)
+                   k_scale=k_scale, q_pos=q_pos, topk_out=topk_out, scores_out=scores_out,
+                   q_mx=q_mx, k_mx=k_mx)
     ws = _workspace(lib.sia_index_workspace_size(ctypes.byref(a)), q.device, workspace)
     wp, wn = _ws_ptr(ws)
     _check(lib.sia_sparse_index_topk(ctypes.byref(a), wp, wn, _ptr(dev_status), _stream_ptr(stream)))
@@ -239,12 +275,12 @@ def sparse_index_topk(q, w, k_cache, page_table, seq_lens, *, top_k, q_scale=Non
 
 
 def index_scores(q, w, k_cache, page_table, seq_lens, *, scores_out, q_scale=None, k_scale=None,
-                 q_pos=None, dev_status=None, stream=None):
+                 q_pos=None, dev_status=None, stream=None, q_mx=None, k_mx=None):
     """The scoring step alone: I[t, s] for every causal position into `scores_out`
     (fp32 [B, J, max_pages_per_seq * page_size]; positions past a query's own are untouched)."""
     lib = load_library()
     a = index_args(q, w, k_cache, page_table, seq_lens, top_k=1, q_scale=q_scale, k_scale=k_scale,
-                   q_pos=q_pos, topk_out=None, scores_out=scores_out)
+                   q_pos=q_pos, topk_out=None, scores_out=scores_out, q_mx=q_mx, k_mx=k_mx)
     _check(lib.sia_index_scores(ctypes.byref(a), _ptr(dev_status), _stream_ptr(stream)))
     return scores_out
 
@@ -261,18 +297,51 @@ def sparse_index_topk_noalloc(q, w, k_cache, page_table, seq_lens, *, top_k, top
 
 
 def sparse_mla_attend(q, kv_cache, page_table, seq_lens, topk, *, d_latent, softmax_scale,
-                      out=None, lse=None, workspace=None, dev_status=None, stream=None):
+                      out=None, lse=None, workspace=None, dev_status=None, stream=None, kv_scale=None):
     """Stage 2: bf16 [B, J, H, d_latent] attention output (and lse when given a buffer)."""
     lib = load_library()
     B, J, H, _ = q.shape
     if out is None:
         out = torch.empty((B, J, H, int(d_latent)), dtype=torch.bfloat16, device=q.device)
     a = attend_args(q, kv_cache, page_table, seq_lens, topk, d_latent=d_latent,
-                    softmax_scale=softmax_scale, out=out, lse=lse)
+                    softmax_scale=softmax_scale, out=out, lse=lse, kv_scale=kv_scale)
     ws = _workspace(lib.sia_attend_workspace_size(ctypes.byref(a)), q.device, workspace)
     wp, wn = _ws_ptr(ws)
     _check(lib.sia_sparse_mla_attend(ctypes.byref(a), wp, wn, _ptr(dev_status), _stream_ptr(stream)))
     return out
+
+
+def cache_append(new_k, new_kv, page_table, seq_lens, k_cache, kv_cache, *, key_format=SIA_KEY_BF16,
+                 kv_format=None, k_scale=None, kv_scale=None, dev_status=None, stream=None):
+    """Write the J new tokens of every sequence (bf16 new_k [B,J,D], new_kv [B,J,DC]) into the
+    paged caches in place, quantising as the formats say (see sia_cache_append in
+    include/sia.h).  kv_format defaults to FP8 when kv_scale is given, else bf16."""
+    lib = load_library()
+    _need(new_k, "new_k", torch.bfloat16, 3)
+    dev = new_k.device
+    _need(new_kv, "new_kv", torch.bfloat16, 3, dev)
+    _need(page_table, "page_table", torch.int32, 2, dev)
+    _need(seq_lens, "seq_lens", torch.int32, 1, dev)
+    key_dtype = torch.bfloat16 if key_format == SIA_KEY_BF16 else torch.float8_e4m3fn
+    _need(k_cache, "k_cache", (key_dtype, torch.uint8) if key_dtype != torch.bfloat16 else key_dtype, 3, dev)
+    if kv_format is None:
+        kv_format = SIA_KV_BF16 if kv_scale is None else SIA_KV_FP8_BLOCK128
+    kv_dtype = torch.bfloat16 if kv_format == SIA_KV_BF16 else (torch.float8_e4m3fn, torch.uint8)
+    _need(kv_cache, "kv_cache", kv_dtype, 3, dev)
+    if k_scale is not None:
+        _need(k_scale, "k_scale", torch.float32 if key_format == SIA_KEY_FP8_POW2 else
+              (torch.uint8, torch.float8_e8m0fnu), None, dev)
+    if kv_scale is not None:
+        _need(kv_scale, "kv_scale", torch.float32, 3, dev)
+    B, J, D = new_k.shape
+    a = AppendArgs()
+    a.batch, a.n_q, a.head_dim, a.d_kv = B, J, D, new_kv.shape[2]
+    a.page_size, a.max_pages_per_seq, a.num_pages = k_cache.shape[1], page_table.shape[1], k_cache.shape[0]
+    a.key_format, a.kv_format = int(key_format), int(kv_format)
+    a.new_k, a.new_kv = _ptr(new_k), _ptr(new_kv)
+    a.page_table, a.seq_lens = _ptr(page_table), _ptr(seq_lens)
+    a.k_cache, a.k_scale, a.kv_cache, a.kv_scale = _ptr(k_cache), _ptr(k_scale), _ptr(kv_cache), _ptr(kv_scale)
+    _check(lib.sia_cache_append(ctypes.byref(a), _ptr(dev_status), _stream_ptr(stream)))
 
 
 def fused_decode_workspace_size(ia: IndexArgs, aa: AttendArgs) -> int:
@@ -281,7 +350,8 @@ def fused_decode_workspace_size(ia: IndexArgs, aa: AttendArgs) -> int:
 
 def fused_decode(q_idx, w, k_cache, q_attn, kv_cache, page_table, seq_lens, *, top_k, d_latent,
                  softmax_scale, q_scale=None, k_scale=None, q_pos=None, topk_out=None, out=None,
-                 lse=None, workspace=None, dev_status=None, stream=None):
+                 lse=None, workspace=None, dev_status=None, stream=None, kv_scale=None, q_mx=None,
+                 k_mx=None):
     """Both stages in one call: returns (out bf16 [B,J,H,d_latent], topk int32 [B,J,K])."""
     lib = load_library()
     B, J = q_idx.shape[:2]
@@ -291,9 +361,9 @@ def fused_decode(q_idx, w, k_cache, q_attn, kv_cache, page_table, seq_lens, *, t
     if out is None:
         out = torch.empty((B, J, H, int(d_latent)), dtype=torch.bfloat16, device=q_idx.device)
     ia = index_args(q_idx, w, k_cache, page_table, seq_lens, top_k=top_k, q_scale=q_scale,
-                    k_scale=k_scale, q_pos=q_pos, topk_out=topk_out)
+                    k_scale=k_scale, q_pos=q_pos, topk_out=topk_out, q_mx=q_mx, k_mx=k_mx)
     aa = attend_args(q_attn, kv_cache, page_table, seq_lens, topk_out, d_latent=d_latent,
-                     softmax_scale=softmax_scale, out=out, lse=lse)
+                     softmax_scale=softmax_scale, out=out, lse=lse, kv_scale=kv_scale)
     ws = _workspace(lib.sia_workspace_size(ctypes.byref(ia), ctypes.byref(aa)), q_idx.device, workspace)
     wp, wn = _ws_ptr(ws)
     _check(lib.sia_fused_decode(ctypes.byref(ia), ctypes.byref(aa), wp, wn, _ptr(dev_status),
@@ -316,10 +386,12 @@ class FusedDecodePlan:
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
         self.ia = index_args(inputs["q_idx"], inputs["w"], inputs["k_cache"], inputs["page_table"],
                              inputs["seq_lens"], top_k=wl.top_k, k_scale=inputs["k_scale"],
-                             q_pos=inputs.get("q_pos"), topk_out=self.topk)
+                             q_pos=inputs.get("q_pos"), topk_out=self.topk, q_mx=inputs.get("q_mx"),
+                             k_mx=inputs.get("k_mx"))
         self.aa = attend_args(inputs["q_attn"], inputs["kv_cache"], inputs["page_table"],
                               inputs["seq_lens"], self.topk, d_latent=wl.d_latent,
-                              softmax_scale=wl.softmax_scale, out=self.out, lse=self.lse)
+                              softmax_scale=wl.softmax_scale, out=self.out, lse=self.lse,
+                              kv_scale=inputs.get("kv_scale"))
         lib = load_library()
         n = lib.sia_workspace_size(ctypes.byref(self.ia), ctypes.byref(self.aa))
         self.ws = torch.empty(max(n, 256), dtype=torch.uint8, device=device)

@@ -34,8 +34,8 @@
 namespace sia {
 namespace {
 
-// Per K stage: 16 bytes of chunk mask, then one fp32 key scale per tile row.
-constexpr uint32_t kStageInfoBytes = 16 + 4 * kIndexTileRows;
+// Per K stage (p.kinfo_bytes): 16 bytes of chunk mask, then the tile rows' key scales (one fp32
+// per row, or with MXFP8 keys one E8M0 byte per 32-element group of each row).
 
 struct IndexBarriers {
   uint64_t k_full[8];
@@ -142,10 +142,17 @@ __device__ void locate_start(const IndexKernelParams& p, IndexBarriers* sb) {
   }
 }
 
-// KBW (64 or 128 bytes per K-block row), NKB (K blocks per row) and FP8 are compile-time so
-// that the MMA issue loop is fully unrolled with constant descriptors: with runtime trip counts
-// each tcgen05.mma took about three times longer to issue.
-template <int NSUB, int KBW, int NKB, bool FP8>
+// KBW (64 or 128 bytes per K-block row), NKB (K blocks per row) and KIND (0 bf16, 1 FP8 E4M3,
+// 2 MXFP8) are compile-time so that the MMA issue loop is fully unrolled with constant
+// descriptors: with runtime trip counts each tcgen05.mma took about three times longer to issue.
+//
+// MXFP8 (one E8M0 scale per 32 elements of q and of each key, "Rapid Adaptation and Inference
+// Optimization", tiered quantisation table, and "Day 0 Inference Adaptation ... for Hybrid
+// Sparse Attention LLMs", section 5.1): one kind::f8f6f4 MMA step covers K = 32 elements, which
+// is exactly one scale group, so every group's partial dot products go to an accumulator of their
+// own, and the epilogue forms d = sum_g D_g * 2^(eq[h,g] + ek[s,g]) before the ReLU.  For
+// integer-valued codes and moderate exponents every term and partial sum is exact in fp32.
+template <int NSUB, int KBW, int NKB, int KIND>
 __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
     index_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
                        const IndexKernelParams p) {
@@ -154,6 +161,10 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   constexpr int kEpiThreads = 128 * NSUB;
+  constexpr bool FP8 = KIND != 0;
+  constexpr bool MX = KIND == 2;
+  constexpr int kGroups = NKB * KBW / 32;   // MX scale groups per row (one MMA K step each)
+  static_assert(!MX || NSUB == 1, "MXFP8 uses one query per group and one sub-block");
 
   if ((smem_u32(smem) & 1023u) != 0) {  // the swizzled layouts need a 1024-byte aligned base
     pdl_wait_primary();
@@ -236,8 +247,10 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
         const bool page_ok = my_page >= 0 && my_page < p.num_pages;
         if (in_range && !page_ok) report(p.status, SIA_DEV_BAD_PAGE);
         const uint32_t valid_mask = __ballot_sync(0xffffffffu, in_range && page_ok);
-        uint8_t* info = smem + p.off_kinfo + stage * kStageInfoBytes;
-        const uint32_t scale_bytes = p.k_scale ? (uint32_t)p.box_rows * 4u : 0u;
+        uint8_t* info = smem + p.off_kinfo + stage * p.kinfo_bytes;
+        const uint32_t row_scale_bytes = MX ? (uint32_t)kGroups : 4u;
+        const void* kscale_src = MX ? static_cast<const void*>(p.k_mx) : static_cast<const void*>(p.k_scale);
+        const uint32_t scale_bytes = kscale_src ? (uint32_t)p.box_rows * row_scale_bytes : 0u;
         if (lane == 0) {
           // per-stage info read by the epilogue: which chunks hold real pages, and (FP8) the
           // per-token key scales of the tile, copied next to the K tile
@@ -255,8 +268,9 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
           for (int kb = 0; kb < NKB; ++kb)
             tma_load_2d_hint(kst + kb * p.k_kblock_bytes + lane * p.box_rows * KBW, &kmap,
                              &sb->k_full[stage], kb * KBW / (FP8 ? 1 : 2), y, stream_policy);
-          if (p.k_scale)
-            bulk_load(info + 16 + lane * p.box_rows * 4, p.k_scale + (long long)y, scale_bytes,
+          if (kscale_src)
+            bulk_load(info + 16 + lane * p.box_rows * row_scale_bytes,
+                      static_cast<const uint8_t*>(kscale_src) + (long long)y * row_scale_bytes, scale_bytes,
                       &sb->k_full[stage]);
         }
         __syncwarp();
@@ -304,7 +318,7 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
             for (int sub = 0; sub < NSUB; ++sub) {
               if (!mbar_wait(&sb->acc_empty[as][sub], aph ^ 1u, wc)) { ok = false; break; }
               tc_fence_after();
-              const uint32_t d_tmem = tmem_base + (uint32_t)((as * NSUB + sub) * p.n_cols);
+              const uint32_t d_tmem = tmem_base + (uint32_t)((as * NSUB + sub) * p.acc_cols);
               const uint32_t b_base = smem_u32(smem + p.off_q + sub * p.q_sub_bytes);
               const uint32_t q_kblock = p.q_kblock_bytes;
 #pragma unroll
@@ -313,7 +327,8 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
                 for (int ks = 0; ks < KBW / 32; ++ks) {
                   const uint64_t ad = umma_smem_desc(a_base + kb * a_kblock + ks * 32, 16, sbo, layout);
                   const uint64_t bd = umma_smem_desc(b_base + kb * q_kblock + ks * 32, 16, sbo, layout);
-                  if (FP8) umma_f8(d_tmem, ad, bd, idesc, (kb | ks) != 0);
+                  if (MX) umma_f8(d_tmem + (uint32_t)((kb * (KBW / 32) + ks) * p.n_cols), ad, bd, idesc, false);
+                  else if (FP8) umma_f8(d_tmem, ad, bd, idesc, (kb | ks) != 0);
                   else umma_f16(d_tmem, ad, bd, idesc, (kb | ks) != 0);
                 }
               umma_commit(&sb->acc_full[as][sub]);
@@ -354,6 +369,8 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
         float* w_s = reinterpret_cast<float*>(smem + p.off_w) + (seg & 1) * w_words;
         int* info_pos = reinterpret_cast<int*>(smem + p.off_info) + (seg & 1) * 16;
         float* info_qs = reinterpret_cast<float*>(smem + p.off_info + 128) + (seg & 1) * 16;
+        // MXFP8: the query's group scales 2^(e - 127) as fp32, [head][group]
+        float* qmx_s = reinterpret_cast<float*>(smem + p.off_qmx) + (seg & 1) * (p.HP * kGroups);
         if (et == 0) {
           // q of the group: one 3-D TMA box (nq_sub queries x HP heads x one K block, heads
           // past H and queries past the batch zero-filled) per (sub-block, K block)
@@ -370,6 +387,15 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
           const int ql = i / p.HP, h = i - ql * p.HP;
           const int j = gi.g * p.qg + ql;
           w_s[i] = (j < p.J && h < p.H) ? p.w[((long long)gi.b * p.J + j) * p.H + h] : 0.0f;
+        }
+        if (MX) {
+          const int j = gi.g;   // one query per group
+          for (int i = et; i < p.HP * kGroups; i += kEpiThreads) {
+            const int h = i / kGroups;
+            const uint32_t code = h < p.H ? p.q_mx[(((long long)gi.b * p.J + j) * p.H + h) * kGroups + i % kGroups] : 127u;
+            // E8M0: 2^(code - 127); code 0 is 2^-127 (a subnormal fp32), 0xFF NaN
+            qmx_s[i] = code == 0xFFu ? __int_as_float(0x7fc00000) : ldexpf(1.0f, (int)code - 127);
+          }
         }
         if (et < p.qg) {
           const int j = gi.g * p.qg + et;
@@ -390,14 +416,47 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
           // landed, and waiting on k_full makes the scales and the chunk mask visible here
           if (!mbar_wait_warp(&sb->k_full[kstage], (uint32_t)(acc_it / p.k_stages) & 1u, wc)) { ok = false; break; }
           tc_fence_after();
-          const uint8_t* info = smem + p.off_kinfo + kstage * kStageInfoBytes;
+          const uint8_t* info = smem + p.off_kinfo + kstage * p.kinfo_bytes;
           // a position whose page id is outside the pool is ranked last (-inf)
           float ks = 1.0f;
-          if (!((*reinterpret_cast<const uint32_t*>(info) >> (row / p.box_rows)) & 1u))
+          const bool page_ok = (*reinterpret_cast<const uint32_t*>(info) >> (row / p.box_rows)) & 1u;
+          if (!page_ok)
             ks = __int_as_float(0xff800000);
-          else if (p.k_scale)
+          else if (!MX && p.k_scale)
             ks = reinterpret_cast<const float*>(info + 16)[row];
-          const uint32_t col0 = (uint32_t)((as * NSUB + sub) * p.n_cols);
+          const uint32_t col0 = (uint32_t)((as * NSUB + sub) * p.acc_cols);
+          if constexpr (MX) {
+            // this position's key group scales, then per 16-head chunk all groups' partial dot
+            // products in one TMEM wait: d_h = sum_g D_g[h] * sq[h][g] * sk[g]
+            float sk[kGroups];
+#pragma unroll
+            for (int g = 0; g < kGroups; ++g) {
+              const uint32_t code = page_ok ? info[16 + row * kGroups + g] : 127u;
+              sk[g] = code == 0xFFu ? __int_as_float(0x7fc00000) : ldexpf(1.0f, (int)code - 127);
+            }
+            const float* wq = w_s;
+            float a4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            for (int hc = 0; hc < 4; ++hc) {
+              if (hc * 16 >= p.H) break;   // warp-uniform
+              uint32_t v[kGroups][16];
+#pragma unroll
+              for (int g = 0; g < kGroups; ++g)
+                tmem_ld16(tmem_addr(tmem_base, quad * 32, col0 + g * p.n_cols + hc * 16), v[g]);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const int h = hc * 16 + i;
+                const float* sq = qmx_s + h * kGroups;
+                float d = 0.0f;
+#pragma unroll
+                for (int g = 0; g < kGroups; ++g) d = fmaf(__uint_as_float(v[g][i]), sq[g] * sk[g], d);
+                a4[i & 3] = fmaf(wq[h], fmaxf(d, 0.0f), a4[i & 3]);
+              }
+            }
+            const float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+            const int pos = info_pos[0];
+            if (s <= pos) p.scores[(out_row0 + gi.g) * p.Lpad + s] = isinf(ks) ? ks : acc;
+          } else {
           // QB queries' columns (up to QB x 64 heads) per TMEM wait: the loads of a batch are in
           // flight together, so each tile pays the TMEM latency once per batch (QB = 1 with two
           // sub-blocks, to stay within the registers of 320 threads)
@@ -438,6 +497,7 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
                 p.scores[(out_row0 + j) * p.Lpad + s] = val;
               }
             }
+          }
           }
           tc_fence_before();
           mbar_arrive(&sb->acc_empty[as][sub]);
@@ -488,8 +548,14 @@ cudaError_t launch_index_score(const IndexKernelParams& p, const CUtensorMap& km
   // (K-block width, K blocks) from the row size: 64 B -> (64, 1), 128 B -> (128, 1), 256 B -> (128, 2)
   const int shape = p.kbw == 64 ? 0 : (p.n_kblocks == 1 ? 1 : 2);
 #define SIA_INDEX_CASE(NS, SH, KB, NK)                                                            \
-  if (p.n_sub == NS && shape == SH) return p.fp8 ? go(index_score_kernel<NS, KB, NK, true>)      \
-                                                 : go(index_score_kernel<NS, KB, NK, false>);
+  if (p.n_sub == NS && shape == SH) return p.fp8 ? go(index_score_kernel<NS, KB, NK, 1>)         \
+                                                 : go(index_score_kernel<NS, KB, NK, 0>);
+  if (p.mx) {
+    if (p.n_sub != 1) return cudaErrorInvalidValue;
+    if (shape == 0) return go(index_score_kernel<1, 64, 1, 2>);
+    if (shape == 1) return go(index_score_kernel<1, 128, 1, 2>);
+    return cudaErrorInvalidValue;   // at most four groups (128 elements) per row
+  }
   SIA_INDEX_CASE(1, 0, 64, 1)
   SIA_INDEX_CASE(1, 1, 128, 1)
   SIA_INDEX_CASE(1, 2, 128, 2)

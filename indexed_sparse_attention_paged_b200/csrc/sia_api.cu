@@ -124,8 +124,17 @@ sia_status check_index(const sia_index_args* a, bool with_topk) {
     return fail(SIA_ERR_INVALID_ARGUMENT, "batch, n_q, top_k, max_pages_per_seq and num_pages must be >= 1");
   if (!a->q || !a->w || !a->k_cache || !a->page_table || !a->seq_lens || (with_topk && !a->topk_out))
     return fail(SIA_ERR_INVALID_ARGUMENT, "q, w, k_cache, page_table, seq_lens and topk_out must be set");
-  if (a->dtype != SIA_BF16 && a->dtype != SIA_FP8_E4M3) return fail(SIA_ERR_UNSUPPORTED, "unknown dtype %d", (int)a->dtype);
+  if (a->dtype != SIA_BF16 && a->dtype != SIA_FP8_E4M3 && a->dtype != SIA_MXFP8)
+    return fail(SIA_ERR_UNSUPPORTED, "unknown dtype %d", (int)a->dtype);
   if (a->n_heads < 1 || a->n_heads > 64) return fail(SIA_ERR_UNSUPPORTED, "n_heads must be 1..64 (got %d)", a->n_heads);
+  if (a->dtype == SIA_MXFP8) {
+    if (!a->q_mx || !a->k_mx) return fail(SIA_ERR_INVALID_ARGUMENT, "MXFP8 needs q_mx and k_mx");
+    if (a->q_scale || a->k_scale) return fail(SIA_ERR_INVALID_ARGUMENT, "MXFP8 takes no q_scale or k_scale");
+    if (a->head_dim != 64 && a->head_dim != 128)
+      return fail(SIA_ERR_UNSUPPORTED, "MXFP8 head_dim must be 64 or 128 (got %d)", a->head_dim);
+  } else if (a->q_mx || a->k_mx) {
+    return fail(SIA_ERR_INVALID_ARGUMENT, "q_mx and k_mx are only for SIA_MXFP8");
+  }
   const int eb = a->dtype == SIA_BF16 ? 2 : 1;
   const int db = a->head_dim * eb;
   if (a->head_dim < 1 || (db != 64 && db != 128 && db != 256))
@@ -133,7 +142,8 @@ sia_status check_index(const sia_index_args* a, bool with_topk) {
   if (!pow2(a->page_size) || a->page_size < 8 || a->page_size > 4096)
     return fail(SIA_ERR_UNSUPPORTED, "page_size must be a power of two in [8, 4096] (got %d)", a->page_size);
   if (!aligned(a->q, 16) || !aligned(a->k_cache, 16) || !aligned(a->w, 4) || !aligned(a->topk_out, 4) ||
-      (a->scores_out && !aligned(a->scores_out, 16)) || (a->k_scale && !aligned(a->k_scale, 16)))
+      (a->scores_out && !aligned(a->scores_out, 16)) || (a->k_scale && !aligned(a->k_scale, 16)) ||
+      (a->k_mx && !aligned(a->k_mx, 16)))
     return fail(SIA_ERR_INVALID_ARGUMENT, "q, k_cache, k_scale and scores_out must be 16-byte aligned, other arrays 4-byte aligned");
   const long long lpad = (long long)a->max_pages_per_seq * a->page_size;
   if (lpad > (1ll << 30)) return fail(SIA_ERR_UNSUPPORTED, "max_pages_per_seq * page_size too large");
@@ -148,6 +158,7 @@ sia_status plan_index(const sia_index_args* a, IndexPlan* pl, bool make_maps, bo
   IndexKernelParams& k = pl->kp;
   memset(&k, 0, sizeof k);
   const int eb = a->dtype == SIA_BF16 ? 2 : 1;
+  const bool mx = a->dtype == SIA_MXFP8;
   k.B = a->batch;
   k.J = a->n_q;
   k.H = a->n_heads;
@@ -160,16 +171,20 @@ sia_status plan_index(const sia_index_args* a, IndexPlan* pl, bool make_maps, bo
   k.kbw = k.d_bytes >= 128 ? 128 : 64;
   k.n_kblocks = k.d_bytes / k.kbw;
   k.ksteps_per_block = k.kbw / 32;
-  k.fp8 = a->dtype == SIA_FP8_E4M3;
+  k.fp8 = a->dtype != SIA_BF16;
+  k.mx = mx ? 1 : 0;
+  k.n_groups = mx ? a->head_dim / 32 : 1;
   // queries sharing one A tile: up to 128 accumulator columns per MMA and two MMAs per tile
   // for a prefill chunk, so that two accumulator stages fit in TMEM (the MMA of the next tile
   // overlaps the epilogue of this one)
-  k.nq_sub = std::max(1, std::min(a->n_q, 128 / k.HP));
-  k.n_sub = (a->n_q > k.nq_sub) ? 2 : 1;
+  // (MXFP8: one query per group; its per-scale-group accumulators take n_groups x the columns)
+  k.nq_sub = mx ? 1 : std::max(1, std::min(a->n_q, 128 / k.HP));
+  k.n_sub = (!mx && a->n_q > k.nq_sub) ? 2 : 1;
   k.qg = k.nq_sub * k.n_sub;
   k.n_cols = k.nq_sub * k.HP;
+  k.acc_cols = k.n_cols * k.n_groups;
   k.groups_per_seq = (a->n_q + k.qg - 1) / k.qg;
-  const int cols_per_stage = k.n_sub * k.n_cols;
+  const int cols_per_stage = k.n_sub * k.acc_cols;
   k.acc_stages = (2 * cols_per_stage <= 512) ? 2 : 1;
   uint32_t cols = (uint32_t)(k.acc_stages * cols_per_stage);
   uint32_t alloc = 32;
@@ -185,8 +200,10 @@ sia_status plan_index(const sia_index_args* a, IndexPlan* pl, bool make_maps, bo
   const uint32_t w_bytes = (uint32_t)round_up((size_t)2 * k.qg * k.HP * 4, 16);  // double-buffered
   const uint32_t info_bytes = 256;
   const uint32_t bar_bytes = 256;
-  const uint32_t kinfo_bytes = 16 + 4 * kIndexTileRows;  // per stage: chunk mask + key scales
-  const uint32_t fixed = q_bytes + w_bytes + info_bytes + bar_bytes;
+  // per stage: chunk mask + key scales (fp32 per row, or one E8M0 byte per group of each row)
+  const uint32_t kinfo_bytes = (uint32_t)round_up(16 + (mx ? k.n_groups : 4) * kIndexTileRows, 16);
+  const uint32_t qmx_bytes = mx ? (uint32_t)round_up((size_t)2 * k.HP * k.n_groups * 4, 16) : 0u;
+  const uint32_t fixed = q_bytes + w_bytes + info_bytes + qmx_bytes + bar_bytes;
   const int limit = max_smem_optin();
   int stages = (int)((limit - (int)fixed) / (int)(k.k_stage_bytes + kinfo_bytes));
   stages = std::min(stages, 8);
@@ -197,12 +214,16 @@ sia_status plan_index(const sia_index_args* a, IndexPlan* pl, bool make_maps, bo
   k.off_w = k.off_q + q_bytes;
   k.off_info = k.off_w + w_bytes;
   k.off_kinfo = k.off_info + info_bytes;
-  k.off_bar = k.off_kinfo + kinfo_bytes * stages;
+  k.kinfo_bytes = kinfo_bytes;
+  k.off_qmx = k.off_kinfo + kinfo_bytes * stages;
+  k.off_bar = k.off_qmx + qmx_bytes;
   k.smem_bytes = k.off_bar + bar_bytes;
   k.q = static_cast<const uint8_t*>(a->q);
   k.q_scale = a->q_scale;
   k.w = a->w;
   k.k_scale = a->k_scale;
+  k.q_mx = a->q_mx;
+  k.k_mx = a->k_mx;
   k.page_table = a->page_table;
   k.seq_lens = a->seq_lens;
   k.q_pos = a->q_pos;
@@ -286,7 +307,7 @@ sia_status check_attend(const sia_attend_args* a) {
     return fail(SIA_ERR_UNSUPPORTED, "top_k must be <= %d (got %d)", 8 * kAttnMaxSplitRows, a->top_k);
   if (!std::isfinite(a->softmax_scale)) return fail(SIA_ERR_INVALID_ARGUMENT, "softmax_scale must be finite");
   if (!aligned(a->q, 16) || !aligned(a->kv_cache, 16) || !aligned(a->out, 16) || !aligned(a->topk, 4) ||
-      (a->lse && !aligned(a->lse, 4)))
+      (a->lse && !aligned(a->lse, 4)) || (a->kv_scale && !aligned(a->kv_scale, 4)))
     return fail(SIA_ERR_INVALID_ARGUMENT, "q, kv_cache and out must be 16-byte aligned");
   if ((long long)a->num_pages * a->page_size > (1ll << 31) - 1)
     return fail(SIA_ERR_UNSUPPORTED, "num_pages * page_size must fit in int32");
@@ -330,6 +351,9 @@ sia_status plan_attend(const sia_attend_args* a, AttendPlan* pl, bool make_maps)
   k.units = (int)(bj * best_s);
   k.q = a->q;
   k.kv = a->kv_cache;
+  k.kv_scale = a->kv_scale;
+  k.kv_fp8 = a->kv_scale ? 1 : 0;
+  k.nblk = (a->d_latent + a->d_rope + 127) / 128;
   k.page_table = a->page_table;
   k.seq_lens = a->seq_lens;
   k.topk = a->topk;
@@ -474,6 +498,57 @@ sia_status sia_fused_decode(const sia_index_args* ia, const sia_attend_args* aa,
   if (st != SIA_OK) return st;
   void* ws2 = ap.ws_part ? static_cast<uint8_t*>(workspace) + round_up(ip.ws_scores, 256) : nullptr;
   return run_attend(&ap, ws2, ap.ws_part, dev_status, s, true);
+}
+
+sia_status sia_cache_append(const sia_append_args* a, int32_t* dev_status, void* stream) {
+  g_last_error[0] = 0;
+  if (!a) return fail(SIA_ERR_INVALID_ARGUMENT, "append args are NULL");
+  if (a->batch < 1 || a->n_q < 1 || a->page_size < 1 || a->max_pages_per_seq < 1 || a->num_pages < 1)
+    return fail(SIA_ERR_INVALID_ARGUMENT, "batch, n_q, page_size, max_pages_per_seq and num_pages must be >= 1");
+  if (!a->new_k || !a->new_kv || !a->page_table || !a->seq_lens || !a->k_cache || !a->kv_cache)
+    return fail(SIA_ERR_INVALID_ARGUMENT, "new_k, new_kv, page_table, seq_lens, k_cache and kv_cache must be set");
+  if (a->key_format != SIA_KEY_BF16 && a->key_format != SIA_KEY_FP8_POW2 && a->key_format != SIA_KEY_MXFP8)
+    return fail(SIA_ERR_UNSUPPORTED, "unknown key format %d", (int)a->key_format);
+  if (a->kv_format != SIA_KV_BF16 && a->kv_format != SIA_KV_FP8_BLOCK128)
+    return fail(SIA_ERR_UNSUPPORTED, "unknown kv format %d", (int)a->kv_format);
+  if (a->head_dim < 32 || a->head_dim > 256 || a->head_dim % 32)
+    return fail(SIA_ERR_UNSUPPORTED, "head_dim must be a multiple of 32 in [32, 256] (got %d)", a->head_dim);
+  if (a->d_kv < 16 || a->d_kv > 1024 || a->d_kv % 2)
+    return fail(SIA_ERR_UNSUPPORTED, "d_kv must be even and in [16, 1024] (got %d)", a->d_kv);
+  if ((a->key_format != SIA_KEY_BF16) != (a->k_scale != nullptr))
+    return fail(SIA_ERR_INVALID_ARGUMENT, "k_scale must be set exactly when the key format is quantised");
+  if ((a->kv_format != SIA_KV_BF16) != (a->kv_scale != nullptr))
+    return fail(SIA_ERR_INVALID_ARGUMENT, "kv_scale must be set exactly when the kv format is FP8");
+  if (!aligned(a->new_k, 2) || !aligned(a->new_kv, 2) || !aligned(a->k_cache, 2) || !aligned(a->kv_cache, 2) ||
+      (a->k_scale && a->key_format == SIA_KEY_FP8_POW2 && !aligned(a->k_scale, 4)) ||
+      (a->kv_scale && !aligned(a->kv_scale, 4)) || !aligned(a->page_table, 4) || !aligned(a->seq_lens, 4))
+    return fail(SIA_ERR_INVALID_ARGUMENT, "misaligned pointer");
+  if ((long long)a->num_pages * a->page_size > (1ll << 31) - 1)
+    return fail(SIA_ERR_UNSUPPORTED, "num_pages * page_size must fit in int32");
+  if ((long long)a->batch * a->n_q > 0x7fffffffll) return fail(SIA_ERR_UNSUPPORTED, "too many tokens");
+  AppendKernelParams k;
+  memset(&k, 0, sizeof k);
+  k.B = a->batch;
+  k.J = a->n_q;
+  k.D = a->head_dim;
+  k.DC = a->d_kv;
+  k.P = a->page_size;
+  k.max_pages = a->max_pages_per_seq;
+  k.num_pages = a->num_pages;
+  k.key_format = (int)a->key_format;
+  k.kv_format = (int)a->kv_format;
+  k.new_k = a->new_k;
+  k.new_kv = a->new_kv;
+  k.page_table = a->page_table;
+  k.seq_lens = a->seq_lens;
+  k.k_cache = a->k_cache;
+  k.k_scale = a->k_scale;
+  k.kv_cache = a->kv_cache;
+  k.kv_scale = a->kv_scale;
+  k.status = dev_status;
+  cudaError_t e = launch_cache_append(k, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cache append launch");
+  return SIA_OK;
 }
 
 const char* sia_status_string(sia_status s) {

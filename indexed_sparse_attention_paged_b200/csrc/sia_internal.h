@@ -30,11 +30,14 @@ struct IndexKernelParams {
   int kbw;                    // bytes per K block row (128 or 64)
   int n_kblocks;              // d_bytes / kbw
   int ksteps_per_block;       // kbw / 32
-  int fp8;
+  int fp8;                    // e4m3 codes (per-token scales, or MXFP8 when mx)
+  int mx;                     // MXFP8: one E8M0 scale per 32 elements of q and of each key
+  int n_groups;               // MX scale groups per row (head_dim / 32)
   int nq_sub;                 // queries per accumulator sub-block
   int n_sub;                  // accumulator sub-blocks per A tile (1 or 2)
   int qg;                     // queries per group = nq_sub * n_sub
   int n_cols;                 // N of one MMA = nq_sub * HP
+  int acc_cols;               // TMEM columns of one accumulator: n_cols, or n_groups * n_cols (MX)
   int groups_per_seq;         // ceil(J / qg)
   int acc_stages;             // accumulator stages in TMEM
   int k_stages;               // K-tile stages in shared memory
@@ -43,11 +46,14 @@ struct IndexKernelParams {
   // shared-memory layout, byte offsets from the 1024-aligned base
   uint32_t off_k, k_stage_bytes, k_kblock_bytes;
   uint32_t off_q, q_sub_bytes, q_kblock_bytes;
-  uint32_t off_w, off_info, off_kinfo, off_bar, smem_bytes;
+  uint32_t off_w, off_info, off_kinfo, off_qmx, off_bar, smem_bytes;
+  uint32_t kinfo_bytes;       // per K stage: chunk mask + the rows' key scales
   const uint8_t* q;
   const float* q_scale;
   const float* w;
   const float* k_scale;
+  const uint8_t* q_mx;        // MX: E8M0 [B, J, H, n_groups]
+  const uint8_t* k_mx;        // MX: E8M0 [num_pages * P, n_groups]
   const int32_t* page_table;
   const int32_t* seq_lens;
   const int32_t* q_pos;
@@ -77,7 +83,10 @@ struct AttnKernelParams {
   int rows_per_split;         // multiple of kAttnTileRows
   int units;                  // B * J * splits
   const void* q;              // bf16 [B*J, H, DL + DR]
-  const void* kv;             // bf16 [num_pages * P, DL + DR]
+  const void* kv;             // bf16 [num_pages * P, DL + DR], or e4m3 codes when kv_fp8
+  const float* kv_scale;      // kv_fp8: fp32 [num_pages * P, nblk], one per 128-element block
+  int kv_fp8;
+  int nblk;                   // ceil((DL + DR) / 128)
   const int32_t* page_table;
   const int32_t* seq_lens;
   const int32_t* topk;
@@ -97,6 +106,22 @@ struct CombineKernelParams {
   float* lse;
 };
 
+// -------------------------------------------------------------------------- paged cache append
+struct AppendKernelParams {
+  int B, J, D, DC, P, max_pages, num_pages;
+  int key_format;             // sia_key_format
+  int kv_format;              // sia_kv_format
+  const void* new_k;          // bf16 [B*J, D]
+  const void* new_kv;         // bf16 [B*J, DC]
+  const int32_t* page_table;
+  const int32_t* seq_lens;
+  void* k_cache;
+  void* k_scale;
+  void* kv_cache;
+  float* kv_scale;
+  int32_t* status;
+};
+
 // Launchers (each returns cudaSuccess or the launch error).  `pdl` asks for programmatic
 // dependent launch on the previous kernel of the stream.
 cudaError_t launch_index_score(const IndexKernelParams& p, const CUtensorMap& kmap, const CUtensorMap& qmap, int grid,
@@ -106,6 +131,7 @@ cudaError_t launch_topk(const TopkKernelParams& p, bool pdl, cudaStream_t stream
 cudaError_t launch_sparse_attend(const AttnKernelParams& p, const CUtensorMap& q_rope,
                                  int n_clusters, bool pdl, cudaStream_t stream);
 cudaError_t launch_combine(const CombineKernelParams& p, bool pdl, cudaStream_t stream);
+cudaError_t launch_cache_append(const AppendKernelParams& p, cudaStream_t stream);
 
 // Shared memory the attention kernel needs for (d_latent, d_rope).
 size_t attend_smem_bytes(int dl, int dr);

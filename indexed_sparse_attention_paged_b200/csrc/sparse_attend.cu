@@ -89,6 +89,14 @@ struct AttnLayout<512, 64> {
     return k < 32 ? (uint32_t)(k >> 3) * (kAttnTileRows * 128) + swizzled_offset(row, (k & 7) * 16, 128)
                   : swizzled_offset(row, (k - 32) * 16, 64);
   }
+  // FP8 main cache (one byte per element, one fp32 scale per 128-element block of the row):
+  // CTA r's 16-element code pieces are 16 latent ones from element 256 r and 2 rope ones from
+  // element 512 + 32 r; its scales are those of blocks 2r, 2r+1 (latent) and 4 (rope)
+  static constexpr int kLatPieces8 = 16, kMaxRopePieces8 = 2, kScalesPerRow = 3, kRopeCodeBytes = 32;
+  __device__ static int rope_pieces8(int) { return 2; }
+  __device__ static int piece_src8(int r, int k) { return k < 16 ? 256 * r + 16 * k : 512 + 32 * r + 16 * (k - 16); }
+  __device__ static int piece_scale8(int k) { return k < 16 ? k >> 3 : 2; }
+  __device__ static int scale_blk8(int r, int which) { return which < 2 ? 2 * r + which : 4; }
 };
 
 template <>
@@ -107,6 +115,13 @@ struct AttnLayout<64, 16> {
   __device__ static uint32_t chunk_dst(int row, int k) {
     return k < 4 ? swizzled_offset(row, k * 16, 64) : swizzled_offset(row, (k - 4) * 16, 32);
   }
+  // FP8 main cache: 2 latent code pieces from element 32 r, and CTA 0's one rope piece (element
+  // 64); the 80-element row is one scale block
+  static constexpr int kLatPieces8 = 2, kMaxRopePieces8 = 1, kScalesPerRow = 1, kRopeCodeBytes = 16;
+  __device__ static int rope_pieces8(int r) { return r == 0 ? 1 : 0; }
+  __device__ static int piece_src8(int r, int k) { return k < 2 ? 32 * r + 16 * k : 64; }
+  __device__ static int piece_scale8(int) { return 0; }
+  __device__ static int scale_blk8(int, int) { return 0; }
 };
 
 // TMEM columns: O [0, kPvN), two logit buffers of kRows fp32 columns, then the CTA's latent
@@ -164,6 +179,7 @@ struct AttnBarriers {
   uint64_t sx_ready, sx_free;
   uint64_t tab_full[2], tab_free[2];
   uint64_t mma_done, pv_done;
+  uint64_t g_loaded[2];             // FP8 cache: every gather thread read its staged codes
   uint32_t tmem_base;
   int abort;
 };
@@ -205,7 +221,21 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
   return v;
 }
 
-template <int DL, int DR>
+// e4m3x2 (two codes in the low 16 bits) -> two fp32, exactly (through f16x2)
+__device__ __forceinline__ void e4m3x2_to_f32(uint32_t codes, float& lo, float& hi) {
+  uint32_t h2;
+  asm("{\n\t.reg .b16 c;\n\tcvt.u16.u32 c, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, c;\n\t}" : "=r"(h2) : "r"(codes));
+  asm("{\n\t.reg .b16 l16, h16;\n\tmov.b32 {l16, h16}, %2;\n\tcvt.f32.f16 %0, l16;\n\tcvt.f32.f16 %1, h16;\n\t}"
+      : "=f"(lo), "=f"(hi)
+      : "r"(h2));
+}
+
+__device__ __forceinline__ void cp_async4_hint(uint32_t dst, const void* src, uint64_t policy) {
+  asm volatile("cp.async.ca.shared.global.L2::cache_hint [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "l"(policy)
+               : "memory");
+}
+
+template <int DL, int DR, bool KV8>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     sparse_attend_kernel(const __grid_constant__ AttnMaps maps, const AttnKernelParams p) {
   static_assert(kAttnThreads == 576, "role layout assumes 18 warps");
@@ -254,6 +284,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     mbar_init(&sb->sx_free, 128);    // arrived by the peer's 128 softmax threads
     mbar_init(&sb->mma_done, 1);
     mbar_init(&sb->pv_done, 1);
+    mbar_init(&sb->g_loaded[0], kProducerWarps * 32);
+    mbar_init(&sb->g_loaded[1], kProducerWarps * 32);
     sb->abort = 0;
     fence_mbarrier_init();
     tma_prefetch_desc(&maps.q_rope);
@@ -337,7 +369,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       for (int i = ptid; i < npages; i += kProducerWarps * 32) {
         const int pg = pt_row[i];
         if (pg >= 0 && pg < p.num_pages)
-          asm volatile("prefetch.global.L2 [%0];" ::"l"(kv + ((size_t)pg * p.P * DC + (size_t)rank * (p.DL / 2)) * 2));
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(kv + ((size_t)pg * p.P * DC + (size_t)rank * (p.DL / 2)) * (KV8 ? 1 : 2)));
       }
     }
     for (int u = cluster_id; u < p.units && ok; u += n_clusters, ++u_it) {
@@ -405,14 +437,114 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_arrive(&sb->tab_full[buf]);
       if (!mbar_wait_warp(&sb->tab_full[buf], (uint32_t)(u_it >> 1) & 1u, wc)) { ok = false; break; }
       const int ntiles = (unit_tiles(buf) + kRows - 1) / kRows;
-      make_pieces();   // (after the table: the two never hold registers at the same time)
-      for (int t = 0; t < ntiles; ++t, ++it) {
-        const int stage = it % kStages, rslot = it % kRopeSlots;
-        if (!mbar_wait_warp(&sb->c_empty[stage], ((uint32_t)(it / kStages) & 1u) ^ 1u, wc)) { ok = false; break; }
-        if (!mbar_wait_warp(&sb->r_empty[rslot], ((uint32_t)(it / kRopeSlots) & 1u) ^ 1u, wc)) { ok = false; break; }
-        gather_tile(smem_u32(smem + Sm::kOffC + stage * Sm::kCStageBytes),
-                    smem_u32(smem + Sm::kOffR + rslot * Sm::kCRopeBytes), rt + t * kRows);
-        asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(&sb->c_full[stage])) : "memory");
+      if constexpr (!KV8) {
+        make_pieces();   // (after the table: the two never hold registers at the same time)
+        for (int t = 0; t < ntiles; ++t, ++it) {
+          const int stage = it % kStages, rslot = it % kRopeSlots;
+          if (!mbar_wait_warp(&sb->c_empty[stage], ((uint32_t)(it / kStages) & 1u) ^ 1u, wc)) { ok = false; break; }
+          if (!mbar_wait_warp(&sb->r_empty[rslot], ((uint32_t)(it / kRopeSlots) & 1u) ^ 1u, wc)) { ok = false; break; }
+          gather_tile(smem_u32(smem + Sm::kOffC + stage * Sm::kCStageBytes),
+                      smem_u32(smem + Sm::kOffR + rslot * Sm::kCRopeBytes), rt + t * kRows);
+          asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(&sb->c_full[stage])) : "memory");
+        }
+      } else {
+        // FP8 main cache ("Rapid Adaptation and Inference Optimization", tiered quantisation
+        // table: FP8 with one scale per 128-element block of the row).  Tile t's e4m3 codes land
+        // by cp.async in the upper half of its own latent stage and rope slot, and the scale of
+        // each of this thread's pieces in a slot of the thread's own at the start of the latent
+        // stage.  One tile later, once this thread's copies of tile t are complete, it reads its
+        // codes and scales, every gather thread agrees that the staging has been read
+        // (g_loaded), and each writes its pieces as bf16 (code x scale, rounded once) into the
+        // swizzled K-major layout the MMAs read.
+        const int npr = Lay::kLatPieces8 + Lay::rope_pieces8((int)rank);
+        constexpr int kP8 = (kRows * (Lay::kLatPieces8 + Lay::kMaxRopePieces8) + kProducerWarps * 32 - 1) /
+                            (kProducerWarps * 32);
+        static_assert((kProducerWarps * 32) * kP8 * 4 <= Sm::kCStageBytes / 2, "scale slots overflow the stage");
+        const uint8_t* kv8 = static_cast<const uint8_t*>(p.kv);
+        auto staged = [&](int row, int k, uint32_t lat_base, uint32_t rope_base) -> uint32_t {
+          return k < Lay::kLatPieces8 ? lat_base + Sm::kCStageBytes / 2 + row * (Lay::kLatPieces8 * 16) + 16 * k
+                                      : rope_base + Sm::kCRopeBytes / 2 + row * Lay::kRopeCodeBytes + 16 * (k - Lay::kLatPieces8);
+        };
+        auto issue8 = [&](uint32_t lat_base, uint32_t rope_base, const int32_t* rows) {
+#pragma unroll
+          for (int j = 0; j < kP8; ++j) {
+            const int i = ptid + j * kProducerWarps * 32;
+            if (i < kRows * npr) {
+              const int row = i / npr, k = i - (i / npr) * npr;
+              const uint32_t pr = (uint32_t)rows[row];
+              const int src = Lay::piece_src8((int)rank, k);
+              cp_async16_hint(staged(row, k, lat_base, rope_base), kv8 + (size_t)pr * DC + src, stream_policy);
+              cp_async4_hint(lat_base + (uint32_t)(ptid * kP8 + j) * 4u,
+                             p.kv_scale + (size_t)pr * p.nblk + src / 128, stream_policy);
+            }
+          }
+          asm volatile("cp.async.commit_group;" ::: "memory");
+        };
+        auto convert8 = [&](int stage, int rslot, int it_) -> bool {
+          const uint32_t lat_base = smem_u32(smem + Sm::kOffC + stage * Sm::kCStageBytes);
+          const uint32_t rope_base = smem_u32(smem + Sm::kOffR + rslot * Sm::kCRopeBytes);
+          uint4 code[kP8];
+          float sc[kP8];
+#pragma unroll
+          for (int j = 0; j < kP8; ++j) {
+            const int i = ptid + j * kProducerWarps * 32;
+            code[j] = make_uint4(0, 0, 0, 0);
+            sc[j] = 0.0f;
+            if (i < kRows * npr) {
+              const int row = i / npr, k = i - (i / npr) * npr;
+              asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                           : "=r"(code[j].x), "=r"(code[j].y), "=r"(code[j].z), "=r"(code[j].w)
+                           : "r"(staged(row, k, lat_base, rope_base)));
+              asm volatile("ld.shared.f32 %0, [%1];" : "=f"(sc[j]) : "r"(lat_base + (uint32_t)(ptid * kP8 + j) * 4u));
+            }
+          }
+          mbar_arrive(&sb->g_loaded[it_ & 1]);
+          if (!mbar_wait_warp(&sb->g_loaded[it_ & 1], (uint32_t)(it_ >> 1) & 1u, wc)) return false;
+#pragma unroll
+          for (int j = 0; j < kP8; ++j) {
+            const int i = ptid + j * kProducerWarps * 32;
+            if (i < kRows * npr) {
+              const int row = i / npr, k = i - (i / npr) * npr;
+              const uint32_t cw[4] = {code[j].x, code[j].y, code[j].z, code[j].w};
+              uint32_t o[8];
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                float a, b, c, d;
+                e4m3x2_to_f32(cw[q] & 0xffffu, a, b);
+                e4m3x2_to_f32(cw[q] >> 16, c, d);
+                o[2 * q] = pack_bf16x2(a * sc[j], b * sc[j]);
+                o[2 * q + 1] = pack_bf16x2(c * sc[j], d * sc[j]);
+              }
+              const bool lat = k < Lay::kLatPieces8;
+              const uint32_t base = lat ? lat_base : rope_base;
+              const int c0 = lat ? 2 * k : Lay::kLatChunks + 2 * (k - Lay::kLatPieces8);
+              st_shared_v4(base + Lay::chunk_dst(row, c0), o[0], o[1], o[2], o[3]);
+              st_shared_v4(base + Lay::chunk_dst(row, c0 + 1), o[4], o[5], o[6], o[7]);
+            }
+          }
+          fence_proxy_async_smem();   // the MMAs read the stage through the async proxy
+          mbar_arrive(&sb->c_full[stage]);
+          return true;
+        };
+        int prev_stage = 0, prev_rslot = 0;
+        for (int t = 0; t < ntiles; ++t, ++it) {
+          const int stage = it % kStages, rslot = it % kRopeSlots;
+          if (!mbar_wait_warp(&sb->c_empty[stage], ((uint32_t)(it / kStages) & 1u) ^ 1u, wc)) { ok = false; break; }
+          if (!mbar_wait_warp(&sb->r_empty[rslot], ((uint32_t)(it / kRopeSlots) & 1u) ^ 1u, wc)) { ok = false; break; }
+          issue8(smem_u32(smem + Sm::kOffC + stage * Sm::kCStageBytes),
+                 smem_u32(smem + Sm::kOffR + rslot * Sm::kCRopeBytes), rt + t * kRows);
+          if (t > 0) {
+            asm volatile("cp.async.wait_group 1;" ::: "memory");   // this thread's copies of tile t-1
+            if (!convert8(prev_stage, prev_rslot, it - 1)) { ok = false; break; }
+          }
+          prev_stage = stage;
+          prev_rslot = rslot;
+        }
+        if (!ok) break;
+        if (ntiles > 0) {
+          asm volatile("cp.async.wait_group 0;" ::: "memory");
+          if (!convert8(prev_stage, prev_rslot, it - 1)) { ok = false; break; }
+        }
       }
     }
     // our copies have landed before we may leave, whether or not the CTA is aborting: every
@@ -830,20 +962,20 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineK
   }
 }
 
-template <int DL, int DR>
+template <int DL, int DR, bool KV8>
 cudaError_t launch_attend_impl(const AttnKernelParams& p, const CUtensorMap& q_rope, int n_clusters,
                                bool pdl, cudaStream_t stream) {
   using Sm = AttnSmem<AttnLayout<DL, DR>>;
   {
     // the warpgroup register split assumes the launch allocation kLaunchRegs per thread
     cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, sparse_attend_kernel<DL, DR>);
+    cudaError_t e = cudaFuncGetAttributes(&fa, sparse_attend_kernel<DL, DR, KV8>);
     if (e != cudaSuccess) return e;
     if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
   }
   // at most two CTAs per SM may share the 512 TMEM columns (kTmemCols each <= 256 when two fit)
   const size_t smem = Sm::kBytes < 100 * 1024 ? 100 * 1024 : Sm::kBytes;
-  cudaError_t e = cudaFuncSetAttribute(sparse_attend_kernel<DL, DR>,
+  cudaError_t e = cudaFuncSetAttribute(sparse_attend_kernel<DL, DR, KV8>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   AttnMaps m;
@@ -867,7 +999,7 @@ cudaError_t launch_attend_impl(const AttnKernelParams& p, const CUtensorMap& q_r
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, sparse_attend_kernel<DL, DR>, m, p);
+  return cudaLaunchKernelEx(&cfg, sparse_attend_kernel<DL, DR, KV8>, m, p);
 }
 
 }  // namespace
@@ -880,8 +1012,12 @@ size_t attend_smem_bytes(int dl, int dr) {
 
 cudaError_t launch_sparse_attend(const AttnKernelParams& p, const CUtensorMap& q_rope,
                                  int n_clusters, bool pdl, cudaStream_t stream) {
-  if (p.DL == 512 && p.DR == 64) return launch_attend_impl<512, 64>(p, q_rope, n_clusters, pdl, stream);
-  if (p.DL == 64 && p.DR == 16) return launch_attend_impl<64, 16>(p, q_rope, n_clusters, pdl, stream);
+  if (p.DL == 512 && p.DR == 64)
+    return p.kv_fp8 ? launch_attend_impl<512, 64, true>(p, q_rope, n_clusters, pdl, stream)
+                    : launch_attend_impl<512, 64, false>(p, q_rope, n_clusters, pdl, stream);
+  if (p.DL == 64 && p.DR == 16)
+    return p.kv_fp8 ? launch_attend_impl<64, 16, true>(p, q_rope, n_clusters, pdl, stream)
+                    : launch_attend_impl<64, 16, false>(p, q_rope, n_clusters, pdl, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -32,3 +32,23 @@ def test_causal_rows_short_of_top_k_count_only_visible_positions():
     ab = bench.algorithmic_bytes(inputs)
     assert ab["kv"] == (100 + 2048) * (512 + 64) * 2
     assert ab["idx_k"] == (100 + 5000) * 128 * 2
+
+
+def test_decode_batch_flops_and_the_roofline_bound():
+    wl = workloads.WORKLOADS[2]
+    inputs = dict(workload=wl, batch=32, n_q=1, seq_lens=torch.full((32,), 8192, dtype=torch.int32))
+    af = bench.algorithmic_flops(inputs)
+    # logits over 576 dims and the output over 512, for 128 heads and 2048 rows, 32 queries
+    assert af["stage2"] == 32 * 2048 * 128 * 2 * (576 + 512) == 18_253_611_008
+    # scoring: 64 heads x 128 dims over every visible position of every query
+    assert af["stage1"] == 32 * 8192 * 64 * 128 * 2
+    pk = {"hbm_gbs": 6542.4, "bf16_tflops": 1663.5, "bf16_tflops_sustained": 1410.5, "source": "test"}
+    ab = bench.algorithmic_bytes(inputs)
+    r = bench.roofline_entry("k", ab["stage2"], af["stage2"], 0.05, pk)
+    # 84.7 MB at 6542 GB/s (12.9 us) is longer than 18.25 GFLOP at 1663.5 TFLOP/s (11.0 us)
+    assert r["bound"] == "hbm" and abs(r["frac"] - r["hbm_frac"]) < 1e-12
+    assert abs(r["hbm_frac"] - ab["stage2"] / 50e-6 / 6542.4e9) < 1e-9
+    assert abs(r["tensor_frac"] - af["stage2"] / 50e-6 / 1663.5e12) < 1e-9
+    rs = bench.roofline_entry("k", ab["stage2"], af["stage2"], 0.05, pk, "bf16_tflops_sustained")
+    # against the sustained peak the contraction takes 12.941 us, the bytes 12.947 us: a tie
+    assert rs["bound"] == "hbm" and abs(rs["tensor_frac"] / rs["hbm_frac"] - 1.0) < 1e-3

@@ -29,7 +29,8 @@ def test_library_exports_every_declared_function(lib):
 
 
 def test_ctypes_structs_match_the_c_layout(tmp_path):
-    fields = {"sia_index_args": sia.IndexArgs, "sia_attend_args": sia.AttendArgs}
+    fields = {"sia_index_args": sia.IndexArgs, "sia_attend_args": sia.AttendArgs,
+              "sia_append_args": sia.AppendArgs}
     lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "sia.h"', "int main(void) {"]
     for cname, cls in fields.items():
         lines.append('printf("%s %%zu\\n", sizeof(%s));' % (cname, cname))
@@ -152,3 +153,30 @@ def test_noalloc_entry_point_clears_a_stale_error_message(lib):
     assert lib.sia_last_error() != b""
     assert lib.sia_sparse_index_topk_noalloc(None, None, None) == sia.SIA_ERR_INVALID_ARGUMENT
     assert b"NULL" in lib.sia_last_error()
+
+
+def _append_args(**kw):
+    a = sia.AppendArgs()
+    a.batch, a.n_q, a.head_dim, a.d_kv, a.page_size = 2, 1, 128, 576, 64
+    a.max_pages_per_seq, a.num_pages = 16, 32
+    a.key_format, a.kv_format = sia.SIA_KEY_BF16, sia.SIA_KV_BF16
+    for name in ("new_k", "new_kv", "page_table", "seq_lens", "k_cache", "kv_cache"):
+        setattr(a, name, 4096)
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(new_k=None), sia.SIA_ERR_INVALID_ARGUMENT),
+    (dict(batch=0), sia.SIA_ERR_INVALID_ARGUMENT),
+    (dict(head_dim=48), sia.SIA_ERR_UNSUPPORTED),
+    (dict(d_kv=2048), sia.SIA_ERR_UNSUPPORTED),
+    (dict(key_format=5), sia.SIA_ERR_UNSUPPORTED),
+    (dict(key_format=sia.SIA_KEY_FP8_POW2), sia.SIA_ERR_INVALID_ARGUMENT),   # k_scale missing
+    (dict(kv_scale=8192), sia.SIA_ERR_INVALID_ARGUMENT),                    # scale for a bf16 cache
+])
+def test_append_arguments_refused_on_the_host(lib, kw, status):
+    a = _append_args(**kw)
+    assert lib.sia_cache_append(ctypes.byref(a), None, None) == status
+    assert lib.sia_last_error() != b""
