@@ -291,6 +291,7 @@ struct AttendPlan {
   CombineKernelParams cp;
   CUtensorMap q_rope;   // the query rows' rope slices (the only TMA load of the attention)
   size_t ws_part;
+  long long records;  // partial-result records (0: every query is written directly)
   int n_clusters;
 };
 
@@ -333,22 +334,38 @@ sia_status plan_attend(const sia_attend_args* a, AttendPlan* pl, bool make_maps)
   k.scale_log2 = a->softmax_scale * 1.4426950408889634f;
   const long long bj = (long long)a->batch * a->n_q;
   const int pairs = std::max(1, sm_count() / 2);
-  // pick the number of Top-K splits that minimises the rows one cluster has to stream
-  const int max_splits = std::max(1, std::min(8, (a->top_k + kAttnTileRows - 1) / kAttnTileRows));
-  const int min_splits = (a->top_k + kAttnMaxSplitRows - 1) / kAttnMaxSplitRows;
-  long long best = -1;
-  int best_s = 1, best_rows = 0;
-  for (int s = min_splits; s <= max_splits; ++s) {
-    const int rows = (int)round_up((size_t)((a->top_k + s - 1) / s), kAttnTileRows);
-    const int s_eff = (a->top_k + rows - 1) / rows;
-    const long long units = bj * s_eff;
-    const long long cost = (units + pairs - 1) / pairs * rows;
-    if (best < 0 || cost < best) { best = cost; best_s = s_eff; best_rows = rows; }
+  // the flat (query, 64-row tile) list split evenly over the CTA pairs (see attn_next_unit)
+  const long long TQ = (a->top_k + kAttnTileRows - 1) / kAttnTileRows;
+  const long long G = bj * TQ;
+  const int C = (int)std::min<long long>(pairs, G);
+  auto pair_start = [&](long long c) { return c * G / C; };
+  auto pair_of_tile = [&](long long g) { return (long long)(((g + 1) * C - 1) / G); };
+  k.tiles_per_q = (int)TQ;
+  k.total_tiles = G;
+  k.n_pairs = C;
+  k.segs_per_q = (int)((TQ + 31) / 32);
+  long long records = 0;
+  int max_slots = 1;
+  if (TQ <= 32) {
+    // only queries with a pair boundary strictly inside them have partial records
+    long long prevq = -1;
+    for (long long c = 1; c < C; ++c) {
+      const long long g = pair_start(c);
+      if (g % TQ == 0 || g / TQ == prevq) continue;
+      prevq = g / TQ;
+      ++records;
+      const long long q0 = prevq * TQ;
+      max_slots = std::max(max_slots, (int)(pair_of_tile(q0 + TQ - 1) - pair_of_tile(q0) + 1));
+    }
+    records *= max_slots;
+  } else {
+    const long long per_pair = std::max<long long>(1, G / C);
+    const long long spanned = std::min<long long>(C, (TQ + per_pair - 1) / per_pair + 1);
+    max_slots = (int)(spanned * k.segs_per_q);
+    records = bj * max_slots;
   }
-  k.splits = best_s;
-  k.rows_per_split = best_rows;
-  if (bj * best_s > 0x7fffffffll) return fail(SIA_ERR_UNSUPPORTED, "too many attention work units");
-  k.units = (int)(bj * best_s);
+  k.max_slots = max_slots;
+  if (records > 0x7fffffffll) return fail(SIA_ERR_UNSUPPORTED, "too many attention partial records");
   k.q = a->q;
   k.kv = a->kv_cache;
   k.kv_scale = a->kv_scale;
@@ -359,18 +376,23 @@ sia_status plan_attend(const sia_attend_args* a, AttendPlan* pl, bool make_maps)
   k.topk = a->topk;
   k.out = static_cast<uint16_t*>(a->out);
   k.lse = a->lse;
-  pl->n_clusters = (int)std::min<long long>(k.units, pairs);
+  pl->n_clusters = C;
+  pl->records = records;
   pl->ws_part = 0;
-  if (k.splits > 1) {
-    const size_t o = round_up((size_t)k.splits * bj * a->n_heads * a->d_latent * 2, 256);
-    const size_t l = round_up((size_t)k.splits * bj * a->n_heads * 4, 256);
+  if (records > 0) {
+    const size_t o = round_up((size_t)records * a->n_heads * a->d_latent * 2, 256);
+    const size_t l = round_up((size_t)records * a->n_heads * 4, 256);
     pl->ws_part = o + l;
   }
   CombineKernelParams& c = pl->cp;
   c.BJ = (int)bj;
   c.H = a->n_heads;
   c.DL = a->d_latent;
-  c.splits = k.splits;
+  c.tiles_per_q = k.tiles_per_q;
+  c.n_pairs = k.n_pairs;
+  c.segs_per_q = k.segs_per_q;
+  c.max_slots = k.max_slots;
+  c.total_tiles = k.total_tiles;
   c.out = k.out;
   c.lse = a->lse;
 
@@ -390,9 +412,8 @@ sia_status run_attend(AttendPlan* pl, void* ws, size_t ws_bytes, int32_t* dev_st
     if (!ws) return fail(SIA_ERR_WORKSPACE, "a workspace of %zu bytes is needed", pl->ws_part);
     if (ws_bytes < pl->ws_part) return fail(SIA_ERR_WORKSPACE, "workspace too small: %zu < %zu", ws_bytes, pl->ws_part);
     if (!aligned(ws, 256)) return fail(SIA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
-    const long long bj = (long long)pl->ap.B * pl->ap.J;
     uint16_t* o = static_cast<uint16_t*>(ws);
-    const size_t ob = round_up((size_t)pl->ap.splits * bj * pl->ap.H * pl->ap.DL * 2, 256);
+    const size_t ob = round_up((size_t)pl->records * pl->ap.H * pl->ap.DL * 2, 256);
     pl->ap.part_o = o;
     pl->ap.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + ob);
     pl->cp.part_o = pl->ap.part_o;
@@ -402,7 +423,7 @@ sia_status run_attend(AttendPlan* pl, void* ws, size_t ws_bytes, int32_t* dev_st
   pl->ap.wait_ns = wait_limit_ns();
   cudaError_t e = launch_sparse_attend(pl->ap, pl->q_rope, pl->n_clusters, pdl_first, stream);
   if (e != cudaSuccess) return cuda_fail(e, "sparse attention launch");
-  if (pl->ap.splits > 1) {
+  if (pl->records > 0) {
     e = launch_combine(pl->cp, true, stream);
     if (e != cudaSuccess) return cuda_fail(e, "split combine launch");
   }

@@ -79,9 +79,11 @@ struct TopkKernelParams {
 struct AttnKernelParams {
   int B, J, H, DL, DR, P, max_pages, num_pages, K;
   float scale_log2;           // softmax_scale * log2(e)
-  int splits;                 // Top-K splits per query (>1 -> partials + combine)
-  int rows_per_split;         // multiple of kAttnTileRows
-  int units;                  // B * J * splits
+  int tiles_per_q;            // ceil(K / kAttnTileRows)
+  long long total_tiles;      // B * J * tiles_per_q
+  int n_pairs;                // CTA pairs (clusters) of the launch
+  int segs_per_q;             // ceil(tiles_per_q / 32)
+  int max_slots;              // partial records per split query
   const void* q;              // bf16 [B*J, H, DL + DR]
   const void* kv;             // bf16 [num_pages * P, DL + DR], or e4m3 codes when kv_fp8
   const float* kv_scale;      // kv_fp8: fp32 [num_pages * P, nblk], one per 128-element block
@@ -92,14 +94,16 @@ struct AttnKernelParams {
   const int32_t* topk;
   uint16_t* out;              // bf16 bits
   float* lse;
-  uint16_t* part_o;           // [splits][B*J][H][DL] bf16, normalised (splits > 1)
-  float* part_lse;            // [splits][B*J][H]
+  uint16_t* part_o;           // [records][H][DL] bf16, normalised
+  float* part_lse;            // [records][H]
   int32_t* status;
   uint64_t wait_ns;           // limit of every bounded in-kernel wait
 };
 
 struct CombineKernelParams {
-  int BJ, H, DL, splits;
+  int BJ, H, DL;
+  int tiles_per_q, n_pairs, segs_per_q, max_slots;
+  long long total_tiles;
   const uint16_t* part_o;
   const float* part_lse;
   uint16_t* out;

@@ -62,7 +62,7 @@ constexpr int kGatherRegs = 64;
 static_assert(128 * kSoftmaxRegs + 256 * kGatherRegs + 128 * kExchangeRegs + 64 * kLaunchRegs <=
                   kAttnThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
-constexpr int kStages = 4;          // latent-row tiles in flight per CTA
+constexpr int kStages = 3;          // latent-row tiles in flight per CTA
 constexpr int kRopeSlots = 2;       // their rope parts (read by S = Q . C^T only) in flight
 constexpr int kRows = kAttnTileRows;
 
@@ -149,10 +149,13 @@ struct AttnSmem {
   static constexpr uint32_t kOffR = kOffC + kStages * kCStageBytes;
   // P (bf16, 128 heads x kRows, 128B-swizzled K-major): the A operand of P . C
   static constexpr uint32_t kOffP = (kOffR + kRopeSlots * kCRopeBytes + 1023u) & ~1023u;
-  static constexpr uint32_t kOffSx = kOffP + 128 * kRows * 2;          // peer logits, fp16
+  // peer logits, fp16, two tiles: the peer's exchange warps fill one while this CTA's softmax
+  // reads the other
+  static constexpr uint32_t kSxBytes = kRows * 128 * 2;
+  static constexpr uint32_t kOffSx = kOffP + 128 * kRows * 2;
   // this CTA's own logits, fp16, two tiles: the exchange warps copy them out of TMEM so that a
   // logit buffer is free for the next product as soon as they have read it
-  static constexpr uint32_t kOffStash = kOffSx + kRows * 128 * 2;
+  static constexpr uint32_t kOffStash = kOffSx + 2 * kSxBytes;
   static constexpr uint32_t kOffRows = kOffStash + 2 * kRows * 128 * 2;
   // per unit (double-buffered): physical cache row of each Top-K entry, validity bits, and
   // each gather warp's lowest position of a -1 entry
@@ -176,7 +179,7 @@ struct AttnBarriers {
   uint64_t q_full, q_empty;       // q in TMEM written by the 128 loader threads / q reusable
   uint64_t q_tma;                 // the rope part of q landed (TMA bytes only)
   uint64_t o_full;
-  uint64_t sx_ready, sx_free;
+  uint64_t sx_ready[2], sx_free[2];
   uint64_t tab_full[2], tab_free[2];
   uint64_t mma_done, pv_done;
   uint64_t g_loaded[2];             // FP8 cache: every gather thread read its staged codes
@@ -219,6 +222,73 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "l"(p));
   return v;
+}
+
+// The work of a call is the flat list of (query, 64-row tile) pairs, query-major with
+// tiles_per_q tiles per query, split evenly between the CTA pairs: pair c takes global tiles
+// [c G / C, (c + 1) G / C).  A unit is the part of that range inside one query and inside one
+// run of 32 tiles of it (at most kAttnMaxSplitRows Top-K entries, the size of the row table).
+// A query covered by one unit gets its output written directly; otherwise every unit writes a
+// partial result (normalised O and log-sum-exp) into a record of the workspace, and
+// combine_kernel merges a query's records.  Records: with at most 32 tiles per query only the
+// queries that straddle a pair boundary have any (at most C - 1 of them), numbered in order;
+// with more, every query has max_slots of them.  Within a query, slot (c - first pair) *
+// segs_per_q + (32-tile run index counted from where pair c starts in the query).
+__device__ __forceinline__ long long attn_pair_start(int c, int C, long long G) { return (long long)c * G / C; }
+
+__device__ __forceinline__ int attn_pair_of_tile(long long g, int C, long long G) {
+  return (int)(((g + 1) * C - 1) / G);
+}
+
+struct AttnUnit {
+  int bj;        // query row (b * J + j)
+  int row0;      // first Top-K entry of the unit
+  int nrows;     // entries in the unit (rows of the last tile may be absent)
+  long long rec; // partial-result record, or -1 when the unit writes the final output
+};
+
+// Record number of query bj's slot `slot` (the host sizes the workspace the same way).
+__device__ __forceinline__ long long attn_record(int TQ, int C, long long G, int max_slots, int bj, int slot) {
+  if (TQ > 32) return (long long)bj * max_slots + slot;
+  // rank of bj among the queries that contain a pair boundary strictly inside them
+  const long long q0 = (long long)bj * TQ;
+  int n = 0, prevq = -1;
+  for (int c = 1; c < C; ++c) {
+    const long long g = attn_pair_start(c, C, G);
+    if (g >= q0) break;
+    const int q = (int)(g / TQ);
+    if (g % TQ != 0 && q != prevq) {
+      ++n;
+      prevq = q;
+    }
+  }
+  return (long long)n * max_slots + slot;
+}
+
+// Next unit of pair `c` from global tile `cursor` (advanced past the unit); false when done.
+__device__ __forceinline__ bool attn_next_unit(const AttnKernelParams& p, int c, long long& cursor, AttnUnit& u) {
+  const long long G = p.total_tiles;
+  const int C = p.n_pairs;
+  const long long g1 = attn_pair_start(c + 1, C, G);
+  if (cursor >= g1) return false;
+  const int TQ = p.tiles_per_q;
+  u.bj = (int)(cursor / TQ);
+  const long long q0 = (long long)u.bj * TQ;
+  const long long seg_end = q0 + (((cursor - q0) >> 5) + 1) * 32;
+  const long long tb = min(min(g1, q0 + TQ), seg_end);
+  u.row0 = (int)(cursor - q0) * kAttnTileRows;
+  u.nrows = min(p.K, (int)(tb - q0) * kAttnTileRows) - u.row0;
+  const int first = attn_pair_of_tile(q0, C, G);
+  const int last = attn_pair_of_tile(q0 + TQ - 1, C, G);
+  if (first == last && TQ <= 32) {
+    u.rec = -1;
+  } else {
+    const long long a = max(q0, attn_pair_start(c, C, G));
+    const int slot = (c - first) * p.segs_per_q + (int)(((cursor - q0) >> 5) - ((a - q0) >> 5));
+    u.rec = attn_record(TQ, C, G, p.max_slots, u.bj, slot);
+  }
+  cursor = tb;
+  return true;
 }
 
 // e4m3x2 (two codes in the low 16 bits) -> two fp32, exactly (through f16x2)
@@ -280,8 +350,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     mbar_init(&sb->q_tma, 1);          // the rope TMA (or a plain arrive when this CTA has none)
     mbar_init(&sb->q_empty, 1);
     mbar_init(&sb->o_full, 1);
-    mbar_init(&sb->sx_ready, 128);   // arrived by the peer's 128 exchange threads
-    mbar_init(&sb->sx_free, 128);    // arrived by the peer's 128 softmax threads
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sb->sx_ready[s], 128);   // arrived by the peer's 128 exchange threads
+      mbar_init(&sb->sx_free[s], 128);    // arrived by the peer's 128 softmax threads
+    }
     mbar_init(&sb->mma_done, 1);
     mbar_init(&sb->pv_done, 1);
     mbar_init(&sb->g_loaded[0], kProducerWarps * 32);
@@ -358,10 +430,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     int it = 0, u_it = 0, q_issued = 0;
     bool ok = true;
     bool waited = false;
-    if (cluster_id < p.units) {
+    long long cursor = (long long)cluster_id * p.total_tiles / p.n_pairs;
+    AttnUnit un;
+    if (cursor < (long long)(cluster_id + 1) * p.total_tiles / p.n_pairs) {
       // While the previous kernel still runs: touch every cache page of the first unit's
       // sequence (address translation and the page-table row warm up before the gather)
-      const int b = (cluster_id / p.splits) / p.J;
+      const int b = (int)(cursor / p.tiles_per_q) / p.J;
       const int L = p.seq_lens[b];
       const int npages = min(p.max_pages, (L + p.P - 1) / p.P);
       const int32_t* pt_row = p.page_table + (long long)b * p.max_pages;
@@ -372,13 +446,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           asm volatile("prefetch.global.L2 [%0];" ::"l"(kv + ((size_t)pg * p.P * DC + (size_t)rank * (p.DL / 2)) * (KV8 ? 1 : 2)));
       }
     }
-    for (int u = cluster_id; u < p.units && ok; u += n_clusters, ++u_it) {
-      const int bj = u / p.splits, split = u - bj * p.splits;
+    while (ok && attn_next_unit(p, cluster_id, cursor, un)) {
+      const int bj = un.bj;
       const int b = bj / p.J;
       const int L = p.seq_lens[b];
       const long long row_base = (long long)bj * p.K;
-      const int row0 = split * p.rows_per_split;
-      const int nrows = min(p.K, row0 + p.rows_per_split) - row0;
+      const int row0 = un.row0;
+      const int nrows = un.nrows;
       const int nrows_pad = (nrows + kRows - 1) / kRows * kRows;
       const int buf = u_it & 1;
       // rope part of the query rows of all heads (TMA; independent of the Top-K list)
@@ -546,6 +620,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (!convert8(prev_stage, prev_rslot, it - 1)) { ok = false; break; }
         }
       }
+      ++u_it;
     }
     // our copies have landed before we may leave, whether or not the CTA is aborting: every
     // cp.async of this thread, and the rope TMA of the last unit (one unit's q at a time: the
@@ -561,7 +636,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint32_t qr_base = smem_u32(smem + Sm::kOffQ);
       int it = 0, u_it = 0;
       bool ok = true;
-      for (int u = cluster_id; u < p.units && ok; u += n_clusters, ++u_it) {
+      long long cursor = (long long)cluster_id * p.total_tiles / p.n_pairs;
+      AttnUnit un;
+      for (; ok && attn_next_unit(p, cluster_id, cursor, un); ++u_it) {
         const int buf = u_it & 1;
         if (!mbar_wait(&sb->tab_full[buf], (uint32_t)(u_it >> 1) & 1u, wc)) { ok = false; break; }
         const int ntiles = (unit_tiles(buf) + kRows - 1) / kRows;
@@ -612,7 +689,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint32_t p_base = smem_u32(smem + Sm::kOffP);
       int it = 0, u_it = 0;
       bool ok = true;
-      for (int u = cluster_id; u < p.units && ok; u += n_clusters, ++u_it) {
+      long long cursor = (long long)cluster_id * p.total_tiles / p.n_pairs;
+      AttnUnit un;
+      for (; ok && attn_next_unit(p, cluster_id, cursor, un); ++u_it) {
         const int buf = u_it & 1;
         if (!mbar_wait(&sb->tab_full[buf], (uint32_t)(u_it >> 1) & 1u, wc)) { ok = false; break; }
         const int ntiles = (unit_tiles(buf) + kRows - 1) / kRows;
@@ -651,8 +730,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t sx_peer = mapa_shared(smem_u32(smem + Sm::kOffSx), peer);
     int s_it = 0, u_it = 0;
     bool ok = true;
-    for (int u = cluster_id; u < p.units && ok; u += n_clusters, ++u_it) {
-      const int bj = u / p.splits;
+    long long cursor = (long long)cluster_id * p.total_tiles / p.n_pairs;
+    AttnUnit un;
+    for (; ok && attn_next_unit(p, cluster_id, cursor, un); ++u_it) {
+      const int bj = un.bj;
       const int buf = u_it & 1;
       {
         // q: head h's dims [rank * kLatDims, +kLatDims) as bf16 pairs, 16 columns per store
@@ -715,13 +796,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           st_shared_v4(smem_u32(smem + Sm::kOffStash + sbuf * (kRows * 128 * 2) + (g * 128 + h) * 16),
                        own[4 * g], own[4 * g + 1], own[4 * g + 2], own[4 * g + 3]);
         mbar_arrive(&sb->own_ready[sbuf]);
-        if (!mbar_wait_warp<true>(&sb->sx_free, ((uint32_t)s_it & 1u) ^ 1u, wc)) { ok = false; break; }
+        if (!mbar_wait_warp<true>(&sb->sx_free[sbuf], ((uint32_t)(s_it >> 1) & 1u) ^ 1u, wc)) { ok = false; break; }
 #pragma unroll
         for (int g = 0; g < kRows / 8; ++g)
-          asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sx_peer + (uint32_t)((g * 128 + h) * 16)),
+          asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sx_peer + sbuf * Sm::kSxBytes + (uint32_t)((g * 128 + h) * 16)),
                        "r"(own[4 * g]), "r"(own[4 * g + 1]), "r"(own[4 * g + 2]), "r"(own[4 * g + 3])
                        : "memory");
-        mbar_arrive_cluster(&sb->sx_ready, peer);
+        mbar_arrive_cluster(&sb->sx_ready[sbuf], peer);
       }
     }
   } else {
@@ -733,8 +814,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     int s_it = 0, u_it = 0, o_it = 0, e_it = 0;
     bool ok = true;
 
-    for (int u = cluster_id; u < p.units && ok; u += n_clusters, ++u_it) {
-      const int bj = u / p.splits, split = u - bj * p.splits;
+    long long cursor = (long long)cluster_id * p.total_tiles / p.n_pairs;
+    AttnUnit un;
+    int last_sbuf = 0;
+    for (; ok && attn_next_unit(p, cluster_id, cursor, un); ++u_it) {
+      const int bj = un.bj;
       const int buf = u_it & 1;
       if (!mbar_wait_warp(&sb->tab_full[buf], (uint32_t)(u_it >> 1) & 1u, wc)) { ok = false; break; }
       const int first_neg = unit_tiles(buf);
@@ -748,13 +832,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int live = first_neg - t * kRows;            // rows past the first -1 are padding
         if (live < kRows) valid &= (1ull << live) - 1ull;
         if (!mbar_wait_warp(&sb->own_ready[sbuf], (uint32_t)(s_it >> 1) & 1u, wc)) { ok = false; break; }
-        if (!mbar_wait_warp<true>(&sb->sx_ready, (uint32_t)s_it & 1u, wc)) { ok = false; break; }
+        if (!mbar_wait_warp<true>(&sb->sx_ready[sbuf], (uint32_t)(s_it >> 1) & 1u, wc)) { ok = false; break; }
+        last_sbuf = sbuf;
         // logits of tile t (base 2) = own fp16 partial + the peer's fp16 partial: both CTAs add
         // the same two values, so their logits agree bit for bit
 #pragma unroll
         for (int g = 0; g < kRows / 8; ++g) {
           const uint4 ov = *reinterpret_cast<const uint4*>(smem + Sm::kOffStash + sbuf * (kRows * 128 * 2) + (g * 128 + h) * 16);
-          const uint4 pv4 = *reinterpret_cast<const uint4*>(smem + Sm::kOffSx + (g * 128 + h) * 16);
+          const uint4 pv4 = *reinterpret_cast<const uint4*>(smem + Sm::kOffSx + sbuf * Sm::kSxBytes + (g * 128 + h) * 16);
           const uint32_t o4[4] = {ov.x, ov.y, ov.z, ov.w};
           const uint32_t q4[4] = {pv4.x, pv4.y, pv4.z, pv4.w};
 #pragma unroll
@@ -769,7 +854,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         mbar_arrive(&sb->own_free[sbuf]);
         // the peer may refill the exchange buffer (the logit values read above are already in
         // registers); after the unit's last tile the buffer first serves the epilogue
-        if (t + 1 < ntiles) mbar_arrive_cluster_relaxed(&sb->sx_free, peer);
+        if (t + 1 < ntiles) mbar_arrive_cluster_relaxed(&sb->sx_free[sbuf], peer);
 
         // online softmax (base 2), lazy rescale
         float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
@@ -846,14 +931,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // buffer (free until the deferred sx_free below): each warp stages 32 heads x 128 bytes
       // per round in a 128B-swizzled 4 KB slice, then writes whole 128-byte runs of 4 heads per
       // instruction
-      uint16_t* obase = (p.splits > 1 ? p.part_o + ((long long)split * p.B * p.J + bj) * p.H * p.DL
-                                      : p.out + (long long)bj * p.H * p.DL) + rank * Lay::kPvN;
+      const bool partial = un.rec >= 0;
+      uint16_t* obase = (partial ? p.part_o + un.rec * p.H * p.DL : p.out + (long long)bj * p.H * p.DL) +
+                        rank * Lay::kPvN;
       if (ntiles > 0) {
         // every softmax warp has read the last tile's peer logits before any slice is reused
         mbar_arrive(&sb->epi_sync);
         if (!mbar_wait_warp(&sb->epi_sync, (uint32_t)e_it & 1u, wc)) { ok = false; break; }
         ++e_it;
-        uint8_t* slice = smem + Sm::kOffSx + quad * 4096;
+        uint8_t* slice = smem + Sm::kOffSx + last_sbuf * Sm::kSxBytes + quad * 4096;
 #pragma unroll 1
         for (int c = 0; c < Lay::kPvN; c += 64) {
           uint32_t w[32];
@@ -889,12 +975,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           *reinterpret_cast<uint4*>(obase + (long long)h * p.DL + c) = make_uint4(0, 0, 0, 0);
       }
       if (real_head && rank == 0) {
-        if (p.splits > 1) p.part_lse[((long long)split * p.B * p.J + bj) * p.H + h] = lse;
+        if (partial) p.part_lse[un.rec * p.H + h] = lse;
         else if (p.lse) p.lse[(long long)bj * p.H + h] = lse;
       }
       if (ntiles > 0) {
         __syncwarp();
-        mbar_arrive_cluster_relaxed(&sb->sx_free, peer);   // deferred from the unit's last tile
+        mbar_arrive_cluster_relaxed(&sb->sx_free[last_sbuf], peer);   // deferred from the unit's last tile
       }
       tc_fence_before();   // our reads of O come before the next unit's first P . C
     }
@@ -908,8 +994,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
 }
 
-// Log-sum-exp merge of the per-split partial results: 256 threads per CTA, 8 output dims per
-// thread (16-byte loads of the bf16 partials), DL/8 threads per (query row, head).
+// Log-sum-exp merge of the partial results of the queries whose units were spread over several
+// records: 256 threads per CTA, 8 output dims per thread (16-byte loads of the bf16 partials),
+// DL/8 threads per (query row, head).  Queries covered by a single unit were written directly.
 constexpr int kCombineThreads = 256;
 
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineKernelParams p) {
@@ -919,47 +1006,71 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineK
   const long long bjh = (long long)blockIdx.x * (kCombineThreads / tph) + threadIdx.x / tph;
   const int d8 = (threadIdx.x % tph) * 8;
   const long long n_bjh = (long long)p.BJ * p.H;
-  if (bjh < n_bjh) {
-    // Splits are merged four at a time: the four log-sum-exps and partial vectors are loaded
-    // together, so a merge of up to four splits waits for one memory latency.
-    float mx = -INFINITY, wsum = 0.0f, o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int s0 = 0; s0 < p.splits; s0 += 4) {
-      float ls[4];
-      uint4 v[4];
+  if (bjh >= n_bjh) return;
+  const int bj = (int)(bjh / p.H), h = (int)(bjh - (long long)bj * p.H);
+  const int TQ = p.tiles_per_q, C = p.n_pairs;
+  const long long G = p.total_tiles;
+  const long long q0 = (long long)bj * TQ;
+  const int first = attn_pair_of_tile(q0, C, G);
+  const int last = attn_pair_of_tile(q0 + TQ - 1, C, G);
+  if (first == last && TQ <= 32) return;
+  const long long rec0 = attn_record(TQ, C, G, p.max_slots, bj, 0);
+  // the query's slots: for each pair c in [first, last], one per 32-tile run it covers
+  float mx = -INFINITY, wsum = 0.0f, o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  int slots[4];
+  int ns = 0;
+  auto merge = [&](int n) {
+    // the log-sum-exps and partial vectors of up to four slots are loaded together, so a
+    // merge of up to four records waits for one memory latency
+    float ls[4];
+    uint4 v[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const bool in = s0 + i < p.splits;
-        const long long e = (long long)(s0 + i) * n_bjh + bjh;
-        ls[i] = in ? p.part_lse[e] : -INFINITY;
-        v[i] = in ? ld_nc_v4(p.part_o + e * p.DL + d8) : make_uint4(0, 0, 0, 0);
-      }
-      float m_new = mx;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) m_new = fmaxf(m_new, ls[i]);
-      if (m_new == -INFINITY) continue;   // every split so far is empty
-      const float c = mx == -INFINITY ? 0.0f : expf(mx - m_new);
-      wsum *= c;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) o[j] *= c;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float wgt = ls[i] == -INFINITY ? 0.0f : expf(ls[i] - m_new);
-        const uint32_t w4[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          o[2 * k] += wgt * __uint_as_float(w4[k] << 16);
-          o[2 * k + 1] += wgt * __uint_as_float(w4[k] & 0xffff0000u);
-        }
-        wsum += wgt;
-      }
-      mx = m_new;
+    for (int i = 0; i < 4; ++i) {
+      const bool in = i < n;
+      const long long e = rec0 + (in ? slots[i] : 0);
+      ls[i] = in ? p.part_lse[e * p.H + h] : -INFINITY;
+      v[i] = in ? ld_nc_v4(p.part_o + (e * p.H + h) * p.DL + d8) : make_uint4(0, 0, 0, 0);
     }
-    const float inv = wsum > 0.0f ? 1.0f / wsum : 0.0f;
-    *reinterpret_cast<uint4*>(p.out + bjh * p.DL + d8) =
-        make_uint4(pack_bf16x2(o[0] * inv, o[1] * inv), pack_bf16x2(o[2] * inv, o[3] * inv),
-                   pack_bf16x2(o[4] * inv, o[5] * inv), pack_bf16x2(o[6] * inv, o[7] * inv));
-    if (d8 == 0 && p.lse) p.lse[bjh] = wsum > 0.0f ? mx + logf(wsum) : -INFINITY;
+    float m_new = mx;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) m_new = fmaxf(m_new, ls[i]);
+    if (m_new == -INFINITY) return;   // every record so far is empty
+    const float c = mx == -INFINITY ? 0.0f : expf(mx - m_new);
+    wsum *= c;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) o[j] *= c;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float wgt = ls[i] == -INFINITY ? 0.0f : expf(ls[i] - m_new);
+      const uint32_t w4[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        o[2 * k] += wgt * __uint_as_float(w4[k] << 16);
+        o[2 * k + 1] += wgt * __uint_as_float(w4[k] & 0xffff0000u);
+      }
+      wsum += wgt;
+    }
+    mx = m_new;
+  };
+  for (int c = first; c <= last; ++c) {
+    const long long a = max(q0, attn_pair_start(c, C, G));
+    const long long b = min(q0 + TQ, attn_pair_start(c + 1, C, G));
+    if (b <= a) continue;
+    const int nseg = (int)(((b - 1 - q0) >> 5) - ((a - q0) >> 5)) + 1;
+    for (int k = 0; k < nseg; ++k) {
+      slots[ns++] = (c - first) * p.segs_per_q + k;
+      if (ns == 4) {
+        merge(4);
+        ns = 0;
+      }
+    }
   }
+  if (ns > 0) merge(ns);
+  const float inv = wsum > 0.0f ? 1.0f / wsum : 0.0f;
+  *reinterpret_cast<uint4*>(p.out + bjh * p.DL + d8) =
+      make_uint4(pack_bf16x2(o[0] * inv, o[1] * inv), pack_bf16x2(o[2] * inv, o[3] * inv),
+                 pack_bf16x2(o[4] * inv, o[5] * inv), pack_bf16x2(o[6] * inv, o[7] * inv));
+  if (d8 == 0 && p.lse) p.lse[bjh] = wsum > 0.0f ? mx + logf(wsum) : -INFINITY;
 }
 
 template <int DL, int DR, bool KV8>
