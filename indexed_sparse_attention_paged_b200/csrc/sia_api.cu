@@ -304,8 +304,8 @@ sia_status check_attend(const sia_attend_args* a) {
   if (!((a->d_latent == 512 && a->d_rope == 64) || (a->d_latent == 64 && a->d_rope == 16)))
     return fail(SIA_ERR_UNSUPPORTED, "(d_latent, d_rope) must be (512, 64) or (64, 16) (got %d, %d)", a->d_latent, a->d_rope);
   if (a->n_heads < 1 || a->n_heads > 128) return fail(SIA_ERR_UNSUPPORTED, "n_heads must be 1..128 (got %d)", a->n_heads);
-  if (a->top_k > 8 * kAttnMaxSplitRows)
-    return fail(SIA_ERR_UNSUPPORTED, "top_k must be <= %d (got %d)", 8 * kAttnMaxSplitRows, a->top_k);
+  if (a->top_k > kAttnMaxSplitRows)
+    return fail(SIA_ERR_UNSUPPORTED, "top_k must be <= %d (got %d)", kAttnMaxSplitRows, a->top_k);
   if (!std::isfinite(a->softmax_scale)) return fail(SIA_ERR_INVALID_ARGUMENT, "softmax_scale must be finite");
   if (!aligned(a->q, 16) || !aligned(a->kv_cache, 16) || !aligned(a->out, 16) || !aligned(a->topk, 4) ||
       (a->lse && !aligned(a->lse, 4)) || (a->kv_scale && !aligned(a->kv_scale, 4)))
@@ -338,34 +338,16 @@ sia_status plan_attend(const sia_attend_args* a, AttendPlan* pl, bool make_maps)
   const long long TQ = (a->top_k + kAttnTileRows - 1) / kAttnTileRows;
   const long long G = bj * TQ;
   const int C = (int)std::min<long long>(pairs, G);
-  auto pair_start = [&](long long c) { return c * G / C; };
-  auto pair_of_tile = [&](long long g) { return (long long)(((g + 1) * C - 1) / G); };
   k.tiles_per_q = (int)TQ;
   k.total_tiles = G;
   k.n_pairs = C;
-  k.segs_per_q = (int)((TQ + 31) / 32);
+  // pieces (and their merge) only when some pair boundary falls inside a query
   long long records = 0;
-  int max_slots = 1;
-  if (TQ <= 32) {
-    // only queries with a pair boundary strictly inside them have partial records
-    long long prevq = -1;
-    for (long long c = 1; c < C; ++c) {
-      const long long g = pair_start(c);
-      if (g % TQ == 0 || g / TQ == prevq) continue;
-      prevq = g / TQ;
-      ++records;
-      const long long q0 = prevq * TQ;
-      max_slots = std::max(max_slots, (int)(pair_of_tile(q0 + TQ - 1) - pair_of_tile(q0) + 1));
+  for (long long c = 1; c < C; ++c)
+    if ((c * G / C) % TQ != 0) {
+      records = 2ll * C;
+      break;
     }
-    records *= max_slots;
-  } else {
-    const long long per_pair = std::max<long long>(1, G / C);
-    const long long spanned = std::min<long long>(C, (TQ + per_pair - 1) / per_pair + 1);
-    max_slots = (int)(spanned * k.segs_per_q);
-    records = bj * max_slots;
-  }
-  k.max_slots = max_slots;
-  if (records > 0x7fffffffll) return fail(SIA_ERR_UNSUPPORTED, "too many attention partial records");
   k.q = a->q;
   k.kv = a->kv_cache;
   k.kv_scale = a->kv_scale;
@@ -381,7 +363,7 @@ sia_status plan_attend(const sia_attend_args* a, AttendPlan* pl, bool make_maps)
   pl->ws_part = 0;
   if (records > 0) {
     const size_t o = round_up((size_t)records * a->n_heads * a->d_latent * 2, 256);
-    const size_t l = round_up((size_t)records * a->n_heads * 4, 256);
+    const size_t l = round_up((size_t)records * 2 * a->n_heads * 4, 256);
     pl->ws_part = o + l;
   }
   CombineKernelParams& c = pl->cp;
@@ -390,8 +372,6 @@ sia_status plan_attend(const sia_attend_args* a, AttendPlan* pl, bool make_maps)
   c.DL = a->d_latent;
   c.tiles_per_q = k.tiles_per_q;
   c.n_pairs = k.n_pairs;
-  c.segs_per_q = k.segs_per_q;
-  c.max_slots = k.max_slots;
   c.total_tiles = k.total_tiles;
   c.out = k.out;
   c.lse = a->lse;

@@ -79,11 +79,9 @@ struct TopkKernelParams {
 struct AttnKernelParams {
   int B, J, H, DL, DR, P, max_pages, num_pages, K;
   float scale_log2;           // softmax_scale * log2(e)
-  int tiles_per_q;            // ceil(K / kAttnTileRows)
+  int tiles_per_q;            // ceil(K / kAttnTileRows) <= 32
   long long total_tiles;      // B * J * tiles_per_q
   int n_pairs;                // CTA pairs (clusters) of the launch
-  int segs_per_q;             // ceil(tiles_per_q / 32)
-  int max_slots;              // partial records per split query
   const void* q;              // bf16 [B*J, H, DL + DR]
   const void* kv;             // bf16 [num_pages * P, DL + DR], or e4m3 codes when kv_fp8
   const float* kv_scale;      // kv_fp8: fp32 [num_pages * P, nblk], one per 128-element block
@@ -94,15 +92,15 @@ struct AttnKernelParams {
   const int32_t* topk;
   uint16_t* out;              // bf16 bits
   float* lse;
-  uint16_t* part_o;           // [records][H][DL] bf16, normalised
-  float* part_lse;            // [records][H]
+  uint16_t* part_o;           // [2 * n_pairs][H][DL] bf16, normalised pieces
+  float* part_lse;            // [2 * n_pairs][2 (CTA of the pair)][H]
   int32_t* status;
   uint64_t wait_ns;           // limit of every bounded in-kernel wait
 };
 
 struct CombineKernelParams {
   int BJ, H, DL;
-  int tiles_per_q, n_pairs, segs_per_q, max_slots;
+  int tiles_per_q, n_pairs;
   long long total_tiles;
   const uint16_t* part_o;
   const float* part_lse;

@@ -51,18 +51,18 @@ constexpr int kPvWarp = 17;     // O += P . C issuer
 // warps 0-3 softmax + epilogue, 4-7 q loader + partial-logit exchange, 8-15 gather, 16 MMA
 constexpr int kAttnThreads = 576;
 // Registers per thread after the split.  The block is launched with kLaunchRegs x 576
-// registers (ptxas' allocation for 576 threads); the softmax warpgroup takes 152 (a tile of
-// fp32 logits), the exchange warpgroup 104, the two gather warpgroups give back down to 64 and
-// the two MMA warps keep the launch value.  The sum stays within the launch allocation, so
-// setmaxnreg.inc never waits for registers that are not there.
+// registers (ptxas' allocation for 576 threads); the softmax warpgroup takes 168 (a tile of
+// fp32 logits and their TMEM loads), the exchange warpgroup 88, the two gather warpgroups give
+// back down to 64 and the two MMA warps keep the launch value.  The sum stays within the launch
+// allocation, so setmaxnreg.inc never waits for registers that are not there.
 constexpr int kLaunchRegs = 96;
-constexpr int kSoftmaxRegs = 152;
-constexpr int kExchangeRegs = 104;
+constexpr int kSoftmaxRegs = 168;
+constexpr int kExchangeRegs = 88;
 constexpr int kGatherRegs = 64;
 static_assert(128 * kSoftmaxRegs + 256 * kGatherRegs + 128 * kExchangeRegs + 64 * kLaunchRegs <=
                   kAttnThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
-constexpr int kStages = 3;          // latent-row tiles in flight per CTA
+constexpr int kStages = 4;          // latent-row tiles in flight per CTA
 constexpr int kRopeSlots = 2;       // their rope parts (read by S = Q . C^T only) in flight
 constexpr int kRows = kAttnTileRows;
 
@@ -91,12 +91,10 @@ struct AttnLayout<512, 64> {
   }
   // FP8 main cache (one byte per element, one fp32 scale per 128-element block of the row):
   // CTA r's 16-element code pieces are 16 latent ones from element 256 r and 2 rope ones from
-  // element 512 + 32 r; its scales are those of blocks 2r, 2r+1 (latent) and 4 (rope)
-  static constexpr int kLatPieces8 = 16, kMaxRopePieces8 = 2, kScalesPerRow = 3, kRopeCodeBytes = 32;
+  // element 512 + 32 r (a piece's scale is that of block element / 128 of the row)
+  static constexpr int kLatPieces8 = 16, kMaxRopePieces8 = 2, kRopeCodeBytes = 32;
   __device__ static int rope_pieces8(int) { return 2; }
   __device__ static int piece_src8(int r, int k) { return k < 16 ? 256 * r + 16 * k : 512 + 32 * r + 16 * (k - 16); }
-  __device__ static int piece_scale8(int k) { return k < 16 ? k >> 3 : 2; }
-  __device__ static int scale_blk8(int r, int which) { return which < 2 ? 2 * r + which : 4; }
 };
 
 template <>
@@ -117,11 +115,9 @@ struct AttnLayout<64, 16> {
   }
   // FP8 main cache: 2 latent code pieces from element 32 r, and CTA 0's one rope piece (element
   // 64); the 80-element row is one scale block
-  static constexpr int kLatPieces8 = 2, kMaxRopePieces8 = 1, kScalesPerRow = 1, kRopeCodeBytes = 16;
+  static constexpr int kLatPieces8 = 2, kMaxRopePieces8 = 1, kRopeCodeBytes = 16;
   __device__ static int rope_pieces8(int r) { return r == 0 ? 1 : 0; }
   __device__ static int piece_src8(int r, int k) { return k < 2 ? 32 * r + 16 * k : 64; }
-  __device__ static int piece_scale8(int) { return 0; }
-  __device__ static int scale_blk8(int, int) { return 0; }
 };
 
 // TMEM columns: O [0, kPvN), two logit buffers of kRows fp32 columns, then the CTA's latent
@@ -149,14 +145,12 @@ struct AttnSmem {
   static constexpr uint32_t kOffR = kOffC + kStages * kCStageBytes;
   // P (bf16, 128 heads x kRows, 128B-swizzled K-major): the A operand of P . C
   static constexpr uint32_t kOffP = (kOffR + kRopeSlots * kCRopeBytes + 1023u) & ~1023u;
-  // peer logits, fp16, two tiles: the peer's exchange warps fill one while this CTA's softmax
-  // reads the other
+  // the peer's partial logits of two tiles, int16 with one power-of-two scale per head: the
+  // peer's exchange warps fill one buffer while this CTA's softmax reads the other
   static constexpr uint32_t kSxBytes = kRows * 128 * 2;
   static constexpr uint32_t kOffSx = kOffP + 128 * kRows * 2;
-  // this CTA's own logits, fp16, two tiles: the exchange warps copy them out of TMEM so that a
-  // logit buffer is free for the next product as soon as they have read it
-  static constexpr uint32_t kOffStash = kOffSx + 2 * kSxBytes;
-  static constexpr uint32_t kOffRows = kOffStash + 2 * kRows * 128 * 2;
+  static constexpr uint32_t kOffSxExp = kOffSx + 2 * kSxBytes;          // [2][128] int32 exponents
+  static constexpr uint32_t kOffRows = kOffSxExp + 2 * 128 * 4;
   // per unit (double-buffered): physical cache row of each Top-K entry, validity bits, and
   // each gather warp's lowest position of a -1 entry
   static constexpr uint32_t kOffMask = kOffRows + 2 * kAttnMaxSplitRows * 4;
@@ -171,8 +165,7 @@ struct AttnSmem {
 struct AttnBarriers {
   uint64_t c_full[kStages], c_empty[kStages];   // a tile's rows landed / latent stage free
   uint64_t r_empty[kRopeSlots];                 // rope slot free (its S = Q . C^T done)
-  uint64_t s_full[2], s_empty[2];   // logits ready in TMEM / read by the exchange warps
-  uint64_t own_ready[2], own_free[2];   // own fp16 logits stashed / read by the softmax
+  uint64_t s_full[2], s_empty[2];   // logits ready in TMEM / read by the exchange and softmax warps
   uint64_t p_full;                  // all softmax threads wrote P (waited by the P . C issuer)
   uint64_t p_empty;                 // P . C of the previous tile done (P buffer and O free)
   uint64_t epi_sync;                // all softmax threads are past the unit's last tile
@@ -195,20 +188,16 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
-  uint32_t r;
-  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-  return r;
-}
+// The partial logits cross to the peer CTA as 16-bit integers with one power-of-two scale per
+// head and tile: x = round(v 2^e), |x| < 2^14.  fma(v, 2^e, kMagic) puts x + 2^15 in the low 16
+// bits of an fp32 in [2^23, 2^24) (where the spacing is 1, so the rounding is to the nearest
+// integer), and the receiver rebuilds 2^23 + x + 2^15 from those bits and removes kMagic exactly.
+constexpr float kMagic = 8421376.0f;   // 2^23 + 2^15
 
-// a + (fp32) the two fp16 halves of h: {a_lo + lo(h), a_hi + hi(h)}, one rounding each
-__device__ __forceinline__ void add_f16x2_to_f32(uint32_t h, float& lo, float& hi) {
-  asm("{\n\t.reg .b16 l16, h16;\n\t"
-      "mov.b32 {l16, h16}, %2;\n\t"
-      "add.rn.f32.f16 %0, l16, %0;\n\t"
-      "add.rn.f32.f16 %1, h16, %1;\n\t}"
-      : "+f"(lo), "+f"(hi)
-      : "r"(h));
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
 }
 
 __device__ __forceinline__ void cp_async16_hint(uint32_t dst, const void* src, uint64_t policy) {
@@ -225,68 +214,38 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
 }
 
 // The work of a call is the flat list of (query, 64-row tile) pairs, query-major with
-// tiles_per_q tiles per query, split evenly between the CTA pairs: pair c takes global tiles
-// [c G / C, (c + 1) G / C).  A unit is the part of that range inside one query and inside one
-// run of 32 tiles of it (at most kAttnMaxSplitRows Top-K entries, the size of the row table).
-// A query covered by one unit gets its output written directly; otherwise every unit writes a
-// partial result (normalised O and log-sum-exp) into a record of the workspace, and
-// combine_kernel merges a query's records.  Records: with at most 32 tiles per query only the
-// queries that straddle a pair boundary have any (at most C - 1 of them), numbered in order;
-// with more, every query has max_slots of them.  Within a query, slot (c - first pair) *
-// segs_per_q + (32-tile run index counted from where pair c starts in the query).
+// tiles_per_q <= 32 tiles per query, split evenly between the CTA pairs: pair c takes global
+// tiles [c G / C, (c + 1) G / C).  A unit is the part of that range inside one query.  A query
+// covered by one unit gets its output written directly; a query that straddles a pair
+// boundary is computed in pieces, each written as a partial result (normalised O and the
+// log-sum-exp of each CTA of the pair) into a record of the workspace, and combine_kernel
+// merges them.  Only a pair's first and last unit can be pieces, so pair c owns records 2c
+// (its first unit) and 2c + 1 (its last unit, when that is another unit).
 __device__ __forceinline__ long long attn_pair_start(int c, int C, long long G) { return (long long)c * G / C; }
-
-__device__ __forceinline__ int attn_pair_of_tile(long long g, int C, long long G) {
-  return (int)(((g + 1) * C - 1) / G);
-}
 
 struct AttnUnit {
   int bj;        // query row (b * J + j)
   int row0;      // first Top-K entry of the unit
   int nrows;     // entries in the unit (rows of the last tile may be absent)
-  long long rec; // partial-result record, or -1 when the unit writes the final output
+  int rec;       // partial-result record, or -1 when the unit writes the final output
 };
 
-// Record number of query bj's slot `slot` (the host sizes the workspace the same way).
-__device__ __forceinline__ long long attn_record(int TQ, int C, long long G, int max_slots, int bj, int slot) {
-  if (TQ > 32) return (long long)bj * max_slots + slot;
-  // rank of bj among the queries that contain a pair boundary strictly inside them
-  const long long q0 = (long long)bj * TQ;
-  int n = 0, prevq = -1;
-  for (int c = 1; c < C; ++c) {
-    const long long g = attn_pair_start(c, C, G);
-    if (g >= q0) break;
-    const int q = (int)(g / TQ);
-    if (g % TQ != 0 && q != prevq) {
-      ++n;
-      prevq = q;
-    }
-  }
-  return (long long)n * max_slots + slot;
-}
+struct AttnRange {
+  long long g0, g1;   // this pair's global tiles
+};
 
-// Next unit of pair `c` from global tile `cursor` (advanced past the unit); false when done.
-__device__ __forceinline__ bool attn_next_unit(const AttnKernelParams& p, int c, long long& cursor, AttnUnit& u) {
-  const long long G = p.total_tiles;
-  const int C = p.n_pairs;
-  const long long g1 = attn_pair_start(c + 1, C, G);
-  if (cursor >= g1) return false;
+// Next unit of the pair from global tile `cursor` (advanced past the unit); false when done.
+__device__ __forceinline__ bool attn_next_unit(const AttnKernelParams& p, int c, const AttnRange& rg,
+                                               long long& cursor, AttnUnit& u) {
+  if (cursor >= rg.g1) return false;
   const int TQ = p.tiles_per_q;
   u.bj = (int)(cursor / TQ);
   const long long q0 = (long long)u.bj * TQ;
-  const long long seg_end = q0 + (((cursor - q0) >> 5) + 1) * 32;
-  const long long tb = min(min(g1, q0 + TQ), seg_end);
+  const long long tb = min(rg.g1, q0 + TQ);
   u.row0 = (int)(cursor - q0) * kAttnTileRows;
   u.nrows = min(p.K, (int)(tb - q0) * kAttnTileRows) - u.row0;
-  const int first = attn_pair_of_tile(q0, C, G);
-  const int last = attn_pair_of_tile(q0 + TQ - 1, C, G);
-  if (first == last && TQ <= 32) {
-    u.rec = -1;
-  } else {
-    const long long a = max(q0, attn_pair_start(c, C, G));
-    const int slot = (c - first) * p.segs_per_q + (int)(((cursor - q0) >> 5) - ((a - q0) >> 5));
-    u.rec = attn_record(TQ, C, G, p.max_slots, u.bj, slot);
-  }
+  const bool piece = q0 < rg.g0 || q0 + TQ > rg.g1;
+  u.rec = piece ? 2 * c + (cursor == rg.g0 ? 0 : 1) : -1;
   cursor = tb;
   return true;
 }
@@ -321,7 +280,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t rank = cluster_ctarank();
   const uint32_t peer = rank ^ 1u;
   const int cluster_id = blockIdx.x >> 1;
-  const int n_clusters = gridDim.x >> 1;
   const bool rope = Lay::has_rope((int)rank);
   const int DC = p.DL + p.DR;
 
@@ -337,9 +295,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     for (int s = 0; s < kRopeSlots; ++s) mbar_init(&sb->r_empty[s], 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sb->s_full[s], 1);
-      mbar_init(&sb->s_empty[s], 128);         // exchange threads
-      mbar_init(&sb->own_ready[s], 128);
-      mbar_init(&sb->own_free[s], 128);
+      mbar_init(&sb->s_empty[s], 256);         // exchange and softmax threads
       mbar_init(&sb->tab_full[s], kProducerWarps * 32);
       mbar_init(&sb->tab_free[s], 128 + 128 + 2);   // softmax, exchange and both MMA threads
     }
@@ -430,9 +386,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     int it = 0, u_it = 0, q_issued = 0;
     bool ok = true;
     bool waited = false;
-    long long cursor = (long long)cluster_id * p.total_tiles / p.n_pairs;
+    const AttnRange rg{attn_pair_start(cluster_id, p.n_pairs, p.total_tiles),
+                      attn_pair_start(cluster_id + 1, p.n_pairs, p.total_tiles)};
+    long long cursor = rg.g0;
     AttnUnit un;
-    if (cursor < (long long)(cluster_id + 1) * p.total_tiles / p.n_pairs) {
+    if (cursor < rg.g1) {
       // While the previous kernel still runs: touch every cache page of the first unit's
       // sequence (address translation and the page-table row warm up before the gather)
       const int b = (int)(cursor / p.tiles_per_q) / p.J;
@@ -446,7 +404,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           asm volatile("prefetch.global.L2 [%0];" ::"l"(kv + ((size_t)pg * p.P * DC + (size_t)rank * (p.DL / 2)) * (KV8 ? 1 : 2)));
       }
     }
-    while (ok && attn_next_unit(p, cluster_id, cursor, un)) {
+    while (ok && attn_next_unit(p, cluster_id, rg, cursor, un)) {
       const int bj = un.bj;
       const int b = bj / p.J;
       const int L = p.seq_lens[b];
@@ -636,9 +594,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint32_t qr_base = smem_u32(smem + Sm::kOffQ);
       int it = 0, u_it = 0;
       bool ok = true;
-      long long cursor = (long long)cluster_id * p.total_tiles / p.n_pairs;
+      const AttnRange rg{attn_pair_start(cluster_id, p.n_pairs, p.total_tiles),
+                      attn_pair_start(cluster_id + 1, p.n_pairs, p.total_tiles)};
+    long long cursor = rg.g0;
       AttnUnit un;
-      for (; ok && attn_next_unit(p, cluster_id, cursor, un); ++u_it) {
+      for (; ok && attn_next_unit(p, cluster_id, rg, cursor, un); ++u_it) {
         const int buf = u_it & 1;
         if (!mbar_wait(&sb->tab_full[buf], (uint32_t)(u_it >> 1) & 1u, wc)) { ok = false; break; }
         const int ntiles = (unit_tiles(buf) + kRows - 1) / kRows;
@@ -689,9 +649,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint32_t p_base = smem_u32(smem + Sm::kOffP);
       int it = 0, u_it = 0;
       bool ok = true;
-      long long cursor = (long long)cluster_id * p.total_tiles / p.n_pairs;
+      const AttnRange rg{attn_pair_start(cluster_id, p.n_pairs, p.total_tiles),
+                      attn_pair_start(cluster_id + 1, p.n_pairs, p.total_tiles)};
+    long long cursor = rg.g0;
       AttnUnit un;
-      for (; ok && attn_next_unit(p, cluster_id, cursor, un); ++u_it) {
+      for (; ok && attn_next_unit(p, cluster_id, rg, cursor, un); ++u_it) {
         const int buf = u_it & 1;
         if (!mbar_wait(&sb->tab_full[buf], (uint32_t)(u_it >> 1) & 1u, wc)) { ok = false; break; }
         const int ntiles = (unit_tiles(buf) + kRows - 1) / kRows;
@@ -721,18 +683,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   } else if (warp >= kFirstExchangeWarp && warp < kFirstExchangeWarp + 4) {
     // ---------------------------------------------------------------- q loader + exchange
     // Per unit: writes this CTA's latent half of every head's query row into TMEM (the A
-    // operand of Q . C^T).  Per tile: reads this CTA's partial logits from TMEM, rounds them
-    // to fp16 (scaled to base 2) and pushes them into the peer CTA's exchange buffer.
+    // operand of Q . C^T).  Per tile: reads this CTA's partial logits from TMEM and pushes them,
+    // scaled to base 2 and encoded as int16 with one power-of-two scale per head (relative
+    // error at most 2^-15 of the head's largest partial), into the peer CTA's exchange buffer.
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kExchangeRegs));
     const int quad = warp & 3;
     const int h = quad * 32 + lane;
     const uint32_t lane_addr = tmem_base + ((uint32_t)(quad * 32) << 16);
     const uint32_t sx_peer = mapa_shared(smem_u32(smem + Sm::kOffSx), peer);
+    const uint32_t sxexp_peer = mapa_shared(smem_u32(smem + Sm::kOffSxExp), peer);
     int s_it = 0, u_it = 0;
     bool ok = true;
-    long long cursor = (long long)cluster_id * p.total_tiles / p.n_pairs;
+    const AttnRange rg{attn_pair_start(cluster_id, p.n_pairs, p.total_tiles),
+                      attn_pair_start(cluster_id + 1, p.n_pairs, p.total_tiles)};
+    long long cursor = rg.g0;
     AttnUnit un;
-    for (; ok && attn_next_unit(p, cluster_id, cursor, un); ++u_it) {
+    for (; ok && attn_next_unit(p, cluster_id, rg, cursor, un); ++u_it) {
       const int bj = un.bj;
       const int buf = u_it & 1;
       {
@@ -774,34 +740,43 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const uint32_t scol = lane_addr + Tm::kS + sbuf * kRows;
         if (!mbar_wait_warp(&sb->s_full[sbuf], (uint32_t)(s_it >> 1) & 1u, wc)) { ok = false; break; }
         tc_fence_after();
-        uint32_t own[kRows / 2];
+        // this CTA's partial logits of head h (base 2) as int16 with one power-of-two scale
+        uint32_t enc[kRows / 2];
+        int e;
         {
           uint32_t r[4][16];   // the whole tile's row in one TMEM wait
 #pragma unroll
           for (int c = 0; c < 4; ++c) tmem_ld16(scol + c * 16, r[c]);
           tmem_wait_ld();
+          float amax = 0.0f;
 #pragma unroll
           for (int c = 0; c < 4; ++c)
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-              own[c * 8 + i] = pack_f16x2(__uint_as_float(r[c][2 * i]) * p.scale_log2,
-                                          __uint_as_float(r[c][2 * i + 1]) * p.scale_log2);
+            for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(__uint_as_float(r[c][i])));
+          amax *= fabsf(p.scale_log2);
+          // e with amax 2^e < 2^14: amax < 2^E for E = (biased exponent of amax) - 126
+          const int E = (int)((__float_as_uint(amax) >> 23) & 0xffu) - 126;
+          e = amax > 0.0f ? min(max(14 - E, -100), 100) : 0;
+          const float sc = p.scale_log2 * __uint_as_float((uint32_t)(127 + e) << 23);
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float y0 = fmaf(__uint_as_float(r[c][2 * i]), sc, kMagic);
+              const float y1 = fmaf(__uint_as_float(r[c][2 * i + 1]), sc, kMagic);
+              enc[c * 8 + i] = prmt(__float_as_uint(y0), __float_as_uint(y1), 0x5410u);
+            }
         }
         tc_fence_before();
         mbar_arrive(&sb->s_empty[sbuf]);   // our reads of these logits are done
-        // own fp16 logits for our softmax (the same values the peer receives)
-        if (!mbar_wait_warp(&sb->own_free[sbuf], ((uint32_t)(s_it >> 1) & 1u) ^ 1u, wc)) { ok = false; break; }
-#pragma unroll
-        for (int g = 0; g < kRows / 8; ++g)
-          st_shared_v4(smem_u32(smem + Sm::kOffStash + sbuf * (kRows * 128 * 2) + (g * 128 + h) * 16),
-                       own[4 * g], own[4 * g + 1], own[4 * g + 2], own[4 * g + 3]);
-        mbar_arrive(&sb->own_ready[sbuf]);
         if (!mbar_wait_warp<true>(&sb->sx_free[sbuf], ((uint32_t)(s_it >> 1) & 1u) ^ 1u, wc)) { ok = false; break; }
 #pragma unroll
         for (int g = 0; g < kRows / 8; ++g)
           asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sx_peer + sbuf * Sm::kSxBytes + (uint32_t)((g * 128 + h) * 16)),
-                       "r"(own[4 * g]), "r"(own[4 * g + 1]), "r"(own[4 * g + 2]), "r"(own[4 * g + 3])
+                       "r"(enc[4 * g]), "r"(enc[4 * g + 1]), "r"(enc[4 * g + 2]), "r"(enc[4 * g + 3])
                        : "memory");
+        asm volatile("st.shared::cluster.b32 [%0], %1;" ::"r"(sxexp_peer + (uint32_t)((sbuf * 128 + h) * 4)), "r"(e)
+                     : "memory");
         mbar_arrive_cluster(&sb->sx_ready[sbuf], peer);
       }
     }
@@ -814,10 +789,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     int s_it = 0, u_it = 0, o_it = 0, e_it = 0;
     bool ok = true;
 
-    long long cursor = (long long)cluster_id * p.total_tiles / p.n_pairs;
+    const AttnRange rg{attn_pair_start(cluster_id, p.n_pairs, p.total_tiles),
+                      attn_pair_start(cluster_id + 1, p.n_pairs, p.total_tiles)};
+    long long cursor = rg.g0;
     AttnUnit un;
     int last_sbuf = 0;
-    for (; ok && attn_next_unit(p, cluster_id, cursor, un); ++u_it) {
+    for (; ok && attn_next_unit(p, cluster_id, rg, cursor, un); ++u_it) {
       const int bj = un.bj;
       const int buf = u_it & 1;
       if (!mbar_wait_warp(&sb->tab_full[buf], (uint32_t)(u_it >> 1) & 1u, wc)) { ok = false; break; }
@@ -831,27 +808,41 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         uint64_t valid = ((uint64_t)mt[2 * t + 1] << 32) | mt[2 * t];
         const int live = first_neg - t * kRows;            // rows past the first -1 are padding
         if (live < kRows) valid &= (1ull << live) - 1ull;
-        if (!mbar_wait_warp(&sb->own_ready[sbuf], (uint32_t)(s_it >> 1) & 1u, wc)) { ok = false; break; }
+        // logits of tile t (base 2) = this CTA's exact fp32 partial (from TMEM) + the peer's
+        // decoded int16 partial, one rounding
+        if (!mbar_wait_warp(&sb->s_full[sbuf], (uint32_t)(s_it >> 1) & 1u, wc)) { ok = false; break; }
+        tc_fence_after();
+        {
+          uint32_t r[4][16];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) tmem_ld16(lane_addr + Tm::kS + sbuf * kRows + c * 16, r[c]);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int i = 0; i < 16; ++i) s[16 * c + i] = __uint_as_float(r[c][i]);
+        }
+        tc_fence_before();
+        mbar_arrive(&sb->s_empty[sbuf]);   // our read of this CTA's partial is done
         if (!mbar_wait_warp<true>(&sb->sx_ready[sbuf], (uint32_t)(s_it >> 1) & 1u, wc)) { ok = false; break; }
         last_sbuf = sbuf;
-        // logits of tile t (base 2) = own fp16 partial + the peer's fp16 partial: both CTAs add
-        // the same two values, so their logits agree bit for bit
+        {
+          const int e = *reinterpret_cast<const int*>(smem + Sm::kOffSxExp + (sbuf * 128 + h) * 4);
+          const float dn = __uint_as_float((uint32_t)(127 - e) << 23);
+          const float bias = -kMagic * dn;
 #pragma unroll
-        for (int g = 0; g < kRows / 8; ++g) {
-          const uint4 ov = *reinterpret_cast<const uint4*>(smem + Sm::kOffStash + sbuf * (kRows * 128 * 2) + (g * 128 + h) * 16);
-          const uint4 pv4 = *reinterpret_cast<const uint4*>(smem + Sm::kOffSx + sbuf * Sm::kSxBytes + (g * 128 + h) * 16);
-          const uint32_t o4[4] = {ov.x, ov.y, ov.z, ov.w};
-          const uint32_t q4[4] = {pv4.x, pv4.y, pv4.z, pv4.w};
+          for (int g = 0; g < kRows / 8; ++g) {
+            const uint4 pv4 = *reinterpret_cast<const uint4*>(smem + Sm::kOffSx + sbuf * Sm::kSxBytes + (g * 128 + h) * 16);
+            const uint32_t q4[4] = {pv4.x, pv4.y, pv4.z, pv4.w};
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            float lo = 0.0f, hi = 0.0f;
-            add_f16x2_to_f32(o4[i], lo, hi);   // exact: fp16 -> fp32
-            add_f16x2_to_f32(q4[i], lo, hi);   // one rounding
-            s[8 * g + 2 * i] = lo;
-            s[8 * g + 2 * i + 1] = hi;
+            for (int i = 0; i < 4; ++i) {
+              const float f0 = __uint_as_float(prmt(q4[i], 0x4B000000u, 0x7610u));
+              const float f1 = __uint_as_float(prmt(q4[i], 0x4B000000u, 0x7632u));
+              s[8 * g + 2 * i] = fmaf(s[8 * g + 2 * i], p.scale_log2, fmaf(f0, dn, bias));
+              s[8 * g + 2 * i + 1] = fmaf(s[8 * g + 2 * i + 1], p.scale_log2, fmaf(f1, dn, bias));
+            }
           }
         }
-        mbar_arrive(&sb->own_free[sbuf]);
         // the peer may refill the exchange buffer (the logit values read above are already in
         // registers); after the unit's last tile the buffer first serves the epilogue
         if (t + 1 < ntiles) mbar_arrive_cluster_relaxed(&sb->sx_free[sbuf], peer);
@@ -932,7 +923,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // per round in a 128B-swizzled 4 KB slice, then writes whole 128-byte runs of 4 heads per
       // instruction
       const bool partial = un.rec >= 0;
-      uint16_t* obase = (partial ? p.part_o + un.rec * p.H * p.DL : p.out + (long long)bj * p.H * p.DL) +
+      uint16_t* obase = (partial ? p.part_o + (long long)un.rec * p.H * p.DL : p.out + (long long)bj * p.H * p.DL) +
                         rank * Lay::kPvN;
       if (ntiles > 0) {
         // every softmax warp has read the last tile's peer logits before any slice is reused
@@ -974,9 +965,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int c = 0; c < Lay::kPvN; c += 8)
           *reinterpret_cast<uint4*>(obase + (long long)h * p.DL + c) = make_uint4(0, 0, 0, 0);
       }
-      if (real_head && rank == 0) {
-        if (partial) p.part_lse[un.rec * p.H + h] = lse;
-        else if (p.lse) p.lse[(long long)bj * p.H + h] = lse;
+      if (real_head) {
+        // a piece records the log-sum-exp of each CTA of the pair (their logits differ in the
+        // last bits: each adds its own exact partial to the peer's decoded one)
+        if (partial) p.part_lse[((long long)un.rec * 2 + rank) * p.H + h] = lse;
+        else if (p.lse && rank == 0) p.lse[(long long)bj * p.H + h] = lse;
       }
       if (ntiles > 0) {
         __syncwarp();
@@ -994,51 +987,52 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
 }
 
-// Log-sum-exp merge of the partial results of the queries whose units were spread over several
-// records: 256 threads per CTA, 8 output dims per thread (16-byte loads of the bf16 partials),
-// DL/8 threads per (query row, head).  Queries covered by a single unit were written directly.
+// Log-sum-exp merge of the pieces of the queries that straddle a CTA-pair boundary.  One
+// (boundary, head) per DL/8 threads, 8 output dims per thread (16-byte loads of the bf16
+// partials); the first boundary inside a query merges all of that query's pieces: the last unit
+// of the pair before it, then the first unit of every pair that starts inside the query.
 constexpr int kCombineThreads = 256;
 
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineKernelParams p) {
   pdl_launch_dependents();  // the dependent waits for this grid's completion before its loads
   pdl_wait_primary();
-  const int tph = p.DL / 8;                               // threads per (row, head)
-  const long long bjh = (long long)blockIdx.x * (kCombineThreads / tph) + threadIdx.x / tph;
+  const int tph = p.DL / 8;                               // threads per (boundary, head)
+  const long long bh = (long long)blockIdx.x * (kCombineThreads / tph) + threadIdx.x / tph;
   const int d8 = (threadIdx.x % tph) * 8;
-  const long long n_bjh = (long long)p.BJ * p.H;
-  if (bjh >= n_bjh) return;
-  const int bj = (int)(bjh / p.H), h = (int)(bjh - (long long)bj * p.H);
+  if (bh >= (long long)(p.n_pairs - 1) * p.H) return;
+  const int c = 1 + (int)(bh / p.H), h = (int)(bh % p.H);
   const int TQ = p.tiles_per_q, C = p.n_pairs;
   const long long G = p.total_tiles;
-  const long long q0 = (long long)bj * TQ;
-  const int first = attn_pair_of_tile(q0, C, G);
-  const int last = attn_pair_of_tile(q0 + TQ - 1, C, G);
-  if (first == last && TQ <= 32) return;
-  const long long rec0 = attn_record(TQ, C, G, p.max_slots, bj, 0);
-  // the query's slots: for each pair c in [first, last], one per 32-tile run it covers
+  const long long g = attn_pair_start(c, C, G);
+  const long long q0 = g / TQ * TQ;
+  if (g == q0) return;                                   // a boundary at a query start
+  if (attn_pair_start(c - 1, C, G) > q0) return;         // an earlier boundary owns this query
+  const int bj = (int)(q0 / TQ);
+  const int rank = d8 >= p.DL / 2 ? 1 : 0;               // the CTA that computed these dims
   float mx = -INFINITY, wsum = 0.0f, o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  int slots[4];
-  int ns = 0;
-  auto merge = [&](int n) {
-    // the log-sum-exps and partial vectors of up to four slots are loaded together, so a
-    // merge of up to four records waits for one memory latency
+  int recs[4];
+  int n = 0;
+  auto merge = [&]() {
+    // the log-sum-exps and partial vectors of up to four pieces are loaded together, so a
+    // merge of up to four pieces waits for one memory latency
     float ls[4];
     uint4 v[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const bool in = i < n;
-      const long long e = rec0 + (in ? slots[i] : 0);
-      ls[i] = in ? p.part_lse[e * p.H + h] : -INFINITY;
+      const long long e = in ? recs[i] : 0;
+      ls[i] = in ? p.part_lse[(e * 2 + rank) * p.H + h] : -INFINITY;
       v[i] = in ? ld_nc_v4(p.part_o + (e * p.H + h) * p.DL + d8) : make_uint4(0, 0, 0, 0);
     }
+    n = 0;
     float m_new = mx;
 #pragma unroll
     for (int i = 0; i < 4; ++i) m_new = fmaxf(m_new, ls[i]);
-    if (m_new == -INFINITY) return;   // every record so far is empty
-    const float c = mx == -INFINITY ? 0.0f : expf(mx - m_new);
-    wsum *= c;
+    if (m_new == -INFINITY) return;   // every piece so far is empty
+    const float cf = mx == -INFINITY ? 0.0f : expf(mx - m_new);
+    wsum *= cf;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) o[j] *= c;
+    for (int j = 0; j < 8; ++j) o[j] *= cf;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const float wgt = ls[i] == -INFINITY ? 0.0f : expf(ls[i] - m_new);
@@ -1052,25 +1046,19 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineK
     }
     mx = m_new;
   };
-  for (int c = first; c <= last; ++c) {
-    const long long a = max(q0, attn_pair_start(c, C, G));
-    const long long b = min(q0 + TQ, attn_pair_start(c + 1, C, G));
-    if (b <= a) continue;
-    const int nseg = (int)(((b - 1 - q0) >> 5) - ((a - q0) >> 5)) + 1;
-    for (int k = 0; k < nseg; ++k) {
-      slots[ns++] = (c - first) * p.segs_per_q + k;
-      if (ns == 4) {
-        merge(4);
-        ns = 0;
-      }
-    }
+  // pair c - 1 holds the query's first piece: its last unit, or its only one when it starts at q0
+  recs[n++] = 2 * (c - 1) + (attn_pair_start(c - 1, C, G) == q0 ? 0 : 1);
+  for (int cc = c; cc < C && attn_pair_start(cc, C, G) < q0 + TQ; ++cc) {
+    recs[n++] = 2 * cc;   // every later pair's first unit
+    if (n == 4) merge();
   }
-  if (ns > 0) merge(ns);
+  if (n > 0) merge();
   const float inv = wsum > 0.0f ? 1.0f / wsum : 0.0f;
-  *reinterpret_cast<uint4*>(p.out + bjh * p.DL + d8) =
+  const long long row = (long long)bj * p.H + h;
+  *reinterpret_cast<uint4*>(p.out + row * p.DL + d8) =
       make_uint4(pack_bf16x2(o[0] * inv, o[1] * inv), pack_bf16x2(o[2] * inv, o[3] * inv),
                  pack_bf16x2(o[4] * inv, o[5] * inv), pack_bf16x2(o[6] * inv, o[7] * inv));
-  if (d8 == 0 && p.lse) p.lse[bjh] = wsum > 0.0f ? mx + logf(wsum) : -INFINITY;
+  if (d8 == 0 && p.lse) p.lse[row] = wsum > 0.0f ? mx + logf(wsum) : -INFINITY;
 }
 
 template <int DL, int DR, bool KV8>
@@ -1136,7 +1124,7 @@ cudaError_t launch_combine(const CombineKernelParams& p, bool pdl, cudaStream_t 
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   const long long per_cta = kCombineThreads / (p.DL / 8);
-  cfg.gridDim = dim3((unsigned)(((long long)p.BJ * p.H + per_cta - 1) / per_cta), 1, 1);
+  cfg.gridDim = dim3((unsigned)(((long long)(p.n_pairs - 1) * p.H + per_cta - 1) / per_cta), 1, 1);
   cfg.blockDim = dim3(kCombineThreads, 1, 1);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;

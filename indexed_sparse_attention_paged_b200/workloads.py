@@ -132,9 +132,10 @@ def make_inputs(wl: Workload, seed: Optional[int] = None, *, batch: Optional[int
 
 def fp8_main_cache(inputs: dict, seed: Optional[int] = None, pow2_scales: bool = False) -> dict:
     """The same workload with its main latent cache drawn in the FP8 format instead: e4m3 codes
-    (N(0, 16^2) samples cast to e4m3, saturating) and one fp32 scale per 128-element block of each
-    row (uniform in [1/64, 1/8), or a power of two 2^e with e uniform in [-6, -3]).  The decoded
-    values have about the spread of the bf16 cache's N(0, 1)."""
+    (N(0, 100^2) samples cast to e4m3, saturating at 448, so that the codes use the format's
+    range) and one fp32 scale per 128-element block of each row (uniform in [1/110, 1/90), or a
+    power of two 2^e with e uniform in [-7, -6]).  The decoded values have about the spread of
+    the bf16 cache's N(0, 1)."""
     wl = inputs["workload"]
     seed = 2000 + wl.number if seed is None else seed
     gen = torch.Generator().manual_seed(seed)
@@ -144,11 +145,11 @@ def fp8_main_cache(inputs: dict, seed: Optional[int] = None, pow2_scales: bool =
     flat = codes.view(pages * P, DC)
     for s0 in range(0, pages * P, 1 << 16):
         e = min(pages * P, s0 + (1 << 16))
-        flat[s0:e] = (torch.randn((e - s0, DC), generator=gen) * 16.0).clamp(-448.0, 448.0).to(torch.float8_e4m3fn)
+        flat[s0:e] = (torch.randn((e - s0, DC), generator=gen) * 100.0).clamp(-448.0, 448.0).to(torch.float8_e4m3fn)
     if pow2_scales:
-        scale = torch.pow(2.0, _randint(gen, -6, -3, (pages, P, nblk)).to(torch.float32))
+        scale = torch.pow(2.0, _randint(gen, -7, -6, (pages, P, nblk)).to(torch.float32))
     else:
-        scale = torch.rand((pages, P, nblk), generator=gen) * (1.0 / 8 - 1.0 / 64) + 1.0 / 64
+        scale = torch.rand((pages, P, nblk), generator=gen) * (1.0 / 90 - 1.0 / 110) + 1.0 / 110
     out = dict(inputs)
     out["kv_cache"] = codes
     out["kv_scale"] = scale

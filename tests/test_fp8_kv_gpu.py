@@ -2,7 +2,11 @@
 128-element block of each row) against the oracle's fp64 dequantise-then-attend, and, with
 power-of-two scales, bit-for-bit equality with the bf16 path on a bf16 cache holding the decoded
 values (the dequantised element is then exact in bf16, so both paths feed identical operands to
-the tensor cores)."""
+the tensor cores).
+
+Tolerance: the kernel rounds each decoded element (code x block scale) once to bf16 before the
+products, a relative error of at most 2^-9; the output is a convex combination of the selected
+rows, so that rounding moves it by at most 2^-9 max|c| on top of the bf16 path's 1e-2."""
 import numpy as np
 import pytest
 import torch
@@ -15,6 +19,13 @@ pytestmark = pytest.mark.gpu
 
 DEV = "cuda:0"
 ATOL = 1e-2
+
+
+def fp8_tol(h):
+    """1e-2 plus the bf16 rounding of the largest decoded element (see the module docstring)."""
+    DC = h["kv_cache"].shape[2]
+    dec = h["kv_cache"].float() * h["kv_scale"].repeat_interleave(128, dim=2)[:, :, :DC]
+    return ATOL + 2.0 ** -9 * float(dec.abs().max())
 
 
 def _topk(h, top_k, seed, fill=1.0):
@@ -66,7 +77,7 @@ def test_fp8_main_cache_attention_matches_the_oracle(name):
                                              kv_scale=h["kv_scale"].numpy())
     assert ost == 0
     err = np.abs(out.float().cpu().numpy() - ref).max()
-    assert err <= ATOL, err
+    assert err <= fp8_tol(h), err
     g = lse.cpu().numpy()
     fin = np.isfinite(ref_lse)
     assert np.all(np.isfinite(g) == fin)
@@ -107,4 +118,4 @@ def test_fused_decode_over_an_fp8_main_cache():
     ref, _, _ = oracle.sparse_attend(h["q_attn"], h["kv_cache"], h["page_table"].numpy(), h["seq_lens"].numpy(),
                                      ref_topk, page_size=wl.page_size, d_latent=wl.d_latent,
                                      scale=wl.softmax_scale, kv_scale=h["kv_scale"].numpy())
-    assert np.abs(out.float().cpu().numpy() - ref).max() <= ATOL
+    assert np.abs(out.float().cpu().numpy() - ref).max() <= fp8_tol(h)
