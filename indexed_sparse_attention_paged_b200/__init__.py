@@ -376,13 +376,17 @@ class FusedDecodePlan:
     step is one C-ABI call with no allocation -- what the benchmark times and what a serving loop
     would capture in a CUDA graph."""
 
-    def __init__(self, inputs: dict, device, *, with_lse: bool = True):
+    def __init__(self, inputs: dict, device, *, with_lse: bool = True, out=None, lse=None, topk=None):
         wl = inputs["workload"]
         self.inputs = inputs
         B, J = inputs["batch"], inputs["n_q"]
-        self.topk = torch.empty((B, J, wl.top_k), dtype=torch.int32, device=device)
-        self.out = torch.empty((B, J, wl.attn_heads, wl.d_latent), dtype=torch.bfloat16, device=device)
-        self.lse = torch.empty((B, J, wl.attn_heads), dtype=torch.float32, device=device) if with_lse else None
+        self.topk = topk if topk is not None else torch.empty((B, J, wl.top_k), dtype=torch.int32, device=device)
+        self.out = out if out is not None else torch.empty((B, J, wl.attn_heads, wl.d_latent), dtype=torch.bfloat16,
+                                                           device=device)
+        if lse is not None:
+            self.lse = lse
+        else:
+            self.lse = torch.empty((B, J, wl.attn_heads), dtype=torch.float32, device=device) if with_lse else None
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
         self.ia = index_args(inputs["q_idx"], inputs["w"], inputs["k_cache"], inputs["page_table"],
                              inputs["seq_lens"], top_k=wl.top_k, k_scale=inputs["k_scale"],

@@ -62,6 +62,9 @@ constexpr int kGatherRegs = 64;
 static_assert(128 * kSoftmaxRegs + 256 * kGatherRegs + 128 * kExchangeRegs + 64 * kLaunchRegs <=
                   kAttnThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
+// setmaxnreg.inc may only raise a warp's count and setmaxnreg.dec only lower it
+static_assert(kSoftmaxRegs >= kLaunchRegs && kGatherRegs <= kLaunchRegs && kExchangeRegs <= kLaunchRegs,
+              "the softmax warpgroup grows, the gather and exchange warpgroups shrink");
 constexpr int kStages = 4;          // latent-row tiles in flight per CTA
 constexpr int kRopeSlots = 2;       // their rope parts (read by S = Q . C^T only) in flight
 constexpr int kRows = kAttnTileRows;
@@ -686,7 +689,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // operand of Q . C^T).  Per tile: reads this CTA's partial logits from TMEM and pushes them,
     // scaled to base 2 and encoded as int16 with one power-of-two scale per head (relative
     // error at most 2^-15 of the head's largest partial), into the peer CTA's exchange buffer.
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kExchangeRegs));
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kExchangeRegs));
     const int quad = warp & 3;
     const int h = quad * 32 + lane;
     const uint32_t lane_addr = tmem_base + ((uint32_t)(quad * 32) << 16);

@@ -329,8 +329,19 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_row_kernel(const TopkKern
     }
     if (lane == 31) sh->wtot[wid] = incl;
     __syncthreads();
-    int before = 0;
-    for (int w = 0; w < wid; ++w) before += sh->wtot[w];
+    // keys in the bins of the warps before this one: an exclusive warp scan of the 32 warp
+    // totals (one load and five shuffles instead of a loop over up to 31 totals)
+    int before;
+    {
+      const int wt = sh->wtot[lane];
+      int sc = wt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, sc, o);
+        if (lane >= o) sc += v;
+      }
+      before = __shfl_sync(0xffffffffu, sc - wt, wid);
+    }
     const int ex = before + incl - (c0 + c1);
     if (ex < krem && krem <= ex + c1) {
       sh->sel_prefix = (prefix << widths[pass]) | (uint32_t)(hi_bin + 1);
