@@ -337,7 +337,8 @@ sia_status plan_attend(const sia_attend_args* a, AttendPlan* pl, bool make_maps)
   // the flat (query, 64-row tile) list split evenly over the CTA pairs (see attn_next_unit)
   const long long TQ = (a->top_k + kAttnTileRows - 1) / kAttnTileRows;
   const long long G = bj * TQ;
-  const int C = (int)std::min<long long>(pairs, G);
+  if (G > 0x7fffffffll) return fail(SIA_ERR_UNSUPPORTED, "batch * n_q * ceil(top_k / 64) must fit in int32");
+  const int C = (int)std::min<long long>(std::min(pairs, kAttnMaxPairs), G);
   k.tiles_per_q = (int)TQ;
   k.total_tiles = G;
   k.n_pairs = C;

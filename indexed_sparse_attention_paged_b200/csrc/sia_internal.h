@@ -17,6 +17,9 @@ constexpr int kIndexTileRows = 128;
 // query's list) may hold.
 constexpr int kAttnTileRows = 64;
 constexpr int kAttnMaxSplitRows = 2048;
+// Most CTA pairs one attention launch uses (148 SMs / 2 on a B200; the merge kernel keeps the
+// pairs' first tiles in shared memory).
+constexpr int kAttnMaxPairs = 128;
 // Largest Top-K slice one CTA keeps in shared memory (keys, 4 bytes each).
 constexpr int kTopkSliceMax = 16384;
 constexpr int kTopkThreads = 512;

@@ -242,7 +242,7 @@ __device__ __forceinline__ bool attn_next_unit(const AttnKernelParams& p, int c,
                                                long long& cursor, AttnUnit& u) {
   if (cursor >= rg.g1) return false;
   const int TQ = p.tiles_per_q;
-  u.bj = (int)(cursor / TQ);
+  u.bj = (int)cursor / TQ;   // G < 2^31
   const long long q0 = (long long)u.bj * TQ;
   const long long tb = min(rg.g1, q0 + TQ);
   u.row0 = (int)(cursor - q0) * kAttnTileRows;
@@ -997,19 +997,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 constexpr int kCombineThreads = 256;
 
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineKernelParams p) {
+  // every pair's first tile, computed once per CTA (one 64-bit division per thread at most)
+  __shared__ long long starts[kAttnMaxPairs + 1];
+  const int TQ = p.tiles_per_q, C = p.n_pairs;
+  const long long G = p.total_tiles;
+  for (int i = threadIdx.x; i <= C; i += kCombineThreads) starts[i] = attn_pair_start(i, C, G);
+  __syncthreads();
   pdl_launch_dependents();  // the dependent waits for this grid's completion before its loads
   pdl_wait_primary();
   const int tph = p.DL / 8;                               // threads per (boundary, head)
   const long long bh = (long long)blockIdx.x * (kCombineThreads / tph) + threadIdx.x / tph;
   const int d8 = (threadIdx.x % tph) * 8;
-  if (bh >= (long long)(p.n_pairs - 1) * p.H) return;
+  if (bh >= (long long)(C - 1) * p.H) return;
   const int c = 1 + (int)(bh / p.H), h = (int)(bh % p.H);
-  const int TQ = p.tiles_per_q, C = p.n_pairs;
-  const long long G = p.total_tiles;
-  const long long g = attn_pair_start(c, C, G);
-  const long long q0 = g / TQ * TQ;
+  const long long g = starts[c];
+  const long long q0 = (long long)((int)g / TQ) * TQ;     // G < 2^31
   if (g == q0) return;                                   // a boundary at a query start
-  if (attn_pair_start(c - 1, C, G) > q0) return;         // an earlier boundary owns this query
+  if (starts[c - 1] > q0) return;                        // an earlier boundary owns this query
   const int bj = (int)(q0 / TQ);
   const int rank = d8 >= p.DL / 2 ? 1 : 0;               // the CTA that computed these dims
   float mx = -INFINITY, wsum = 0.0f, o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -1050,8 +1054,8 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineK
     mx = m_new;
   };
   // pair c - 1 holds the query's first piece: its last unit, or its only one when it starts at q0
-  recs[n++] = 2 * (c - 1) + (attn_pair_start(c - 1, C, G) == q0 ? 0 : 1);
-  for (int cc = c; cc < C && attn_pair_start(cc, C, G) < q0 + TQ; ++cc) {
+  recs[n++] = 2 * (c - 1) + (starts[c - 1] == q0 ? 0 : 1);
+  for (int cc = c; cc < C && starts[cc] < q0 + TQ; ++cc) {
     recs[n++] = 2 * cc;   // every later pair's first unit
     if (n == 4) merge();
   }

@@ -61,7 +61,9 @@ def test_emulated_ranks_reproduce_the_whole_chunk(T, N, top_k):
     got = cp_prefill.restore_order(parts, T, N).float().cpu().numpy()
     torch.cuda.synchronize()
     ref = _oracle_chunk(wl, h, new_k, new_kv, T, top_k)
-    assert np.abs(got - ref).max() <= 1e-2
+    # the first queries of a chunk attend to a handful of rows: their outputs reach magnitudes
+    # where the bf16 output's own rounding (up to 2^-9 |ref|) adds to the 1e-2
+    assert np.all(np.abs(got - ref) <= 1e-2 + 2.0 ** -9 * np.abs(ref))
 
 
 def test_world_size_one_nccl_run():
@@ -84,5 +86,5 @@ def test_world_size_one_nccl_run():
     finally:
         dist.destroy_process_group()
     ref = _oracle_chunk(wl, h, new_k, new_kv, T, top_k)
-    assert np.abs(full.float().cpu().numpy() - ref).max() <= 1e-2
+    assert np.all(np.abs(full.float().cpu().numpy() - ref) <= 1e-2 + 2.0 ** -9 * np.abs(ref))
     assert torch.equal(own, full)

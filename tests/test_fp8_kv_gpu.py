@@ -6,7 +6,8 @@ the tensor cores).
 
 Tolerance: the kernel rounds each decoded element (code x block scale) once to bf16 before the
 products, a relative error of at most 2^-9; the output is a convex combination of the selected
-rows, so that rounding moves it by at most 2^-9 max|c| on top of the bf16 path's 1e-2."""
+rows, so that rounding moves it by at most 2^-9 max|c| on top of the bf16 path's 1e-2; the
+bf16 output's own rounding (2^-9 |ref|) is added as in the other stress cases."""
 import numpy as np
 import pytest
 import torch
@@ -76,8 +77,8 @@ def test_fp8_main_cache_attention_matches_the_oracle(name):
                                              d_latent=wl.d_latent, scale=wl.softmax_scale,
                                              kv_scale=h["kv_scale"].numpy())
     assert ost == 0
-    err = np.abs(out.float().cpu().numpy() - ref).max()
-    assert err <= fp8_tol(h), err
+    err = np.abs(out.float().cpu().numpy() - ref)
+    assert np.all(err <= fp8_tol(h) + 2.0 ** -9 * np.abs(ref)), err.max()
     g = lse.cpu().numpy()
     fin = np.isfinite(ref_lse)
     assert np.all(np.isfinite(g) == fin)
@@ -118,4 +119,4 @@ def test_fused_decode_over_an_fp8_main_cache():
     ref, _, _ = oracle.sparse_attend(h["q_attn"], h["kv_cache"], h["page_table"].numpy(), h["seq_lens"].numpy(),
                                      ref_topk, page_size=wl.page_size, d_latent=wl.d_latent,
                                      scale=wl.softmax_scale, kv_scale=h["kv_scale"].numpy())
-    assert np.abs(out.float().cpu().numpy() - ref).max() <= fp8_tol(h)
+    assert np.all(np.abs(out.float().cpu().numpy() - ref) <= fp8_tol(h) + 2.0 ** -9 * np.abs(ref))

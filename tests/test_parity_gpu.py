@@ -93,7 +93,14 @@ def check_index_case(h, top_k, rows=None):
     return got_topk
 
 
-def check_attend_case(h, topk_np, rows=None):
+def out_tol(ref):
+    """1e-2 plus the bf16 output's own rounding (half an ulp, at most 2^-9 |ref|).  The five
+    workloads meet the plain 1e-2; for few-row lists or very peaked softmaxes the output can reach
+    magnitudes of 2-4, where its bf16 rounding alone is up to 0.0078."""
+    return ATOL + 2.0 ** -9 * np.abs(ref)
+
+
+def check_attend_case(h, topk_np, rows=None, stress=False):
     d = workloads.to_device(h, DEV)
     got, got_lse, st = run_attend(h, d, topk_np)
     assert st == 0
@@ -107,7 +114,8 @@ def check_attend_case(h, topk_np, rows=None):
         b, j = divmod(int(r), J)
         err = np.abs(got[b, j] - ref[b, j])
         worst = max(worst, float(err.max()))
-        assert err.max() <= ATOL, "row (%d,%d): max-abs error %.3g" % (b, j, err.max())
+        tol = out_tol(ref[b, j]) if stress else ATOL
+        assert np.all(err <= tol), "row (%d,%d): max-abs error %.3g" % (b, j, err.max())
         e_lse = np.abs(got_lse[b, j] - ref_lse[b, j])
         fin = np.isfinite(ref_lse[b, j])
         assert np.all(np.isfinite(got_lse[b, j]) == fin)
@@ -349,8 +357,9 @@ def test_full_size_workload(num):
 # ------------------------------------------------------------------ harder attention inputs
 
 def test_attend_wide_logits_within_tolerance():
-    """Queries scaled by 12 make the logits span about +-40 (natural units), where the fp16
-    rounding of each CTA's partial logit is largest; the output must still be within 1e-2."""
+    """Queries scaled by 12 make the logits span about +-40 (natural units), where any rounding of
+    the partial logits exchanged between the two CTAs would show most; the softmax is then peaked
+    on few rows, so the output is compared within 1e-2 plus its own bf16 rounding."""
     h = workloads.make_inputs(workloads.WORKLOADS[2], seq_lens=[4000, 6000, 2500])
     h["q_attn"] = (h["q_attn"].float() * 12.0).to(torch.bfloat16)
     topk = _random_topk(h, 2048, seed=21)
@@ -365,7 +374,7 @@ def test_attend_wide_logits_within_tolerance():
         z.append((q @ c.T) * wl.softmax_scale)
     span = max(float(x.max()) for x in z)
     assert span > 30.0
-    worst = check_attend_case(h, topk)
+    worst = check_attend_case(h, topk, stress=True)
     print("wide logits (max %.1f): worst max-abs error %.3g" % (span, worst))
 
 
