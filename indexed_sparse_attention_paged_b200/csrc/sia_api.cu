@@ -291,7 +291,8 @@ struct AttendPlan {
   CombineKernelParams cp;
   CUtensorMap q_rope;   // the query rows' rope slices (the only TMA load of the attention)
   size_t ws_part;
-  long long records;  // partial-result records (0: every query is written directly)
+  long long records;  // partial-result records in the workspace (two per pair)
+  bool merge;         // some query straddles a pair boundary: launch the merge
   int n_clusters;
 };
 
@@ -317,7 +318,9 @@ sia_status check_attend(const sia_attend_args* a) {
   return SIA_OK;
 }
 
-sia_status plan_attend(const sia_attend_args* a, AttendPlan* pl, bool make_maps) {
+// busy_sms: SMs that the preceding grid on the stream holds while this one is launched (the
+// Top-K grid in the fused call); the pairs that can only start once it leaves get less work.
+sia_status plan_attend(const sia_attend_args* a, AttendPlan* pl, bool make_maps, int busy_sms = 0) {
   sia_status st = check_attend(a);
   if (st != SIA_OK) return st;
   AttnKernelParams& k = pl->ap;
@@ -340,13 +343,26 @@ sia_status plan_attend(const sia_attend_args* a, AttendPlan* pl, bool make_maps)
   if (G > 0x7fffffffll) return fail(SIA_ERR_UNSUPPORTED, "batch * n_q * ceil(top_k / 64) must fit in int32");
   const int C = (int)std::min<long long>(std::min(pairs, kAttnMaxPairs), G);
   k.tiles_per_q = (int)TQ;
-  k.total_tiles = G;
-  k.n_pairs = C;
-  // pieces (and their merge) only when some pair boundary falls inside a query
-  long long records = 0;
-  for (long long c = 1; c < C; ++c)
-    if ((c * G / C) % TQ != 0) {
-      records = 2ll * C;
+  k.split.G = G;
+  k.split.C = C;
+  k.split.n_early = C;
+  k.split.w_early = 1;
+  k.split.w_late = 1;
+  if (busy_sms > 0) {
+    // the late pairs start about when the preceding grid ends, a few microseconds into a stage
+    // of some tens: 7/8 of the work of an early pair
+    k.split.n_early = std::max(0, std::min(C, (sm_count() - busy_sms) / 2));
+    k.split.w_early = 8;
+    k.split.w_late = 7;
+  }
+  // pieces (and their merge) only when some pair boundary falls inside a query; the workspace
+  // holds the two records of every pair whenever there is more than one pair, so that its size
+  // does not depend on how the pairs are weighted
+  const long long records = C > 1 ? 2ll * C : 0;
+  pl->merge = false;
+  for (int c = 1; c < C; ++c)
+    if (attn_pair_start(k.split, c) % TQ != 0) {
+      pl->merge = true;
       break;
     }
   k.q = a->q;
@@ -363,7 +379,7 @@ sia_status plan_attend(const sia_attend_args* a, AttendPlan* pl, bool make_maps)
   pl->records = records;
   pl->ws_part = 0;
   if (records > 0) {
-    const size_t o = round_up((size_t)records * a->n_heads * a->d_latent * 2, 256);
+    const size_t o = round_up((size_t)records * a->n_heads * a->d_latent * 4, 256);
     const size_t l = round_up((size_t)records * 2 * a->n_heads * 4, 256);
     pl->ws_part = o + l;
   }
@@ -372,8 +388,7 @@ sia_status plan_attend(const sia_attend_args* a, AttendPlan* pl, bool make_maps)
   c.H = a->n_heads;
   c.DL = a->d_latent;
   c.tiles_per_q = k.tiles_per_q;
-  c.n_pairs = k.n_pairs;
-  c.total_tiles = k.total_tiles;
+  c.split = k.split;
   c.out = k.out;
   c.lse = a->lse;
 
@@ -393,8 +408,8 @@ sia_status run_attend(AttendPlan* pl, void* ws, size_t ws_bytes, int32_t* dev_st
     if (!ws) return fail(SIA_ERR_WORKSPACE, "a workspace of %zu bytes is needed", pl->ws_part);
     if (ws_bytes < pl->ws_part) return fail(SIA_ERR_WORKSPACE, "workspace too small: %zu < %zu", ws_bytes, pl->ws_part);
     if (!aligned(ws, 256)) return fail(SIA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
-    uint16_t* o = static_cast<uint16_t*>(ws);
-    const size_t ob = round_up((size_t)pl->records * pl->ap.H * pl->ap.DL * 2, 256);
+    float* o = static_cast<float*>(ws);
+    const size_t ob = round_up((size_t)pl->records * pl->ap.H * pl->ap.DL * 4, 256);
     pl->ap.part_o = o;
     pl->ap.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + ob);
     pl->cp.part_o = pl->ap.part_o;
@@ -404,7 +419,7 @@ sia_status run_attend(AttendPlan* pl, void* ws, size_t ws_bytes, int32_t* dev_st
   pl->ap.wait_ns = wait_limit_ns();
   cudaError_t e = launch_sparse_attend(pl->ap, pl->q_rope, pl->n_clusters, pdl_first, stream);
   if (e != cudaSuccess) return cuda_fail(e, "sparse attention launch");
-  if (pl->records > 0) {
+  if (pl->merge) {
     e = launch_combine(pl->cp, true, stream);
     if (e != cudaSuccess) return cuda_fail(e, "split combine launch");
   }
@@ -490,7 +505,9 @@ sia_status sia_fused_decode(const sia_index_args* ia, const sia_attend_args* aa,
   AttendPlan ap;
   sia_status st = plan_index(ia, &ip, true);
   if (st != SIA_OK) return st;
-  st = plan_attend(aa, &ap, true);
+  // the Top-K grid holds one SM per CTA while the attention grid is launched
+  const long long topk_ctas = (long long)ip.tp.B * ip.tp.J * ip.tp.cluster;
+  st = plan_attend(aa, &ap, true, (int)std::min<long long>(topk_ctas, sm_count()));
   if (st != SIA_OK) return st;
   const size_t need = round_up(ip.ws_scores, 256) + round_up(ap.ws_part, 256);
   if (need && (!workspace || ws_bytes < need || !aligned(workspace, 256)))

@@ -79,12 +79,30 @@ struct TopkKernelParams {
 };
 
 // -------------------------------------------------------------------------- attention
+// How the flat (query, 64-row tile) list is divided between the CTA pairs of an attention
+// launch: pair c takes tiles [start(c), start(c + 1)) with start(c) = G W(c) / W(C), where the
+// first n_early pairs weigh w_early and the others w_late.  In the fused call the pairs launched
+// last can only become resident when the Top-K grid's CTAs leave their SMs, so they get less.
+struct AttnSplit {
+  long long G;                // total tiles
+  int C;                      // pairs
+  int n_early, w_early, w_late;
+};
+
+__host__ __device__ inline long long attn_weight_before(const AttnSplit& s, int c) {
+  const int e = c < s.n_early ? c : s.n_early;
+  return (long long)s.w_early * e + (long long)s.w_late * (c - e);
+}
+
+__host__ __device__ inline long long attn_pair_start(const AttnSplit& s, int c) {
+  return s.G * attn_weight_before(s, c) / attn_weight_before(s, s.C);
+}
+
 struct AttnKernelParams {
   int B, J, H, DL, DR, P, max_pages, num_pages, K;
   float scale_log2;           // softmax_scale * log2(e)
   int tiles_per_q;            // ceil(K / kAttnTileRows) <= 32
-  long long total_tiles;      // B * J * tiles_per_q
-  int n_pairs;                // CTA pairs (clusters) of the launch
+  AttnSplit split;            // the pairs' ranges of the flat tile list
   const void* q;              // bf16 [B*J, H, DL + DR]
   const void* kv;             // bf16 [num_pages * P, DL + DR], or e4m3 codes when kv_fp8
   const float* kv_scale;      // kv_fp8: fp32 [num_pages * P, nblk], one per 128-element block
@@ -95,7 +113,7 @@ struct AttnKernelParams {
   const int32_t* topk;
   uint16_t* out;              // bf16 bits
   float* lse;
-  uint16_t* part_o;           // [2 * n_pairs][H][DL] bf16, normalised pieces
+  float* part_o;              // [2 * n_pairs][H][DL] fp32, normalised pieces
   float* part_lse;            // [2 * n_pairs][2 (CTA of the pair)][H]
   int32_t* status;
   uint64_t wait_ns;           // limit of every bounded in-kernel wait
@@ -103,9 +121,9 @@ struct AttnKernelParams {
 
 struct CombineKernelParams {
   int BJ, H, DL;
-  int tiles_per_q, n_pairs;
-  long long total_tiles;
-  const uint16_t* part_o;
+  int tiles_per_q;
+  AttnSplit split;
+  const float* part_o;
   const float* part_lse;
   uint16_t* out;
   float* lse;

@@ -11,26 +11,27 @@
 //
 // Design (B200).  All 128 heads of a query form the M = 128 side of every MMA.  The output
 // accumulator O [128 heads x 512 dims] fp32 would fill the whole 256 KB of TMEM, so a CLUSTER
-// OF TWO CTAs shares one (query, Top-K split):
+// OF TWO CTAs shares each piece of work:
 //   - CTA r owns output dims [r*DL/2, (r+1)*DL/2) and gathers only its half of each latent row
 //     (plus half of the rope dims), so together the pair reads each 1152-byte row once;
 //   - each CTA computes a partial S = Q_r . C_r^T over its own dims, with its latent half of Q
 //     held in TMEM (the A operand of the MMA) and only the rope part of Q in shared memory;
-//   - the partials are rounded to fp16 (scaled to base 2); each CTA keeps its own in a shared
-//     stash and sends it to the peer through distributed shared memory, and each softmax adds
-//     the same two fp16 values, so both CTAs see bit-identical logits and take the same
-//     decisions;
+//   - the partials cross to the peer through distributed shared memory as int16 with one
+//     power-of-two scale per head and half tile, and each CTA adds the peer's decoded partial
+//     to its own exact fp32 one (read straight from TMEM);
 //   - P (bf16) is written to a 128B-swizzled shared buffer and is the A operand of
 //     O_r += P . C_r.
-// Warp roles (576 threads): softmax + epilogue (warps 0-3), TMEM q loading and the logit
-// exchange (4-7), the row gather (8-15), the S = Q C^T issuer (16) and the P . C issuer (17);
-// setmaxnreg splits the registers between them.  Rows are gathered with 16-byte cp.async from a
-// per-unit table of physical cache rows into swizzled K-major tiles (four latent stages, a
-// separate two-slot rope ring); the same tile serves as the K-major B operand of Q.C^T and as
-// the MN-major B operand of P.C.  Rescaling of O is lazy: only when a head's running max grows
-// by more than 2^8.  Splits of the Top-K list (to fill the GPU at small batch) write normalised
-// bf16 partials and an fp32 log-sum-exp per split that combine_kernel merges.  Every pipeline
-// wait is an mbarrier wait with a bounded spin.
+// Warp roles (576 threads): two softmax warpgroups (warps 0-3 and 4-7; each owns 32 of a tile's
+// 64 rows for all heads, and does that half's logit exchange, its part of the q load into TMEM
+// and half of the output columns), the row gather (8-15), the S = Q C^T issuer (16) and the
+// P . C issuer (17); setmaxnreg splits the registers between them.  Rows are gathered with
+// 16-byte cp.async from a per-unit table of physical cache rows into swizzled K-major tiles (four
+// latent stages, a separate two-slot rope ring); the same tile serves as the K-major B operand
+// of Q.C^T and as the MN-major B operand of P.C.  Rescaling of O is lazy: only when a head's
+// running max grows by more than 2^8.  The (query, 64-row tile) work is split evenly over all CTA
+// pairs; queries that straddle a pair boundary are computed in pieces (normalised bf16 partials
+// and log-sum-exps) that combine_kernel merges.  Every pipeline wait is an mbarrier wait with a
+// bounded spin.
 #include <cuda.h>
 #include <cuda_fp16.h>
 
@@ -44,27 +45,25 @@ namespace sia {
 namespace {
 
 constexpr int kProducerWarps = 8;   // cp.async gather (+ TMA for the rope part of q)
-constexpr int kFirstExchangeWarp = 4;
 constexpr int kFirstProducerWarp = 8;
 constexpr int kMmaWarp = 16;    // S = Q . C^T issuer (and TMEM owner)
 constexpr int kPvWarp = 17;     // O += P . C issuer
-// warps 0-3 softmax + epilogue, 4-7 q loader + partial-logit exchange, 8-15 gather, 16 MMA
+// warps 0-7 softmax, partial-logit exchange, q loader and epilogue (two warpgroups, one per half
+// of each tile's rows), 8-15 gather, 16 S = Q . C^T issuer, 17 O += P . C issuer
 constexpr int kAttnThreads = 576;
 // Registers per thread after the split.  The block is launched with kLaunchRegs x 576
-// registers (ptxas' allocation for 576 threads); the softmax warpgroup takes 168 (a tile of
-// fp32 logits and their TMEM loads), the exchange warpgroup 88, the two gather warpgroups give
-// back down to 64 and the two MMA warps keep the launch value.  The sum stays within the launch
-// allocation, so setmaxnreg.inc never waits for registers that are not there.
+// registers (ptxas' allocation for 576 threads); the two softmax warpgroups take 128 each (half a
+// tile of fp32 logits and their TMEM loads), the two gather warpgroups give back down to 64 and
+// the two MMA warps keep the launch value.  The sum stays within the launch allocation, so
+// setmaxnreg.inc never waits for registers that are not there.
 constexpr int kLaunchRegs = 96;
-constexpr int kSoftmaxRegs = 168;
-constexpr int kExchangeRegs = 88;
+constexpr int kSoftmaxRegs = 128;
 constexpr int kGatherRegs = 64;
-static_assert(128 * kSoftmaxRegs + 256 * kGatherRegs + 128 * kExchangeRegs + 64 * kLaunchRegs <=
-                  kAttnThreads * kLaunchRegs,
+static_assert(256 * kSoftmaxRegs + 256 * kGatherRegs + 64 * kLaunchRegs <= kAttnThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
 // setmaxnreg.inc may only raise a warp's count and setmaxnreg.dec only lower it
-static_assert(kSoftmaxRegs >= kLaunchRegs && kGatherRegs <= kLaunchRegs && kExchangeRegs <= kLaunchRegs,
-              "the softmax warpgroup grows, the gather and exchange warpgroups shrink");
+static_assert(kSoftmaxRegs >= kLaunchRegs && kGatherRegs <= kLaunchRegs,
+              "the softmax warpgroups grow, the gather warpgroups shrink");
 constexpr int kStages = 4;          // latent-row tiles in flight per CTA
 constexpr int kRopeSlots = 2;       // their rope parts (read by S = Q . C^T only) in flight
 constexpr int kRows = kAttnTileRows;
@@ -152,8 +151,11 @@ struct AttnSmem {
   // peer's exchange warps fill one buffer while this CTA's softmax reads the other
   static constexpr uint32_t kSxBytes = kRows * 128 * 2;
   static constexpr uint32_t kOffSx = kOffP + 128 * kRows * 2;
-  static constexpr uint32_t kOffSxExp = kOffSx + 2 * kSxBytes;          // [2][128] int32 exponents
-  static constexpr uint32_t kOffRows = kOffSxExp + 2 * 128 * 4;
+  static constexpr uint32_t kOffSxExp = kOffSx + 2 * kSxBytes;      // [2 tiles][2 halves][128] int32
+  // the two softmax warpgroups' per-head tile maxima [2 tiles][2][128] and unit sums [2][128]
+  static constexpr uint32_t kOffMx = kOffSxExp + 2 * 2 * 128 * 4;
+  static constexpr uint32_t kOffL = kOffMx + 2 * 2 * 128 * 4;
+  static constexpr uint32_t kOffRows = kOffL + 2 * 128 * 4;
   // per unit (double-buffered): physical cache row of each Top-K entry, validity bits, and
   // each gather warp's lowest position of a -1 entry
   static constexpr uint32_t kOffMask = kOffRows + 2 * kAttnMaxSplitRows * 4;
@@ -168,14 +170,15 @@ struct AttnSmem {
 struct AttnBarriers {
   uint64_t c_full[kStages], c_empty[kStages];   // a tile's rows landed / latent stage free
   uint64_t r_empty[kRopeSlots];                 // rope slot free (its S = Q . C^T done)
-  uint64_t s_full[2], s_empty[2];   // logits ready in TMEM / read by the exchange and softmax warps
+  uint64_t s_full[2], s_empty[2];   // logits ready in TMEM / read by both softmax warpgroups
+  uint64_t mx_bar[2];               // both warpgroups wrote their half's per-head tile max
   uint64_t p_full;                  // all softmax threads wrote P (waited by the P . C issuer)
   uint64_t p_empty;                 // P . C of the previous tile done (P buffer and O free)
   uint64_t epi_sync;                // all softmax threads are past the unit's last tile
   uint64_t q_full, q_empty;       // q in TMEM written by the 128 loader threads / q reusable
   uint64_t q_tma;                 // the rope part of q landed (TMA bytes only)
   uint64_t o_full;
-  uint64_t sx_ready[2], sx_free[2];
+  uint64_t sx_ready[2][2], sx_free[2][2];   // [tile][half]: the peer's half landed / was read
   uint64_t tab_full[2], tab_free[2];
   uint64_t mma_done, pv_done;
   uint64_t g_loaded[2];             // FP8 cache: every gather thread read its staged codes
@@ -217,14 +220,13 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
 }
 
 // The work of a call is the flat list of (query, 64-row tile) pairs, query-major with
-// tiles_per_q <= 32 tiles per query, split evenly between the CTA pairs: pair c takes global
-// tiles [c G / C, (c + 1) G / C).  A unit is the part of that range inside one query.  A query
+// tiles_per_q <= 32 tiles per query, divided between the CTA pairs (AttnSplit): pair c takes
+// global tiles [start(c), start(c + 1)).  A unit is the part of that range inside one query.  A query
 // covered by one unit gets its output written directly; a query that straddles a pair
 // boundary is computed in pieces, each written as a partial result (normalised O and the
 // log-sum-exp of each CTA of the pair) into a record of the workspace, and combine_kernel
 // merges them.  Only a pair's first and last unit can be pieces, so pair c owns records 2c
 // (its first unit) and 2c + 1 (its last unit, when that is another unit).
-__device__ __forceinline__ long long attn_pair_start(int c, int C, long long G) { return (long long)c * G / C; }
 
 struct AttnUnit {
   int bj;        // query row (b * J + j)
@@ -298,21 +300,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     for (int s = 0; s < kRopeSlots; ++s) mbar_init(&sb->r_empty[s], 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sb->s_full[s], 1);
-      mbar_init(&sb->s_empty[s], 256);         // exchange and softmax threads
+      mbar_init(&sb->s_empty[s], 256);         // both softmax warpgroups
+      mbar_init(&sb->mx_bar[s], 256);
       mbar_init(&sb->tab_full[s], kProducerWarps * 32);
-      mbar_init(&sb->tab_free[s], 128 + 128 + 2);   // softmax, exchange and both MMA threads
+      mbar_init(&sb->tab_free[s], 256 + 2);   // both softmax warpgroups and both MMA threads
     }
-    mbar_init(&sb->p_full, 128);
+    mbar_init(&sb->p_full, 256);
     mbar_init(&sb->p_empty, 1);
-    mbar_init(&sb->epi_sync, 128);
-    mbar_init(&sb->q_full, 128);       // the 128 TMEM writers
+    mbar_init(&sb->epi_sync, 256);
+    mbar_init(&sb->q_full, 256);       // the 256 TMEM writers
     mbar_init(&sb->q_tma, 1);          // the rope TMA (or a plain arrive when this CTA has none)
     mbar_init(&sb->q_empty, 1);
     mbar_init(&sb->o_full, 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&sb->sx_ready[s], 128);   // arrived by the peer's 128 exchange threads
-      mbar_init(&sb->sx_free[s], 128);    // arrived by the peer's 128 softmax threads
-    }
+    for (int s = 0; s < 2; ++s)
+      for (int g = 0; g < 2; ++g) {
+        mbar_init(&sb->sx_ready[s][g], 128);   // arrived by the peer's warpgroup g
+        mbar_init(&sb->sx_free[s][g], 128);
+      }
     mbar_init(&sb->mma_done, 1);
     mbar_init(&sb->pv_done, 1);
     mbar_init(&sb->g_loaded[0], kProducerWarps * 32);
@@ -389,8 +393,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     int it = 0, u_it = 0, q_issued = 0;
     bool ok = true;
     bool waited = false;
-    const AttnRange rg{attn_pair_start(cluster_id, p.n_pairs, p.total_tiles),
-                      attn_pair_start(cluster_id + 1, p.n_pairs, p.total_tiles)};
+    const AttnRange rg{attn_pair_start(p.split, cluster_id), attn_pair_start(p.split, cluster_id + 1)};
     long long cursor = rg.g0;
     AttnUnit un;
     if (cursor < rg.g1) {
@@ -597,8 +600,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint32_t qr_base = smem_u32(smem + Sm::kOffQ);
       int it = 0, u_it = 0;
       bool ok = true;
-      const AttnRange rg{attn_pair_start(cluster_id, p.n_pairs, p.total_tiles),
-                      attn_pair_start(cluster_id + 1, p.n_pairs, p.total_tiles)};
+      const AttnRange rg{attn_pair_start(p.split, cluster_id), attn_pair_start(p.split, cluster_id + 1)};
     long long cursor = rg.g0;
       AttnUnit un;
       for (; ok && attn_next_unit(p, cluster_id, rg, cursor, un); ++u_it) {
@@ -652,8 +654,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint32_t p_base = smem_u32(smem + Sm::kOffP);
       int it = 0, u_it = 0;
       bool ok = true;
-      const AttnRange rg{attn_pair_start(cluster_id, p.n_pairs, p.total_tiles),
-                      attn_pair_start(cluster_id + 1, p.n_pairs, p.total_tiles)};
+      const AttnRange rg{attn_pair_start(p.split, cluster_id), attn_pair_start(p.split, cluster_id + 1)};
     long long cursor = rg.g0;
       AttnUnit un;
       for (; ok && attn_next_unit(p, cluster_id, rg, cursor, un); ++u_it) {
@@ -683,43 +684,50 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_drain(&sb->pv_done, 0, p.status);    // every O += P . C product done
     }
     __syncwarp();
-  } else if (warp >= kFirstExchangeWarp && warp < kFirstExchangeWarp + 4) {
-    // ---------------------------------------------------------------- q loader + exchange
-    // Per unit: writes this CTA's latent half of every head's query row into TMEM (the A
-    // operand of Q . C^T).  Per tile: reads this CTA's partial logits from TMEM and pushes them,
-    // scaled to base 2 and encoded as int16 with one power-of-two scale per head (relative
-    // error at most 2^-15 of the head's largest partial), into the peer CTA's exchange buffer.
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kExchangeRegs));
+  } else {
+    // ---------------------------------------------------------------- softmax + exchange
+    // Two warpgroups (warps 0-3 and 4-7, two warps per SM sub-partition); thread = head h =
+    // TMEM lane, warpgroup wg owns rows [32 wg, 32 wg + 32) of every 64-row tile.  Per tile a
+    // warpgroup reads its half of this CTA's partial logits from TMEM, sends them to the peer CTA
+    // as int16 with one power-of-two scale per head (relative error at most 2^-15 of the half's
+    // largest partial), adds the peer's decoded half to its exact own partial (one rounding),
+    // agrees with the other warpgroup on each head's tile max through shared memory, and writes
+    // its half of P.  Per unit it also loads its part of q into TMEM and, at the end, its half of
+    // the output columns.
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
+    constexpr int kHalf = kRows / 2;
+    const int wg = warp >> 2;
     const int quad = warp & 3;
-    const int h = quad * 32 + lane;
+    const int h = quad * 32 + lane;   // head = TMEM lane
     const uint32_t lane_addr = tmem_base + ((uint32_t)(quad * 32) << 16);
     const uint32_t sx_peer = mapa_shared(smem_u32(smem + Sm::kOffSx), peer);
     const uint32_t sxexp_peer = mapa_shared(smem_u32(smem + Sm::kOffSxExp), peer);
-    int s_it = 0, u_it = 0;
+    float* mxbuf = reinterpret_cast<float*>(smem + Sm::kOffMx);   // [2 tiles][2 warpgroups][128]
+    float* lbuf = reinterpret_cast<float*>(smem + Sm::kOffL);     // [2 warpgroups][128]
+    int s_it = 0, u_it = 0, o_it = 0, e_it = 0;
     bool ok = true;
-    const AttnRange rg{attn_pair_start(cluster_id, p.n_pairs, p.total_tiles),
-                      attn_pair_start(cluster_id + 1, p.n_pairs, p.total_tiles)};
+
+    const AttnRange rg{attn_pair_start(p.split, cluster_id), attn_pair_start(p.split, cluster_id + 1)};
     long long cursor = rg.g0;
     AttnUnit un;
+    int last_sbuf = 0;
     for (; ok && attn_next_unit(p, cluster_id, rg, cursor, un); ++u_it) {
       const int bj = un.bj;
       const int buf = u_it & 1;
       {
-        // q: head h's dims [rank * kLatDims, +kLatDims) as bf16 pairs, 16 columns per store
+        // q: head h's dims [rank * kLatDims, +kLatDims) as bf16 pairs, 16 columns per store;
+        // the warpgroups split the column groups
         if (!mbar_wait_warp(&sb->q_empty, ((uint32_t)u_it & 1u) ^ 1u, wc)) { ok = false; break; }
         const bool real = h < p.H;
         const uint8_t* qrow = static_cast<const uint8_t*>(p.q) + ((long long)bj * p.H + (real ? h : 0)) * (DC * 2) +
                               (size_t)rank * Lay::kLatDims * 2;
         constexpr int kGroups = Lay::kLatDims / 32;   // 64 bytes = 16 columns each
-        // pull the whole row share into L2 first, so the grouped loads below wait on L2, not DRAM
-        if (real) {
-#pragma unroll
-          for (int g = 0; g < kGroups; g += 2)
-            asm volatile("prefetch.global.L2 [%0];" ::"l"(qrow + g * 64));
-        }
+        const int g_lo = wg == 0 ? 0 : (kGroups + 1) / 2, g_hi = wg == 0 ? (kGroups + 1) / 2 : kGroups;
+        if (real)
+          for (int g = g_lo; g < g_hi; g += 2) asm volatile("prefetch.global.L2 [%0];" ::"l"(qrow + g * 64));
         tc_fence_after();
 #pragma unroll 1
-        for (int g = 0; g < kGroups; ++g) {
+        for (int g = g_lo; g < g_hi; ++g) {
           uint32_t w[16];
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
@@ -736,133 +744,101 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         mbar_arrive(&sb->q_full);
       }
       if (!mbar_wait_warp(&sb->tab_full[buf], (uint32_t)(u_it >> 1) & 1u, wc)) { ok = false; break; }
-      const int ntiles = (unit_tiles(buf) + kRows - 1) / kRows;
-      mbar_arrive(&sb->tab_free[buf]);
+      const int first_neg = unit_tiles(buf);
+      const int ntiles = (first_neg + kRows - 1) / kRows;
+      const uint32_t* mt = mask_tab + buf * (kAttnMaxSplitRows / 32);
+      float m = -INFINITY, l = 0.0f;   // m is the same in both warpgroups; l covers this half
+      float s[kHalf];
       for (int t = 0; t < ntiles; ++t, ++s_it) {
         const int sbuf = s_it & 1;
-        const uint32_t scol = lane_addr + Tm::kS + sbuf * kRows;
+        uint32_t valid = mt[2 * t + wg];                  // this half's 32 rows
+        const int live = first_neg - t * kRows - wg * kHalf;   // rows past the first -1 are padding
+        if (live < kHalf) valid &= live > 0 ? (1u << live) - 1u : 0u;
         if (!mbar_wait_warp(&sb->s_full[sbuf], (uint32_t)(s_it >> 1) & 1u, wc)) { ok = false; break; }
         tc_fence_after();
-        // this CTA's partial logits of head h (base 2) as int16 with one power-of-two scale
-        uint32_t enc[kRows / 2];
+        uint32_t enc[kHalf / 2];
         int e;
         {
-          uint32_t r[4][16];   // the whole tile's row in one TMEM wait
+          uint32_t r[2][16];
 #pragma unroll
-          for (int c = 0; c < 4; ++c) tmem_ld16(scol + c * 16, r[c]);
+          for (int c = 0; c < 2; ++c) tmem_ld16(lane_addr + Tm::kS + sbuf * kRows + wg * kHalf + c * 16, r[c]);
           tmem_wait_ld();
           float amax = 0.0f;
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
+          for (int c = 0; c < 2; ++c)
 #pragma unroll
-            for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(__uint_as_float(r[c][i])));
+            for (int i = 0; i < 16; ++i) {
+              s[16 * c + i] = __uint_as_float(r[c][i]);
+              amax = fmaxf(amax, fabsf(s[16 * c + i]));
+            }
           amax *= fabsf(p.scale_log2);
           // e with amax 2^e < 2^14: amax < 2^E for E = (biased exponent of amax) - 126
           const int E = (int)((__float_as_uint(amax) >> 23) & 0xffu) - 126;
           e = amax > 0.0f ? min(max(14 - E, -100), 100) : 0;
           const float sc = p.scale_log2 * __uint_as_float((uint32_t)(127 + e) << 23);
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const float y0 = fmaf(__uint_as_float(r[c][2 * i]), sc, kMagic);
-              const float y1 = fmaf(__uint_as_float(r[c][2 * i + 1]), sc, kMagic);
-              enc[c * 8 + i] = prmt(__float_as_uint(y0), __float_as_uint(y1), 0x5410u);
-            }
+          for (int i = 0; i < kHalf / 2; ++i) {
+            const float y0 = fmaf(s[2 * i], sc, kMagic);
+            const float y1 = fmaf(s[2 * i + 1], sc, kMagic);
+            enc[i] = prmt(__float_as_uint(y0), __float_as_uint(y1), 0x5410u);
+          }
         }
         tc_fence_before();
-        mbar_arrive(&sb->s_empty[sbuf]);   // our reads of these logits are done
-        if (!mbar_wait_warp<true>(&sb->sx_free[sbuf], ((uint32_t)(s_it >> 1) & 1u) ^ 1u, wc)) { ok = false; break; }
+        mbar_arrive(&sb->s_empty[sbuf]);   // this warpgroup's reads of the partial are done
+        // send this half to the peer (the peer's same warpgroup reads it)
+        if (!mbar_wait_warp<true>(&sb->sx_free[sbuf][wg], ((uint32_t)(s_it >> 1) & 1u) ^ 1u, wc)) { ok = false; break; }
 #pragma unroll
-        for (int g = 0; g < kRows / 8; ++g)
-          asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sx_peer + sbuf * Sm::kSxBytes + (uint32_t)((g * 128 + h) * 16)),
-                       "r"(enc[4 * g]), "r"(enc[4 * g + 1]), "r"(enc[4 * g + 2]), "r"(enc[4 * g + 3])
+        for (int gi = 0; gi < kHalf / 8; ++gi) {
+          const uint32_t dst = sx_peer + sbuf * Sm::kSxBytes + (uint32_t)(((wg * (kHalf / 8) + gi) * 128 + h) * 16);
+          asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(enc[4 * gi]),
+                       "r"(enc[4 * gi + 1]), "r"(enc[4 * gi + 2]), "r"(enc[4 * gi + 3])
                        : "memory");
-        asm volatile("st.shared::cluster.b32 [%0], %1;" ::"r"(sxexp_peer + (uint32_t)((sbuf * 128 + h) * 4)), "r"(e)
-                     : "memory");
-        mbar_arrive_cluster(&sb->sx_ready[sbuf], peer);
-      }
-    }
-  } else {
-    // ---------------------------------------------------------------- softmax + epilogue
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
-    const int quad = warp & 3;
-    const int h = quad * 32 + lane;   // head = TMEM lane
-    const uint32_t lane_addr = tmem_base + ((uint32_t)(quad * 32) << 16);
-    int s_it = 0, u_it = 0, o_it = 0, e_it = 0;
-    bool ok = true;
-
-    const AttnRange rg{attn_pair_start(cluster_id, p.n_pairs, p.total_tiles),
-                      attn_pair_start(cluster_id + 1, p.n_pairs, p.total_tiles)};
-    long long cursor = rg.g0;
-    AttnUnit un;
-    int last_sbuf = 0;
-    for (; ok && attn_next_unit(p, cluster_id, rg, cursor, un); ++u_it) {
-      const int bj = un.bj;
-      const int buf = u_it & 1;
-      if (!mbar_wait_warp(&sb->tab_full[buf], (uint32_t)(u_it >> 1) & 1u, wc)) { ok = false; break; }
-      const int first_neg = unit_tiles(buf);
-      const int ntiles = (first_neg + kRows - 1) / kRows;
-      const uint32_t* mt = mask_tab + buf * (kAttnMaxSplitRows / 32);
-      float m = -INFINITY, l = 0.0f;
-      float s[kRows];
-      for (int t = 0; t < ntiles; ++t, ++s_it) {
-        const int sbuf = s_it & 1;
-        uint64_t valid = ((uint64_t)mt[2 * t + 1] << 32) | mt[2 * t];
-        const int live = first_neg - t * kRows;            // rows past the first -1 are padding
-        if (live < kRows) valid &= (1ull << live) - 1ull;
-        // logits of tile t (base 2) = this CTA's exact fp32 partial (from TMEM) + the peer's
-        // decoded int16 partial, one rounding
-        if (!mbar_wait_warp(&sb->s_full[sbuf], (uint32_t)(s_it >> 1) & 1u, wc)) { ok = false; break; }
-        tc_fence_after();
-        {
-          uint32_t r[4][16];
-#pragma unroll
-          for (int c = 0; c < 4; ++c) tmem_ld16(lane_addr + Tm::kS + sbuf * kRows + c * 16, r[c]);
-          tmem_wait_ld();
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-#pragma unroll
-            for (int i = 0; i < 16; ++i) s[16 * c + i] = __uint_as_float(r[c][i]);
         }
-        tc_fence_before();
-        mbar_arrive(&sb->s_empty[sbuf]);   // our read of this CTA's partial is done
-        if (!mbar_wait_warp<true>(&sb->sx_ready[sbuf], (uint32_t)(s_it >> 1) & 1u, wc)) { ok = false; break; }
+        asm volatile("st.shared::cluster.b32 [%0], %1;" ::"r"(sxexp_peer + (uint32_t)(((sbuf * 2 + wg) * 128 + h) * 4)), "r"(e)
+                     : "memory");
+        mbar_arrive_cluster(&sb->sx_ready[sbuf][wg], peer);
+        // the peer's half for the same rows: logit = own exact partial + decoded peer partial
+        if (!mbar_wait_warp<true>(&sb->sx_ready[sbuf][wg], (uint32_t)(s_it >> 1) & 1u, wc)) { ok = false; break; }
         last_sbuf = sbuf;
         {
-          const int e = *reinterpret_cast<const int*>(smem + Sm::kOffSxExp + (sbuf * 128 + h) * 4);
-          const float dn = __uint_as_float((uint32_t)(127 - e) << 23);
+          const int pe = *reinterpret_cast<const int*>(smem + Sm::kOffSxExp + ((sbuf * 2 + wg) * 128 + h) * 4);
+          const float dn = __uint_as_float((uint32_t)(127 - pe) << 23);
           const float bias = -kMagic * dn;
 #pragma unroll
-          for (int g = 0; g < kRows / 8; ++g) {
-            const uint4 pv4 = *reinterpret_cast<const uint4*>(smem + Sm::kOffSx + sbuf * Sm::kSxBytes + (g * 128 + h) * 16);
+          for (int gi = 0; gi < kHalf / 8; ++gi) {
+            const uint4 pv4 = *reinterpret_cast<const uint4*>(smem + Sm::kOffSx + sbuf * Sm::kSxBytes +
+                                                              ((wg * (kHalf / 8) + gi) * 128 + h) * 16);
             const uint32_t q4[4] = {pv4.x, pv4.y, pv4.z, pv4.w};
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const float f0 = __uint_as_float(prmt(q4[i], 0x4B000000u, 0x7610u));
               const float f1 = __uint_as_float(prmt(q4[i], 0x4B000000u, 0x7632u));
-              s[8 * g + 2 * i] = fmaf(s[8 * g + 2 * i], p.scale_log2, fmaf(f0, dn, bias));
-              s[8 * g + 2 * i + 1] = fmaf(s[8 * g + 2 * i + 1], p.scale_log2, fmaf(f1, dn, bias));
+              s[8 * gi + 2 * i] = fmaf(s[8 * gi + 2 * i], p.scale_log2, fmaf(f0, dn, bias));
+              s[8 * gi + 2 * i + 1] = fmaf(s[8 * gi + 2 * i + 1], p.scale_log2, fmaf(f1, dn, bias));
             }
           }
         }
-        // the peer may refill the exchange buffer (the logit values read above are already in
-        // registers); after the unit's last tile the buffer first serves the epilogue
-        if (t + 1 < ntiles) mbar_arrive_cluster_relaxed(&sb->sx_free[sbuf], peer);
+        // the peer may refill its half of the exchange buffer; after the unit's last tile the
+        // buffer first serves the epilogue (released there)
+        if (t + 1 < ntiles) mbar_arrive_cluster_relaxed(&sb->sx_free[sbuf][wg], peer);
 
-        // online softmax (base 2), lazy rescale
+        // online softmax (base 2), lazy rescale; the two halves agree on the tile max
         float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-        if (valid == ~0ull) {
+        if (valid == ~0u) {
 #pragma unroll
-          for (int i = 0; i < kRows; ++i) mx[i & 3] = fmaxf(mx[i & 3], s[i]);
+          for (int i = 0; i < kHalf; ++i) mx[i & 3] = fmaxf(mx[i & 3], s[i]);
         } else {
 #pragma unroll
-          for (int i = 0; i < kRows; ++i) {
-            s[i] = (valid >> i & 1ull) ? s[i] : -INFINITY;
+          for (int i = 0; i < kHalf; ++i) {
+            s[i] = (valid >> i & 1u) ? s[i] : -INFINITY;
             mx[i & 3] = fmaxf(mx[i & 3], s[i]);
           }
         }
-        const float mt_ = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+        const float mine = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+        mxbuf[(sbuf * 2 + wg) * 128 + h] = mine;
+        mbar_arrive(&sb->mx_bar[sbuf]);
+        if (!mbar_wait_warp(&sb->mx_bar[sbuf], (uint32_t)(s_it >> 1) & 1u, wc)) { ok = false; break; }
+        const float mt_ = fmaxf(mine, mxbuf[(sbuf * 2 + (wg ^ 1)) * 128 + h]);
         float alpha = 1.0f;
         const bool need = mt_ > m + 8.0f;
         if (need) {
@@ -873,13 +849,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (m != -INFINITY) {
           // masked logits are -inf and m is finite: their exp2 is exactly 0
 #pragma unroll
-          for (int i = 0; i < kRows; ++i) {
+          for (int i = 0; i < kHalf; ++i) {
             s[i] = fast_exp2(s[i] - m);
             ps[i & 3] += s[i];
           }
         } else {
 #pragma unroll
-          for (int i = 0; i < kRows; ++i) s[i] = 0.0f;
+          for (int i = 0; i < kHalf; ++i) s[i] = 0.0f;
         }
         l = l * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
 
@@ -887,9 +863,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (!mbar_wait_warp(&sb->p_empty, ((uint32_t)s_it & 1u) ^ 1u, wc)) { ok = false; break; }
         tc_fence_after();
         if (__any_sync(0xffffffffu, need && t > 0)) {
-          // O holds the tiles < t of this unit: rescale it
+          // O holds the tiles < t of this unit: each warpgroup rescales half of its columns
 #pragma unroll 1
-          for (int c = 0; c < Lay::kPvN; c += 16) {
+          for (int c = wg * (Lay::kPvN / 2); c < (wg + 1) * (Lay::kPvN / 2); c += 16) {
             uint32_t r[16];
             tmem_ld16(lane_addr + Tm::kO + c, r);
             tmem_wait_ld();
@@ -899,10 +875,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
           tmem_wait_st();
         }
-        // P (bf16) into shared memory: this head's row of kRows values, 128B-swizzled
+        // this half of P (bf16) into shared memory: head h's row, K columns [32 wg, 32 wg + 32)
 #pragma unroll
-        for (int k = 0; k < kRows / 8; ++k)
-          st_shared_v4(smem_u32(smem + Sm::kOffP + swizzled_offset((uint32_t)h, (uint32_t)k * 16, 128)),
+        for (int k = 0; k < kHalf / 8; ++k)
+          st_shared_v4(smem_u32(smem + Sm::kOffP + swizzled_offset((uint32_t)h, (uint32_t)(wg * (kHalf / 8) + k) * 16, 128)),
                        pack_bf16x2(s[8 * k], s[8 * k + 1]), pack_bf16x2(s[8 * k + 2], s[8 * k + 3]),
                        pack_bf16x2(s[8 * k + 4], s[8 * k + 5]), pack_bf16x2(s[8 * k + 6], s[8 * k + 7]));
         fence_proxy_async_smem();
@@ -915,68 +891,115 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (ntiles > 0) {
         if (!mbar_wait_warp(&sb->o_full, (uint32_t)o_it & 1u, wc)) { ok = false; break; }
         ++o_it;
+        // every thread has read the last tile's peer logits before a staging slice is reused,
+        // and the two halves' sums are visible
+        lbuf[wg * 128 + h] = l;
+        mbar_arrive(&sb->epi_sync);
+        if (!mbar_wait_warp(&sb->epi_sync, (uint32_t)e_it & 1u, wc)) { ok = false; break; }
+        ++e_it;
+        l += lbuf[(wg ^ 1) * 128 + h];
       }
       tc_fence_after();
       const bool any = ntiles > 0 && l > 0.0f;
       const float inv = any ? 1.0f / l : 0.0f;
       const float lse = any ? (m + log2f(l)) * 0.69314718055994530942f : -INFINITY;
       const bool real_head = h < p.H;
-      // O rows (bf16: the output, or a split's normalised partial) go out through the exchange
-      // buffer (free until the deferred sx_free below): each warp stages 32 heads x 128 bytes
-      // per round in a 128B-swizzled 4 KB slice, then writes whole 128-byte runs of 4 heads per
-      // instruction
+      // O rows (the bf16 output, or a piece's normalised fp32 partial): each warpgroup writes
+      // half of this CTA's columns, staged through a 128B-swizzled 4 KB slice per warp
+      // (warpgroup 0 in the P buffer, free once the unit's last P . C is done; warpgroup 1 in the
+      // exchange buffer of the last tile, released below) so that each global store writes four
+      // whole 128-byte runs
       const bool partial = un.rec >= 0;
-      uint16_t* obase = (partial ? p.part_o + (long long)un.rec * p.H * p.DL : p.out + (long long)bj * p.H * p.DL) +
-                        rank * Lay::kPvN;
+      const int c_lo = wg * (Lay::kPvN / 2), c_hi = (wg + 1) * (Lay::kPvN / 2);
       if (ntiles > 0) {
-        // every softmax warp has read the last tile's peer logits before any slice is reused
-        mbar_arrive(&sb->epi_sync);
-        if (!mbar_wait_warp(&sb->epi_sync, (uint32_t)e_it & 1u, wc)) { ok = false; break; }
-        ++e_it;
-        uint8_t* slice = smem + Sm::kOffSx + last_sbuf * Sm::kSxBytes + quad * 4096;
+        uint8_t* slice = (wg == 0 ? smem + Sm::kOffP : smem + Sm::kOffSx + last_sbuf * Sm::kSxBytes) + quad * 4096;
+        if (!partial) {
+          // the output, bf16: 64 columns (128 bytes) per head and round
+          uint16_t* obase = p.out + (long long)bj * p.H * p.DL + rank * Lay::kPvN;
 #pragma unroll 1
-        for (int c = 0; c < Lay::kPvN; c += 64) {
-          uint32_t w[32];
-          {
-            // four loads in flight per TMEM wait (a wait per load made the epilogue latency bound)
-            uint32_t r[4][16];
+          for (int c = c_lo; c < c_hi; c += 64) {
+            uint32_t w[32];
+            {
+              // four loads in flight per TMEM wait (a wait per load made the epilogue latency bound)
+              uint32_t r[4][16];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) tmem_ld16(lane_addr + Tm::kO + c + 16 * q, r[q]);   // past kPvN: not stored
-            tmem_wait_ld();
+              for (int q = 0; q < 4; ++q) tmem_ld16(lane_addr + Tm::kO + c + 16 * q, r[q]);   // past c_hi: not stored
+              tmem_wait_ld();
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
+              for (int q = 0; q < 4; ++q)
 #pragma unroll
-              for (int i = 0; i < 8; ++i)
-                w[8 * q + i] = pack_bf16x2(__uint_as_float(r[q][2 * i]) * inv, __uint_as_float(r[q][2 * i + 1]) * inv);
+                for (int i = 0; i < 8; ++i)
+                  w[8 * q + i] = pack_bf16x2(__uint_as_float(r[q][2 * i]) * inv, __uint_as_float(r[q][2 * i + 1]) * inv);
+            }
+            __syncwarp();
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              st_shared_v4(smem_u32(slice + lane * 128 + ((k ^ (lane & 7)) * 16)), w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+            __syncwarp();
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const int r = 4 * k + (lane >> 3), blk = lane & 7;
+              const int head = quad * 32 + r;
+              const uint4 v = *reinterpret_cast<const uint4*>(slice + r * 128 + ((blk ^ (r & 7)) * 16));
+              if (head < p.H && c + 8 * blk < c_hi)
+                *reinterpret_cast<uint4*>(obase + (long long)head * p.DL + c + 8 * blk) = v;
+            }
           }
-          __syncwarp();
+        } else {
+          // a piece, fp32 (the merge rounds once, to the bf16 output): 32 columns per round
+          float* obase = p.part_o + (long long)un.rec * p.H * p.DL + rank * Lay::kPvN;
+#pragma unroll 1
+          for (int c = c_lo; c < c_hi; c += 32) {
+            uint32_t w[32];
+            {
+              uint32_t r[2][16];
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            st_shared_v4(smem_u32(slice + lane * 128 + ((k ^ (lane & 7)) * 16)), w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
-          __syncwarp();
+              for (int q = 0; q < 2; ++q) tmem_ld16(lane_addr + Tm::kO + c + 16 * q, r[q]);   // past c_hi: not stored
+              tmem_wait_ld();
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const int r = 4 * k + (lane >> 3), blk = lane & 7;
-            const int head = quad * 32 + r;
-            const uint4 v = *reinterpret_cast<const uint4*>(slice + r * 128 + ((blk ^ (r & 7)) * 16));
-            if (head < p.H && c + 8 * blk < Lay::kPvN)
-              *reinterpret_cast<uint4*>(obase + (long long)head * p.DL + c + 8 * blk) = v;
+              for (int q = 0; q < 2; ++q)
+#pragma unroll
+                for (int i = 0; i < 16; ++i) w[16 * q + i] = __float_as_uint(__uint_as_float(r[q][i]) * inv);
+            }
+            __syncwarp();
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              st_shared_v4(smem_u32(slice + lane * 128 + ((k ^ (lane & 7)) * 16)), w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+            __syncwarp();
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const int r = 4 * k + (lane >> 3), blk = lane & 7;
+              const int head = quad * 32 + r;
+              const uint4 v = *reinterpret_cast<const uint4*>(slice + r * 128 + ((blk ^ (r & 7)) * 16));
+              if (head < p.H && c + 4 * blk < c_hi)
+                *reinterpret_cast<uint4*>(obase + (long long)head * p.DL + c + 4 * blk) = v;
+            }
           }
         }
       } else if (real_head) {
         // empty list: zeros (the exchange buffer may already hold the peer's next logits)
-        for (int c = 0; c < Lay::kPvN; c += 8)
-          *reinterpret_cast<uint4*>(obase + (long long)h * p.DL + c) = make_uint4(0, 0, 0, 0);
+        if (!partial) {
+          uint16_t* obase = p.out + (long long)bj * p.H * p.DL + rank * Lay::kPvN;
+          for (int c = c_lo; c < c_hi; c += 8)
+            *reinterpret_cast<uint4*>(obase + (long long)h * p.DL + c) = make_uint4(0, 0, 0, 0);
+        } else {
+          float* obase = p.part_o + (long long)un.rec * p.H * p.DL + rank * Lay::kPvN;
+          for (int c = c_lo; c < c_hi; c += 4)
+            *reinterpret_cast<uint4*>(obase + (long long)h * p.DL + c) = make_uint4(0, 0, 0, 0);
+        }
       }
-      if (real_head) {
+      if (real_head && wg == 0) {
         // a piece records the log-sum-exp of each CTA of the pair (their logits differ in the
         // last bits: each adds its own exact partial to the peer's decoded one)
         if (partial) p.part_lse[((long long)un.rec * 2 + rank) * p.H + h] = lse;
         else if (p.lse && rank == 0) p.lse[(long long)bj * p.H + h] = lse;
       }
-      if (ntiles > 0) {
+      if (ntiles > 0 && wg == 1) {
+        // warpgroup 1 staged through the whole exchange buffer of the last tile: it releases
+        // both halves (deferred from that tile)
         __syncwarp();
-        mbar_arrive_cluster_relaxed(&sb->sx_free[last_sbuf], peer);   // deferred from the unit's last tile
+        mbar_arrive_cluster_relaxed(&sb->sx_free[last_sbuf][0], peer);
+        mbar_arrive_cluster_relaxed(&sb->sx_free[last_sbuf][1], peer);
       }
       tc_fence_before();   // our reads of O come before the next unit's first P . C
     }
@@ -991,7 +1014,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 }
 
 // Log-sum-exp merge of the pieces of the queries that straddle a CTA-pair boundary.  One
-// (boundary, head) per DL/8 threads, 8 output dims per thread (16-byte loads of the bf16
+// (boundary, head) per DL/8 threads, 8 output dims per thread (two 16-byte loads of the fp32
 // partials); the first boundary inside a query merges all of that query's pieces: the last unit
 // of the pair before it, then the first unit of every pair that starts inside the query.
 constexpr int kCombineThreads = 256;
@@ -999,9 +1022,8 @@ constexpr int kCombineThreads = 256;
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineKernelParams p) {
   // every pair's first tile, computed once per CTA (one 64-bit division per thread at most)
   __shared__ long long starts[kAttnMaxPairs + 1];
-  const int TQ = p.tiles_per_q, C = p.n_pairs;
-  const long long G = p.total_tiles;
-  for (int i = threadIdx.x; i <= C; i += kCombineThreads) starts[i] = attn_pair_start(i, C, G);
+  const int TQ = p.tiles_per_q, C = p.split.C;
+  for (int i = threadIdx.x; i <= C; i += kCombineThreads) starts[i] = attn_pair_start(p.split, i);
   __syncthreads();
   pdl_launch_dependents();  // the dependent waits for this grid's completion before its loads
   pdl_wait_primary();
@@ -1023,13 +1045,15 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineK
     // the log-sum-exps and partial vectors of up to four pieces are loaded together, so a
     // merge of up to four pieces waits for one memory latency
     float ls[4];
-    uint4 v[4];
+    uint4 v[4][2];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const bool in = i < n;
       const long long e = in ? recs[i] : 0;
       ls[i] = in ? p.part_lse[(e * 2 + rank) * p.H + h] : -INFINITY;
-      v[i] = in ? ld_nc_v4(p.part_o + (e * p.H + h) * p.DL + d8) : make_uint4(0, 0, 0, 0);
+      const float* src = p.part_o + (e * p.H + h) * p.DL + d8;
+      v[i][0] = in ? ld_nc_v4(src) : make_uint4(0, 0, 0, 0);
+      v[i][1] = in ? ld_nc_v4(src + 4) : make_uint4(0, 0, 0, 0);
     }
     n = 0;
     float m_new = mx;
@@ -1043,12 +1067,9 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineK
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const float wgt = ls[i] == -INFINITY ? 0.0f : expf(ls[i] - m_new);
-      const uint32_t w4[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+      const uint32_t w8[8] = {v[i][0].x, v[i][0].y, v[i][0].z, v[i][0].w, v[i][1].x, v[i][1].y, v[i][1].z, v[i][1].w};
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        o[2 * k] += wgt * __uint_as_float(w4[k] << 16);
-        o[2 * k + 1] += wgt * __uint_as_float(w4[k] & 0xffff0000u);
-      }
+      for (int k = 0; k < 8; ++k) o[k] += wgt * __uint_as_float(w8[k]);
       wsum += wgt;
     }
     mx = m_new;
@@ -1131,7 +1152,7 @@ cudaError_t launch_combine(const CombineKernelParams& p, bool pdl, cudaStream_t 
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   const long long per_cta = kCombineThreads / (p.DL / 8);
-  cfg.gridDim = dim3((unsigned)(((long long)(p.n_pairs - 1) * p.H + per_cta - 1) / per_cta), 1, 1);
+  cfg.gridDim = dim3((unsigned)(((long long)(p.split.C - 1) * p.H + per_cta - 1) / per_cta), 1, 1);
   cfg.blockDim = dim3(kCombineThreads, 1, 1);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
