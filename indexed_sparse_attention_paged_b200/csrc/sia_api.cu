@@ -48,6 +48,27 @@ int sm_count() {
   return n;
 }
 
+// CTA pairs of the attention grid that run at once on the current device: half the SMs, or
+// fewer when the GPCs' SM counts leave some SMs that no 2-CTA cluster can use.  A grid with
+// more pairs than this would run the extra ones as a second wave.
+int attend_pairs(int dl, int dr, bool kv8) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+  static std::atomic<int> cached[64][2];   // + 1, so that 0 means "not looked up yet"
+  const int half = std::max(1, sm_count() / 2);
+  const bool small = dl != 512;
+  if (dev < 0 || dev >= 64 || small) {
+    const int n = attend_max_clusters(dl, dr, kv8);
+    return n > 0 ? std::min(half, n) : half;
+  }
+  const int c = cached[dev][kv8 ? 1 : 0].load(std::memory_order_relaxed);
+  if (c > 0) return c - 1;
+  const int n = attend_max_clusters(dl, dr, kv8);
+  const int pairs = n > 0 ? std::min(half, n) : half;
+  cached[dev][kv8 ? 1 : 0].store(pairs + 1, std::memory_order_relaxed);
+  return pairs;
+}
+
 int max_smem_optin() {
   int dev = 0, v = 232448;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
@@ -336,19 +357,26 @@ sia_status plan_attend(const sia_attend_args* a, AttendPlan* pl, bool make_maps,
   k.K = a->top_k;
   k.scale_log2 = a->softmax_scale * 1.4426950408889634f;
   const long long bj = (long long)a->batch * a->n_q;
-  const int pairs = std::max(1, sm_count() / 2);
+  const int pairs = attend_pairs(a->d_latent, a->d_rope, a->kv_scale != nullptr);
   // the flat (query, 64-row tile) list split evenly over the CTA pairs (see attn_next_unit)
   const long long TQ = (a->top_k + kAttnTileRows - 1) / kAttnTileRows;
   const long long G = bj * TQ;
   if (G > 0x7fffffffll) return fail(SIA_ERR_UNSUPPORTED, "batch * n_q * ceil(top_k / 64) must fit in int32");
-  const int C = (int)std::min<long long>(std::min(pairs, kAttnMaxPairs), G);
+  // With at most as many queries as pairs, every query gets the same number s of pairs and the
+  // even split then puts each pair inside one query (pair c's range starts at c TQ / s): a pair
+  // that moves on to a second query pays that query's start (its query rows, its first gathers)
+  // and the first one's output on its critical path, which costs more than the few tiles an
+  // uneven count saves.  With more queries than pairs, the flat list is split evenly.
+  const bool per_query = bj <= pairs;
+  const int C = per_query ? (int)(std::min<long long>(pairs / bj, TQ) * bj)
+                          : (int)std::min<long long>(std::min(pairs, kAttnMaxPairs), G);
   k.tiles_per_q = (int)TQ;
   k.split.G = G;
   k.split.C = C;
   k.split.n_early = C;
   k.split.w_early = 1;
   k.split.w_late = 1;
-  if (busy_sms > 0) {
+  if (busy_sms > 0 && !per_query) {
     // the late pairs start about when the preceding grid ends, a few microseconds into a stage
     // of some tens: 7/8 of the work of an early pair
     k.split.n_early = std::max(0, std::min(C, (sm_count() - busy_sms) / 2));

@@ -158,6 +158,8 @@ cudaError_t launch_cache_append(const AppendKernelParams& p, cudaStream_t stream
 
 // Shared memory the attention kernel needs for (d_latent, d_rope).
 size_t attend_smem_bytes(int dl, int dr);
+// 2-CTA clusters of the attention kernel the current device holds at once; 0 if unknown.
+int attend_max_clusters(int dl, int dr, bool kv8);
 
 // Limit of every bounded in-kernel wait, in nanoseconds (set by sia_set_wait_limit_ns).
 uint64_t wait_limit_ns();

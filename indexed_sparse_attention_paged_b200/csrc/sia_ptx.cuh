@@ -77,6 +77,22 @@ __device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint64_t* bar, uint3
       : "memory");
 }
 
+// One arrival per warp, for barriers counted in warps: __syncwarp orders every lane's prior
+// accesses (and their fences) before lane 0's arrive, and 32 arrivals on one barrier word would
+// serialise.  All 32 lanes must call it at the same point.
+__device__ __forceinline__ void mbar_arrive_warp(uint64_t* bar) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+__device__ __forceinline__ void mbar_arrive_cluster_warp(uint64_t* bar, uint32_t cta) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive_cluster(bar, cta);
+}
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed_warp(uint64_t* bar, uint32_t cta) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive_cluster_relaxed(bar, cta);
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -168,6 +184,26 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity, int32
   }
 }
 
+// ------------------------------------------------------------------ bulk copies inside a cluster
+
+// Arrive on the barrier at the same offset in CTA `cta` of the cluster, adding `bytes` to the
+// transaction count its current phase waits for (the bytes of a bulk copy issued next).
+__device__ __forceinline__ void mbar_arrive_expect_tx_remote(uint64_t* bar, uint32_t cta, uint32_t bytes);
+
+// Bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned) from this CTA's shared
+// memory to shared::cluster address `dst`; its bytes complete on the barrier at shared::cluster
+// address `bar` (no multicast).
+__device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(dst), "r"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// this thread's committed bulk copies have read their sources
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// this thread's committed bulk copies are complete
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // ------------------------------------------------------------------ proxies, PDL, cluster
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -215,6 +251,12 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t local, uint32_t cta) {
 }
 
 // 16-byte load from cluster shared memory (no memory clobber, so several can be in flight).
+__device__ __forceinline__ void mbar_arrive_expect_tx_remote(uint64_t* bar, uint32_t cta, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.relaxed.cluster.shared::cluster.b64 _, [%0], %1;"
+               ::"r"(mapa_shared(smem_u32(bar), cta)), "r"(bytes)
+               : "memory");
+}
+
 __device__ __forceinline__ uint4 ld_cluster_v4(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];"

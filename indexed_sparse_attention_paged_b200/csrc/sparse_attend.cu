@@ -147,23 +147,29 @@ struct AttnSmem {
   static constexpr uint32_t kOffR = kOffC + kStages * kCStageBytes;
   // P (bf16, 128 heads x kRows, 128B-swizzled K-major): the A operand of P . C
   static constexpr uint32_t kOffP = (kOffR + kRopeSlots * kCRopeBytes + 1023u) & ~1023u;
-  // the peer's partial logits of two tiles, int16 with one power-of-two scale per head: the
-  // peer's exchange warps fill one buffer while this CTA's softmax reads the other
-  static constexpr uint32_t kSxBytes = kRows * 128 * 2;
+  // Partial-logit exchange.  One block per half of a tile's rows (one softmax warpgroup): 32
+  // rows x 128 heads of int16 codes ([row / 8][head] in 16-byte groups of 8 rows), then the 128
+  // heads' power-of-two scale exponents (int32).  Sx holds the blocks the peer copies in for two
+  // tiles ([tile parity][half]); Xs this CTA's own two halves, staged for those bulk copies.
+  static constexpr uint32_t kSxCodes = (kRows / 2) * 128 * 2;
+  static constexpr uint32_t kSxHalf = kSxCodes + 128 * 4;
   static constexpr uint32_t kOffSx = kOffP + 128 * kRows * 2;
-  static constexpr uint32_t kOffSxExp = kOffSx + 2 * kSxBytes;      // [2 tiles][2 halves][128] int32
+  static constexpr uint32_t kOffXs = kOffSx + 4 * kSxHalf;
   // the two softmax warpgroups' per-head tile maxima [2 tiles][2][128] and unit sums [2][128]
-  static constexpr uint32_t kOffMx = kOffSxExp + 2 * 2 * 128 * 4;
+  static constexpr uint32_t kOffMx = kOffXs + 2 * kSxHalf;
   static constexpr uint32_t kOffL = kOffMx + 2 * 2 * 128 * 4;
+  // the physical cache row of each Top-K entry of the unit being gathered (read by the gather
+  // threads only, which rebuild it between units), then per unit (double-buffered) the validity
+  // bits and each gather warp's lowest position of a -1 entry
   static constexpr uint32_t kOffRows = kOffL + 2 * 128 * 4;
-  // per unit (double-buffered): physical cache row of each Top-K entry, validity bits, and
-  // each gather warp's lowest position of a -1 entry
-  static constexpr uint32_t kOffMask = kOffRows + 2 * kAttnMaxSplitRows * 4;
+  static constexpr uint32_t kOffMask = kOffRows + kAttnMaxSplitRows * 4;
   static constexpr uint32_t kOffFirstNeg = kOffMask + 2 * (kAttnMaxSplitRows / 8);
   static constexpr uint32_t kOffBar = kOffFirstNeg + 2 * kProducerWarps * 4;
   static constexpr uint32_t kBarBytes = 512;
   static constexpr uint32_t kBytes = kOffBar + kBarBytes;
   static_assert(kOffP % 1024 == 0, "P must sit on a 1024-byte swizzle atom");
+  static_assert(kSxHalf % 16 == 0 && kOffSx % 16 == 0 && kOffXs % 16 == 0, "bulk copies move 16-byte units");
+  static_assert(2 * kSxHalf >= 4 * 4096, "a tile's two halves also stage one warpgroup's output slices");
   static_assert(kBytes <= 232448, "shared memory over the 227 KB a CTA may opt into");
 };
 
@@ -179,6 +185,8 @@ struct AttnBarriers {
   uint64_t q_tma;                 // the rope part of q landed (TMA bytes only)
   uint64_t o_full;
   uint64_t sx_ready[2][2], sx_free[2][2];   // [tile][half]: the peer's half landed / was read
+  uint64_t xs_free[2], xs_full[2];          // [half]: staging reusable / staged by all 128 threads
+  uint64_t g_sync;                          // every gather thread issued the unit's tiles
   uint64_t tab_full[2], tab_free[2];
   uint64_t mma_done, pv_done;
   uint64_t g_loaded[2];             // FP8 cache: every gather thread read its staged codes
@@ -278,7 +286,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   using Tm = AttnTmem<Lay>;
   extern __shared__ __align__(1024) uint8_t smem[];
   AttnBarriers* sb = reinterpret_cast<AttnBarriers*>(smem + Sm::kOffBar);
-  int32_t* rows_tab = reinterpret_cast<int32_t*>(smem + Sm::kOffRows);        // [2][max rows]
+  int32_t* rows_tab = reinterpret_cast<int32_t*>(smem + Sm::kOffRows);        // [max rows]
   uint32_t* mask_tab = reinterpret_cast<uint32_t*>(smem + Sm::kOffMask);      // [2][max rows/32]
   int32_t* fneg_tab = reinterpret_cast<int32_t*>(smem + Sm::kOffFirstNeg);    // [2][gather warps]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -300,27 +308,32 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     for (int s = 0; s < kRopeSlots; ++s) mbar_init(&sb->r_empty[s], 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sb->s_full[s], 1);
-      mbar_init(&sb->s_empty[s], 256);         // both softmax warpgroups
-      mbar_init(&sb->mx_bar[s], 256);
-      mbar_init(&sb->tab_full[s], kProducerWarps * 32);
-      mbar_init(&sb->tab_free[s], 256 + 2);   // both softmax warpgroups and both MMA threads
+      mbar_init(&sb->s_empty[s], 8);           // the 8 softmax warps (one arrival per warp)
+      mbar_init(&sb->mx_bar[s], 8);
+      mbar_init(&sb->tab_full[s], kProducerWarps);
+      mbar_init(&sb->tab_free[s], 8 + 2);     // the softmax warps and both MMA threads
     }
-    mbar_init(&sb->p_full, 256);
+    mbar_init(&sb->p_full, 8);
     mbar_init(&sb->p_empty, 1);
-    mbar_init(&sb->epi_sync, 256);
-    mbar_init(&sb->q_full, 256);       // the 256 TMEM writers
+    mbar_init(&sb->epi_sync, 8);
+    mbar_init(&sb->q_full, 8);         // the 8 warps writing q into TMEM
     mbar_init(&sb->q_tma, 1);          // the rope TMA (or a plain arrive when this CTA has none)
     mbar_init(&sb->q_empty, 1);
     mbar_init(&sb->o_full, 1);
     for (int s = 0; s < 2; ++s)
       for (int g = 0; g < 2; ++g) {
-        mbar_init(&sb->sx_ready[s][g], 128);   // arrived by the peer's warpgroup g
-        mbar_init(&sb->sx_free[s][g], 128);
+        mbar_init(&sb->sx_ready[s][g], 1);   // the peer's copy: its leader's arrive + the bytes
+        mbar_init(&sb->sx_free[s][g], 4);    // the 4 warps of the peer's warpgroup g
       }
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(&sb->xs_free[g], 1);
+      mbar_init(&sb->xs_full[g], 4);
+    }
+    mbar_init(&sb->g_sync, kProducerWarps);
     mbar_init(&sb->mma_done, 1);
     mbar_init(&sb->pv_done, 1);
-    mbar_init(&sb->g_loaded[0], kProducerWarps * 32);
-    mbar_init(&sb->g_loaded[1], kProducerWarps * 32);
+    mbar_init(&sb->g_loaded[0], kProducerWarps);
+    mbar_init(&sb->g_loaded[1], kProducerWarps);
     sb->abort = 0;
     fence_mbarrier_init();
     tma_prefetch_desc(&maps.q_rope);
@@ -396,19 +409,30 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const AttnRange rg{attn_pair_start(p.split, cluster_id), attn_pair_start(p.split, cluster_id + 1)};
     long long cursor = rg.g0;
     AttnUnit un;
-    if (cursor < rg.g1) {
-      // While the previous kernel still runs: touch every cache page of the first unit's
-      // sequence (address translation and the page-table row warm up before the gather)
-      const int b = (int)(cursor / p.tiles_per_q) / p.J;
+    // Touch every cache page of sequence b (one line of this CTA's half per page): the address
+    // translations and the page-table row are then warm when the unit's rows are gathered.  A
+    // unit that started on cold translations waited microseconds for its first tile.
+    auto touch_pages = [&](int b) {
       const int L = p.seq_lens[b];
       const int npages = min(p.max_pages, (L + p.P - 1) / p.P);
       const int32_t* pt_row = p.page_table + (long long)b * p.max_pages;
-      const uint8_t* kv = static_cast<const uint8_t*>(p.kv);
       for (int i = ptid; i < npages; i += kProducerWarps * 32) {
         const int pg = pt_row[i];
         if (pg >= 0 && pg < p.num_pages)
           asm volatile("prefetch.global.L2 [%0];" ::"l"(kv + ((size_t)pg * p.P * DC + (size_t)rank * (p.DL / 2)) * (KV8 ? 1 : 2)));
       }
+    };
+    // while the previous kernel still runs: the sequences of all of this pair's units, and the
+    // latent half of their query rows that this CTA loads into TMEM at each unit's start
+    if (cursor < rg.g1) {
+      const int bj_lo = (int)(rg.g0 / p.tiles_per_q), bj_hi = (int)((rg.g1 - 1) / p.tiles_per_q);
+      for (int b = bj_lo / p.J; b <= bj_hi / p.J; ++b) touch_pages(b);
+      constexpr int kLines = Lay::kLatDims * 2 >= 128 ? Lay::kLatDims * 2 / 128 : 1;   // 128-byte lines per head row
+      for (int bj = bj_lo; bj <= bj_hi; ++bj)
+        for (int i = ptid; i < p.H * kLines; i += kProducerWarps * 32)
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(static_cast<const uint8_t*>(p.q) +
+                                                        ((size_t)bj * p.H + i / kLines) * (DC * 2) +
+                                                        (size_t)rank * Lay::kLatDims * 2 + (i % kLines) * 128));
     }
     while (ok && attn_next_unit(p, cluster_id, rg, cursor, un)) {
       const int bj = un.bj;
@@ -438,7 +462,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // resolve this unit's Top-K entries to physical cache rows: 8 entries per thread, all
       // loads of a thread in flight at once
       if (!mbar_wait_warp(&sb->tab_free[buf], ((uint32_t)(u_it >> 1) & 1u) ^ 1u, wc)) { ok = false; break; }
-      int32_t* rt = rows_tab + buf * kAttnMaxSplitRows;
+      int32_t* rt = rows_tab;
       uint32_t* mt = mask_tab + buf * (kAttnMaxSplitRows / 32);
       const int32_t* tk = p.topk + row_base + row0;
       const int32_t* pt_row = p.page_table + (long long)b * p.max_pages;
@@ -451,6 +475,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
 #pragma unroll
       for (int k = 0; k < kPer; ++k) pg[k] = (idx[k] >= 0 && idx[k] < L) ? pt_row[idx[k] / p.P] : -1;
+      // the row table is rewritten once every gather thread has issued the previous unit's tiles
+      if (u_it > 0 && !mbar_wait_warp(&sb->g_sync, (uint32_t)(u_it - 1) & 1u, wc)) { ok = false; break; }
       int fneg = nrows;
 #pragma unroll
       for (int k = 0; k < kPer; ++k) {
@@ -472,7 +498,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) fneg = min(fneg, __shfl_xor_sync(0xffffffffu, fneg, o));
       if (lane == 0) fneg_tab[buf * kProducerWarps + pwarp] = fneg;
-      mbar_arrive(&sb->tab_full[buf]);
+      mbar_arrive_warp(&sb->tab_full[buf]);
       if (!mbar_wait_warp(&sb->tab_full[buf], (uint32_t)(u_it >> 1) & 1u, wc)) { ok = false; break; }
       const int ntiles = (unit_tiles(buf) + kRows - 1) / kRows;
       if constexpr (!KV8) {
@@ -536,7 +562,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               asm volatile("ld.shared.f32 %0, [%1];" : "=f"(sc[j]) : "r"(lat_base + (uint32_t)(ptid * kP8 + j) * 4u));
             }
           }
-          mbar_arrive(&sb->g_loaded[it_ & 1]);
+          mbar_arrive_warp(&sb->g_loaded[it_ & 1]);
           if (!mbar_wait_warp(&sb->g_loaded[it_ & 1], (uint32_t)(it_ >> 1) & 1u, wc)) return false;
 #pragma unroll
           for (int j = 0; j < kP8; ++j) {
@@ -584,6 +610,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (!convert8(prev_stage, prev_rslot, it - 1)) { ok = false; break; }
         }
       }
+      if (!ok) break;
+      mbar_arrive_warp(&sb->g_sync);   // this warp is done with the row table
       ++u_it;
     }
     // our copies have landed before we may leave, whether or not the CTA is aborting: every
@@ -701,7 +729,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int h = quad * 32 + lane;   // head = TMEM lane
     const uint32_t lane_addr = tmem_base + ((uint32_t)(quad * 32) << 16);
     const uint32_t sx_peer = mapa_shared(smem_u32(smem + Sm::kOffSx), peer);
-    const uint32_t sxexp_peer = mapa_shared(smem_u32(smem + Sm::kOffSxExp), peer);
+    const bool leader = (threadIdx.x & 127) == 0;   // issues this warpgroup's bulk copies
     float* mxbuf = reinterpret_cast<float*>(smem + Sm::kOffMx);   // [2 tiles][2 warpgroups][128]
     float* lbuf = reinterpret_cast<float*>(smem + Sm::kOffL);     // [2 warpgroups][128]
     int s_it = 0, u_it = 0, o_it = 0, e_it = 0;
@@ -715,178 +743,215 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int bj = un.bj;
       const int buf = u_it & 1;
       {
-        // q: head h's dims [rank * kLatDims, +kLatDims) as bf16 pairs, 16 columns per store;
-        // the warpgroups split the column groups
-        if (!mbar_wait_warp(&sb->q_empty, ((uint32_t)u_it & 1u) ^ 1u, wc)) { ok = false; break; }
+        // q: head h's dims [rank * kLatDims, +kLatDims) as bf16 pairs, 16 columns (64 bytes) per
+        // TMEM store; the warpgroups split the column groups.  All of a thread's loads are in
+        // flight at once (the gather warps fetched the rows into L2 at the start).
+        constexpr int kGroups = Lay::kLatDims / 32;
+        constexpr int kGPer = (kGroups + 1) / 2;
+        const int g_lo = wg == 0 ? 0 : kGPer, g_hi = wg == 0 ? kGPer : kGroups;
         const bool real = h < p.H;
-        const uint8_t* qrow = static_cast<const uint8_t*>(p.q) + ((long long)bj * p.H + (real ? h : 0)) * (DC * 2) +
-                              (size_t)rank * Lay::kLatDims * 2;
-        constexpr int kGroups = Lay::kLatDims / 32;   // 64 bytes = 16 columns each
-        const int g_lo = wg == 0 ? 0 : (kGroups + 1) / 2, g_hi = wg == 0 ? (kGroups + 1) / 2 : kGroups;
-        if (real)
-          for (int g = g_lo; g < g_hi; g += 2) asm volatile("prefetch.global.L2 [%0];" ::"l"(qrow + g * 64));
-        tc_fence_after();
-#pragma unroll 1
-        for (int g = g_lo; g < g_hi; ++g) {
-          uint32_t w[16];
+        const size_t q_off = ((size_t)(real ? h : 0)) * (DC * 2) + (size_t)rank * Lay::kLatDims * 2;
+        const uint8_t* qrow = static_cast<const uint8_t*>(p.q) + (size_t)bj * p.H * (DC * 2) + q_off;
+        uint4 qv[kGPer][4];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const uint4 v = real ? ld_nc_v4(qrow + g * 64 + 16 * i) : make_uint4(0, 0, 0, 0);
-            w[4 * i] = v.x;
-            w[4 * i + 1] = v.y;
-            w[4 * i + 2] = v.z;
-            w[4 * i + 3] = v.w;
+        for (int j = 0; j < kGPer; ++j)
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            qv[j][i] = real && g_lo + j < g_hi ? ld_nc_v4(qrow + (g_lo + j) * 64 + 16 * i) : make_uint4(0, 0, 0, 0);
+        if (!mbar_wait_warp(&sb->q_empty, ((uint32_t)u_it & 1u) ^ 1u, wc)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int j = 0; j < kGPer; ++j) {
+          if (g_lo + j < g_hi) {   // warp-uniform
+            const uint32_t w[16] = {qv[j][0].x, qv[j][0].y, qv[j][0].z, qv[j][0].w, qv[j][1].x, qv[j][1].y,
+                                    qv[j][1].z, qv[j][1].w, qv[j][2].x, qv[j][2].y, qv[j][2].z, qv[j][2].w,
+                                    qv[j][3].x, qv[j][3].y, qv[j][3].z, qv[j][3].w};
+            tmem_st16(lane_addr + Tm::kQ + (uint32_t)(16 * (g_lo + j)), w);
           }
-          tmem_st16(lane_addr + Tm::kQ + (uint32_t)(16 * g), w);
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&sb->q_full);
+        mbar_arrive_warp(&sb->q_full);
       }
       if (!mbar_wait_warp(&sb->tab_full[buf], (uint32_t)(u_it >> 1) & 1u, wc)) { ok = false; break; }
       const int first_neg = unit_tiles(buf);
       const int ntiles = (first_neg + kRows - 1) / kRows;
       const uint32_t* mt = mask_tab + buf * (kAttnMaxSplitRows / 32);
       float m = -INFINITY, l = 0.0f;   // m is the same in both warpgroups; l covers this half
-      float s[kHalf];
-      for (int t = 0; t < ntiles; ++t, ++s_it) {
-        const int sbuf = s_it & 1;
-        uint32_t valid = mt[2 * t + wg];                  // this half's 32 rows
-        const int live = first_neg - t * kRows - wg * kHalf;   // rows past the first -1 are padding
-        if (live < kHalf) valid &= live > 0 ? (1u << live) - 1u : 0u;
-        if (!mbar_wait_warp(&sb->s_full[sbuf], (uint32_t)(s_it >> 1) & 1u, wc)) { ok = false; break; }
-        tc_fence_after();
-        uint32_t enc[kHalf / 2];
-        int e;
-        {
-          uint32_t r[2][16];
-#pragma unroll
-          for (int c = 0; c < 2; ++c) tmem_ld16(lane_addr + Tm::kS + sbuf * kRows + wg * kHalf + c * 16, r[c]);
-          tmem_wait_ld();
-          float amax = 0.0f;
-#pragma unroll
-          for (int c = 0; c < 2; ++c)
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              s[16 * c + i] = __uint_as_float(r[c][i]);
-              amax = fmaxf(amax, fabsf(s[16 * c + i]));
-            }
-          amax *= fabsf(p.scale_log2);
-          // e with amax 2^e < 2^14: amax < 2^E for E = (biased exponent of amax) - 126
-          const int E = (int)((__float_as_uint(amax) >> 23) & 0xffu) - 126;
-          e = amax > 0.0f ? min(max(14 - E, -100), 100) : 0;
-          const float sc = p.scale_log2 * __uint_as_float((uint32_t)(127 + e) << 23);
-#pragma unroll
-          for (int i = 0; i < kHalf / 2; ++i) {
-            const float y0 = fmaf(s[2 * i], sc, kMagic);
-            const float y1 = fmaf(s[2 * i + 1], sc, kMagic);
-            enc[i] = prmt(__float_as_uint(y0), __float_as_uint(y1), 0x5410u);
+      // Software pipeline over the unit's tiles: pass t first sends tile t+1's partial logits to
+      // the peer (read from TMEM, encoded, stored into the peer's exchange buffer), then finishes
+      // tile t, whose peer half arrived during pass t-1, so each DSMEM transfer overlaps the
+      // softmax of the tile before it.  s holds this warpgroup's exact fp32 partials of tile t,
+      // sn those of tile t+1.
+      float s[kHalf], sn[kHalf];
+      const int it0 = s_it;
+      for (int t = -1; t < ntiles; ++t) {
+        if (t + 1 < ntiles) {
+          const int it1 = it0 + t + 1, sb1 = it1 & 1;
+          // This half's partial logits go to the peer as int16 codes with one power-of-two scale
+          // per head, staged here and copied into the peer's buffer of the same tile parity and
+          // half with one bulk copy by the warpgroup's leader.  The staging is reused once the
+          // previous copy has read it.
+          if (leader) {
+            bulk_wait_read_all();
+            mbar_arrive(&sb->xs_free[wg]);
           }
-        }
-        tc_fence_before();
-        mbar_arrive(&sb->s_empty[sbuf]);   // this warpgroup's reads of the partial are done
-        // send this half to the peer (the peer's same warpgroup reads it)
-        if (!mbar_wait_warp<true>(&sb->sx_free[sbuf][wg], ((uint32_t)(s_it >> 1) & 1u) ^ 1u, wc)) { ok = false; break; }
+          if (!mbar_wait_warp(&sb->xs_free[wg], (uint32_t)it1 & 1u, wc)) { ok = false; break; }
+          if (!mbar_wait_warp(&sb->s_full[sb1], (uint32_t)(it1 >> 1) & 1u, wc)) { ok = false; break; }
+          tc_fence_after();
+          uint8_t* xs = smem + Sm::kOffXs + wg * Sm::kSxHalf;
+          {
+            uint32_t r[2][16];
 #pragma unroll
-        for (int gi = 0; gi < kHalf / 8; ++gi) {
-          const uint32_t dst = sx_peer + sbuf * Sm::kSxBytes + (uint32_t)(((wg * (kHalf / 8) + gi) * 128 + h) * 16);
-          asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(enc[4 * gi]),
-                       "r"(enc[4 * gi + 1]), "r"(enc[4 * gi + 2]), "r"(enc[4 * gi + 3])
-                       : "memory");
-        }
-        asm volatile("st.shared::cluster.b32 [%0], %1;" ::"r"(sxexp_peer + (uint32_t)(((sbuf * 2 + wg) * 128 + h) * 4)), "r"(e)
-                     : "memory");
-        mbar_arrive_cluster(&sb->sx_ready[sbuf][wg], peer);
-        // the peer's half for the same rows: logit = own exact partial + decoded peer partial
-        if (!mbar_wait_warp<true>(&sb->sx_ready[sbuf][wg], (uint32_t)(s_it >> 1) & 1u, wc)) { ok = false; break; }
-        last_sbuf = sbuf;
-        {
-          const int pe = *reinterpret_cast<const int*>(smem + Sm::kOffSxExp + ((sbuf * 2 + wg) * 128 + h) * 4);
-          const float dn = __uint_as_float((uint32_t)(127 - pe) << 23);
-          const float bias = -kMagic * dn;
-#pragma unroll
-          for (int gi = 0; gi < kHalf / 8; ++gi) {
-            const uint4 pv4 = *reinterpret_cast<const uint4*>(smem + Sm::kOffSx + sbuf * Sm::kSxBytes +
-                                                              ((wg * (kHalf / 8) + gi) * 128 + h) * 16);
-            const uint32_t q4[4] = {pv4.x, pv4.y, pv4.z, pv4.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const float f0 = __uint_as_float(prmt(q4[i], 0x4B000000u, 0x7610u));
-              const float f1 = __uint_as_float(prmt(q4[i], 0x4B000000u, 0x7632u));
-              s[8 * gi + 2 * i] = fmaf(s[8 * gi + 2 * i], p.scale_log2, fmaf(f0, dn, bias));
-              s[8 * gi + 2 * i + 1] = fmaf(s[8 * gi + 2 * i + 1], p.scale_log2, fmaf(f1, dn, bias));
-            }
-          }
-        }
-        // the peer may refill its half of the exchange buffer; after the unit's last tile the
-        // buffer first serves the epilogue (released there)
-        if (t + 1 < ntiles) mbar_arrive_cluster_relaxed(&sb->sx_free[sbuf][wg], peer);
-
-        // online softmax (base 2), lazy rescale; the two halves agree on the tile max
-        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-        if (valid == ~0u) {
-#pragma unroll
-          for (int i = 0; i < kHalf; ++i) mx[i & 3] = fmaxf(mx[i & 3], s[i]);
-        } else {
-#pragma unroll
-          for (int i = 0; i < kHalf; ++i) {
-            s[i] = (valid >> i & 1u) ? s[i] : -INFINITY;
-            mx[i & 3] = fmaxf(mx[i & 3], s[i]);
-          }
-        }
-        const float mine = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-        mxbuf[(sbuf * 2 + wg) * 128 + h] = mine;
-        mbar_arrive(&sb->mx_bar[sbuf]);
-        if (!mbar_wait_warp(&sb->mx_bar[sbuf], (uint32_t)(s_it >> 1) & 1u, wc)) { ok = false; break; }
-        const float mt_ = fmaxf(mine, mxbuf[(sbuf * 2 + (wg ^ 1)) * 128 + h]);
-        float alpha = 1.0f;
-        const bool need = mt_ > m + 8.0f;
-        if (need) {
-          alpha = fast_exp2(m - mt_);   // 0 when m is -inf
-          m = mt_;
-        }
-        float ps[4] = {0.f, 0.f, 0.f, 0.f};
-        if (m != -INFINITY) {
-          // masked logits are -inf and m is finite: their exp2 is exactly 0
-#pragma unroll
-          for (int i = 0; i < kHalf; ++i) {
-            s[i] = fast_exp2(s[i] - m);
-            ps[i & 3] += s[i];
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < kHalf; ++i) s[i] = 0.0f;
-        }
-        l = l * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
-
-        // P . C of the previous tile must be done: it reads the P buffer, and O is rescaled
-        if (!mbar_wait_warp(&sb->p_empty, ((uint32_t)s_it & 1u) ^ 1u, wc)) { ok = false; break; }
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, need && t > 0)) {
-          // O holds the tiles < t of this unit: each warpgroup rescales half of its columns
-#pragma unroll 1
-          for (int c = wg * (Lay::kPvN / 2); c < (wg + 1) * (Lay::kPvN / 2); c += 16) {
-            uint32_t r[16];
-            tmem_ld16(lane_addr + Tm::kO + c, r);
+            for (int c = 0; c < 2; ++c) tmem_ld16(lane_addr + Tm::kS + sb1 * kRows + wg * kHalf + c * 16, r[c]);
             tmem_wait_ld();
+            float amax = 0.0f;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-            tmem_st16(lane_addr + Tm::kO + c, r);
+            for (int c = 0; c < 2; ++c)
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                sn[16 * c + i] = __uint_as_float(r[c][i]);
+                amax = fmaxf(amax, fabsf(sn[16 * c + i]));
+              }
+            amax *= fabsf(p.scale_log2);
+            // e with amax 2^e < 2^14: amax < 2^E for E = (biased exponent of amax) - 126
+            const int E = (int)((__float_as_uint(amax) >> 23) & 0xffu) - 126;
+            const int e = amax > 0.0f ? min(max(14 - E, -100), 100) : 0;
+            const float sc = p.scale_log2 * __uint_as_float((uint32_t)(127 + e) << 23);
+#pragma unroll
+            for (int gi = 0; gi < kHalf / 8; ++gi) {
+              uint32_t enc[4];
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const float y0 = fmaf(sn[8 * gi + 2 * i], sc, kMagic);
+                const float y1 = fmaf(sn[8 * gi + 2 * i + 1], sc, kMagic);
+                enc[i] = prmt(__float_as_uint(y0), __float_as_uint(y1), 0x5410u);
+              }
+              st_shared_v4(smem_u32(xs + (gi * 128 + h) * 16), enc[0], enc[1], enc[2], enc[3]);
+            }
+            *reinterpret_cast<int*>(xs + Sm::kSxCodes + h * 4) = e;
           }
-          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive_warp(&sb->s_empty[sb1]);   // this warpgroup's reads of the partial are done
+          fence_proxy_async_smem();           // the copy reads the staging through the async proxy
+          mbar_arrive_warp(&sb->xs_full[wg]);
+          bool sent = true;
+          if (leader) {
+            // the peer's buffer was last released either after its reads of tile it1 - 2
+            // (nothing to order against the copy) or, when that tile ended the previous unit,
+            // after the peer staged its output through it (generic stores: acquire them)
+            const uint32_t par = ((uint32_t)(it1 >> 1) & 1u) ^ 1u;
+            sent = mbar_wait(&sb->xs_full[wg], (uint32_t)it1 & 1u, wc) &&
+                   (t == 0 ? mbar_wait<true>(&sb->sx_free[sb1][wg], par, wc) : mbar_wait(&sb->sx_free[sb1][wg], par, wc));
+            if (sent) {
+              mbar_arrive_expect_tx_remote(&sb->sx_ready[sb1][wg], peer, Sm::kSxHalf);
+              bulk_copy_to_cluster(sx_peer + (uint32_t)((sb1 * 2 + wg) * Sm::kSxHalf), smem_u32(xs), Sm::kSxHalf,
+                                   mapa_shared(smem_u32(&sb->sx_ready[sb1][wg]), peer));
+              bulk_commit();
+            }
+          }
+          if (!__shfl_sync(0xffffffffu, sent, 0)) { ok = false; break; }
         }
-        // this half of P (bf16) into shared memory: head h's row, K columns [32 wg, 32 wg + 32)
+        if (t >= 0) {
+          const int it = it0 + t, sbuf = it & 1;
+          uint32_t valid = mt[2 * t + wg];                  // this half's 32 rows
+          const int live = first_neg - t * kRows - wg * kHalf;   // rows past the first -1 are padding
+          if (live < kHalf) valid &= live > 0 ? (1u << live) - 1u : 0u;
+          // the peer's half for the same rows: logit = own exact partial + decoded peer partial
+          // (the bytes come from the peer's bulk copy: the barrier's completion makes them visible)
+          if (!mbar_wait_warp(&sb->sx_ready[sbuf][wg], (uint32_t)(it >> 1) & 1u, wc)) { ok = false; break; }
+          last_sbuf = sbuf;
+          {
+            const uint8_t* rx = smem + Sm::kOffSx + (sbuf * 2 + wg) * Sm::kSxHalf;
+            const int pe = *reinterpret_cast<const int*>(rx + Sm::kSxCodes + h * 4);
+            const float dn = __uint_as_float((uint32_t)(127 - pe) << 23);
+            const float bias = -kMagic * dn;
 #pragma unroll
-        for (int k = 0; k < kHalf / 8; ++k)
-          st_shared_v4(smem_u32(smem + Sm::kOffP + swizzled_offset((uint32_t)h, (uint32_t)(wg * (kHalf / 8) + k) * 16, 128)),
-                       pack_bf16x2(s[8 * k], s[8 * k + 1]), pack_bf16x2(s[8 * k + 2], s[8 * k + 3]),
-                       pack_bf16x2(s[8 * k + 4], s[8 * k + 5]), pack_bf16x2(s[8 * k + 6], s[8 * k + 7]));
-        fence_proxy_async_smem();
-        tc_fence_before();
-        mbar_arrive(&sb->p_full);   // P written (and O rescaled) by this thread
+            for (int gi = 0; gi < kHalf / 8; ++gi) {
+              const uint4 pv4 = *reinterpret_cast<const uint4*>(rx + (gi * 128 + h) * 16);
+              const uint32_t q4[4] = {pv4.x, pv4.y, pv4.z, pv4.w};
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const float f0 = __uint_as_float(prmt(q4[i], 0x4B000000u, 0x7610u));
+                const float f1 = __uint_as_float(prmt(q4[i], 0x4B000000u, 0x7632u));
+                s[8 * gi + 2 * i] = fmaf(s[8 * gi + 2 * i], p.scale_log2, fmaf(f0, dn, bias));
+                s[8 * gi + 2 * i + 1] = fmaf(s[8 * gi + 2 * i + 1], p.scale_log2, fmaf(f1, dn, bias));
+              }
+            }
+          }
+          // the peer may refill its half of the exchange buffer; after the unit's last tile the
+          // buffer first serves the epilogue (released there)
+          if (t + 1 < ntiles) mbar_arrive_cluster_relaxed_warp(&sb->sx_free[sbuf][wg], peer);
+
+          // online softmax (base 2), lazy rescale; the two halves agree on the tile max
+          float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+          if (valid == ~0u) {
+#pragma unroll
+            for (int i = 0; i < kHalf; ++i) mx[i & 3] = fmaxf(mx[i & 3], s[i]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < kHalf; ++i) {
+              s[i] = (valid >> i & 1u) ? s[i] : -INFINITY;
+              mx[i & 3] = fmaxf(mx[i & 3], s[i]);
+            }
+          }
+          const float mine = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+          mxbuf[(sbuf * 2 + wg) * 128 + h] = mine;
+          mbar_arrive_warp(&sb->mx_bar[sbuf]);
+          if (!mbar_wait_warp(&sb->mx_bar[sbuf], (uint32_t)(it >> 1) & 1u, wc)) { ok = false; break; }
+          const float mt_ = fmaxf(mine, mxbuf[(sbuf * 2 + (wg ^ 1)) * 128 + h]);
+          float alpha = 1.0f;
+          const bool need = mt_ > m + 8.0f;
+          if (need) {
+            alpha = fast_exp2(m - mt_);   // 0 when m is -inf
+            m = mt_;
+          }
+          float ps[4] = {0.f, 0.f, 0.f, 0.f};
+          if (m != -INFINITY) {
+            // masked logits are -inf and m is finite: their exp2 is exactly 0
+#pragma unroll
+            for (int i = 0; i < kHalf; ++i) {
+              s[i] = fast_exp2(s[i] - m);
+              ps[i & 3] += s[i];
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < kHalf; ++i) s[i] = 0.0f;
+          }
+          l = l * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
+
+          // P . C of the previous tile must be done: it reads the P buffer, and O is rescaled
+          if (!mbar_wait_warp(&sb->p_empty, ((uint32_t)it & 1u) ^ 1u, wc)) { ok = false; break; }
+          tc_fence_after();
+          if (__any_sync(0xffffffffu, need && t > 0)) {
+            // O holds the tiles < t of this unit: each warpgroup rescales half of its columns
+#pragma unroll 1
+            for (int c = wg * (Lay::kPvN / 2); c < (wg + 1) * (Lay::kPvN / 2); c += 16) {
+              uint32_t r[16];
+              tmem_ld16(lane_addr + Tm::kO + c, r);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+              tmem_st16(lane_addr + Tm::kO + c, r);
+            }
+            tmem_wait_st();
+          }
+          // this half of P (bf16) into shared memory: head h's row, K columns [32 wg, 32 wg + 32)
+#pragma unroll
+          for (int k = 0; k < kHalf / 8; ++k)
+            st_shared_v4(smem_u32(smem + Sm::kOffP + swizzled_offset((uint32_t)h, (uint32_t)(wg * (kHalf / 8) + k) * 16, 128)),
+                         pack_bf16x2(s[8 * k], s[8 * k + 1]), pack_bf16x2(s[8 * k + 2], s[8 * k + 3]),
+                         pack_bf16x2(s[8 * k + 4], s[8 * k + 5]), pack_bf16x2(s[8 * k + 6], s[8 * k + 7]));
+          fence_proxy_async_smem();
+          tc_fence_before();
+          mbar_arrive_warp(&sb->p_full);   // P written (and O rescaled) by this warp
+        }
+#pragma unroll
+        for (int i = 0; i < kHalf; ++i) s[i] = sn[i];
       }
+      s_it = it0 + ntiles;
       if (!ok) break;
-      mbar_arrive(&sb->tab_free[buf]);
+      mbar_arrive_warp(&sb->tab_free[buf]);
       // ---- unit epilogue: normalise O and write it out
       if (ntiles > 0) {
         if (!mbar_wait_warp(&sb->o_full, (uint32_t)o_it & 1u, wc)) { ok = false; break; }
@@ -894,7 +959,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // every thread has read the last tile's peer logits before a staging slice is reused,
         // and the two halves' sums are visible
         lbuf[wg * 128 + h] = l;
-        mbar_arrive(&sb->epi_sync);
+        mbar_arrive_warp(&sb->epi_sync);
         if (!mbar_wait_warp(&sb->epi_sync, (uint32_t)e_it & 1u, wc)) { ok = false; break; }
         ++e_it;
         l += lbuf[(wg ^ 1) * 128 + h];
@@ -912,7 +977,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const bool partial = un.rec >= 0;
       const int c_lo = wg * (Lay::kPvN / 2), c_hi = (wg + 1) * (Lay::kPvN / 2);
       if (ntiles > 0) {
-        uint8_t* slice = (wg == 0 ? smem + Sm::kOffP : smem + Sm::kOffSx + last_sbuf * Sm::kSxBytes) + quad * 4096;
+        uint8_t* slice = (wg == 0 ? smem + Sm::kOffP : smem + Sm::kOffSx + last_sbuf * 2 * Sm::kSxHalf) + quad * 4096;
         if (!partial) {
           // the output, bf16: 64 columns (128 bytes) per head and round
           uint16_t* obase = p.out + (long long)bj * p.H * p.DL + rank * Lay::kPvN;
@@ -998,11 +1063,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // warpgroup 1 staged through the whole exchange buffer of the last tile: it releases
         // both halves (deferred from that tile)
         __syncwarp();
-        mbar_arrive_cluster_relaxed(&sb->sx_free[last_sbuf][0], peer);
-        mbar_arrive_cluster_relaxed(&sb->sx_free[last_sbuf][1], peer);
+        fence_proxy_async_smem();   // the peer's next bulk copy into this buffer comes after our stores
+        mbar_arrive_cluster_warp(&sb->sx_free[last_sbuf][0], peer);
+        mbar_arrive_cluster_warp(&sb->sx_free[last_sbuf][1], peer);
       }
       tc_fence_before();   // our reads of O come before the next unit's first P . C
     }
+    // drain: this CTA's bulk copies into the peer are complete before the final cluster barrier
+    if (leader) bulk_wait_all();
   }
   tc_fence_before();
   __syncthreads();
@@ -1089,10 +1157,44 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineK
   if (d8 == 0 && p.lse) p.lse[row] = wsum > 0.0f ? mx + logf(wsum) : -INFINITY;
 }
 
+// The dynamic shared memory of a launch: at most two CTAs per SM may share the 512 TMEM columns
+// (kTmemCols each <= 256 when two fit), so a small layout still takes 100 KB.
+template <int DL, int DR>
+size_t attend_launch_smem() {
+  using Sm = AttnSmem<AttnLayout<DL, DR>>;
+  return Sm::kBytes < 100 * 1024 ? 100 * 1024 : Sm::kBytes;
+}
+
+// How many 2-CTA clusters of the kernel the device holds at once (0 if the runtime cannot say).
+// A cluster's CTAs must sit in one GPC, so this can be below half the SM count.
+template <int DL, int DR, bool KV8>
+int attend_clusters_impl() {
+  const size_t smem = attend_launch_smem<DL, DR>();
+  if (cudaFuncSetAttribute(sparse_attend_kernel<DL, DR, KV8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return 0;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.gridDim = dim3(2, 1, 1);
+  cfg.blockDim = dim3(kAttnThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, sparse_attend_kernel<DL, DR, KV8>, &cfg) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+
 template <int DL, int DR, bool KV8>
 cudaError_t launch_attend_impl(const AttnKernelParams& p, const CUtensorMap& q_rope, int n_clusters,
                                bool pdl, cudaStream_t stream) {
-  using Sm = AttnSmem<AttnLayout<DL, DR>>;
   {
     // the warpgroup register split assumes the launch allocation kLaunchRegs per thread
     cudaFuncAttributes fa;
@@ -1100,8 +1202,7 @@ cudaError_t launch_attend_impl(const AttnKernelParams& p, const CUtensorMap& q_r
     if (e != cudaSuccess) return e;
     if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
   }
-  // at most two CTAs per SM may share the 512 TMEM columns (kTmemCols each <= 256 when two fit)
-  const size_t smem = Sm::kBytes < 100 * 1024 ? 100 * 1024 : Sm::kBytes;
+  const size_t smem = attend_launch_smem<DL, DR>();
   cudaError_t e = cudaFuncSetAttribute(sparse_attend_kernel<DL, DR, KV8>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -1134,6 +1235,14 @@ cudaError_t launch_attend_impl(const AttnKernelParams& p, const CUtensorMap& q_r
 size_t attend_smem_bytes(int dl, int dr) {
   if (dl == 512 && dr == 64) return AttnSmem<AttnLayout<512, 64>>::kBytes;
   if (dl == 64 && dr == 16) return AttnSmem<AttnLayout<64, 16>>::kBytes;
+  return 0;
+}
+
+int attend_max_clusters(int dl, int dr, bool kv8) {
+  if (dl == 512 && dr == 64)
+    return kv8 ? attend_clusters_impl<512, 64, true>() : attend_clusters_impl<512, 64, false>();
+  if (dl == 64 && dr == 16)
+    return kv8 ? attend_clusters_impl<64, 16, true>() : attend_clusters_impl<64, 16, false>();
   return 0;
 }
 
