@@ -779,11 +779,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint32_t* mt = mask_tab + buf * (kAttnMaxSplitRows / 32);
       float m = -INFINITY, l = 0.0f;   // m is the same in both warpgroups; l covers this half
       // Software pipeline over the unit's tiles: pass t first sends tile t+1's partial logits to
-      // the peer (read from TMEM, encoded, stored into the peer's exchange buffer), then finishes
-      // tile t, whose peer half arrived during pass t-1, so each DSMEM transfer overlaps the
-      // softmax of the tile before it.  s holds this warpgroup's exact fp32 partials of tile t,
-      // sn those of tile t+1.
-      float s[kHalf], sn[kHalf];
+      // the peer (read from TMEM, encoded, staged, bulk-copied), then finishes tile t, whose peer
+      // half arrived during pass t-1, so each DSMEM transfer overlaps the softmax of the tile
+      // before it.  Tile t's exact fp32 partials are read from TMEM a second time when it is
+      // finished (a tile's S buffer is released only then; the S issuer still runs two tiles
+      // ahead with its two buffers), which keeps one tile of logits in registers, not two.
+      float s[kHalf];
       const int it0 = s_it;
       for (int t = -1; t < ntiles; ++t) {
         if (t + 1 < ntiles) {
@@ -809,10 +810,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
             for (int c = 0; c < 2; ++c)
 #pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                sn[16 * c + i] = __uint_as_float(r[c][i]);
-                amax = fmaxf(amax, fabsf(sn[16 * c + i]));
-              }
+              for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(__uint_as_float(r[c][i])));
             amax *= fabsf(p.scale_log2);
             // e with amax 2^e < 2^14: amax < 2^E for E = (biased exponent of amax) - 126
             const int E = (int)((__float_as_uint(amax) >> 23) & 0xffu) - 126;
@@ -823,16 +821,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               uint32_t enc[4];
 #pragma unroll
               for (int i = 0; i < 4; ++i) {
-                const float y0 = fmaf(sn[8 * gi + 2 * i], sc, kMagic);
-                const float y1 = fmaf(sn[8 * gi + 2 * i + 1], sc, kMagic);
+                const int j = 8 * gi + 2 * i;   // row pair (j, j + 1) of this half
+                const float y0 = fmaf(__uint_as_float(r[j >> 4][j & 15]), sc, kMagic);
+                const float y1 = fmaf(__uint_as_float(r[(j + 1) >> 4][(j + 1) & 15]), sc, kMagic);
                 enc[i] = prmt(__float_as_uint(y0), __float_as_uint(y1), 0x5410u);
               }
               st_shared_v4(smem_u32(xs + (gi * 128 + h) * 16), enc[0], enc[1], enc[2], enc[3]);
             }
             *reinterpret_cast<int*>(xs + Sm::kSxCodes + h * 4) = e;
           }
-          tc_fence_before();
-          mbar_arrive_warp(&sb->s_empty[sb1]);   // this warpgroup's reads of the partial are done
           fence_proxy_async_smem();           // the copy reads the staging through the async proxy
           mbar_arrive_warp(&sb->xs_full[wg]);
           bool sent = true;
@@ -858,6 +855,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const int live = first_neg - t * kRows - wg * kHalf;   // rows past the first -1 are padding
           if (live < kHalf) valid &= live > 0 ? (1u << live) - 1u : 0u;
           // the peer's half for the same rows: logit = own exact partial + decoded peer partial
+          {
+            // this half's exact partials of tile t, read again; then the S buffer is free
+            uint32_t r[2][16];
+#pragma unroll
+            for (int c = 0; c < 2; ++c) tmem_ld16(lane_addr + Tm::kS + sbuf * kRows + wg * kHalf + c * 16, r[c]);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+#pragma unroll
+              for (int i = 0; i < 16; ++i) s[16 * c + i] = __uint_as_float(r[c][i]);
+          }
+          tc_fence_before();
+          mbar_arrive_warp(&sb->s_empty[sbuf]);   // this warpgroup's reads of the partial are done
           // (the bytes come from the peer's bulk copy: the barrier's completion makes them visible)
           if (!mbar_wait_warp(&sb->sx_ready[sbuf][wg], (uint32_t)(it >> 1) & 1u, wc)) { ok = false; break; }
           last_sbuf = sbuf;
@@ -946,8 +956,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           tc_fence_before();
           mbar_arrive_warp(&sb->p_full);   // P written (and O rescaled) by this warp
         }
-#pragma unroll
-        for (int i = 0; i < kHalf; ++i) s[i] = sn[i];
       }
       s_it = it0 + ntiles;
       if (!ok) break;
