@@ -534,7 +534,7 @@ sia_status sia_fused_decode(const sia_index_args* ia, const sia_attend_args* aa,
   sia_status st = plan_index(ia, &ip, true);
   if (st != SIA_OK) return st;
   // the Top-K grid holds one SM per CTA while the attention grid is launched
-  const long long topk_ctas = (long long)ip.tp.B * ip.tp.J * ip.tp.cluster;
+  const long long topk_ctas = topk_grid_ctas(ip.tp);
   st = plan_attend(aa, &ap, true, (int)std::min<long long>(topk_ctas, sm_count()));
   if (st != SIA_OK) return st;
   const size_t need = round_up(ip.ws_scores, 256) + round_up(ap.ws_part, 256);

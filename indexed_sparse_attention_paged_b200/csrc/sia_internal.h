@@ -149,6 +149,8 @@ struct AppendKernelParams {
 // dependent launch on the previous kernel of the stream.
 cudaError_t launch_index_score(const IndexKernelParams& p, const CUtensorMap& kmap, const CUtensorMap& qmap, int grid,
                                bool pdl, cudaStream_t stream);
+// CTAs of the Top-K grid launch_topk starts for these parameters.
+long long topk_grid_ctas(const TopkKernelParams& p);
 cudaError_t launch_topk(const TopkKernelParams& p, bool pdl, cudaStream_t stream);
 // q_rope: 2-D map over the query rows [B*J*H, DL+DR] whose box is one CTA's rope slice of 128 heads
 cudaError_t launch_sparse_attend(const AttnKernelParams& p, const CUtensorMap& q_rope,

@@ -11,9 +11,9 @@
 // Three MSB-first radix passes (11, 11, 10 bits) find the exact K-th largest key T; the
 // selection is then every key > T plus the lowest-positioned keys == T, compacted in position
 // order with prefix sums, which makes the output ascending without a sort.
-//   - Rows of up to 16384 positions (topk_row_kernel): one CTA of 1024 threads per row, 16
-//     consecutive keys per thread in registers, shared-memory histograms with plain atomics,
-//     three barriers per pass.
+//   - Rows of up to 16384 positions (topk_row_kernel): 1024 threads per row (512 and two rows
+//     per CTA for rows of up to 8192), 16 consecutive keys per thread in registers,
+//     shared-memory histograms with plain atomics, three barriers per pass.
 //   - Longer rows (topk_kernel): a thread-block cluster of 2-16 CTAs per row, each keeping a
 //     slice of the keys in shared memory; the per-CTA digit histograms are summed across the
 //     cluster through distributed shared memory.
@@ -213,24 +213,39 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkKernelP
 
 
 // ---------------------------------------------------------------------------------------------
-// Rows of at most kRowKeys positions: one CTA of 1024 threads per query row, each thread holding
-// 16 consecutive keys in registers (its share is contiguous, so thread order is position order).
+// Rows of at most kRowKeys positions: one CTA of 1024 threads holds R rows, a group of 1024 / R
+// threads per row, each thread holding 16 consecutive keys in registers (its share is
+// contiguous, so thread order is position order).  Two rows per CTA when rows have at most 8192
+// positions: the same threads per row, half the SMs (the attention grid launched behind this
+// one gets them).  Each group synchronises on its own named barrier.
 constexpr int kRowThreads = 1024;
 constexpr int kRowPer = 16;
 constexpr int kRowKeys = kRowThreads * kRowPer;
 
 struct RowShared {
   uint32_t hist[2][kBins];          // alternate passes use alternate histograms
-  int wtot[kRowThreads / 32];       // per-warp totals of the bin scan
-  int warp_a[kRowThreads / 32];
-  int warp_b[kRowThreads / 32];
+  int wtot[32];                     // per-warp totals of the bin scan
+  int warp_a[32];
+  int warp_b[32];
   uint32_t sel_prefix;
   int sel_krem;
 };
 
-// Exclusive prefix sums of (a, b) over the CTA's threads in thread order, and their totals.
-__device__ __forceinline__ void row_scan2(int a, int b, int& ea, int& eb, int& ta, int& tb, RowShared* sh) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+template <int R>
+__device__ __forceinline__ void group_sync(int g) {
+  if (R == 1) {
+    __syncthreads();
+  } else {
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + g), "n"(kRowThreads / R) : "memory");
+  }
+}
+
+// Exclusive prefix sums of (a, b) over the group's threads in thread order, and their totals.
+template <int R>
+__device__ __forceinline__ void row_scan2(int a, int b, int& ea, int& eb, int& ta, int& tb, RowShared* sh, int g,
+                                          int gt) {
+  constexpr int kWarps = kRowThreads / R / 32;
+  const int lane = gt & 31, warp = gt >> 5;
   int ia = a, ib = b;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -238,50 +253,58 @@ __device__ __forceinline__ void row_scan2(int a, int b, int& ea, int& eb, int& t
     if (lane >= o) { ia += va; ib += vb; }
   }
   if (lane == 31) { sh->warp_a[warp] = ia; sh->warp_b[warp] = ib; }
-  __syncthreads();
+  group_sync<R>(g);
   if (warp == 0) {
-    int xa = sh->warp_a[lane], xb = sh->warp_b[lane];
+    const int xa = lane < kWarps ? sh->warp_a[lane] : 0, xb = lane < kWarps ? sh->warp_b[lane] : 0;
     int sa = xa, sb_ = xb;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int va = __shfl_up_sync(0xffffffffu, sa, o), vb = __shfl_up_sync(0xffffffffu, sb_, o);
       if (lane >= o) { sa += va; sb_ += vb; }
     }
-    sh->warp_a[lane] = sa - xa;   // exclusive warp offsets
-    sh->warp_b[lane] = sb_ - xb;
+    if (lane < kWarps) {
+      sh->warp_a[lane] = sa - xa;   // exclusive warp offsets
+      sh->warp_b[lane] = sb_ - xb;
+    }
     if (lane == 31) { sh->sel_prefix = (uint32_t)sa; sh->sel_krem = sb_; }   // totals (scratch)
   }
-  __syncthreads();
+  group_sync<R>(g);
   ea = sh->warp_a[warp] + ia - a;
   eb = sh->warp_b[warp] + ib - b;
   ta = (int)sh->sel_prefix;
   tb = sh->sel_krem;
-  __syncthreads();
+  group_sync<R>(g);
 }
 
+template <int R>
 __global__ void __launch_bounds__(kRowThreads, 1) topk_row_kernel(const TopkKernelParams p) {
-  __shared__ RowShared shm;
-  RowShared* sh = &shm;
-  const int tid = threadIdx.x;
-  const long long row = blockIdx.x;
-  const int b = (int)(row / p.J), j = (int)(row - (long long)b * p.J);
-  int32_t* out = p.topk + row * p.K;
+  constexpr int kGT = kRowThreads / R;     // threads per row
+  constexpr int kWarps = kGT / 32;
+  constexpr int kBpt = kBins / kGT;        // histogram bins per thread in the bin scan
+  __shared__ RowShared shm[R];
+  const int g = threadIdx.x / kGT, gt = threadIdx.x - g * kGT;
+  RowShared* sh = &shm[g];
+  const long long row = (long long)blockIdx.x * R + g;
+  const long long nrows = (long long)p.B * p.J;
 
   pdl_wait_primary();  // scores come from the previous kernel on the stream
   // the next kernel (attention) may be scheduled now: it only reads our output after its own
   // griddepcontrol.wait, which waits for this whole grid to finish
   pdl_launch_dependents();
+  if (row >= nrows) return;   // a whole group (the grid's last CTA when the rows are odd)
 
+  const int b = (int)(row / p.J), j = (int)(row - (long long)b * p.J);
+  int32_t* out = p.topk + row * p.K;
   bool bad = false;
   const int pos = query_position(p.seq_lens, p.q_pos, p.J, b, j, p.Lpad, &bad);
-  if (bad && tid == 0) report(p.status, SIA_DEV_BAD_POSITION);
+  if (bad && gt == 0) report(p.status, SIA_DEV_BAD_POSITION);
   const int n = pos + 1;
   if (n <= p.K) {
-    for (int i = tid; i < p.K; i += kRowThreads) out[i] = i < n ? i : -1;
+    for (int i = gt; i < p.K; i += kGT) out[i] = i < n ? i : -1;
     return;
   }
-  // this thread's keys: positions [tid*16, tid*16+16) of the visible range
-  const int base = tid * kRowPer;
+  // this thread's keys: positions [gt*16, gt*16+16) of the visible range
+  const int base = gt * kRowPer;
   uint32_t key[kRowPer];
   const float* src = p.scores + row * p.Lpad + base;
   if (base + kRowPer <= n) {
@@ -303,37 +326,41 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_row_kernel(const TopkKern
   int krem = p.K;
   const int shifts[3] = {21, 10, 0};
   const int widths[3] = {11, 11, 10};
-  for (int i = tid; i < kBins; i += kRowThreads) sh->hist[0][i] = 0;
-  __syncthreads();
+  for (int i = gt; i < kBins; i += kGT) sh->hist[0][i] = 0;
+  group_sync<R>(g);
 #pragma unroll 1
   for (int pass = 0; pass < 3; ++pass) {
     uint32_t* hist = sh->hist[pass & 1];
     // the other histogram is cleared for the next pass (nobody reads it in this one)
-    for (int i = tid; i < kBins; i += kRowThreads) sh->hist[(pass + 1) & 1][i] = 0;
+    for (int i = gt; i < kBins; i += kGT) sh->hist[(pass + 1) & 1][i] = 0;
     const int sh_ = shifts[pass], hi_shift = sh_ + widths[pass];
     const uint32_t dmask = (1u << widths[pass]) - 1u;
 #pragma unroll
     for (int i = 0; i < kRowPer; ++i)
       if (i < nmine && (pass == 0 || (key[i] >> hi_shift) == prefix)) atomicAdd(&hist[(key[i] >> sh_) & dmask], 1u);
-    __syncthreads();
-    // thread t owns bins 2t, 2t+1 counted from the top; "above" = keys in higher bins, by a warp
-    // scan plus the totals of the warps before (each warp adds those up itself)
-    const int lane = tid & 31, wid = tid >> 5;
-    const int hi_bin = kBins - 2 - 2 * tid;        // reversed: thread 0 owns the two top bins
-    const int c1 = (int)hist[hi_bin + 1], c0 = (int)hist[hi_bin];
-    int incl = c0 + c1;
+    group_sync<R>(g);
+    // thread gt owns kBpt consecutive bins counted from the top; "above" = keys in higher bins,
+    // by a warp scan plus the totals of the warps before (each warp scans those itself)
+    const int lane = gt & 31, wid = gt >> 5;
+    const int lo_bin = kBins - kBpt * (gt + 1);   // thread 0 owns the top bins
+    int cnt[kBpt];
+    int mine = 0;
+#pragma unroll
+    for (int k = 0; k < kBpt; ++k) {
+      cnt[k] = (int)hist[lo_bin + kBpt - 1 - k];   // cnt[0] is this thread's highest bin
+      mine += cnt[k];
+    }
+    int incl = mine;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int v = __shfl_up_sync(0xffffffffu, incl, o);
       if (lane >= o) incl += v;
     }
     if (lane == 31) sh->wtot[wid] = incl;
-    __syncthreads();
-    // keys in the bins of the warps before this one: an exclusive warp scan of the 32 warp
-    // totals (one load and five shuffles instead of a loop over up to 31 totals)
+    group_sync<R>(g);
     int before;
     {
-      const int wt = sh->wtot[lane];
+      const int wt = lane < kWarps ? sh->wtot[lane] : 0;
       int sc = wt;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -342,28 +369,29 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_row_kernel(const TopkKern
       }
       before = __shfl_sync(0xffffffffu, sc - wt, wid);
     }
-    const int ex = before + incl - (c0 + c1);
-    if (ex < krem && krem <= ex + c1) {
-      sh->sel_prefix = (prefix << widths[pass]) | (uint32_t)(hi_bin + 1);
-      sh->sel_krem = krem - ex;
-    } else if (ex + c1 < krem && krem <= ex + c1 + c0) {
-      sh->sel_prefix = (prefix << widths[pass]) | (uint32_t)hi_bin;
-      sh->sel_krem = krem - ex - c1;
+    int ex = before + incl - mine;   // keys in bins above this thread's
+#pragma unroll
+    for (int k = 0; k < kBpt; ++k) {
+      if (ex < krem && krem <= ex + cnt[k]) {
+        sh->sel_prefix = (prefix << widths[pass]) | (uint32_t)(lo_bin + kBpt - 1 - k);
+        sh->sel_krem = krem - ex;
+      }
+      ex += cnt[k];
     }
-    __syncthreads();
+    group_sync<R>(g);
     prefix = sh->sel_prefix;
     krem = sh->sel_krem;
   }
   const uint32_t T = prefix;
 
-  int gt = 0, eq = 0;
+  int gtc = 0, eqc = 0;
 #pragma unroll
   for (int i = 0; i < kRowPer; ++i) {
-    gt += (i < nmine && key[i] > T);
-    eq += (i < nmine && key[i] == T);
+    gtc += (i < nmine && key[i] > T);
+    eqc += (i < nmine && key[i] == T);
   }
   int ex_gt, ex_eq, tot_gt, tot_eq;
-  row_scan2(gt, eq, ex_gt, ex_eq, tot_gt, tot_eq, sh);
+  row_scan2<R>(gtc, eqc, ex_gt, ex_eq, tot_gt, tot_eq, sh, g, gt);
   int gt_before = ex_gt, eq_before = ex_eq;
 #pragma unroll
   for (int i = 0; i < kRowPer; ++i) {
@@ -380,11 +408,22 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_row_kernel(const TopkKern
 
 }  // namespace
 
+long long topk_grid_ctas(const TopkKernelParams& p) {
+  const long long rows = (long long)p.B * p.J;
+  if (p.Lpad <= kRowKeys) return p.Lpad <= kRowKeys / 2 ? (rows + 3) / 4 * 2 : rows;
+  return rows * p.cluster;
+}
+
 cudaError_t launch_topk(const TopkKernelParams& p, bool pdl, cudaStream_t stream) {
   if (p.Lpad <= kRowKeys) {
+    const long long rows = (long long)p.B * p.J;
+    const bool two = p.Lpad <= kRowKeys / 2;   // two rows per CTA
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    cfg.gridDim = dim3((unsigned)((long long)p.B * p.J), 1, 1);
+    cudaLaunchAttribute attr[2];
+    // two rows per CTA and CTA pairs launched as 2-CTA clusters: a cluster sits on an SM pair,
+    // so the grid blocks as few SM pairs as possible for the 2-CTA clusters of the attention
+    // grid launched behind it (a lone CTA on an SM pair leaves its neighbour unusable to them)
+    cfg.gridDim = dim3((unsigned)(two ? (rows + 3) / 4 * 2 : rows), 1, 1);
     cfg.blockDim = dim3(kRowThreads, 1, 1);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = stream;
@@ -394,9 +433,16 @@ cudaError_t launch_topk(const TopkKernelParams& p, bool pdl, cudaStream_t stream
       attr[na].val.programmaticStreamSerializationAllowed = 1;
       ++na;
     }
+    if (two) {
+      attr[na].id = cudaLaunchAttributeClusterDimension;
+      attr[na].val.clusterDim.x = 2;
+      attr[na].val.clusterDim.y = 1;
+      attr[na].val.clusterDim.z = 1;
+      ++na;
+    }
     cfg.attrs = attr;
     cfg.numAttrs = na;
-    return cudaLaunchKernelEx(&cfg, topk_row_kernel, p);
+    return two ? cudaLaunchKernelEx(&cfg, topk_row_kernel<2>, p) : cudaLaunchKernelEx(&cfg, topk_row_kernel<1>, p);
   }
   const size_t smem = sizeof(TopkShared) + (size_t)p.slice * sizeof(uint32_t);
   cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
