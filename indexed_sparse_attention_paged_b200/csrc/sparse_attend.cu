@@ -48,23 +48,26 @@ constexpr int kProducerWarps = 8;   // cp.async gather (+ TMA for the rope part 
 constexpr int kFirstProducerWarp = 8;
 constexpr int kMmaWarp = 16;    // S = Q . C^T issuer (and TMEM owner)
 constexpr int kPvWarp = 17;     // O += P . C issuer
-// warps 0-7 softmax, partial-logit exchange, q loader and epilogue (two warpgroups, one per half
-// of each tile's rows), 8-15 gather, 16 S = Q . C^T issuer, 17 O += P . C issuer
+// warps 0-3 softmax, 4-7 partial-logit exchange (both also load q and write the output), 8-15
+// gather, 16 S = Q . C^T issuer, 17 O += P . C issuer
 constexpr int kAttnThreads = 576;
 // Registers per thread after the split.  The block is launched with kLaunchRegs x 576
-// registers (ptxas' allocation for 576 threads); the two softmax warpgroups take 128 each (half a
-// tile of fp32 logits and their TMEM loads), the two gather warpgroups give back down to 64 and
+// registers (ptxas' allocation for 576 threads); the softmax warpgroup takes kSoftmaxRegs (a
+// tile's 64 fp32 logits per thread plus the rescale of O), the exchange warpgroup kExchangeRegs
+// (a tile's 64 partials per thread), the two gather warpgroups give back down to kGatherRegs and
 // the two MMA warps keep the launch value.  The sum stays within the launch allocation, so
 // setmaxnreg.inc never waits for registers that are not there.
 constexpr int kLaunchRegs = 96;
-constexpr int kSoftmaxRegs = 128;
+constexpr int kSoftmaxRegs = 152;
+constexpr int kExchangeRegs = 104;
 constexpr int kGatherRegs = 64;
-static_assert(256 * kSoftmaxRegs + 256 * kGatherRegs + 64 * kLaunchRegs <= kAttnThreads * kLaunchRegs,
+static_assert(128 * kSoftmaxRegs + 128 * kExchangeRegs + 256 * kGatherRegs + 64 * kLaunchRegs <=
+                  kAttnThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
 // setmaxnreg.inc may only raise a warp's count and setmaxnreg.dec only lower it
-static_assert(kSoftmaxRegs >= kLaunchRegs && kGatherRegs <= kLaunchRegs,
-              "the softmax warpgroups grow, the gather warpgroups shrink");
-constexpr int kStages = 4;          // latent-row tiles in flight per CTA
+static_assert(kSoftmaxRegs >= kLaunchRegs && kExchangeRegs >= kLaunchRegs && kGatherRegs <= kLaunchRegs,
+              "the softmax and exchange warpgroups grow, the gather warpgroups shrink");
+constexpr int kStages = 3;          // latent-row tiles in flight per CTA
 constexpr int kRopeSlots = 2;       // their rope parts (read by S = Q . C^T only) in flight
 constexpr int kRows = kAttnTileRows;
 
@@ -145,19 +148,20 @@ struct AttnSmem {
   static constexpr uint32_t kOffQ = 0;                                  // rope part of q only
   static constexpr uint32_t kOffC = (kOffQ + kQRopeBytes + 1023u) & ~1023u;
   static constexpr uint32_t kOffR = kOffC + kStages * kCStageBytes;
+
+  // Partial-logit exchange, one block per tile: 64 rows x 128 heads of int16 codes ([row / 8]
+  // [head] in 16-byte groups of 8 rows), then the 128 heads' power-of-two scale exponents
+  // (int32).  Sx holds the blocks the peer copies in and the stash this CTA's own blocks, two
+  // tiles each (by tile parity); a stash block is read by this CTA's softmax and is the source of
+  // the copy to the peer.
+  static constexpr uint32_t kSxCodes = kRows * 128 * 2;
+  static constexpr uint32_t kSxBlock = kSxCodes + 128 * 4;
   // P (bf16, 128 heads x kRows, 128B-swizzled K-major): the A operand of P . C
   static constexpr uint32_t kOffP = (kOffR + kRopeSlots * kCRopeBytes + 1023u) & ~1023u;
-  // Partial-logit exchange.  One block per half of a tile's rows (one softmax warpgroup): 32
-  // rows x 128 heads of int16 codes ([row / 8][head] in 16-byte groups of 8 rows), then the 128
-  // heads' power-of-two scale exponents (int32).  Sx holds the blocks the peer copies in for two
-  // tiles ([tile parity][half]); Xs this CTA's own two halves, staged for those bulk copies.
-  static constexpr uint32_t kSxCodes = (kRows / 2) * 128 * 2;
-  static constexpr uint32_t kSxHalf = kSxCodes + 128 * 4;
   static constexpr uint32_t kOffSx = kOffP + 128 * kRows * 2;
-  static constexpr uint32_t kOffXs = kOffSx + 4 * kSxHalf;
-  // the two softmax warpgroups' per-head tile maxima [2 tiles][2][128] and unit sums [2][128]
-  static constexpr uint32_t kOffMx = kOffXs + 2 * kSxHalf;
-  static constexpr uint32_t kOffL = kOffMx + 2 * 2 * 128 * 4;
+  static constexpr uint32_t kOffStash = kOffSx + 2 * kSxBlock;
+  // each head's sum and max of the softmax (read by the other warpgroup at a unit's end)
+  static constexpr uint32_t kOffL = kOffStash + 2 * kSxBlock;
   // the physical cache row of each Top-K entry of the unit being gathered (read by the gather
   // threads only, which rebuild it between units), then per unit (double-buffered) the validity
   // bits and each gather warp's lowest position of a -1 entry
@@ -168,24 +172,23 @@ struct AttnSmem {
   static constexpr uint32_t kBarBytes = 512;
   static constexpr uint32_t kBytes = kOffBar + kBarBytes;
   static_assert(kOffP % 1024 == 0, "P must sit on a 1024-byte swizzle atom");
-  static_assert(kSxHalf % 16 == 0 && kOffSx % 16 == 0 && kOffXs % 16 == 0, "bulk copies move 16-byte units");
-  static_assert(2 * kSxHalf >= 4 * 4096, "a tile's two halves also stage one warpgroup's output slices");
+  static_assert(kSxBlock % 16 == 0 && kOffSx % 16 == 0 && kOffStash % 16 == 0, "bulk copies move 16-byte units");
+  static_assert(kSxBlock >= 4 * 4096, "an exchange block also stages one warpgroup's output slices");
   static_assert(kBytes <= 232448, "shared memory over the 227 KB a CTA may opt into");
 };
 
 struct AttnBarriers {
   uint64_t c_full[kStages], c_empty[kStages];   // a tile's rows landed / latent stage free
   uint64_t r_empty[kRopeSlots];                 // rope slot free (its S = Q . C^T done)
-  uint64_t s_full[2], s_empty[2];   // logits ready in TMEM / read by both softmax warpgroups
-  uint64_t mx_bar[2];               // both warpgroups wrote their half's per-head tile max
+  uint64_t s_full[2], s_empty[2];   // partial logits in TMEM / read by the exchange warps
+  uint64_t stash_full[2], own_free[2];  // own block stashed / decoded by the softmax and copied
   uint64_t p_full;                  // all softmax threads wrote P (waited by the P . C issuer)
   uint64_t p_empty;                 // P . C of the previous tile done (P buffer and O free)
   uint64_t epi_sync;                // all softmax threads are past the unit's last tile
   uint64_t q_full, q_empty;       // q in TMEM written by the 128 loader threads / q reusable
   uint64_t q_tma;                 // the rope part of q landed (TMA bytes only)
   uint64_t o_full;
-  uint64_t sx_ready[2][2], sx_free[2][2];   // [tile][half]: the peer's half landed / was read
-  uint64_t xs_free[2], xs_full[2];          // [half]: staging reusable / staged by all 128 threads
+  uint64_t sx_ready[2], sx_free[2];  // [tile parity]: the peer's block landed / was decoded
   uint64_t g_sync;                          // every gather thread issued the unit's tiles
   uint64_t tab_full[2], tab_free[2];
   uint64_t mma_done, pv_done;
@@ -308,26 +311,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     for (int s = 0; s < kRopeSlots; ++s) mbar_init(&sb->r_empty[s], 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sb->s_full[s], 1);
-      mbar_init(&sb->s_empty[s], 8);           // the 8 softmax warps (one arrival per warp)
-      mbar_init(&sb->mx_bar[s], 8);
+      mbar_init(&sb->s_empty[s], 4);           // the 4 exchange warps (one arrival per warp)
+      mbar_init(&sb->stash_full[s], 4);        // the 4 exchange warps
+      mbar_init(&sb->own_free[s], 4 + 1);      // the 4 softmax warps and the copy's issuer
       mbar_init(&sb->tab_full[s], kProducerWarps);
       mbar_init(&sb->tab_free[s], 8 + 2);     // the softmax warps and both MMA threads
     }
-    mbar_init(&sb->p_full, 8);
+    mbar_init(&sb->p_full, 4);
     mbar_init(&sb->p_empty, 1);
     mbar_init(&sb->epi_sync, 8);
     mbar_init(&sb->q_full, 8);         // the 8 warps writing q into TMEM
     mbar_init(&sb->q_tma, 1);          // the rope TMA (or a plain arrive when this CTA has none)
     mbar_init(&sb->q_empty, 1);
     mbar_init(&sb->o_full, 1);
-    for (int s = 0; s < 2; ++s)
-      for (int g = 0; g < 2; ++g) {
-        mbar_init(&sb->sx_ready[s][g], 1);   // the peer's copy: its leader's arrive + the bytes
-        mbar_init(&sb->sx_free[s][g], 4);    // the 4 warps of the peer's warpgroup g
-      }
-    for (int g = 0; g < 2; ++g) {
-      mbar_init(&sb->xs_free[g], 1);
-      mbar_init(&sb->xs_full[g], 4);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sb->sx_ready[s], 1);   // the peer's copy: its issuer's arrive + the bytes
+      mbar_init(&sb->sx_free[s], 4);    // the peer's 4 softmax warps
     }
     mbar_init(&sb->g_sync, kProducerWarps);
     mbar_init(&sb->mma_done, 1);
@@ -714,31 +713,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- softmax + exchange
-    // Two warpgroups (warps 0-3 and 4-7, two warps per SM sub-partition); thread = head h =
-    // TMEM lane, warpgroup wg owns rows [32 wg, 32 wg + 32) of every 64-row tile.  Per tile a
-    // warpgroup reads its half of this CTA's partial logits from TMEM, sends them to the peer CTA
-    // as int16 with one power-of-two scale per head (relative error at most 2^-15 of the half's
-    // largest partial), adds the peer's decoded half to its exact own partial (one rounding),
-    // agrees with the other warpgroup on each head's tile max through shared memory, and writes
-    // its half of P.  Per unit it also loads its part of q into TMEM and, at the end, its half of
-    // the output columns.
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
-    constexpr int kHalf = kRows / 2;
-    const int wg = warp >> 2;
+    // Two warpgroups, thread = head h = TMEM lane in both.  The exchange warpgroup (warps 4-7)
+    // reads each tile's partial logits out of TMEM (the S buffer is free again at once), encodes
+    // them as int16 with one power-of-two scale per head (relative error at most 2^-15 of the
+    // head's largest partial in the tile) into a local stash, and bulk-copies the stash into the
+    // peer CTA's buffer.  The softmax warpgroup (warps 0-3) decodes its own stash and the peer's
+    // block and adds them: both CTAs add the same two values, so their logits are bit-identical.
+    // Per unit both warpgroups load half of q into TMEM and write half of the output columns.
+    // One copy of the warpgroups' code per role, each behind its own register count.
+    auto role = [&](auto wg_c) __attribute__((always_inline)) {
+    constexpr int wg = decltype(wg_c)::value;
     const int quad = warp & 3;
     const int h = quad * 32 + lane;   // head = TMEM lane
     const uint32_t lane_addr = tmem_base + ((uint32_t)(quad * 32) << 16);
     const uint32_t sx_peer = mapa_shared(smem_u32(smem + Sm::kOffSx), peer);
-    const bool leader = (threadIdx.x & 127) == 0;   // issues this warpgroup's bulk copies
-    float* mxbuf = reinterpret_cast<float*>(smem + Sm::kOffMx);   // [2 tiles][2 warpgroups][128]
-    float* lbuf = reinterpret_cast<float*>(smem + Sm::kOffL);     // [2 warpgroups][128]
+    const bool leader = threadIdx.x == 128;   // issues the exchange warpgroup's bulk copies
+    float* lbuf = reinterpret_cast<float*>(smem + Sm::kOffL);     // [sum, max][128]
     int s_it = 0, u_it = 0, o_it = 0, e_it = 0;
     bool ok = true;
 
     const AttnRange rg{attn_pair_start(p.split, cluster_id), attn_pair_start(p.split, cluster_id + 1)};
     long long cursor = rg.g0;
     AttnUnit un;
-    int last_sbuf = 0;
     for (; ok && attn_next_unit(p, cluster_id, rg, cursor, un); ++u_it) {
       const int bj = un.bj;
       const int buf = u_it & 1;
@@ -777,38 +773,34 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int first_neg = unit_tiles(buf);
       const int ntiles = (first_neg + kRows - 1) / kRows;
       const uint32_t* mt = mask_tab + buf * (kAttnMaxSplitRows / 32);
-      float m = -INFINITY, l = 0.0f;   // m is the same in both warpgroups; l covers this half
-      // Software pipeline over the unit's tiles: pass t first sends tile t+1's partial logits to
-      // the peer (read from TMEM, encoded, staged, bulk-copied), then finishes tile t, whose peer
-      // half arrived during pass t-1, so each DSMEM transfer overlaps the softmax of the tile
-      // before it.  Tile t's exact fp32 partials are read from TMEM a second time when it is
-      // finished (a tile's S buffer is released only then; the S issuer still runs two tiles
-      // ahead with its two buffers), which keeps one tile of logits in registers, not two.
-      float s[kHalf];
+      float m = -INFINITY, l = 0.0f;   // the softmax warpgroup's running max and sum of head h
       const int it0 = s_it;
-      for (int t = -1; t < ntiles; ++t) {
-        if (t + 1 < ntiles) {
-          const int it1 = it0 + t + 1, sb1 = it1 & 1;
-          // This half's partial logits go to the peer as int16 codes with one power-of-two scale
-          // per head, staged here and copied into the peer's buffer of the same tile parity and
-          // half with one bulk copy by the warpgroup's leader.  The staging is reused once the
-          // previous copy has read it.
-          if (leader) {
-            bulk_wait_read_all();
-            mbar_arrive(&sb->xs_free[wg]);
-          }
-          if (!mbar_wait_warp(&sb->xs_free[wg], (uint32_t)it1 & 1u, wc)) { ok = false; break; }
-          if (!mbar_wait_warp(&sb->s_full[sb1], (uint32_t)(it1 >> 1) & 1u, wc)) { ok = false; break; }
+      if (wg == 1) {
+        // ---- exchange warpgroup
+        for (int t = 0; t < ntiles; ++t) {
+          const int it = it0 + t, sb1 = it & 1;
+          if (!mbar_wait_warp(&sb->s_full[sb1], (uint32_t)(it >> 1) & 1u, wc)) { ok = false; break; }
           tc_fence_after();
-          uint8_t* xs = smem + Sm::kOffXs + wg * Sm::kSxHalf;
-          {
-            uint32_t r[2][16];
+          uint32_t r[4][16];
 #pragma unroll
-            for (int c = 0; c < 2; ++c) tmem_ld16(lane_addr + Tm::kS + sb1 * kRows + wg * kHalf + c * 16, r[c]);
-            tmem_wait_ld();
+          for (int c = 0; c < 4; ++c) tmem_ld16(lane_addr + Tm::kS + sb1 * kRows + c * 16, r[c]);
+          tmem_wait_ld();
+          tc_fence_before();
+          mbar_arrive_warp(&sb->s_empty[sb1]);   // the S buffer may be refilled
+          // the stash of tile it - 2 is free once the softmax decoded it and its copy to the
+          // peer read it (the most recent copy, tile it - 1's, may still be in flight)
+          if (it >= 2) {
+            if (leader) {
+              bulk_wait_read_prior();
+              mbar_arrive(&sb->own_free[sb1]);
+            }
+            if (!mbar_wait_warp(&sb->own_free[sb1], (uint32_t)((it >> 1) - 1) & 1u, wc)) { ok = false; break; }
+          }
+          uint8_t* xs = smem + Sm::kOffStash + sb1 * Sm::kSxBlock;
+          {
             float amax = 0.0f;
 #pragma unroll
-            for (int c = 0; c < 2; ++c)
+            for (int c = 0; c < 4; ++c)
 #pragma unroll
               for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(__uint_as_float(r[c][i])));
             amax *= fabsf(p.scale_log2);
@@ -817,11 +809,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const int e = amax > 0.0f ? min(max(14 - E, -100), 100) : 0;
             const float sc = p.scale_log2 * __uint_as_float((uint32_t)(127 + e) << 23);
 #pragma unroll
-            for (int gi = 0; gi < kHalf / 8; ++gi) {
+            for (int gi = 0; gi < kRows / 8; ++gi) {   // 16-byte group gi: rows [8 gi, 8 gi + 8)
               uint32_t enc[4];
 #pragma unroll
               for (int i = 0; i < 4; ++i) {
-                const int j = 8 * gi + 2 * i;   // row pair (j, j + 1) of this half
+                const int j = 8 * gi + 2 * i;
                 const float y0 = fmaf(__uint_as_float(r[j >> 4][j & 15]), sc, kMagic);
                 const float y1 = fmaf(__uint_as_float(r[(j + 1) >> 4][(j + 1) & 15]), sc, kMagic);
                 enc[i] = prmt(__float_as_uint(y0), __float_as_uint(y1), 0x5410u);
@@ -830,86 +822,90 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             }
             *reinterpret_cast<int*>(xs + Sm::kSxCodes + h * 4) = e;
           }
-          fence_proxy_async_smem();           // the copy reads the staging through the async proxy
-          mbar_arrive_warp(&sb->xs_full[wg]);
+          fence_proxy_async_smem();   // the copy reads the stash through the async proxy
+          mbar_arrive_warp(&sb->stash_full[sb1]);
           bool sent = true;
           if (leader) {
-            // the peer's buffer was last released either after its reads of tile it1 - 2
-            // (nothing to order against the copy) or, when that tile ended the previous unit,
-            // after the peer staged its output through it (generic stores: acquire them)
-            const uint32_t par = ((uint32_t)(it1 >> 1) & 1u) ^ 1u;
-            sent = mbar_wait(&sb->xs_full[wg], (uint32_t)it1 & 1u, wc) &&
-                   (t == 0 ? mbar_wait<true>(&sb->sx_free[sb1][wg], par, wc) : mbar_wait(&sb->sx_free[sb1][wg], par, wc));
+            // the peer's buffer of this parity was last released either after its softmax
+            // decoded tile it - 2 (nothing to order against the copy) or, when that tile ended
+            // the previous unit (it is this unit's second tile), after the peer staged its
+            // output through it (generic stores: acquire them)
+            const uint32_t par = ((uint32_t)(it >> 1) & 1u) ^ 1u;
+            sent = mbar_wait(&sb->stash_full[sb1], (uint32_t)(it >> 1) & 1u, wc) &&
+                   (t == 1 ? mbar_wait<true>(&sb->sx_free[sb1], par, wc) : mbar_wait(&sb->sx_free[sb1], par, wc));
             if (sent) {
-              mbar_arrive_expect_tx_remote(&sb->sx_ready[sb1][wg], peer, Sm::kSxHalf);
-              bulk_copy_to_cluster(sx_peer + (uint32_t)((sb1 * 2 + wg) * Sm::kSxHalf), smem_u32(xs), Sm::kSxHalf,
-                                   mapa_shared(smem_u32(&sb->sx_ready[sb1][wg]), peer));
+              mbar_arrive_expect_tx_remote(&sb->sx_ready[sb1], peer, Sm::kSxBlock);
+              bulk_copy_to_cluster(sx_peer + (uint32_t)(sb1 * Sm::kSxBlock), smem_u32(xs), Sm::kSxBlock,
+                                   mapa_shared(smem_u32(&sb->sx_ready[sb1]), peer));
               bulk_commit();
             }
           }
           if (!__shfl_sync(0xffffffffu, sent, 0)) { ok = false; break; }
         }
-        if (t >= 0) {
+      } else {
+        // ---- softmax warpgroup: all 64 rows of each tile per thread.  Online softmax in base 2
+        // with lazy rescaling of O (only when a head's max grows by more than 2^8).
+        for (int t = 0; t < ntiles; ++t) {
           const int it = it0 + t, sbuf = it & 1;
-          uint32_t valid = mt[2 * t + wg];                  // this half's 32 rows
-          const int live = first_neg - t * kRows - wg * kHalf;   // rows past the first -1 are padding
-          if (live < kHalf) valid &= live > 0 ? (1u << live) - 1u : 0u;
-          // the peer's half for the same rows: logit = own exact partial + decoded peer partial
-          {
-            // this half's exact partials of tile t, read again; then the S buffer is free
-            uint32_t r[2][16];
-#pragma unroll
-            for (int c = 0; c < 2; ++c) tmem_ld16(lane_addr + Tm::kS + sbuf * kRows + wg * kHalf + c * 16, r[c]);
-            tmem_wait_ld();
-#pragma unroll
-            for (int c = 0; c < 2; ++c)
-#pragma unroll
-              for (int i = 0; i < 16; ++i) s[16 * c + i] = __uint_as_float(r[c][i]);
+          uint32_t valid0 = mt[2 * t], valid1 = mt[2 * t + 1];
+          const int live = first_neg - t * kRows;   // rows past the first -1 are padding
+          if (live < 32) {
+            valid0 &= live > 0 ? (1u << live) - 1u : 0u;
+            valid1 = 0u;
+          } else if (live < 64) {
+            valid1 &= (1u << (live - 32)) - 1u;
           }
-          tc_fence_before();
-          mbar_arrive_warp(&sb->s_empty[sbuf]);   // this warpgroup's reads of the partial are done
-          // (the bytes come from the peer's bulk copy: the barrier's completion makes them visible)
-          if (!mbar_wait_warp(&sb->sx_ready[sbuf][wg], (uint32_t)(it >> 1) & 1u, wc)) { ok = false; break; }
-          last_sbuf = sbuf;
+          // this CTA's partials (stash) plus the peer's (its bulk copy; the barrier's completion
+          // makes the bytes visible): logit = decoded own + decoded peer, in that order on both
+          if (!mbar_wait_warp(&sb->stash_full[sbuf], (uint32_t)(it >> 1) & 1u, wc)) { ok = false; break; }
+          if (!mbar_wait_warp(&sb->sx_ready[sbuf], (uint32_t)(it >> 1) & 1u, wc)) { ok = false; break; }
+          float s[kRows];
           {
-            const uint8_t* rx = smem + Sm::kOffSx + (sbuf * 2 + wg) * Sm::kSxHalf;
-            const int pe = *reinterpret_cast<const int*>(rx + Sm::kSxCodes + h * 4);
-            const float dn = __uint_as_float((uint32_t)(127 - pe) << 23);
-            const float bias = -kMagic * dn;
+            const uint8_t* own = smem + Sm::kOffStash + sbuf * Sm::kSxBlock;
+            const uint8_t* prx = smem + Sm::kOffSx + sbuf * Sm::kSxBlock;
+            const int e0 = *reinterpret_cast<const int*>(own + Sm::kSxCodes + h * 4);
+            const int e1 = *reinterpret_cast<const int*>(prx + Sm::kSxCodes + h * 4);
+            const float dn0 = __uint_as_float((uint32_t)(127 - e0) << 23), bias0 = -kMagic * dn0;
+            const float dn1 = __uint_as_float((uint32_t)(127 - e1) << 23), bias1 = -kMagic * dn1;
+            // rank 0 adds (own, peer) and rank 1 (peer, own): the same two values in the same
+            // order on both CTAs
+            const uint8_t* first = rank == 0 ? own : prx;
+            const uint8_t* second = rank == 0 ? prx : own;
+            const float dnA = rank == 0 ? dn0 : dn1, biasA = rank == 0 ? bias0 : bias1;
+            const float dnB = rank == 0 ? dn1 : dn0, biasB = rank == 0 ? bias1 : bias0;
 #pragma unroll
-            for (int gi = 0; gi < kHalf / 8; ++gi) {
-              const uint4 pv4 = *reinterpret_cast<const uint4*>(rx + (gi * 128 + h) * 16);
-              const uint32_t q4[4] = {pv4.x, pv4.y, pv4.z, pv4.w};
+            for (int gi = 0; gi < kRows / 8; ++gi) {
+              const uint4 a4 = *reinterpret_cast<const uint4*>(first + (gi * 128 + h) * 16);
+              const uint4 b4 = *reinterpret_cast<const uint4*>(second + (gi * 128 + h) * 16);
+              const uint32_t qa[4] = {a4.x, a4.y, a4.z, a4.w}, qb[4] = {b4.x, b4.y, b4.z, b4.w};
 #pragma unroll
               for (int i = 0; i < 4; ++i) {
-                const float f0 = __uint_as_float(prmt(q4[i], 0x4B000000u, 0x7610u));
-                const float f1 = __uint_as_float(prmt(q4[i], 0x4B000000u, 0x7632u));
-                s[8 * gi + 2 * i] = fmaf(s[8 * gi + 2 * i], p.scale_log2, fmaf(f0, dn, bias));
-                s[8 * gi + 2 * i + 1] = fmaf(s[8 * gi + 2 * i + 1], p.scale_log2, fmaf(f1, dn, bias));
+                const float a0 = fmaf(__uint_as_float(prmt(qa[i], 0x4B000000u, 0x7610u)), dnA, biasA);
+                const float a1 = fmaf(__uint_as_float(prmt(qa[i], 0x4B000000u, 0x7632u)), dnA, biasA);
+                const float b0 = fmaf(__uint_as_float(prmt(qb[i], 0x4B000000u, 0x7610u)), dnB, biasB);
+                const float b1 = fmaf(__uint_as_float(prmt(qb[i], 0x4B000000u, 0x7632u)), dnB, biasB);
+                s[8 * gi + 2 * i] = a0 + b0;
+                s[8 * gi + 2 * i + 1] = a1 + b1;
               }
             }
           }
-          // the peer may refill its half of the exchange buffer; after the unit's last tile the
-          // buffer first serves the epilogue (released there)
-          if (t + 1 < ntiles) mbar_arrive_cluster_relaxed_warp(&sb->sx_free[sbuf][wg], peer);
-
-          // online softmax (base 2), lazy rescale; the two halves agree on the tile max
+          // both blocks are in registers: the stash may be rewritten (with the copy's read) and
+          // the peer may refill our buffer; after the unit's last tile the peer's block first
+          // stages the epilogue's output (released there)
+          mbar_arrive_warp(&sb->own_free[sbuf]);
+          if (t + 1 < ntiles) mbar_arrive_cluster_relaxed_warp(&sb->sx_free[sbuf], peer);
           float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-          if (valid == ~0u) {
+          if ((valid0 & valid1) == ~0u) {
 #pragma unroll
-            for (int i = 0; i < kHalf; ++i) mx[i & 3] = fmaxf(mx[i & 3], s[i]);
+            for (int i = 0; i < kRows; ++i) mx[i & 3] = fmaxf(mx[i & 3], s[i]);
           } else {
 #pragma unroll
-            for (int i = 0; i < kHalf; ++i) {
-              s[i] = (valid >> i & 1u) ? s[i] : -INFINITY;
+            for (int i = 0; i < kRows; ++i) {
+              s[i] = (((i < 32 ? valid0 : valid1) >> (i & 31)) & 1u) ? s[i] : -INFINITY;
               mx[i & 3] = fmaxf(mx[i & 3], s[i]);
             }
           }
-          const float mine = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-          mxbuf[(sbuf * 2 + wg) * 128 + h] = mine;
-          mbar_arrive_warp(&sb->mx_bar[sbuf]);
-          if (!mbar_wait_warp(&sb->mx_bar[sbuf], (uint32_t)(it >> 1) & 1u, wc)) { ok = false; break; }
-          const float mt_ = fmaxf(mine, mxbuf[(sbuf * 2 + (wg ^ 1)) * 128 + h]);
+          const float mt_ = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
           float alpha = 1.0f;
           const bool need = mt_ > m + 8.0f;
           if (need) {
@@ -920,13 +916,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (m != -INFINITY) {
             // masked logits are -inf and m is finite: their exp2 is exactly 0
 #pragma unroll
-            for (int i = 0; i < kHalf; ++i) {
+            for (int i = 0; i < kRows; ++i) {
               s[i] = fast_exp2(s[i] - m);
               ps[i & 3] += s[i];
             }
           } else {
 #pragma unroll
-            for (int i = 0; i < kHalf; ++i) s[i] = 0.0f;
+            for (int i = 0; i < kRows; ++i) s[i] = 0.0f;
           }
           l = l * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
 
@@ -934,22 +930,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (!mbar_wait_warp(&sb->p_empty, ((uint32_t)it & 1u) ^ 1u, wc)) { ok = false; break; }
           tc_fence_after();
           if (__any_sync(0xffffffffu, need && t > 0)) {
-            // O holds the tiles < t of this unit: each warpgroup rescales half of its columns
+            // O holds the tiles < t of this unit
 #pragma unroll 1
-            for (int c = wg * (Lay::kPvN / 2); c < (wg + 1) * (Lay::kPvN / 2); c += 16) {
-              uint32_t r[16];
-              tmem_ld16(lane_addr + Tm::kO + c, r);
+            for (int c = 0; c < Lay::kPvN; c += 16) {
+              uint32_t rr[16];
+              tmem_ld16(lane_addr + Tm::kO + c, rr);
               tmem_wait_ld();
 #pragma unroll
-              for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-              tmem_st16(lane_addr + Tm::kO + c, r);
+              for (int i = 0; i < 16; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * alpha);
+              tmem_st16(lane_addr + Tm::kO + c, rr);
             }
             tmem_wait_st();
           }
-          // this half of P (bf16) into shared memory: head h's row, K columns [32 wg, 32 wg + 32)
+          // P (bf16) into shared memory: head h's row, K columns = the tile's 64 rows
 #pragma unroll
-          for (int k = 0; k < kHalf / 8; ++k)
-            st_shared_v4(smem_u32(smem + Sm::kOffP + swizzled_offset((uint32_t)h, (uint32_t)(wg * (kHalf / 8) + k) * 16, 128)),
+          for (int k = 0; k < kRows / 8; ++k)
+            st_shared_v4(smem_u32(smem + Sm::kOffP + swizzled_offset((uint32_t)h, (uint32_t)k * 16, 128)),
                          pack_bf16x2(s[8 * k], s[8 * k + 1]), pack_bf16x2(s[8 * k + 2], s[8 * k + 3]),
                          pack_bf16x2(s[8 * k + 4], s[8 * k + 5]), pack_bf16x2(s[8 * k + 6], s[8 * k + 7]));
           fence_proxy_async_smem();
@@ -964,13 +960,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (ntiles > 0) {
         if (!mbar_wait_warp(&sb->o_full, (uint32_t)o_it & 1u, wc)) { ok = false; break; }
         ++o_it;
-        // every thread has read the last tile's peer logits before a staging slice is reused,
-        // and the two halves' sums are visible
-        lbuf[wg * 128 + h] = l;
+        // the softmax warpgroup has decoded the last tile (so the peer-logit buffer may stage
+        // output), and the exchange warpgroup takes each head's max and sum from it
+        if (wg == 0) {
+          lbuf[h] = l;
+          lbuf[128 + h] = m;
+        }
         mbar_arrive_warp(&sb->epi_sync);
         if (!mbar_wait_warp(&sb->epi_sync, (uint32_t)e_it & 1u, wc)) { ok = false; break; }
         ++e_it;
-        l += lbuf[(wg ^ 1) * 128 + h];
+        if (wg == 1) {
+          l = lbuf[h];
+          m = lbuf[128 + h];
+        }
       }
       tc_fence_after();
       const bool any = ntiles > 0 && l > 0.0f;
@@ -979,13 +981,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const bool real_head = h < p.H;
       // O rows (the bf16 output, or a piece's normalised fp32 partial): each warpgroup writes
       // half of this CTA's columns, staged through a 128B-swizzled 4 KB slice per warp
-      // (warpgroup 0 in the P buffer, free once the unit's last P . C is done; warpgroup 1 in the
-      // exchange buffer of the last tile, released below) so that each global store writes four
-      // whole 128-byte runs
+      // (the softmax warpgroup in the P buffer, free once the unit's last P . C is done; the
+      // exchange warpgroup in the last tile's peer-logit block, released to the peer only
+      // afterwards) so that each global store writes four whole 128-byte runs
       const bool partial = un.rec >= 0;
       const int c_lo = wg * (Lay::kPvN / 2), c_hi = (wg + 1) * (Lay::kPvN / 2);
       if (ntiles > 0) {
-        uint8_t* slice = (wg == 0 ? smem + Sm::kOffP : smem + Sm::kOffSx + last_sbuf * 2 * Sm::kSxHalf) + quad * 4096;
+        uint8_t* slice = (wg == 0 ? smem + Sm::kOffP : smem + Sm::kOffSx + ((it0 + ntiles - 1) & 1) * Sm::kSxBlock) + quad * 4096;
         if (!partial) {
           // the output, bf16: 64 columns (128 bytes) per head and round
           uint16_t* obase = p.out + (long long)bj * p.H * p.DL + rank * Lay::kPvN;
@@ -1068,17 +1070,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         else if (p.lse && rank == 0) p.lse[(long long)bj * p.H + h] = lse;
       }
       if (ntiles > 0 && wg == 1) {
-        // warpgroup 1 staged through the whole exchange buffer of the last tile: it releases
-        // both halves (deferred from that tile)
+        // the exchange warpgroup staged its output through the peer-logit buffer of the last
+        // tile: it releases that buffer to the peer now (deferred from the tile)
         __syncwarp();
         fence_proxy_async_smem();   // the peer's next bulk copy into this buffer comes after our stores
-        mbar_arrive_cluster_warp(&sb->sx_free[last_sbuf][0], peer);
-        mbar_arrive_cluster_warp(&sb->sx_free[last_sbuf][1], peer);
+        mbar_arrive_cluster_warp(&sb->sx_free[(it0 + ntiles - 1) & 1], peer);
       }
       tc_fence_before();   // our reads of O come before the next unit's first P . C
     }
     // drain: this CTA's bulk copies into the peer are complete before the final cluster barrier
     if (leader) bulk_wait_all();
+    };
+    if (warp < 4) {
+      asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
+      role(std::integral_constant<int, 0>{});
+    } else {
+      asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kExchangeRegs));
+      role(std::integral_constant<int, 1>{});
+    }
   }
   tc_fence_before();
   __syncthreads();
