@@ -649,6 +649,32 @@ class DecodeBench:
         }
 
 
+def bind_to_gpu_cpus(dev_index: int):
+    """Restrict this process to the CPUs NVML names as local to the GPU (its NUMA node), so that
+    the pinned host buffers of the end-to-end loop are allocated next to the GPU's PCIe root.
+    A process setting, not a GPU one; returns (cpus kept, the previous affinity) or None."""
+    try:
+        import pynvml
+        import torch
+        before = os.sched_getaffinity(0)
+        pr = torch.cuda.get_device_properties(dev_index)
+        bus = "%08x:%02x:%02x.0" % (pr.pci_domain_id, pr.pci_bus_id, pr.pci_device_id)
+        pynvml.nvmlInit()
+        try:
+            handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            words = (os.cpu_count() + 63) // 64
+            mask = pynvml.nvmlDeviceGetCpuAffinity(handle, words)
+        finally:
+            pynvml.nvmlShutdown()
+        cpus = {64 * w + b for w, m in enumerate(mask) for b in range(64) if (int(m) >> b) & 1} & before
+        if not cpus or cpus == before:
+            return None
+        os.sched_setaffinity(0, cpus)
+        return sorted(cpus), before
+    except Exception:
+        return None
+
+
 def main():
     args = parse()
     rank = int(os.environ.get("RANK", "0"))
@@ -666,6 +692,7 @@ def main():
     cuda_build.build()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    binding = bind_to_gpu_cpus(local)
     if world > 1:
         dist.init_process_group("nccl", device_id=dev, timeout=__import__("datetime").timedelta(seconds=120))
 
@@ -739,7 +766,9 @@ def main():
                 "loop": ("pipelined: 2 buffer slots, copy-in / compute / copy-out streams" if pipelined
                          else "serial: copy-in, fused call, copy-out on one stream") +
                         "; one packed pinned-host copy per direction per step",
-                "serial_ms_per_step": serial_ms},
+                "serial_ms_per_step": serial_ms,
+                "host_cpus": ("%d CPUs local to the GPU (NVML affinity)" % len(binding[0])) if binding
+                             else "unrestricted"},
         "gpu_launches": db.kernels_per_step * args.steps,
         "clocks": dict(clocks, window="nvidia-smi every 200 ms over a %.1f s soak of the same steps "
                                       "right before the timed region, the timed region and the "
@@ -773,6 +802,8 @@ def main():
         line["workloads"] = subs
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
+        if binding:
+            os.sched_setaffinity(0, binding[1])   # the oracle runs on all of the host's cores again
         n = max(4, min(16, oracle.num_threads()))
         line["cpu_baseline"] = cpu_baseline(host, list(range(n)))
     if rank == 0:
