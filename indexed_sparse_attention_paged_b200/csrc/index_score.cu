@@ -475,7 +475,8 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
               if (q0 + qq >= p.nq_sub) break;
               const int qloc = sub * p.nq_sub + q0 + qq;
               const float4* wq = reinterpret_cast<const float4*>(w_s + qloc * p.HP);
-              // four independent partial sums over the heads (w from shared memory, 4 per load)
+              // four independent partial sums over the heads (w from shared memory, 4 per load),
+              // updated two at a time by packed fp32 FMAs (each lane rounds as fmaf does)
               float a4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
               for (int hc = 0; hc < 4; ++hc) {
@@ -483,10 +484,10 @@ __global__ void __launch_bounds__(64 + 128 * NSUB, 1)
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                   const float4 wv = wq[hc * 4 + i];
-                  a4[0] = fmaf(wv.x, fmaxf(__uint_as_float(v[qq][hc][4 * i]), 0.0f), a4[0]);
-                  a4[1] = fmaf(wv.y, fmaxf(__uint_as_float(v[qq][hc][4 * i + 1]), 0.0f), a4[1]);
-                  a4[2] = fmaf(wv.z, fmaxf(__uint_as_float(v[qq][hc][4 * i + 2]), 0.0f), a4[2]);
-                  a4[3] = fmaf(wv.w, fmaxf(__uint_as_float(v[qq][hc][4 * i + 3]), 0.0f), a4[3]);
+                  fma_f32x2(a4[0], a4[1], wv.x, wv.y, fmaxf(__uint_as_float(v[qq][hc][4 * i]), 0.0f),
+                            fmaxf(__uint_as_float(v[qq][hc][4 * i + 1]), 0.0f));
+                  fma_f32x2(a4[2], a4[3], wv.z, wv.w, fmaxf(__uint_as_float(v[qq][hc][4 * i + 2]), 0.0f),
+                            fmaxf(__uint_as_float(v[qq][hc][4 * i + 3]), 0.0f));
                 }
               }
               const float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);

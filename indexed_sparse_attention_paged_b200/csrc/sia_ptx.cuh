@@ -206,6 +206,21 @@ __device__ __forceinline__ void bulk_wait_read_prior() { asm volatile("cp.async.
 // this thread's committed bulk copies are complete
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// ------------------------------------------------------------------ packed fp32 arithmetic
+
+// (d0, d1) = (a0 * b0 + d0, a1 * b1 + d1): two independent fp32 fused multiply-adds, each
+// rounded once to nearest even, issued as one sm_100 instruction on a register pair.
+__device__ __forceinline__ void fma_f32x2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %5};\n\t"
+      "mov.b64 rc, {%0, %1};\n\t"
+      "fma.rn.f32x2 rc, ra, rb, rc;\n\t"
+      "mov.b64 {%0, %1}, rc;\n\t}"
+      : "+f"(d0), "+f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
 // ------------------------------------------------------------------ proxies, PDL, cluster
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
