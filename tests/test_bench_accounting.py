@@ -52,3 +52,25 @@ def test_decode_batch_flops_and_the_roofline_bound():
     rs = bench.roofline_entry("k", ab["stage2"], af["stage2"], 0.05, pk, "bf16_tflops_sustained")
     # against the sustained peak the contraction takes 12.941 us, the bytes 12.947 us: a tie
     assert rs["bound"] == "hbm" and abs(rs["tensor_frac"] / rs["hbm_frac"] - 1.0) < 1e-3
+
+
+def test_recorded_dram_traffic_is_from_the_current_sources():
+    """The `traffic` the bench line carries comes from profiles/traffic.json, and only when that
+    capture was taken on the kernel sources as they are now (a hash of csrc/).  Every stage the
+    bench reports has such a record, and it is not far from the algorithmic bytes (a capture of
+    another workload, or of a kernel that re-reads its inputs, would be)."""
+    import json
+    import os
+    rec = json.load(open(os.path.join(os.path.dirname(bench.__file__), "profiles", "traffic.json")))
+    assert set(rec) >= {"index_topk", "sparse_attend"}
+    for stage in ("index_topk", "sparse_attend"):
+        assert rec[stage]["source_sha"] == bench.source_sha(), stage
+        assert rec[stage]["workload"] == "decode_b32_ctx8k"
+        assert bench.recorded_traffic(stage) == rec[stage]["dram_bytes_per_launch"]
+        assert "ncu" in rec[stage]["command"] and "--clock-control none" in rec[stage]["command"]
+    wl = workloads.WORKLOADS[2]
+    inputs = dict(workload=wl, batch=32, n_q=1, seq_lens=torch.full((32,), 8192, dtype=torch.int32))
+    ab = bench.algorithmic_bytes(inputs)
+    # the attention reads the selected rows once; the indexer reads every visible key once
+    assert 0.9 * ab["kv"] < rec["sparse_attend"]["dram_bytes_per_launch"] < 1.2 * (ab["total"] - ab["idx_k"])
+    assert 0.95 * ab["idx_k"] < rec["index_topk"]["dram_bytes_per_launch"] < 1.1 * ab["idx_k"] + 4e6
