@@ -1,5 +1,5 @@
 // sia_ptx.cuh -- thin inline-PTX wrappers for sm_100a used by the libsia kernels:
-// mbarriers (with bounded waits), TMA tensor loads (tiled and gather4), tcgen05 tensor-core
+// mbarriers (with bounded waits), TMA tensor loads (tiled), bulk copies, tcgen05 tensor-core
 // MMA / TMEM access, cluster shared memory, and programmatic dependent launch.
 #pragma once
 
